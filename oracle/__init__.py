@@ -1,0 +1,52 @@
+"""CPU oracle for LServe-style unified sparse attention -- TEST INFRASTRUCTURE ONLY.
+
+Plain, slow, fp64 numpy restatement of what the hot path computes, written
+from the LServe explainer page ("MLSys 2025論文解説: LServe — 統一疎アテンション
+による長文脈LLM推論の効率化", arXiv 2502.14866) and the LServe abstract page
+("LServe: Efficient Long-sequence LLM Serving with Unified Sparse Attention").
+
+Only tests, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline leg may
+import this package.  It shares no code with the CUDA library and imports
+nothing from it.  Inputs arrive as bf16 bit patterns (uint16) and are widened
+exactly to float64 here.
+
+Section references used throughout (all on the LServe explainer page unless
+stated otherwise):
+  [TD-static]   技術的詳細 › 静的スパーシティ (streaming heads, Lambda mask)
+  [TD-dynamic]  技術的詳細 › 動的スパーシティ, the equation for S^j
+  [TD-paging]   技術的詳細 › 階層的ページング (N_P = g * N_L, max-reduction)
+  [TD-unified]  技術的詳細 › 統一ブロックスパースアテンション (figure; 1/(1-r))
+  [TD-reuse]    技術的詳細 › Reusable Page Selection (k = 4, Table 6)
+  [Abstract]    LServe abstract page (block-wise skipping; constant page budget)
+
+Readings where the pages are silent (each is listed in the design notes):
+  R1 GQA: one page choice per KV head, ranked by the SUM over its G query
+     heads of S^j.                                          (parity unpinned)
+  R2 partial pages: only valid tokens count; empty logical pages are skipped.
+  R3 retrieval heads use pure top-K, nothing force-included.
+  R4 ties go to the lowest page index; selections are reported ascending.
+  R5 streaming decode is page-granular: sink pages [0, ceil(S/N_P)) plus every
+     page holding one of the last L tokens.
+  R6 Lambda prefill: block row i sees blocks {0..sink-1} and
+     [i - local + 1, i] (the diagonal counts as local).   (parity unpinned)
+  R7 retrieval heads in prefill are dense causal.
+  R8 softmax scale is a parameter (1/sqrt(D) in the harness); scores unscaled.
+"""
+from .lserve import (  # noqa: F401
+    widen_bf16,
+    page_stats,
+    head_scores,
+    logical_scores,
+    physical_scores,
+    select_top_k,
+    retrieval_pages,
+    streaming_pages,
+    page_tokens,
+    decode_attention,
+    decode_pair,
+    kv_blocks,
+    computed_blocks,
+    theoretical_speedup,
+    prefill_rows,
+    prefill_flops,
+)

@@ -1,0 +1,205 @@
+"""fp64 oracle functions -- test infrastructure only (see package docstring).
+
+Every function follows one step of the method in the page's order:
+  stats (k_min/k_max per logical page) -> S^j -> physical max -> top-K ->
+  attention over the chosen pages; and, for prefill, the block iterator ->
+  causal softmax attention over the allowed blocks.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+
+def widen_bf16(u16) -> np.ndarray:
+    """bf16 bit patterns -> float64 (exact: a bf16 is the top half of a float32)."""
+    u = np.asarray(u16, dtype=np.uint16)
+    return (u.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+# --- decode: page statistics [TD-dynamic] ------------------------------------
+
+def page_stats(k: np.ndarray, N_L: int):
+    """Channel-wise k_min^j / k_max^j of each logical page j.
+
+    [TD-dynamic]: k_min^j[i] and k_max^j[i] are the min and max of channel i
+    over the keys of logical page j.  R2: a partial last page uses only its
+    valid tokens.  k is [n][D] float64; returns two [ceil(n/N_L)][D] arrays.
+    """
+    n, D = k.shape
+    J = -(-n // N_L)
+    full = n // N_L
+    kmin = np.empty((J, D))
+    kmax = np.empty((J, D))
+    pages = k[:full * N_L].reshape(full, N_L, D)   # page j = rows [j*N_L, (j+1)*N_L)
+    kmin[:full] = pages.min(axis=1)
+    kmax[:full] = pages.max(axis=1)
+    if J > full:                                   # partial last page: valid rows only
+        kmin[full] = k[full * N_L:].min(axis=0)
+        kmax[full] = k[full * N_L:].max(axis=0)
+    return kmin, kmax
+
+
+# --- decode: query-centric score [TD-dynamic, Eq. S^j] --------------------------
+
+def head_scores(q: np.ndarray, kmin: np.ndarray, kmax: np.ndarray) -> np.ndarray:
+    """s[h, j] = sum_{i=1..D} max(q_h[i] * k_max^j[i], q_h[i] * k_min^j[i]).
+
+    [TD-dynamic], the equation for S^j, for each query head h of q [G][D].
+    """
+    q3 = q[:, None, :]
+    return np.maximum(q3 * kmax[None, :, :], q3 * kmin[None, :, :]).sum(axis=2)
+
+
+def logical_scores(q: np.ndarray, kmin: np.ndarray, kmax: np.ndarray) -> np.ndarray:
+    """S^j for one KV head: reading R1, the sum over its G query heads of s[h, j]."""
+    return head_scores(q, kmin, kmax).sum(axis=0)
+
+
+# --- decode: logical -> physical max [TD-paging] --------------------------------
+
+def physical_scores(S: np.ndarray, g: int) -> np.ndarray:
+    """P^m = max of S^j over the (valid) logical pages j in [m*g, m*g + g).
+
+    [TD-paging]: a physical page of N_P = g * N_L tokens is scored by the
+    max-reduction of the scores of the logical pages it contains.
+    """
+    M = -(-len(S) // g)
+    return np.array([S[m * g:min((m + 1) * g, len(S))].max() for m in range(M)])
+
+
+# --- decode: top-K physical pages [TD-unified figure "Top-K物理ページ"] --------------
+
+def select_top_k(P: np.ndarray, K: int) -> list:
+    """The K highest-scoring physical pages (all of them if there are <= K).
+
+    Ordering by (score descending, index ascending) puts ties on the lowest
+    index (R4); the chosen set is returned in ascending page order.  [Abstract]:
+    the page budget K is a constant, independent of the context length.
+    """
+    order = sorted(range(len(P)), key=lambda m: (-P[m], m))
+    return sorted(order[:min(K, len(P))])
+
+
+def retrieval_pages(q, k, n, N_L, N_P, K):
+    """Retrieval-head page choice for one (sequence, KV head):
+    stats -> S^j -> P^m -> top-K.  Returns (sel, P, S)."""
+    kmin, kmax = page_stats(k[:n], N_L)
+    S = logical_scores(q, kmin, kmax)
+    P = physical_scores(S, N_P // N_L)
+    return select_top_k(P, K), P, S
+
+
+def streaming_pages(n: int, N_P: int, sink: int, local: int) -> list:
+    """Pages a streaming head attends at decode (reading R5 of the Lambda mask
+    [TD-static]): the sink pages [0, ceil(sink/N_P)) plus every page holding one
+    of the last `local` tokens; ascending, without duplicates."""
+    npages = -(-n // N_P)
+    sink_pages = set(range(min(-(-sink // N_P), npages)))
+    first_local = max(0, n - local) // N_P
+    return sorted(sink_pages | set(range(first_local, npages)))
+
+
+def page_tokens(pages, n: int, N_P: int) -> np.ndarray:
+    """Valid token positions of the given physical pages (R2)."""
+    out = [np.arange(m * N_P, min((m + 1) * N_P, n)) for m in pages]
+    return np.concatenate(out) if out else np.zeros(0, dtype=np.int64)
+
+
+# --- decode attention [TD-unified; "Top-K物理ページ" / "Λ型マスク"] -----------------
+
+def decode_attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, tokens, scale: float):
+    """softmax(scale * q k_t) weighted sum of v_t over the given tokens, per head.
+
+    q [G][D], k/v [n][D]; returns (o [G][D], lse [G]) with lse the natural log
+    of sum_t exp(scale * q.k_t).  An empty token set gives o = 0, lse = -inf.
+    """
+    tokens = np.asarray(tokens, dtype=np.int64)
+    G, D = q.shape
+    if tokens.size == 0:
+        return np.zeros((G, D)), np.full(G, -np.inf)
+    z = scale * (q @ k[tokens].T)              # [G][T]
+    zmax = z.max(axis=1, keepdims=True)
+    e = np.exp(z - zmax)
+    lsum = e.sum(axis=1)
+    o = (e @ v[tokens]) / lsum[:, None]
+    return o, zmax[:, 0] + np.log(lsum)
+
+
+def decode_pair(q, k, v, n, kind, N_L, N_P, K, sink, local, scale):
+    """One (sequence, KV head) of a decode step: retrieval heads pick top-K
+    pages by S^j, streaming heads take sink + local pages; then attention.
+    Returns (o [G][D], lse [G], pages)."""
+    if kind == 0:
+        pages = retrieval_pages(q, k, n, N_L, N_P, K)[0]
+    else:
+        pages = streaming_pages(n, N_P, sink, local)
+    o, lse = decode_attention(q, k, v, page_tokens(pages, n, N_P), scale)
+    return o, lse, pages
+
+
+# --- prefill: block iterator [TD-static, TD-unified] ---------------------------
+
+def kv_blocks(i: int, kind: int, sink_blocks: int, local_blocks: int) -> list:
+    """KV blocks that query block row i visits.
+
+    Retrieval heads (kind 0): every block j <= i (dense causal, R7).
+    Streaming heads (kind 1): the Lambda mask [TD-static] -- sink blocks
+    [0, sink_blocks) and local blocks [i - local_blocks + 1, i] (R6).
+    """
+    if kind == 0:
+        return list(range(i + 1))
+    sink = set(range(min(sink_blocks, i + 1)))
+    local = set(range(max(0, i - local_blocks + 1), i + 1))
+    return sorted(sink | local)
+
+
+def computed_blocks(nblocks: int, kind: int, sink_blocks: int, local_blocks: int) -> int:
+    """Number of (query block, key block) tiles one head computes."""
+    return sum(len(kv_blocks(i, kind, sink_blocks, local_blocks)) for i in range(nblocks))
+
+
+def theoretical_speedup(nonempty: int, total: int) -> float:
+    """[TD-unified]: at block sparsity r = 1 - nonempty/total the ideal
+    speedup over computing every block is 1 / (1 - r)."""
+    r = 1.0 - nonempty / total
+    return 1.0 / (1.0 - r)
+
+
+def prefill_flops(T, H_q, H_kv, D, block, head_kind, sink_blocks, local_blocks) -> float:
+    """Work counted as the pages count it: full block tiles, 2 matmuls of
+    2*block*block*D flops each, per query head."""
+    nb = -(-T // block)
+    G = H_q // H_kv
+    tiles = sum(G * computed_blocks(nb, int(head_kind[h]), sink_blocks, local_blocks)
+                for h in range(H_kv))
+    return tiles * 4.0 * block * block * D
+
+
+# --- prefill attention [TD-unified; Abstract "skipped block-wise"] -------------
+
+def prefill_rows(q: np.ndarray, k: np.ndarray, v: np.ndarray, kind: int, block: int,
+                 sink_blocks: int, local_blocks: int, scale: float, rows):
+    """Causal softmax attention of the given query rows of ONE query head over
+    the keys of the blocks kv_blocks() allows (keys s <= t only).
+
+    q [rows][D] holds the query vectors of `rows` (token positions);
+    k, v [T][D] the head's keys/values.  Returns (o [rows][D], lse [rows]).
+    """
+    rows = np.asarray(rows, dtype=np.int64)
+    T, D = k.shape
+    o = np.empty((len(rows), D))
+    lse = np.empty(len(rows))
+    for r, t in enumerate(rows):
+        i = int(t) // block
+        keys = np.concatenate([np.arange(j * block, min((j + 1) * block, T))
+                               for j in kv_blocks(i, kind, sink_blocks, local_blocks)])
+        keys = keys[keys <= t]
+        z = scale * (k[keys] @ q[r])
+        zmax = z.max()
+        e = np.exp(z - zmax)
+        lsum = e.sum()
+        o[r] = (e @ v[keys]) / lsum
+        lse[r] = zmax + math.log(lsum)
+    return o, lse
