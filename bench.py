@@ -1,0 +1,483 @@
+"""Benchmark of the LServe-style sparse attention hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+Workload (synthetic, seeded): the Llama-3-8B-shaped decode layer -- batch 4,
+64K context, 32 query / 8 KV heads, D=128, bf16 paged KV (N_L=16, N_P=64),
+half the KV heads streaming (sink 128 + local 512), top-64 physical pages for
+the retrieval heads, selection reused over 4 decode steps.  The layer is
+replicated over 32 layers (Llama-3-8B depth), each with its own KV / stats /
+selection buffers, so one step streams ~1.5 GB -- far more than the 126 MB L2.
+
+A step is one decode token through the 32 layers: every 4th step runs
+page selection (lserve_page_select) before attention in each layer, the
+others reuse it; every step runs lserve_sparse_decode_attn per layer.  Steps
+are replayed from two CUDA graphs (with / without selection).
+
+Reported (one JSON line, rank 0):
+  value      touched-HBM GB/s of the decode steps, summed over ranks
+  us_per_layer_step, ms_per_step
+  stages     each call timed alone: selection, attention, the full stats
+             build, and the block-sparse prefill TFLOP/s on the 128K workload
+  roofline   for the dominant call (decode attention) against the measured
+             HBM copy bandwidth
+  e2e        the same step with the step's q copied host->device and the
+             output read back device->host inside the timed region
+  cpu_baseline  the fp64 oracle on a bounded sample of the same step
+Multi-GPU (torchrun): every rank runs its own replica (weak scaling, no
+collective on the data path); time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+LAYERS = 32
+REUSE = 4
+DEFAULT_STEPS = 6000
+DEFAULT_WARMUP = 8
+METRIC = "sparse decode attn µs/step & HBM GB/s; block-sparse prefill TFLOP/s"
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), float(p.get("bf16_tflops_sustained",
+                                                                        p["bf16_tflops"])), "measured"
+    except Exception:
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+# --- algorithmic byte / flop accounting (what the chosen sparsity touches) ----
+
+def decode_bytes(w):
+    """Bytes one decode step of one layer must move, amortising selection over
+    the reuse interval.  KV: valid tokens of the attended pages, K and V, D*2
+    bytes each.  Selection: the stats of every valid logical page of the
+    retrieval heads (2*D*2 bytes), the q vectors, scores and selection."""
+    import oracle
+    D, NP, NL = w.D, w.N_P, w.N_L
+    kv = 0
+    stats = 0
+    for b in range(w.B):
+        n = int(w.ctx_lens[b])
+        npages = -(-n // NP)
+        for h in range(w.H_kv):
+            if w.head_kind[h] == 0:
+                # top-K pages; the count of valid tokens depends only on whether the
+                # partial last page is selected -- bound it by full pages
+                k = min(w.top_k, npages)
+                kv += k * NP * D * 2 * 2
+                stats += (-(-n // NL)) * 2 * D * 2
+            else:
+                pages = oracle.streaming_pages(n, NP, w.sink, w.local)
+                toks = len(oracle.page_tokens(pages, n, NP))
+                kv += toks * D * 2 * 2
+    q = w.B * w.H_q * D * 2
+    out = w.B * w.H_q * D * 2
+    sel_io = q + w.B * w.H_kv * (w.max_pages * 4 + w.top_k * 4 + 4)
+    attn = kv + q + out
+    select = stats + sel_io
+    return dict(attn=attn, select=select, step=attn + select / REUSE, kv=kv, stats=stats)
+
+
+def stats_build_bytes(w):
+    """lserve_page_stats full build: read K of the retrieval heads, write stats."""
+    rd = wr = 0
+    for b in range(w.B):
+        n = int(w.ctx_lens[b])
+        for h in range(w.H_kv):
+            if w.head_kind[h] == 0:
+                rd += n * w.D * 2
+                wr += (-(-n // w.N_L)) * 2 * w.D * 2
+    return rd + wr
+
+
+# --- clocks sampling ----------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index, uuid=None):
+        self.sel = ["-i", uuid] if uuid else ["-i", str(device_index)]
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "--query-gpu=" + self.FIELDS,
+                                          "--format=csv,noheader,nounits", "-lms", "200"] + self.sel,
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = []
+        for line in out.strip().splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append(dict(sm=float(parts[1]), smax=float(parts[2]), power=float(parts[3]),
+                                 hw=parts[5], hwt=parts[6], swt=parts[7], swp=parts[8]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+        sm = np.array([r["sm"] for r in rows])
+        reasons = set()
+        for r in rows:
+            for key, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"),
+                              ("swt", "sw_thermal_slowdown"), ("swp", "sw_power_cap")):
+                if r[key].lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": float(rows[0]["smax"]),
+                "reasons": sorted(reasons), "samples": len(rows),
+                "power_w_max": float(max(r["power"] for r in rows))}
+
+
+# --- distributed plumbing -------------------------------------------------------
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def max_over_ranks(x, ws, device):
+    if ws == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# --- the CPU oracle baseline ----------------------------------------------------
+
+def oracle_step_sample(w, budget_s=12.0, max_pairs=None):
+    """Time the oracle's decode step (stats of the retrieval heads already
+    built, as on the GPU; then S^j -> P^m -> top-K -> attention per pair) on a
+    bounded sample of (sequence, KV head) pairs; returns seconds per layer-step
+    extrapolated from the pairs timed, and what was sampled."""
+    import oracle
+    try:
+        from threadpoolctl import threadpool_limits
+        lim = threadpool_limits(1)
+    except Exception:
+        lim = None
+    G = w.G
+    scale = 1.0 / math.sqrt(w.D)
+    pairs = [(b, h) for b in range(w.B) for h in range(w.H_kv)]
+    t_sel = t_attn = 0.0
+    done = 0
+    t_start = time.perf_counter()
+    for (b, h) in pairs:
+        n = int(w.ctx_lens[b])
+        q = oracle.widen_bf16(w.q[b, h * G:(h + 1) * G])
+        k = oracle.widen_bf16(w.k_seq(b, h))
+        v = oracle.widen_bf16(w.v_seq(b, h))
+        if w.head_kind[h] == 0:
+            kmin, kmax = oracle.page_stats(k, w.N_L)      # built once, not timed (GPU: not per step)
+            t0 = time.perf_counter()
+            P = oracle.physical_scores(oracle.logical_scores(q, kmin, kmax), w.g)
+            pages = oracle.select_top_k(P, w.top_k)
+            t1 = time.perf_counter()
+            t_sel += t1 - t0
+        else:
+            t1 = time.perf_counter()
+            pages = oracle.streaming_pages(n, w.N_P, w.sink, w.local)
+        oracle.decode_attention(q, k, v, oracle.page_tokens(pages, n, w.N_P), scale)
+        t_attn += time.perf_counter() - t1
+        done += 1
+        if time.perf_counter() - t_start > budget_s or (max_pairs and done >= max_pairs):
+            break
+    if lim is not None:
+        lim.unregister() if hasattr(lim, "unregister") else None
+    frac = done / len(pairs)
+    per_step = (t_sel / REUSE + t_attn) / frac
+    return per_step, f"{done} of {len(pairs)} (sequence, KV head) pairs of one layer-step, " \
+                     f"selection amortised over {REUSE} steps, 1 thread"
+
+
+def reference_arm(args):
+    """The oracle as the reference arm: same metric / unit / config."""
+    ws, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    import synth
+    w = synth.llama3_8b_decode()
+    acct = decode_bytes(w)
+    total_s, steps_done = 0.0, 0
+    sample = None
+    for _ in range(max(1, args.warmup // 4)):
+        oracle_step_sample(w, budget_s=2.0, max_pairs=2)
+    t0 = time.perf_counter()
+    per_step, sample = oracle_step_sample(w, budget_s=20.0)
+    total_s = time.perf_counter() - t0
+    value = acct["step"] * LAYERS / (per_step * LAYERS) / 1e9
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus,
+        "steps": 1, "warmup": args.warmup, "ms_per_step": per_step * LAYERS * 1e3,
+        "us_per_layer_step": per_step * 1e6, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(w),
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                         "sample": sample + f"; {total_s:.1f} s of CPU work"},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+    return 0
+
+
+def workload_config(w):
+    return {"workload": f"{w.name}: B={w.B} n={int(w.ctx_lens[0])} H_q={w.H_q} H_kv={w.H_kv} D={w.D} "
+                        f"N_L={w.N_L} N_P={w.N_P} top_k={w.top_k} sink={w.sink} local={w.local} "
+                        f"reuse={REUSE}",
+            "layers": LAYERS, "global_batch": w.B, "seq_len": int(w.ctx_lens[0]),
+            "parallelism": "replica per GPU",
+            "l2": f"inputs larger than L2: {LAYERS} layer replicas, each step streams all of them"}
+
+
+# --- the CUDA path ----------------------------------------------------------------
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=DEFAULT_STEPS)
+    ap.add_argument("--warmup", type=int, default=DEFAULT_WARMUP)
+    ap.add_argument("--impl", default="lserve", choices=["lserve", "reference"])
+    ap.add_argument("--no-prefill", action="store_true", help="skip the prefill stage")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+    if args.impl == "reference":
+        return reference_arm(args)
+
+    import torch
+    ws, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    import block_sparse_attention_page_b200 as lserve
+    import synth
+    from synth.device import DecodeBuffers
+
+    hbm_peak, tc_peak, tc_sustained, peak_src = peaks()
+    w = synth.llama3_8b_decode()
+    buf = DecodeBuffers(w, device=dev, layers=LAYERS)
+    d = lserve.paged_desc(w.B, w.H_q, w.H_kv, w.D, w.N_L, w.N_P, w.max_pages, w.num_pool_pages)
+    scale = 1.0 / math.sqrt(w.D)
+    ws_dec = lserve.alloc_workspace(lserve.workspace_size(lserve.OP_DECODE, d, w.top_k), device=dev)
+    ws_sel = lserve.alloc_workspace(lserve.workspace_size(lserve.OP_SELECT, d, w.top_k), device=dev)
+    outs = [torch.empty_like(buf.out) for _ in range(LAYERS)]
+    qs = [buf.q.clone() for _ in range(LAYERS)]
+    stream = torch.cuda.Stream(device=dev)
+    acct = decode_bytes(w)
+
+    def stats_all():
+        for l in range(LAYERS):
+            lserve.page_stats(d, buf.k_pools[l], buf.block_table, buf.ctx_lens, buf.head_kind,
+                              buf.stats[l])
+
+    def select(l):
+        lserve.page_select(d, qs[l], buf.stats[l], buf.block_table, buf.ctx_lens, buf.head_kind,
+                           w.top_k, buf.sel[l], buf.sel_count[l], workspace=ws_sel)
+
+    def attn(l):
+        lserve.sparse_decode_attn(d, qs[l], buf.k_pools[l], buf.v_pools[l], buf.block_table,
+                                  buf.ctx_lens, buf.head_kind, buf.sel[l], buf.sel_count[l], w.top_k,
+                                  w.sink, w.local, scale, outs[l], None, workspace=ws_dec)
+
+    with torch.cuda.stream(stream):
+        stats_all()
+        for l in range(LAYERS):
+            select(l)
+            attn(l)
+    torch.cuda.synchronize()
+    assert lserve.read_device_status(stream) == lserve.OK
+
+    def capture(fn):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            fn()
+        return g
+
+    g_sel = capture(lambda: [(select(l), attn(l)) for l in range(LAYERS)])
+    g_reuse = capture(lambda: [attn(l) for l in range(LAYERS)])
+    g_select_only = capture(lambda: [select(l) for l in range(LAYERS)])
+    g_stats = capture(stats_all)
+
+    def run_steps(k0, k):
+        for t in range(k0, k0 + k):
+            (g_sel if t % REUSE == 0 else g_reuse).replay()
+
+    def timed(fn, reps=1):
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        if ws > 1:
+            torch.distributed.barrier()
+        e0.record(stream)
+        with torch.cuda.stream(stream):
+            for _ in range(reps):
+                fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        if ws > 1:
+            torch.distributed.barrier()
+        return e0.elapsed_time(e1) / 1e3
+
+    # warm-up (untimed), then exactly K steps
+    with torch.cuda.stream(stream):
+        run_steps(0, args.warmup)
+    torch.cuda.synchronize()
+    sampler = ClockSampler(local, getattr(torch.cuda.get_device_properties(dev), "uuid", None))
+    sampler.start() if rank == 0 else None
+    time.sleep(0.3)
+    elapsed = timed(lambda: run_steps(0, args.steps))
+    clocks = sampler.stop() if rank == 0 else None
+    elapsed = max_over_ranks(elapsed, ws, dev)
+    step_bytes = acct["step"] * LAYERS
+    value = step_bytes * args.steps * ws / elapsed / 1e9
+    us_layer = elapsed / (args.steps * LAYERS) * 1e6
+
+    # stages, each alone (graph replays, CUDA events on the launching stream)
+    reps = 20
+    t_attn = timed(lambda: g_reuse.replay(), reps) / (reps * LAYERS)
+    t_sel = timed(lambda: g_select_only.replay(), reps) / (reps * LAYERS)
+    t_stats = timed(lambda: g_stats.replay(), 3) / (3 * LAYERS)
+    sb = stats_build_bytes(w)
+    attn_gbs = acct["attn"] / t_attn / 1e9
+    stages = {
+        "attention": {"us": t_attn * 1e6, "GB/s": attn_gbs, "frac": attn_gbs / hbm_peak,
+                      "bytes": acct["attn"]},
+        "selection": {"us": t_sel * 1e6, "GB/s": acct["select"] / t_sel / 1e9,
+                      "frac": acct["select"] / t_sel / 1e9 / hbm_peak, "bytes": acct["select"]},
+        "stats_build": {"us": t_stats * 1e6, "GB/s": sb / t_stats / 1e9,
+                        "frac": sb / t_stats / 1e9 / hbm_peak, "bytes": sb},
+    }
+    del g_stats
+
+    # e2e: per step, copy the step's q (all layers) host->device from pinned memory,
+    # run the step, read every layer's output back to pinned host memory
+    q_host = torch.empty((LAYERS,) + tuple(buf.q.shape), dtype=torch.bfloat16).pin_memory()
+    o_host = torch.empty((LAYERS,) + tuple(buf.out.shape), dtype=torch.bfloat16).pin_memory()
+    q_host.copy_(torch.stack([q.cpu() for q in qs]))
+    q_dev = torch.empty_like(q_host, device=dev)
+
+    def e2e_step(t):
+        q_dev.copy_(q_host, non_blocking=True)
+        for l in range(LAYERS):
+            qs[l].copy_(q_dev[l], non_blocking=True)
+        (g_sel if t % REUSE == 0 else g_reuse).replay()
+        for l in range(LAYERS):
+            o_host[l].copy_(outs[l], non_blocking=True)
+
+    e2e_steps = min(args.steps, 400)
+    with torch.cuda.stream(stream):
+        for t in range(args.warmup):
+            e2e_step(t)
+    t_e2e = timed(lambda: [e2e_step(t) for t in range(e2e_steps)])
+    t_e2e = max_over_ranks(t_e2e, ws, dev)
+    h2d = q_host.numel() * 2
+    d2h = o_host.numel() * 2
+    e2e = {"value": step_bytes * e2e_steps * ws / t_e2e / 1e9, "unit": "GB/s",
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+           "ms_per_step": t_e2e / e2e_steps * 1e3}
+
+    launches = args.steps * LAYERS * 2 + (-(-args.steps // REUSE)) * LAYERS * 2
+    result = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": ws, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": elapsed / args.steps * 1e3,
+        "us_per_layer_step": us_layer, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": workload_config(w),
+        "roofline": {"bound": "hbm", "kernel": "lserve_sparse_decode_attn (split + combine)",
+                     "achieved": attn_gbs, "peak": hbm_peak, "unit": "GB/s",
+                     "frac": attn_gbs / hbm_peak, "traffic": None,
+                     "peak_source": f"{peak_src} hbm_gbs (copy)"},
+        "stages": stages,
+        "e2e": e2e,
+        "gpu_launches": launches,
+        "clocks": clocks,
+    }
+    del g_sel, g_reuse, g_select_only
+    buf = None
+    torch.cuda.empty_cache()
+
+    if not args.no_prefill:
+        result["stages"]["prefill"] = prefill_stage(lserve, synth, dev, stream, tc_peak, timed)
+
+    if rank == 0 and not args.no_cpu_baseline:
+        per_step, sample = oracle_step_sample(w, budget_s=15.0)
+        cpu_val = acct["step"] / per_step / 1e9
+        result["cpu_baseline"] = {"value": cpu_val, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                                  "sample": sample}
+    if rank == 0:
+        print(json.dumps(result))
+    if ws > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+def prefill_stage(lserve, synth, dev, stream, tc_peak, timed):
+    """Block-sparse prefill on the 128K workload: TFLOP/s over computed blocks."""
+    import torch
+    import oracle
+    w = synth.prefill_128k()
+    d = lserve.prefill_desc(w.T, w.H_q, w.H_kv, w.D, w.block, w.sink_blocks, w.local_blocks)
+    need = lserve.workspace_size(lserve.OP_PREFILL, d)
+    try:
+        from synth.device import PrefillBuffers
+        pb = PrefillBuffers(w, device=dev)
+        wsb = lserve.alloc_workspace(need, device=dev)
+        scale = 1.0 / math.sqrt(w.D)
+
+        def run():
+            lserve.blocksparse_prefill(d, pb.q, pb.k, pb.v, list(w.head_kind), scale, pb.out, None,
+                                       workspace=wsb, stream=stream)
+        with torch.cuda.stream(stream):
+            run()
+        torch.cuda.synchronize()
+        t = timed(run, 3) / 3
+    except lserve.LServeError as e:
+        return {"unavailable": str(e)}
+    flops = oracle.prefill_flops(w.T, w.H_q, w.H_kv, w.D, w.block, w.head_kind, w.sink_blocks,
+                                 w.local_blocks)
+    tf = flops / t / 1e12
+    return {"ms": t * 1e3, "TFLOP/s": tf, "frac": tf / tc_peak, "flops": flops,
+            "workload": f"{w.name}: T={w.T} H_q={w.H_q} H_kv={w.H_kv} D={w.D} block={w.block} "
+                        f"Lambda({w.sink_blocks},{w.local_blocks}) on KV heads 4-7"}
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,168 @@
+"""Thin Python binding of liblserve.so (LServe-style unified sparse attention
+hot path on B200 / sm_100a).
+
+Every function here only marshals arguments -- torch tensors in, raw device
+pointers and the current CUDA stream out -- and calls the C-ABI function of
+the same name declared in include/lserve.h.  All computation happens in the
+library's CUDA kernels.  There is no fallback: if liblserve.so is missing or
+cannot be loaded, importing this package raises.
+
+Layouts (see include/lserve.h):
+  q            bf16 [B][H_q][D]
+  k/v pool     bf16 [num_pool_pages][H_kv][N_P][D]
+  stats pool   bf16 [num_pool_pages][H_kv][N_P/N_L][2][D]
+  block_table  int32 [B][max_pages]     ctx_lens int32 [B]
+  head_kind    uint8 [H_kv] (0 retrieval, 1 streaming)
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_TIMEOUT, ERR_BOUNDS = range(7)
+OP_STATS, OP_SELECT, OP_DECODE, OP_PREFILL = range(4)
+
+EXPORTED = [
+    "lserve_page_stats", "lserve_page_select", "lserve_sparse_decode_attn",
+    "lserve_blocksparse_prefill", "lserve_workspace_size", "lserve_read_device_status",
+    "lserve_set_wait_limit_cycles", "lserve_debug_wait_timeout", "lserve_status_string",
+    "lserve_bounds_checked",
+]
+
+
+class LServeError(RuntimeError):
+    def __init__(self, fn, status, msg):
+        super().__init__(f"{fn} failed: status {status} ({msg})")
+        self.status = status
+
+
+class PagedDesc(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in (
+        "batch", "num_q_heads", "num_kv_heads", "head_dim", "logical_page", "physical_page",
+        "max_pages_per_seq", "num_pool_pages")]
+
+
+class PrefillDesc(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in (
+        "seq_len", "num_q_heads", "num_kv_heads", "head_dim", "block_q", "block_k",
+        "sink_blocks", "local_blocks")]
+
+
+def library_path() -> str:
+    return os.path.join(_HERE, "liblserve.so")
+
+
+def _load(path):
+    if not os.path.exists(path):
+        raise ImportError(f"{path} not built: run `python -m block_sparse_attention_page_b200.build`")
+    lib = ctypes.CDLL(path)
+    vp, i32, sz, u64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t, ctypes.c_uint64
+    P = ctypes.POINTER
+    lib.lserve_page_stats.argtypes = [P(PagedDesc), vp, vp, vp, vp, vp, i32, vp]
+    lib.lserve_page_select.argtypes = [P(PagedDesc), vp, vp, vp, vp, vp, i32, vp, vp, vp, vp, sz, vp]
+    lib.lserve_sparse_decode_attn.argtypes = [P(PagedDesc), vp, vp, vp, vp, vp, vp, vp, vp, i32, i32,
+                                              i32, ctypes.c_float, vp, vp, vp, sz, vp]
+    lib.lserve_blocksparse_prefill.argtypes = [P(PrefillDesc), vp, vp, vp, vp, ctypes.c_float, vp, vp,
+                                               vp, sz, vp]
+    lib.lserve_workspace_size.argtypes = [ctypes.c_int, vp, i32]
+    lib.lserve_workspace_size.restype = sz
+    lib.lserve_read_device_status.argtypes = [vp]
+    lib.lserve_set_wait_limit_cycles.argtypes = [u64]
+    lib.lserve_set_wait_limit_cycles.restype = None
+    lib.lserve_debug_wait_timeout.argtypes = [u64, vp]
+    lib.lserve_status_string.argtypes = [ctypes.c_int]
+    lib.lserve_status_string.restype = ctypes.c_char_p
+    for name in ("lserve_page_stats", "lserve_page_select", "lserve_sparse_decode_attn",
+                 "lserve_blocksparse_prefill", "lserve_read_device_status", "lserve_debug_wait_timeout",
+                 "lserve_bounds_checked"):
+        getattr(lib, name).restype = ctypes.c_int
+    return lib
+
+
+lib = _load(library_path())
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(fn, status):
+    if status != OK:
+        raise LServeError(fn, status, lib.lserve_status_string(status).decode())
+
+
+def status_string(status: int) -> str:
+    return lib.lserve_status_string(status).decode()
+
+
+def paged_desc(B, H_q, H_kv, D, N_L, N_P, max_pages, num_pool_pages) -> PagedDesc:
+    return PagedDesc(B, H_q, H_kv, D, N_L, N_P, max_pages, num_pool_pages)
+
+
+def prefill_desc(T, H_q, H_kv, D, block, sink_blocks, local_blocks) -> PrefillDesc:
+    return PrefillDesc(T, H_q, H_kv, D, block, block, sink_blocks, local_blocks)
+
+
+def workspace_size(op: int, desc, top_k: int = 0) -> int:
+    return lib.lserve_workspace_size(op, ctypes.byref(desc), top_k)
+
+
+def page_stats(desc, k_pool, block_table, ctx_lens, head_kind, stats_pool, first_logical_page=0,
+               stream=None):
+    _check("lserve_page_stats", lib.lserve_page_stats(
+        ctypes.byref(desc), _ptr(k_pool), _ptr(block_table), _ptr(ctx_lens), _ptr(head_kind),
+        _ptr(stats_pool), first_logical_page, _stream(stream)))
+
+
+def page_select(desc, q, stats_pool, block_table, ctx_lens, head_kind, top_k, sel, sel_count,
+                phys_scores=None, workspace=None, stream=None):
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check("lserve_page_select", lib.lserve_page_select(
+        ctypes.byref(desc), _ptr(q), _ptr(stats_pool), _ptr(block_table), _ptr(ctx_lens),
+        _ptr(head_kind), top_k, _ptr(sel), _ptr(sel_count), _ptr(phys_scores), _ptr(workspace),
+        ws_bytes, _stream(stream)))
+
+
+def sparse_decode_attn(desc, q, k_pool, v_pool, block_table, ctx_lens, head_kind, sel, sel_count,
+                       top_k, sink_tokens, local_tokens, softmax_scale, out, lse=None,
+                       workspace=None, stream=None):
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check("lserve_sparse_decode_attn", lib.lserve_sparse_decode_attn(
+        ctypes.byref(desc), _ptr(q), _ptr(k_pool), _ptr(v_pool), _ptr(block_table), _ptr(ctx_lens),
+        _ptr(head_kind), _ptr(sel), _ptr(sel_count), top_k, sink_tokens, local_tokens,
+        float(softmax_scale), _ptr(out), _ptr(lse), _ptr(workspace), ws_bytes, _stream(stream)))
+
+
+def blocksparse_prefill(desc, q, k, v, head_kind_host, softmax_scale, out, lse=None, workspace=None,
+                        stream=None):
+    hk = (ctypes.c_uint8 * len(head_kind_host))(*[int(x) for x in head_kind_host])
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check("lserve_blocksparse_prefill", lib.lserve_blocksparse_prefill(
+        ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), ctypes.cast(hk, ctypes.c_void_p),
+        float(softmax_scale), _ptr(out), _ptr(lse), _ptr(workspace), ws_bytes, _stream(stream)))
+
+
+def read_device_status(stream=None) -> int:
+    return lib.lserve_read_device_status(_stream(stream))
+
+
+def set_wait_limit_cycles(cycles: int) -> None:
+    lib.lserve_set_wait_limit_cycles(cycles)
+
+
+def debug_wait_timeout(cycles: int, stream=None):
+    _check("lserve_debug_wait_timeout", lib.lserve_debug_wait_timeout(cycles, _stream(stream)))
+
+
+def alloc_workspace(nbytes: int, device="cuda") -> torch.Tensor:
+    """Caller-owned workspace (256-byte aligned by the caching allocator)."""
+    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)

@@ -1,0 +1,371 @@
+// C-ABI entry points of liblserve.so (declared in include/lserve.h): argument
+// validation, tensor-map encoding, workspace carving and kernel launches.
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstring>
+#include <mutex>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "prefill.h"
+
+namespace lserve {
+
+__device__ unsigned int g_status = 0;
+
+namespace {
+
+constexpr uint64_t kDefaultWaitLimit = 4000000000ull;  // ~2 s at 1.9 GHz
+uint64_t g_wait_limit = kDefaultWaitLimit;
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int sm_count_current() {
+  static std::mutex mu;
+  static int cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  std::lock_guard<std::mutex> lock(mu);
+  if (cache[dev] == 0) {
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    cache[dev] = v;
+  }
+  return cache[dev];
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return (PFN_cuTensorMapEncodeTiled_v12000) nullptr;
+    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  }();
+  return fn;
+}
+
+}  // namespace
+
+// 2-D bf16 tensor map [rows][cols] (row pitch `pitch_elems`), 128-byte swizzle,
+// box of box_rows x 64 columns.
+bool make_map_2d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint64_t pitch_elems,
+                 uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {pitch_elems * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t es[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+cudaError_t set_smem_once(const void* kernel, int bytes) {
+  struct Entry {
+    const void* fn;
+    int dev;
+    int bytes;
+  };
+  static std::mutex mu;
+  static Entry done[256];
+  static int ndone = 0;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(mu);
+  for (int i = 0; i < ndone; ++i)
+    if (done[i].fn == kernel && done[i].dev == dev && done[i].bytes >= bytes) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e != cudaSuccess) return e;
+  if (ndone < 256) done[ndone++] = Entry{kernel, dev, bytes};
+  return cudaSuccess;
+}
+
+uint64_t wait_limit() { return g_wait_limit; }
+int current_sm_count() { return sm_count_current(); }
+
+// Device address of g_status on the current device (cached per device).
+unsigned int* device_status_word() {
+  static std::mutex mu;
+  static unsigned int* cache[64] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!cache[dev]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_status) != cudaSuccess) return nullptr;
+    cache[dev] = static_cast<unsigned int*>(ptr);
+  }
+  return cache[dev];
+}
+
+static __global__ void wait_timeout_probe_kernel(uint64_t cycles, unsigned int* status) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+    // nobody arrives: the bounded wait must give up and raise the flag
+    (void)mbar_wait(&bar, 0, cycles, status);
+  }
+}
+
+cudaError_t launch_wait_timeout_probe(uint64_t cycles, unsigned int* status, cudaStream_t stream) {
+  wait_timeout_probe_kernel<<<1, 32, 0, stream>>>(cycles, status);
+  return cudaGetLastError();
+}
+
+}  // namespace lserve
+
+using namespace lserve;
+
+namespace {
+
+bool valid_paged(const lserve_paged_desc* d) {
+  if (!d) return false;
+  if (d->batch < 1 || d->num_kv_heads < 1 || d->num_q_heads < d->num_kv_heads) return false;
+  if (d->num_q_heads % d->num_kv_heads) return false;
+  if (d->logical_page < 1 || d->physical_page < d->logical_page) return false;
+  if (d->physical_page % d->logical_page) return false;
+  if (d->max_pages_per_seq < 1 || d->num_pool_pages < 1) return false;
+  return true;
+}
+
+int supported_paged(const lserve_paged_desc* d) {
+  const int G = d->num_q_heads / d->num_kv_heads;
+  if (d->head_dim != 64 && d->head_dim != 128) return LSERVE_ERR_UNSUPPORTED;
+  if (G != 1 && G != 2 && G != 4 && G != 8) return LSERVE_ERR_UNSUPPORTED;
+  if (d->logical_page != 8 && d->logical_page != 16 && d->logical_page != 32 && d->logical_page != 64)
+    return LSERVE_ERR_UNSUPPORTED;
+  if (d->physical_page % kDecodeTile || d->physical_page > 1024) return LSERVE_ERR_UNSUPPORTED;
+  const long long rows = (long long)d->num_pool_pages * d->num_kv_heads * d->physical_page;
+  if (rows >= (1ll << 31)) return LSERVE_ERR_UNSUPPORTED;
+  return LSERVE_OK;
+}
+
+size_t select_ws(const lserve_paged_desc* d) {
+  return ((size_t)d->batch * d->num_kv_heads * d->max_pages_per_seq * 4 + 255) / 256 * 256;
+}
+
+size_t decode_ws(const lserve_paged_desc* d) {
+  const int sms = current_sm_count();
+  if (sms <= 0) return 0;
+  const int G = d->num_q_heads / d->num_kv_heads;
+  const int wpc = decode_warps_per_cta(d->head_dim, G);
+  if (wpc <= 0) return 0;
+  return decode_workspace_bytes(d->batch * d->num_kv_heads, decode_num_ctas(sms) * wpc, G,
+                                d->head_dim);
+}
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? LSERVE_OK : LSERVE_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+const char* lserve_status_string(int s) {
+  switch (s) {
+    case LSERVE_OK: return "ok";
+    case LSERVE_ERR_INVALID_ARG: return "invalid argument";
+    case LSERVE_ERR_UNSUPPORTED: return "unsupported shape or parameter";
+    case LSERVE_ERR_WORKSPACE: return "workspace missing or too small";
+    case LSERVE_ERR_CUDA: return "CUDA runtime error";
+    case LSERVE_ERR_TIMEOUT: return "bounded device wait timed out";
+    case LSERVE_ERR_BOUNDS: return "index out of range (page skipped)";
+    default: return "unknown status";
+  }
+}
+
+int lserve_bounds_checked(void) { return kCheckBounds ? 1 : 0; }
+
+void lserve_set_wait_limit_cycles(uint64_t cycles) {
+  g_wait_limit = cycles ? cycles : kDefaultWaitLimit;
+}
+
+size_t lserve_workspace_size(int op, const void* desc, int32_t top_k) {
+  (void)top_k;
+  if (!desc) return 0;
+  switch (op) {
+    case LSERVE_OP_STATS: {
+      const auto* d = static_cast<const lserve_paged_desc*>(desc);
+      return valid_paged(d) ? 0 : 0;
+    }
+    case LSERVE_OP_SELECT: {
+      const auto* d = static_cast<const lserve_paged_desc*>(desc);
+      return valid_paged(d) ? select_ws(d) : 0;
+    }
+    case LSERVE_OP_DECODE: {
+      const auto* d = static_cast<const lserve_paged_desc*>(desc);
+      if (!valid_paged(d) || supported_paged(d) != LSERVE_OK) return 0;
+      return decode_ws(d);
+    }
+    case LSERVE_OP_PREFILL:
+      return prefill_workspace_bytes(static_cast<const lserve_prefill_desc*>(desc));
+    default:
+      return 0;
+  }
+}
+
+int lserve_read_device_status(void* stream) {
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return LSERVE_ERR_CUDA;
+  unsigned int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_status, sizeof(v)) != cudaSuccess) return LSERVE_ERR_CUDA;
+  const unsigned int zero = 0;
+  if (cudaMemcpyToSymbol(g_status, &zero, sizeof(zero)) != cudaSuccess) return LSERVE_ERR_CUDA;
+  if (v & (1u << LSERVE_ERR_TIMEOUT)) return LSERVE_ERR_TIMEOUT;
+  if (v & (1u << LSERVE_ERR_BOUNDS)) return LSERVE_ERR_BOUNDS;
+  return LSERVE_OK;
+}
+
+int lserve_debug_wait_timeout(uint64_t cycles, void* stream) {
+  if (cycles == 0 || cycles > (1ull << 40)) return LSERVE_ERR_INVALID_ARG;
+  unsigned int* st = device_status_word();
+  if (!st) return LSERVE_ERR_CUDA;
+  return cuda_status(launch_wait_timeout_probe(cycles, st, static_cast<cudaStream_t>(stream)));
+}
+
+int lserve_page_stats(const lserve_paged_desc* desc, const void* k_pool, const int32_t* block_table,
+                      const int32_t* ctx_lens, const uint8_t* head_kind, void* stats_pool,
+                      int32_t first_logical_page, void* stream) {
+  if (!valid_paged(desc)) return LSERVE_ERR_INVALID_ARG;
+  if (!k_pool || !block_table || !ctx_lens || !head_kind || !stats_pool) return LSERVE_ERR_INVALID_ARG;
+  if (!aligned(k_pool, 16) || !aligned(stats_pool, 16) || !aligned(block_table, 4) ||
+      !aligned(ctx_lens, 4))
+    return LSERVE_ERR_INVALID_ARG;
+  if (first_logical_page < 0) return LSERVE_ERR_INVALID_ARG;
+  const int st = supported_paged(desc);
+  if (st != LSERVE_OK) return st;
+  StatsParams p;
+  p.k_pool = static_cast<const __nv_bfloat16*>(k_pool);
+  p.block_table = block_table;
+  p.ctx_lens = ctx_lens;
+  p.head_kind = head_kind;
+  p.stats_pool = static_cast<__nv_bfloat16*>(stats_pool);
+  p.batch = desc->batch;
+  p.num_kv_heads = desc->num_kv_heads;
+  p.logical_page = desc->logical_page;
+  p.physical_page = desc->physical_page;
+  p.max_pages = desc->max_pages_per_seq;
+  p.num_pool_pages = desc->num_pool_pages;
+  p.first_logical_page = first_logical_page;
+  p.status = device_status_word();
+  if (!p.status) return LSERVE_ERR_CUDA;
+  const int g = desc->physical_page / desc->logical_page;
+  const long long max_lp = (long long)desc->max_pages_per_seq * g;
+  if (max_lp >= (1ll << 30)) return LSERVE_ERR_UNSUPPORTED;
+  return cuda_status(launch_page_stats(p, desc->head_dim, (int)max_lp, static_cast<cudaStream_t>(stream)));
+}
+
+int lserve_page_select(const lserve_paged_desc* desc, const void* q, const void* stats_pool,
+                       const int32_t* block_table, const int32_t* ctx_lens, const uint8_t* head_kind,
+                       int32_t top_k, int32_t* sel, int32_t* sel_count, float* phys_scores,
+                       void* workspace, size_t workspace_bytes, void* stream) {
+  if (!valid_paged(desc)) return LSERVE_ERR_INVALID_ARG;
+  if (!q || !stats_pool || !block_table || !ctx_lens || !head_kind || !sel || !sel_count)
+    return LSERVE_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(stats_pool, 16) || !aligned(sel, 4) || !aligned(sel_count, 4) ||
+      !aligned(block_table, 4) || !aligned(ctx_lens, 4) || (phys_scores && !aligned(phys_scores, 4)))
+    return LSERVE_ERR_INVALID_ARG;
+  if (top_k < 1 || top_k > desc->max_pages_per_seq) return LSERVE_ERR_INVALID_ARG;
+  const int st = supported_paged(desc);
+  if (st != LSERVE_OK) return st;
+  if (desc->max_pages_per_seq > kTopkMaxPages) return LSERVE_ERR_UNSUPPORTED;
+  float* scores = phys_scores;
+  if (!scores) {
+    if (!workspace || workspace_bytes < select_ws(desc) || !aligned(workspace, 16))
+      return LSERVE_ERR_WORKSPACE;
+    scores = static_cast<float*>(workspace);
+  }
+  SelectParams p;
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.stats_pool = static_cast<const __nv_bfloat16*>(stats_pool);
+  p.block_table = block_table;
+  p.ctx_lens = ctx_lens;
+  p.head_kind = head_kind;
+  p.scores = scores;
+  p.sel = sel;
+  p.sel_count = sel_count;
+  p.batch = desc->batch;
+  p.num_q_heads = desc->num_q_heads;
+  p.num_kv_heads = desc->num_kv_heads;
+  p.logical_page = desc->logical_page;
+  p.physical_page = desc->physical_page;
+  p.max_pages = desc->max_pages_per_seq;
+  p.num_pool_pages = desc->num_pool_pages;
+  p.top_k = top_k;
+  p.status = device_status_word();
+  if (!p.status) return LSERVE_ERR_CUDA;
+  return cuda_status(launch_page_select(p, desc->head_dim, static_cast<cudaStream_t>(stream)));
+}
+
+int lserve_sparse_decode_attn(const lserve_paged_desc* desc, const void* q, const void* k_pool,
+                              const void* v_pool, const int32_t* block_table, const int32_t* ctx_lens,
+                              const uint8_t* head_kind, const int32_t* sel, const int32_t* sel_count,
+                              int32_t top_k, int32_t sink_tokens, int32_t local_tokens,
+                              float softmax_scale, void* out, float* lse, void* workspace,
+                              size_t workspace_bytes, void* stream) {
+  if (!valid_paged(desc)) return LSERVE_ERR_INVALID_ARG;
+  if (!q || !k_pool || !v_pool || !block_table || !ctx_lens || !head_kind || !sel || !sel_count || !out)
+    return LSERVE_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k_pool, 16) || !aligned(v_pool, 16) || !aligned(out, 16) ||
+      !aligned(block_table, 4) || !aligned(ctx_lens, 4) || !aligned(sel, 4) || !aligned(sel_count, 4) ||
+      (lse && !aligned(lse, 4)))
+    return LSERVE_ERR_INVALID_ARG;
+  if (top_k < 1 || top_k > desc->max_pages_per_seq) return LSERVE_ERR_INVALID_ARG;
+  if (sink_tokens < 0 || local_tokens < 0 || !std::isfinite(softmax_scale)) return LSERVE_ERR_INVALID_ARG;
+  const int st = supported_paged(desc);
+  if (st != LSERVE_OK) return st;
+  const size_t need = decode_ws(desc);
+  if (need == 0) return LSERVE_ERR_CUDA;
+  if (!workspace || workspace_bytes < need || !aligned(workspace, 256)) return LSERVE_ERR_WORKSPACE;
+  const int D = desc->head_dim, G = desc->num_q_heads / desc->num_kv_heads;
+  const uint64_t rows = (uint64_t)desc->num_pool_pages * desc->num_kv_heads * desc->physical_page;
+  CUtensorMap kmap, vmap;
+  if (!make_map_2d(&kmap, k_pool, rows, D, D, kDecodeTile) ||
+      !make_map_2d(&vmap, v_pool, rows, D, D, kDecodeTile))
+    return LSERVE_ERR_CUDA;
+  const int P = desc->batch * desc->num_kv_heads;
+  DecodeParams p;
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.block_table = block_table;
+  p.ctx_lens = ctx_lens;
+  p.head_kind = head_kind;
+  p.sel = sel;
+  p.sel_count = sel_count;
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.lse = lse;
+  p.pair_tiles = static_cast<int32_t*>(workspace);
+  p.partial = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
+                                       ((size_t)(P + 1) * 4 + 255) / 256 * 256);
+  p.batch = desc->batch;
+  p.num_q_heads = desc->num_q_heads;
+  p.num_kv_heads = desc->num_kv_heads;
+  p.physical_page = desc->physical_page;
+  p.max_pages = desc->max_pages_per_seq;
+  p.num_pool_pages = desc->num_pool_pages;
+  p.top_k = top_k;
+  p.sink = sink_tokens;
+  p.local = local_tokens;
+  p.tiles_per_page = desc->physical_page / kDecodeTile;
+  p.num_warps = 0;  // set by launch_decode
+  p.scale_log2 = softmax_scale * 1.4426950408889634f;
+  p.wait_limit = wait_limit();
+  p.status = device_status_word();
+  if (!p.status) return LSERVE_ERR_CUDA;
+  return cuda_status(
+      launch_decode(p, kmap, vmap, D, G, decode_num_ctas(current_sm_count()), static_cast<cudaStream_t>(stream)));
+}
+
+int lserve_blocksparse_prefill(const lserve_prefill_desc* desc, const void* q, const void* k,
+                               const void* v, const uint8_t* head_kind_host, float softmax_scale,
+                               void* out, float* lse, void* workspace, size_t workspace_bytes,
+                               void* stream) {
+  return prefill_entry(desc, q, k, v, head_kind_host, softmax_scale, out, lse, workspace,
+                       workspace_bytes, static_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"

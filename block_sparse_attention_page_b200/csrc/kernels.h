@@ -1,0 +1,91 @@
+// Internal launch interface between the C-ABI layer (api.cu) and the kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace lserve {
+
+constexpr int kStatsWarps = 8;   // warps per CTA of the stats kernel
+constexpr int kScoreWarps = 8;   // warps per CTA of the score kernel
+constexpr int kScorePagesPerWarp = 2;
+constexpr int kTopkThreads = 512;
+constexpr int kTopkMaxPages = 32768;
+
+struct StatsParams {
+  const __nv_bfloat16* k_pool;
+  const int32_t* block_table;
+  const int32_t* ctx_lens;
+  const uint8_t* head_kind;
+  __nv_bfloat16* stats_pool;
+  unsigned int* status;
+  int batch, num_kv_heads, logical_page, physical_page, max_pages, num_pool_pages;
+  int first_logical_page;
+};
+
+struct SelectParams {
+  const __nv_bfloat16* q;
+  const __nv_bfloat16* stats_pool;
+  const int32_t* block_table;
+  const int32_t* ctx_lens;
+  const uint8_t* head_kind;
+  float* scores;          // [B][H_kv][max_pages]
+  int32_t* sel;           // [B][H_kv][top_k]
+  int32_t* sel_count;     // [B][H_kv]
+  unsigned int* status;
+  int batch, num_q_heads, num_kv_heads, logical_page, physical_page, max_pages, num_pool_pages;
+  int top_k;
+};
+
+// Decode split: the tiles of all (sequence, KV head) pairs are laid end to end
+// and cut into equal ranges, one per consumer warp of a persistent grid.
+constexpr int kDecodeTile = 32;       // tokens per tile
+constexpr int kDecodeWarps = 6;       // consumer warps per CTA
+constexpr int kDecodeStages = 2;      // tiles in flight per warp
+
+struct DecodeParams {
+  const __nv_bfloat16* q;
+  const int32_t* block_table;
+  const int32_t* ctx_lens;
+  const uint8_t* head_kind;
+  const int32_t* sel;
+  const int32_t* sel_count;
+  __nv_bfloat16* out;
+  float* lse;
+  int32_t* pair_tiles;    // workspace [P + 1]: exclusive prefix of tiles per pair
+  float* partial;         // workspace: o [(num_warps + P)][G][D], then (m, l) [..][G][2]
+  unsigned int* status;
+  int batch, num_q_heads, num_kv_heads, physical_page, max_pages, num_pool_pages;
+  int top_k, sink, local;
+  int tiles_per_page;
+  int num_warps;          // consumer warps in the whole grid
+  float scale_log2;       // softmax_scale * log2(e)
+  uint64_t wait_limit;
+};
+
+cudaError_t launch_page_stats(const StatsParams& p, int D, int max_logical_pages,
+                              cudaStream_t stream);
+cudaError_t launch_page_select(const SelectParams& p, int D, cudaStream_t stream);
+cudaError_t launch_decode(const DecodeParams& p, const CUtensorMap& kmap, const CUtensorMap& vmap,
+                          int D, int G, int num_ctas, cudaStream_t stream);
+size_t decode_workspace_bytes(int pairs, int num_warps, int G, int D);
+int decode_num_ctas(int sm_count);
+size_t decode_smem_bytes(int D, int G);
+int decode_warps_per_cta(int D, int G);
+
+cudaError_t launch_wait_timeout_probe(uint64_t cycles, unsigned int* status, cudaStream_t stream);
+
+// Raises a kernel's dynamic shared memory limit once per (kernel, device), so
+// that later calls (e.g. during CUDA-graph capture) launch without it.
+cudaError_t set_smem_once(const void* kernel, int bytes);
+
+// host helpers shared by the entry points (api.cu)
+bool make_map_2d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint64_t pitch_elems,
+                 uint32_t box_rows);
+uint64_t wait_limit();
+int current_sm_count();
+unsigned int* device_status_word();
+
+}  // namespace lserve

@@ -1,0 +1,208 @@
+/*
+ * lserve.h -- C ABI of liblserve.so: the hot path of LServe-style unified
+ * sparse attention on one NVIDIA B200 (sm_100a).
+ *
+ * Source of the method: the LServe explainer page "MLSys 2025論文解説: LServe —
+ * 統一疎アテンションによる長文脈LLM推論の効率化" (arXiv 2502.14866) and the LServe
+ * abstract page "LServe: Efficient Long-sequence LLM Serving with Unified Sparse
+ * Attention".  Section names below are that explainer's.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  - bf16 tensors are IEEE bfloat16 (uint16 storage).  All pointers except
+ *    those named *_host are DEVICE pointers owned by the caller; the library
+ *    keeps no reference after the call returns and allocates nothing.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *    stream).  Calls only enqueue work; results are ready when the stream is.
+ *  - Every call validates its arguments on the host first.  On failure it
+ *    returns a non-zero lserve_status and launches nothing.  A launch error
+ *    reported by the CUDA runtime returns LSERVE_ERR_CUDA.
+ *  - Kernels never trap.  Waits on hardware barriers are bounded; a wait that
+ *    runs out sets a device status flag (LSERVE_ERR_TIMEOUT) that
+ *    lserve_read_device_status() returns.  Block-table entries, selected page
+ *    ordinals and page counts are checked per page: an entry out of range sets
+ *    LSERVE_ERR_BOUNDS and the offending page is skipped (never read).
+ *  - Stateless and thread-safe, apart from one cached driver entry point and
+ *    a per-device cache of the SM count.
+ *
+ * Paged KV cache layout (the "page" and "block table" of hierarchical paging,
+ * 技術的詳細 › 階層的ページング)
+ *  - k_pool, v_pool : bf16 [num_pool_pages][H_kv][N_P][D]; one (page, head)
+ *                     is N_P * D contiguous elements.
+ *  - block_table    : int32 [B][max_pages_per_seq]; entry m is the pool id of
+ *                     physical page m (tokens [m*N_P, (m+1)*N_P)) of sequence b.
+ *  - ctx_lens       : int32 [B]; n_b, the number of valid tokens of sequence b.
+ *                     Tokens at positions >= n_b of the last page are ignored.
+ *  - head_kind      : uint8 [H_kv] (device) -- 0 = retrieval head, 1 = streaming
+ *                     head (技術的詳細 › 静的スパーシティ).
+ *  - stats_pool     : bf16 [num_pool_pages][H_kv][g][2][D], g = N_P / N_L;
+ *                     [..][0][:] = k_min, [..][1][:] = k_max of logical page
+ *                     (pool page, head, sub-page), indexed by the same pool id.
+ *  - q              : bf16 [B][H_q][D]; query head hq uses KV head hq / G,
+ *                     G = H_q / H_kv.
+ */
+#ifndef LSERVE_H_
+#define LSERVE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  LSERVE_OK = 0,
+  LSERVE_ERR_INVALID_ARG = 1, /* null pointer, bad size, misaligned pointer      */
+  LSERVE_ERR_UNSUPPORTED = 2, /* valid but not built: e.g. D not in {64, 128}    */
+  LSERVE_ERR_WORKSPACE = 3,   /* workspace missing or smaller than required      */
+  LSERVE_ERR_CUDA = 4,        /* the CUDA runtime reported an error              */
+  LSERVE_ERR_TIMEOUT = 5,     /* a bounded device wait ran out                   */
+  LSERVE_ERR_BOUNDS = 6       /* a page index was out of range (page skipped)   */
+} lserve_status;
+
+typedef enum { LSERVE_OP_STATS = 0, LSERVE_OP_SELECT = 1, LSERVE_OP_DECODE = 2, LSERVE_OP_PREFILL = 3 } lserve_op;
+
+/* Shapes of the paged decode calls. */
+typedef struct {
+  int32_t batch;             /* B >= 1                                              */
+  int32_t num_q_heads;       /* H_q, a multiple of H_kv                             */
+  int32_t num_kv_heads;      /* H_kv >= 1; G = H_q / H_kv in {1, 2, 4, 8}           */
+  int32_t head_dim;          /* D in {64, 128}                                      */
+  int32_t logical_page;      /* N_L in {8, 16, 32, 64}                              */
+  int32_t physical_page;     /* N_P = g * N_L, g >= 1; N_P in {32, 64, 128, 256}    */
+  int32_t max_pages_per_seq; /* row length of block_table                           */
+  int32_t num_pool_pages;    /* first dimension of k_pool / v_pool / stats_pool     */
+} lserve_paged_desc;
+
+/* Shapes of the prefill call.  Q [T][H_q][D], K/V [T][H_kv][D], O [T][H_q][D]. */
+typedef struct {
+  int32_t seq_len;      /* T >= 1                                                   */
+  int32_t num_q_heads;  /* H_q, a multiple of H_kv                                  */
+  int32_t num_kv_heads; /* H_kv                                                     */
+  int32_t head_dim;     /* D = 128 (64 also accepted)                               */
+  int32_t block_q;      /* query block, == block_k, 128                             */
+  int32_t block_k;      /* key block                                                */
+  int32_t sink_blocks;  /* Lambda mask: leading blocks every streaming row sees     */
+  int32_t local_blocks; /* Lambda mask: blocks [i - local + 1, i] (diagonal counts) */
+} lserve_prefill_desc;
+
+/*
+ * lserve_page_stats -- channel-wise k_min / k_max of every logical page.
+ * [技術的詳細 › 動的スパーシティ: k_min^j[i], k_max^j[i] are the min / max of channel
+ *  i over the keys of logical page j; 階層的ページング: logical pages of N_L tokens
+ *  inside physical pages of N_P = g * N_L tokens.]
+ *
+ * For each sequence b, RETRIEVAL head h (streaming heads are skipped) and
+ * logical page j >= first_logical_page with j * N_L < n_b, writes k_min and
+ * k_max over the valid tokens [j*N_L, min((j+1)*N_L, n_b)) into stats_pool at
+ * pool id block_table[b][j / g], sub-page j % g.  Results are exact (min/max of
+ * bf16 values).  first_logical_page = 0 rebuilds everything; a larger value
+ * refreshes only the pages from there on (e.g. the page a decode step filled).
+ * Reads ~n*D*2 bytes of K per (b, h), writes 1/(N_L/2) of that.
+ */
+int lserve_page_stats(const lserve_paged_desc* desc, const void* k_pool, const int32_t* block_table,
+                      const int32_t* ctx_lens, const uint8_t* head_kind, void* stats_pool,
+                      int32_t first_logical_page, void* stream);
+
+/*
+ * lserve_page_select -- query-centric page scores and top-K physical pages.
+ * [技術的詳細 › 動的スパーシティ, the equation
+ *    S^j = sum_{i=1..D} max(q[i] * k_max^j[i], q[i] * k_min^j[i]);
+ *  階層的ページング: a physical page scores the max of its logical pages;
+ *  統一ブロックスパースアテンション figure: "Top-K物理ページ"; Reusable Page Selection:
+ *  the result may be reused for k consecutive decode steps (default 4).]
+ *
+ * For each (b, retrieval KV head h): S^j is summed over the G query heads of h
+ * (GQA reading), in fp32 from exact bf16 x bf16 products; P^m = max over the
+ * valid logical pages of physical page m; then the top_k largest P^m, ties to
+ * the lowest m.  Outputs:
+ *   sel         int32 [B][H_kv][top_k]: chosen page ORDINALS m (not pool ids),
+ *               ascending, padded with -1.  Streaming heads: all -1.
+ *   sel_count   int32 [B][H_kv]: min(top_k, ceil(n_b / N_P)); 0 for streaming.
+ *   phys_scores float [B][H_kv][max_pages_per_seq] or NULL; entries past the
+ *               sequence's pages and for streaming heads are left untouched.
+ * workspace: lserve_workspace_size(LSERVE_OP_SELECT, desc, top_k) bytes (used
+ * for the scores when phys_scores is NULL).  1 <= top_k <= max_pages_per_seq.
+ */
+int lserve_page_select(const lserve_paged_desc* desc, const void* q, const void* stats_pool,
+                       const int32_t* block_table, const int32_t* ctx_lens, const uint8_t* head_kind,
+                       int32_t top_k, int32_t* sel, int32_t* sel_count, float* phys_scores,
+                       void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * lserve_sparse_decode_attn -- one decode step of paged GQA attention over the
+ * pages each head keeps.
+ * [統一ブロックスパースアテンション figure: retrieval heads attend the top-K
+ *  physical pages, streaming heads the Lambda-shaped sink + local blocks;
+ *  技術的詳細 › 静的スパーシティ: sink tokens and recent local tokens.]
+ *
+ * Retrieval head h of sequence b attends every valid token of the pages
+ * sel[b][h][0 .. sel_count[b][h]) (page ordinals, as lserve_page_select writes
+ * them).  A streaming head attends the pages [0, ceil(sink_tokens / N_P)) and
+ * every page holding one of the last local_tokens tokens.  Each of the G query
+ * heads computes softmax(softmax_scale * q.k) . v in fp32 (split over pages,
+ * merged by a log-sum-exp combine pass) and writes:
+ *   out  bf16 [B][H_q][D]
+ *   lse  float [B][H_q] natural-log sum of exp(scale * q.k), or NULL.
+ * A head with no token to attend (n_b = 0) gets out = 0, lse = -inf.
+ * workspace: lserve_workspace_size(LSERVE_OP_DECODE, desc, top_k) bytes.
+ */
+int lserve_sparse_decode_attn(const lserve_paged_desc* desc, const void* q, const void* k_pool,
+                              const void* v_pool, const int32_t* block_table, const int32_t* ctx_lens,
+                              const uint8_t* head_kind, const int32_t* sel, const int32_t* sel_count,
+                              int32_t top_k, int32_t sink_tokens, int32_t local_tokens,
+                              float softmax_scale, void* out, float* lse, void* workspace,
+                              size_t workspace_bytes, void* stream);
+
+/*
+ * lserve_blocksparse_prefill -- causal block-sparse flash attention for one
+ * sequence.
+ * [統一ブロックスパースアテンション: retrieval heads "block-sparse attention, static
+ *  pattern" (dense causal here), streaming heads the Lambda mask of sink and
+ *  local blocks; the ideal speedup at block sparsity r is 1/(1-r).  Abstract
+ *  page: computation on less important tokens is skipped block-wise.]
+ *
+ * Query block row i of a head whose KV head is retrieval visits key blocks
+ * 0..i; a streaming head visits [0, sink_blocks) and [i-local_blocks+1, i].
+ * Causal masking applies inside the diagonal block.  QK^T and PV run on the
+ * tcgen05 tensor cores (bf16 in, fp32 accumulate in tensor memory); softmax in
+ * fp32.  head_kind_host is a HOST array uint8 [H_kv].
+ *   q   bf16 [T][H_q][D], k / v bf16 [T][H_kv][D] (16-byte aligned)
+ *   out bf16 [T][H_q][D]; lse float [H_q][T] (natural log) or NULL.
+ * workspace: lserve_workspace_size(LSERVE_OP_PREFILL, desc, 0) bytes.
+ */
+int lserve_blocksparse_prefill(const lserve_prefill_desc* desc, const void* q, const void* k,
+                               const void* v, const uint8_t* head_kind_host, float softmax_scale,
+                               void* out, float* lse, void* workspace, size_t workspace_bytes,
+                               void* stream);
+
+/* Bytes of workspace `op` needs for these shapes on the CURRENT device
+ * (desc points to lserve_paged_desc, or lserve_prefill_desc for PREFILL).
+ * Returns 0 for invalid shapes. */
+size_t lserve_workspace_size(int op, const void* desc, int32_t top_k);
+
+/* Synchronises `stream`, returns the first device-side error flag raised since
+ * the last call (LSERVE_ERR_TIMEOUT / LSERVE_ERR_BOUNDS) or LSERVE_OK, and
+ * clears the flags of the current device. */
+int lserve_read_device_status(void* stream);
+
+/* Upper bound, in SM clock cycles, of every bounded device wait started after
+ * this call (default 4e9, about two seconds).  0 restores the default. */
+void lserve_set_wait_limit_cycles(uint64_t cycles);
+
+/* Diagnostic: launches one CTA that waits on a hardware barrier nobody
+ * arrives at, bounded by `cycles`; lserve_read_device_status() must then
+ * report LSERVE_ERR_TIMEOUT.  Exercises the timeout path without a fault. */
+int lserve_debug_wait_timeout(uint64_t cycles, void* stream);
+
+const char* lserve_status_string(int status);
+
+/* 1: page-level index checks are compiled into every kernel. */
+int lserve_bounds_checked(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LSERVE_H_ */
