@@ -112,6 +112,9 @@ class ClockSampler:
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
     def __init__(self, device_index, uuid=None):
+        if uuid is not None:
+            uuid = str(uuid)
+            uuid = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
         self.sel = ["-i", uuid] if uuid else ["-i", str(device_index)]
         self.proc = None
 

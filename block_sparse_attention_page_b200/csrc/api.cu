@@ -85,6 +85,20 @@ cudaError_t set_smem_once(const void* kernel, int bytes) {
   return cudaSuccess;
 }
 
+// Contiguous bf16 tensor [d2][d1][d0] (rank 2 or 3), box b0 x b1 x b2, 128-byte swizzle.
+bool make_map_tiled(CUtensorMap* m, const void* base, int rank, uint64_t d0, uint64_t d1, uint64_t d2,
+                    uint32_t b0, uint32_t b1, uint32_t b2) {
+  auto fn = encode_fn();
+  if (!fn || rank < 2 || rank > 3) return false;
+  cuuint64_t dims[3] = {d0, d1, d2};
+  cuuint64_t strides[2] = {d0 * 2, d0 * d1 * 2};
+  cuuint32_t box[3] = {b0, b1, b2};
+  cuuint32_t es[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(base), dims,
+            strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 uint64_t wait_limit() { return g_wait_limit; }
 int current_sm_count() { return sm_count_current(); }
 

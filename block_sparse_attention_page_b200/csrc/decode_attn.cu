@@ -388,7 +388,9 @@ decode_attn_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
 }
 
 // One warp per (pair, query head of the pair): merge the partials of the warps
-// whose tile ranges overlap the pair.
+// whose tile ranges overlap the pair.  Lanes take one segment each (32 at a
+// time): the max and the weighted row sum are warp reductions, then every lane
+// accumulates its D/32 channels over the segments with independent loads.
 __global__ void __launch_bounds__(128)
 decode_combine_kernel(const __grid_constant__ DecodeParams p, int G, int D) {
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
@@ -405,24 +407,42 @@ decode_combine_kernel(const __grid_constant__ DecodeParams p, int G, int D) {
   float acc[4] = {0.f, 0.f, 0.f, 0.f};
   float M = -INFINITY, Lsum = 0.f;
   if (T1 > T0) {
-    auto start = [&](long long w) { return U * w / NW; };
-    long long w = (T0 * NW) / U;
-    while (w + 1 < NW && start(w + 1) <= T0) ++w;
-    while (w > 0 && start(w) > T0) --w;
-    // pass 1: the running max over segments
-    for (long long ww = w; ww < NW && start(ww) < T1; ++ww) {
-      if (start(ww + 1) <= start(ww) || start(ww + 1) <= T0) continue;
-      M = fmaxf(M, pml[((size_t)(ww + pair) * G + g) * 2]);
-    }
-    if (M > -INFINITY) {
-      for (long long ww = w; ww < NW && start(ww) < T1; ++ww) {
-        if (start(ww + 1) <= start(ww) || start(ww + 1) <= T0) continue;
-        const size_t slot = (size_t)(ww + pair);
-        const float2 ml = *reinterpret_cast<const float2*>(pml + (slot * G + g) * 2);
-        const float wgt = exp2f(ml.x - M);
-        Lsum += wgt * ml.y;
-        const float* src = po + (slot * G + g) * D + lane * CPL;
-        for (int j = 0; j < CPL; ++j) acc[j] += wgt * src[j];
+    // first warp whose range holds tile T0: start(w) = floor(U*w/NW) <= T0 < start(w+1)
+    long long w0 = (T0 * NW) / U;
+    while (w0 + 1 < NW && (U * (w0 + 1)) / NW <= T0) ++w0;
+    while (w0 > 0 && (U * w0) / NW > T0) --w0;
+    // last warp whose range holds tile T1 - 1
+    long long w1 = ((T1 - 1) * NW) / U;
+    while (w1 + 1 < NW && (U * (w1 + 1)) / NW <= T1 - 1) ++w1;
+    while (w1 > 0 && (U * w1) / NW > T1 - 1) --w1;
+    for (long long base = w0; base <= w1; base += 32) {
+      const long long ww = base + lane;
+      float m_s = -INFINITY, l_s = 0.f;
+      bool has = false;
+      if (ww <= w1) {
+        const long long s0 = (U * ww) / NW, s1 = (U * (ww + 1)) / NW;
+        has = s1 > s0;  // warps with an empty range wrote nothing
+        if (has) {
+          const float2 ml = *reinterpret_cast<const float2*>(pml + ((size_t)(ww + pair) * G + g) * 2);
+          m_s = ml.x;
+          l_s = ml.y;
+        }
+      }
+      const float Mc = warp_max(m_s);
+      const float Mn = fmaxf(M, Mc);
+      if (!(Mn > -INFINITY)) continue;
+      const float rescale = exp2f(M - Mn);  // 0 when M was -inf
+      const float w_s = has ? exp2f(m_s - Mn) : 0.f;
+      Lsum = Lsum * rescale + warp_sum(w_s * l_s);
+      for (int j = 0; j < CPL; ++j) acc[j] *= rescale;
+      M = Mn;
+      const int nseg = (int)min(32ll, w1 - base + 1);
+#pragma unroll 4
+      for (int i = 0; i < nseg; ++i) {
+        const float wi = __shfl_sync(0xffffffffu, w_s, i);
+        if (wi == 0.f) continue;
+        const float* src = po + ((size_t)(base + i + pair) * G + g) * D + lane * CPL;
+        for (int j = 0; j < CPL; ++j) acc[j] = fmaf(wi, src[j], acc[j]);
       }
     }
   }

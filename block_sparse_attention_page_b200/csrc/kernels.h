@@ -84,6 +84,8 @@ cudaError_t set_smem_once(const void* kernel, int bytes);
 // host helpers shared by the entry points (api.cu)
 bool make_map_2d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint64_t pitch_elems,
                  uint32_t box_rows);
+bool make_map_tiled(CUtensorMap* m, const void* base, int rank, uint64_t d0, uint64_t d1, uint64_t d2,
+                    uint32_t b0, uint32_t b1, uint32_t b2);
 uint64_t wait_limit();
 int current_sm_count();
 unsigned int* device_status_word();

@@ -1,13 +1,485 @@
-// Block-sparse prefill: placeholder until the tcgen05 kernel lands.
+// lserve_blocksparse_prefill: causal block-sparse flash attention on the
+// sm_100a tensor cores (LServe explainer, 統一ブロックスパースアテンション: retrieval
+// heads dense causal, streaming heads the Lambda mask of sink + local blocks,
+// ideal speedup 1/(1-r) at block sparsity r; abstract page: computation on
+// less important tokens is skipped block-wise).
+//
+// One CTA per SM, persistent over work tiles (query head, 128-row query tile).
+// Tiles are ordered by decreasing cost (dense heads, last query tiles first)
+// and dealt to CTAs in a snake order, so every SM ends up with a similar
+// number of key tiles.  The key-tile iterator visits only the non-empty tiles
+// of the row (all j <= i for dense heads; sink tiles and the local window for
+// streaming heads) -- the block skipping of the method.
+//
+// Warp roles (192 threads):
+//   warp 0     TMA producer: Q tile, then K and V tiles into two-stage rings
+//              (3-D tensor maps over [T][H][D], 128-byte swizzle, no multicast)
+//   warp 1     tensor-memory owner and single-thread MMA issuer:
+//                S_j = Q K_j^T  -> TMEM (two fp32 128x128 buffers, ping-pong)
+//                O  += P_j V_j  -> TMEM (fp32 128 x D), P from shared memory
+//   warps 2-5  softmax: thread r owns query row r (TMEM lane r); loads S_j,
+//              masks, keeps the running max / row sum in fp32, writes P_j as
+//              bf16 into shared memory (swizzled like a TMA tile), rescales O
+//              in TMEM only when the row max grows by more than 2^8, and runs
+//              the epilogue O / l -> bf16 and the log-sum-exp.
+// MMA order S_0, S_1, PV_0, S_2, PV_1, ... keeps the tensor core on S_{j+1}
+// while the softmax warps work on S_j.
+#include <algorithm>
+#include <cmath>
+#include <cstring>
+
+#include "common.cuh"
+#include "kernels.h"
 #include "prefill.h"
+#include "tcgen05.cuh"
 
 namespace lserve {
 
-size_t prefill_workspace_bytes(const lserve_prefill_desc*) { return 0; }
+namespace {
 
-int prefill_entry(const lserve_prefill_desc*, const void*, const void*, const void*, const uint8_t*,
-                  float, void*, float*, void*, size_t, cudaStream_t) {
-  return LSERVE_ERR_UNSUPPORTED;
+constexpr int kBM = 128;            // query rows per tile (MMA M)
+constexpr int kBN = 128;            // keys per key tile (MMA N of S, K of PV)
+constexpr int kThreads = 192;
+constexpr float kRescaleLog2 = 8.0f;  // rescale O only when the max grows by > 2^8
+constexpr int kMaxHeads = 256;
+
+struct PrefillParams {
+  __nv_bfloat16* out;
+  float* lse;
+  unsigned int* status;
+  uint64_t wait_limit;
+  float scale_log2;
+  int T, H_q, H_kv, G;
+  int mask_block, sink_blocks, local_blocks;
+  int n_qt;               // query tiles per head
+  int n_dense, n_stream;  // query heads whose KV head is retrieval / streaming
+  uint8_t dense_heads[kMaxHeads];
+  uint8_t stream_heads[kMaxHeads];
+  uint8_t kv_kind[kMaxHeads];
+};
+
+template <int D>
+struct Layout {
+  static constexpr int kBox = kBM * 128;          // one 64-column swizzled box: 16 KiB
+  static constexpr int kTile = kBox * (D / 64);   // a Q, K or V tile
+  static constexpr int kQ = 0;
+  static constexpr int kK = kQ + kTile;           // 2 stages
+  static constexpr int kV = kK + 2 * kTile;       // 2 stages
+  static constexpr int kP = kV + 2 * kTile;       // P: 128 x 128 bf16, 2 boxes
+  static constexpr int kBar = kP + 2 * kBox;
+  static constexpr int kNumBars = 17;
+  static constexpr int kBytes = kBar + kNumBars * 8 + 16;
+};
+
+struct TileRef {
+  int hq, qt;
+};
+
+__device__ __forceinline__ TileRef tile_at(const PrefillParams& p, int idx) {
+  const int nd = p.n_dense * p.n_qt;
+  if (idx < nd) return {p.dense_heads[idx % p.n_dense], p.n_qt - 1 - idx / p.n_dense};
+  idx -= nd;
+  return {p.stream_heads[idx % p.n_stream], p.n_qt - 1 - idx / p.n_stream};
+}
+
+// round r of CTA c: snake order over the cost-sorted tile list
+__device__ __forceinline__ int cta_tile(int r, int c, int grid) {
+  return r * grid + ((r & 1) ? grid - 1 - c : c);
+}
+
+// Key tiles a query tile visits: [0, a_end) then [b_begin, b_end).
+struct KvRange {
+  int a_end, b_begin, b_end;
+  __device__ int count() const { return a_end + (b_end - b_begin); }
+  __device__ int at(int j) const { return j < a_end ? j : b_begin + (j - a_end); }
+};
+
+__device__ __forceinline__ KvRange kv_range(const PrefillParams& p, int kind, int qt) {
+  if (kind == 0) return {qt + 1, qt + 1, qt + 1};
+  const int R = kBN / p.mask_block;  // mask blocks per tile
+  const int st = min((p.sink_blocks * p.mask_block + kBN - 1) / kBN, qt + 1);
+  const int first_kb = max(0, qt * R - p.local_blocks + 1);
+  const int lt = max((first_kb * p.mask_block) / kBN, st);
+  return {st, lt, qt + 1};
+}
+
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, uint64_t limit,
+                                          unsigned int* status) {
+  const bool ok = mbar_wait(bar, parity, limit, status);
+  return __all_sync(0xffffffffu, ok);
+}
+
+}  // namespace
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+prefill_kernel(const __grid_constant__ PrefillParams p, const __grid_constant__ CUtensorMap qmap,
+               const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap) {
+  using L = Layout<D>;
+  constexpr int NBOX = D / 64;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
+  uint64_t* q_full = bars + 0;
+  uint64_t* q_empty = bars + 1;
+  uint64_t* k_full = bars + 2;   // [2]
+  uint64_t* k_empty = bars + 4;  // [2]
+  uint64_t* v_full = bars + 6;   // [2]
+  uint64_t* v_empty = bars + 8;  // [2]
+  uint64_t* s_full = bars + 10;  // [2]
+  uint64_t* s_free = bars + 12;  // [2]
+  uint64_t* p_full = bars + 14;
+  uint64_t* p_free = bars + 15;
+  uint64_t* o_free = bars + 16;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::kBar + L::kNumBars * 8);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&k_full[s], 1);
+      mbar_init(&k_empty[s], 1);
+      mbar_init(&v_full[s], 1);
+      mbar_init(&v_empty[s], 1);
+      mbar_init(&s_full[s], 1);
+      mbar_init(&s_free[s], 128);
+    }
+    mbar_init(p_full, 128);
+    mbar_init(p_free, 1);
+    mbar_init(o_free, 128);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tc::alloc(tmem_holder, 512);
+    tc::relinquish();
+  }
+  tc::fence_before();
+  __syncthreads();
+  tc::fence_after();
+  const uint32_t tmem = *tmem_holder;
+  const uint32_t tmem_o = tmem + 2 * kBN;  // columns [256, 256 + D)
+
+  const int total = (p.n_dense + p.n_stream) * p.n_qt;
+  const int grid = gridDim.x;
+  const uint64_t lim = p.wait_limit;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      tma_prefetch_desc(&qmap);
+      tma_prefetch_desc(&kmap);
+      tma_prefetch_desc(&vmap);
+      int q_use = 0, kv_use = 0;
+      for (int r = 0;; ++r) {
+        const int idx = cta_tile(r, blockIdx.x, grid);
+        if (idx >= total) break;
+        const TileRef t = tile_at(p, idx);
+        const int hkv = t.hq / p.G;
+        const KvRange kr = kv_range(p, p.kv_kind[hkv], t.qt);
+        if (q_use > 0 && !mbar_wait(q_empty, (q_use - 1) & 1, lim, p.status)) break;
+        mbar_arrive_expect_tx(q_full, L::kTile);
+        for (int bx = 0; bx < NBOX; ++bx)
+          tma_load_3d(smem + L::kQ + bx * L::kBox, &qmap, bx * 64, t.hq, t.qt * kBM, q_full);
+        ++q_use;
+        bool ok = true;
+        const int nkv = kr.count();
+        for (int j = 0; j < nkv && ok; ++j) {
+          const int kt = kr.at(j);
+          const int s = kv_use & 1, n = kv_use >> 1;
+          if (n > 0 && !mbar_wait(&k_empty[s], (n - 1) & 1, lim, p.status)) { ok = false; break; }
+          mbar_arrive_expect_tx(&k_full[s], L::kTile);
+          for (int bx = 0; bx < NBOX; ++bx)
+            tma_load_3d(smem + L::kK + s * L::kTile + bx * L::kBox, &kmap, bx * 64, hkv, kt * kBN,
+                        &k_full[s]);
+          if (n > 0 && !mbar_wait(&v_empty[s], (n - 1) & 1, lim, p.status)) { ok = false; break; }
+          mbar_arrive_expect_tx(&v_full[s], L::kTile);
+          for (int bx = 0; bx < NBOX; ++bx)
+            tma_load_3d(smem + L::kV + s * L::kTile + bx * L::kBox, &vmap, bx * 64, hkv, kt * kBN,
+                        &v_full[s]);
+          ++kv_use;
+        }
+        if (!ok) break;
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = tc::idesc_bf16_f32(kBM, kBN, false, false);
+      constexpr uint32_t idesc_pv = tc::idesc_bf16_f32(kBM, D, false, true);
+      const uint32_t q_addr = smem_u32(smem + L::kQ);
+      const uint32_t p_addr = smem_u32(smem + L::kP);
+      int q_use = 0, kv_base = 0, s_count = 0, pv_count = 0, tile_count = 0;
+      bool ok = true;
+      for (int r = 0; ok; ++r) {
+        const int idx = cta_tile(r, blockIdx.x, grid);
+        if (idx >= total) break;
+        const TileRef t = tile_at(p, idx);
+        const KvRange kr = kv_range(p, p.kv_kind[t.hq / p.G], t.qt);
+        const int nkv = kr.count();
+        if (!mbar_wait(q_full, q_use & 1, lim, p.status)) break;
+        ++q_use;
+        tc::fence_after();
+        auto issue_s = [&](int j) -> bool {
+          const int kvi = kv_base + j, s = kvi & 1, n = kvi >> 1;
+          const int sb = s_count & 1, sn = s_count >> 1;
+          if (sn > 0 && !mbar_wait(&s_free[sb], (sn - 1) & 1, lim, p.status)) return false;
+          if (!mbar_wait(&k_full[s], n & 1, lim, p.status)) return false;
+          tc::fence_after();
+          const uint32_t k_addr = smem_u32(smem + L::kK + s * L::kTile);
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk / 4) * L::kBox + (kk % 4) * 32;
+            tc::mma_ss(tmem + sb * kBN, tc::smem_desc_sw128(q_addr + off, 16, 1024),
+                       tc::smem_desc_sw128(k_addr + off, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
+          }
+          tc::commit(&s_full[sb]);
+          tc::commit(&k_empty[s]);
+          if (j == nkv - 1) tc::commit(q_empty);
+          ++s_count;
+          return true;
+        };
+        auto issue_pv = [&](int j) -> bool {
+          const int kvi = kv_base + j, s = kvi & 1, n = kvi >> 1;
+          if (!mbar_wait(p_full, pv_count & 1, lim, p.status)) return false;
+          if (j == 0 && tile_count > 0 && !mbar_wait(o_free, (tile_count - 1) & 1, lim, p.status))
+            return false;
+          if (!mbar_wait(&v_full[s], n & 1, lim, p.status)) return false;
+          tc::fence_after();
+          const uint32_t v_addr = smem_u32(smem + L::kV + s * L::kTile);
+#pragma unroll
+          for (int kk = 0; kk < kBN / 16; ++kk) {
+            const uint32_t poff = (kk / 4) * L::kBox + (kk % 4) * 32;
+            tc::mma_ss(tmem_o, tc::smem_desc_sw128(p_addr + poff, 16, 1024),
+                       tc::smem_desc_sw128(v_addr + kk * 16 * 128, L::kBox, 1024), idesc_pv,
+                       (j > 0 || kk > 0) ? 1u : 0u);
+          }
+          tc::commit(&v_empty[s]);
+          tc::commit(p_free);
+          ++pv_count;
+          return true;
+        };
+        ok = issue_s(0);
+        for (int j = 1; j < nkv && ok; ++j) ok = issue_s(j) && issue_pv(j - 1);
+        if (ok) ok = issue_pv(nkv - 1);
+        kv_base += nkv;
+        ++tile_count;
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ softmax
+    const int quad = warp & 3;                 // TMEM lane quarter of this warp
+    const int row = quad * 32 + lane;          // query row within the tile
+    const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+    uint8_t* p_row = smem + L::kP + row * 128;
+    int s_count = 0, pv_count = 0;
+    bool ok = true;
+    for (int r = 0; ok; ++r) {
+      const int idx = cta_tile(r, blockIdx.x, grid);
+      if (idx >= total) break;
+      const TileRef t = tile_at(p, idx);
+      const int kind = p.kv_kind[t.hq / p.G];
+      const KvRange kr = kv_range(p, kind, t.qt);
+      const int nkv = kr.count();
+      const int q = t.qt * kBM + row;
+      float m = -INFINITY, l = 0.f;
+      for (int j = 0; j < nkv; ++j) {
+        const int kt = kr.at(j);
+        const int sb = s_count & 1, sn = s_count >> 1;
+        if (!warp_wait(&s_full[sb], sn & 1, lim, p.status)) { ok = false; break; }
+        tc::fence_after();
+        float x[kBN];
+#pragma unroll
+        for (int c = 0; c < kBN / 32; ++c) {
+          uint32_t u[32];
+          tc::ld32(tmem + lane_off + sb * kBN + c * 32, u);
+          tc::wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) x[c * 32 + i] = __uint_as_float(u[i]);
+        }
+        tc::fence_before();
+        mbar_arrive(&s_free[sb]);
+        ++s_count;
+        const bool need_mask = kt == t.qt || (kt + 1) * kBN > p.T || (kind == 1 && p.mask_block < kBN);
+        if (need_mask) {
+          const int qb = q / p.mask_block;
+#pragma unroll
+          for (int i = 0; i < kBN; ++i) {
+            const int k = kt * kBN + i;
+            const int kb = k / p.mask_block;
+            const bool allowed = k <= q && k < p.T &&
+                                 (kind == 0 || kb < p.sink_blocks || qb - kb < p.local_blocks);
+            if (!allowed) x[i] = -INFINITY;
+          }
+        }
+        float mt = -INFINITY;
+#pragma unroll
+        for (int i = 0; i < kBN; ++i) mt = fmaxf(mt, x[i]);
+        const float m_new = fmaxf(m, mt * p.scale_log2);
+        float alpha = 1.f;
+        bool rescale = false;
+        if (j == 0) {
+          m = m_new;
+        } else if (m_new > m + kRescaleLog2) {
+          alpha = tc::ex2(m - m_new);
+          m = m_new;
+          rescale = true;
+        }
+        const float mu = (m == -INFINITY) ? 0.f : m;
+        float rs = 0.f;
+#pragma unroll
+        for (int i = 0; i < kBN; ++i) {
+          x[i] = tc::ex2(fmaf(x[i], p.scale_log2, -mu));
+          rs += x[i];
+        }
+        l = l * alpha + rs;
+        // P_j may overwrite P_{j-1} (and O may be rescaled) once PV_{j-1} is done
+        if (pv_count > 0 && !warp_wait(p_free, (pv_count - 1) & 1, lim, p.status)) { ok = false; break; }
+        tc::fence_after();
+        if (rescale) {
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t u[32];
+            tc::ld32(tmem_o + lane_off + c * 32, u);
+            tc::wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) u[i] = __float_as_uint(__uint_as_float(u[i]) * alpha);
+            tc::st32(tmem_o + lane_off + c * 32, u);
+          }
+          tc::wait_st();
+        }
+#pragma unroll
+        for (int c = 0; c < kBN / 8; ++c) {
+          uint4 w;
+          w.x = float2_to_bf16x2(x[c * 8 + 0], x[c * 8 + 1]);
+          w.y = float2_to_bf16x2(x[c * 8 + 2], x[c * 8 + 3]);
+          w.z = float2_to_bf16x2(x[c * 8 + 4], x[c * 8 + 5]);
+          w.w = float2_to_bf16x2(x[c * 8 + 6], x[c * 8 + 7]);
+          *reinterpret_cast<uint4*>(p_row + (c / 8) * L::kBox + (((c % 8) ^ (row & 7)) << 4)) = w;
+        }
+        fence_proxy_async_smem();
+        tc::fence_before();
+        mbar_arrive(p_full);
+        ++pv_count;
+      }
+      if (!ok) break;
+      // ---- epilogue: O / l -> bf16, log-sum-exp
+      if (!warp_wait(p_free, (pv_count - 1) & 1, lim, p.status)) break;
+      tc::fence_after();
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+      __nv_bfloat16* orow = p.out + ((size_t)q * p.H_q + t.hq) * D;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t u[32];
+        tc::ld32(tmem_o + lane_off + c * 32, u);
+        tc::wait_ld();
+        if (q < p.T) {
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            uint4 w;
+            w.x = float2_to_bf16x2(__uint_as_float(u[v * 8 + 0]) * inv, __uint_as_float(u[v * 8 + 1]) * inv);
+            w.y = float2_to_bf16x2(__uint_as_float(u[v * 8 + 2]) * inv, __uint_as_float(u[v * 8 + 3]) * inv);
+            w.z = float2_to_bf16x2(__uint_as_float(u[v * 8 + 4]) * inv, __uint_as_float(u[v * 8 + 5]) * inv);
+            w.w = float2_to_bf16x2(__uint_as_float(u[v * 8 + 6]) * inv, __uint_as_float(u[v * 8 + 7]) * inv);
+            *reinterpret_cast<uint4*>(orow + c * 32 + v * 8) = w;
+          }
+        }
+      }
+      if (p.lse != nullptr && q < p.T)
+        p.lse[(size_t)t.hq * p.T + q] = l > 0.f ? (m + __log2f(l)) * 0.69314718055994530942f : -INFINITY;
+      tc::fence_before();
+      mbar_arrive(o_free);
+    }
+  }
+  tc::fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc::fence_after();
+    tc::dealloc(tmem, 512);
+  }
+}
+
+// --- host side ------------------------------------------------------------------
+
+static bool make_map_3d(CUtensorMap* m, const void* base, uint64_t T, uint64_t H, uint64_t D) {
+  // [T][H][D] bf16, box = 64 channels x 1 head x 128 tokens, 128-byte swizzle
+  return make_map_tiled(m, base, 3, D, H, T, 64, 1, 128);
+}
+
+size_t prefill_workspace_bytes(const lserve_prefill_desc* d) {
+  (void)d;
+  return 0;  // the schedule is closed-form; nothing to stage
+}
+
+int prefill_entry(const lserve_prefill_desc* d, const void* q, const void* k, const void* v,
+                  const uint8_t* head_kind_host, float softmax_scale, void* out, float* lse,
+                  void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  (void)workspace;
+  (void)workspace_bytes;
+  if (!d || !q || !k || !v || !head_kind_host || !out) return LSERVE_ERR_INVALID_ARG;
+  if (d->seq_len < 1 || d->num_kv_heads < 1 || d->num_q_heads < d->num_kv_heads ||
+      d->num_q_heads % d->num_kv_heads)
+    return LSERVE_ERR_INVALID_ARG;
+  if (d->block_q != d->block_k || d->sink_blocks < 0 || d->local_blocks < 1)
+    return LSERVE_ERR_INVALID_ARG;
+  if (!(softmax_scale > 0.f) || !std::isfinite(softmax_scale)) return LSERVE_ERR_INVALID_ARG;
+  auto al = [](const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15) == 0; };
+  if (!al(q) || !al(k) || !al(v) || !al(out) || (lse && (reinterpret_cast<uintptr_t>(lse) & 3)))
+    return LSERVE_ERR_INVALID_ARG;
+  if (d->head_dim != 64 && d->head_dim != 128) return LSERVE_ERR_UNSUPPORTED;
+  if (d->block_q != 64 && d->block_q != 128) return LSERVE_ERR_UNSUPPORTED;
+  if (d->num_q_heads > kMaxHeads || d->num_kv_heads > kMaxHeads) return LSERVE_ERR_UNSUPPORTED;
+  for (int h = 0; h < d->num_kv_heads; ++h)
+    if (head_kind_host[h] > 1) return LSERVE_ERR_INVALID_ARG;
+
+  PrefillParams p;
+  memset(&p, 0, sizeof(p));
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.lse = lse;
+  p.status = device_status_word();
+  if (!p.status) return LSERVE_ERR_CUDA;
+  p.wait_limit = wait_limit();
+  p.scale_log2 = softmax_scale * 1.4426950408889634f;
+  p.T = d->seq_len;
+  p.H_q = d->num_q_heads;
+  p.H_kv = d->num_kv_heads;
+  p.G = d->num_q_heads / d->num_kv_heads;
+  p.mask_block = d->block_q;
+  p.sink_blocks = d->sink_blocks;
+  p.local_blocks = d->local_blocks;
+  p.n_qt = (d->seq_len + kBM - 1) / kBM;
+  for (int h = 0; h < d->num_kv_heads; ++h) p.kv_kind[h] = head_kind_host[h];
+  for (int hq = 0; hq < d->num_q_heads; ++hq) {
+    if (head_kind_host[hq / p.G] == 0)
+      p.dense_heads[p.n_dense++] = (uint8_t)hq;
+    else
+      p.stream_heads[p.n_stream++] = (uint8_t)hq;
+  }
+  CUtensorMap qm, km, vm;
+  if (!make_map_3d(&qm, q, d->seq_len, d->num_q_heads, d->head_dim) ||
+      !make_map_3d(&km, k, d->seq_len, d->num_kv_heads, d->head_dim) ||
+      !make_map_3d(&vm, v, d->seq_len, d->num_kv_heads, d->head_dim))
+    return LSERVE_ERR_CUDA;
+  const int sms = current_sm_count();
+  if (sms <= 0) return LSERVE_ERR_CUDA;
+  const int tiles = d->num_q_heads * p.n_qt;
+  const int grid = tiles < sms ? tiles : sms;
+  cudaError_t e;
+  // more than half of the SM's shared memory: one CTA per SM, so the 512-column
+  // tensor-memory allocation never waits on a co-resident CTA
+  const int kOneCtaSmem = 118 * 1024;
+  if (d->head_dim == 128) {
+    const int smem = std::max(Layout<128>::kBytes + 1024, kOneCtaSmem);
+    e = set_smem_once((const void*)prefill_kernel<128>, smem);
+    if (e != cudaSuccess) return LSERVE_ERR_CUDA;
+    prefill_kernel<128><<<grid, kThreads, smem, stream>>>(p, qm, km, vm);
+  } else {
+    const int smem = std::max(Layout<64>::kBytes + 1024, kOneCtaSmem);
+    e = set_smem_once((const void*)prefill_kernel<64>, smem);
+    if (e != cudaSuccess) return LSERVE_ERR_CUDA;
+    prefill_kernel<64><<<grid, kThreads, smem, stream>>>(p, qm, km, vm);
+  }
+  return cudaGetLastError() == cudaSuccess ? LSERVE_OK : LSERVE_ERR_CUDA;
 }
 
 }  // namespace lserve
