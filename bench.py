@@ -267,6 +267,7 @@ def workload_config(w):
 # --- the CUDA path ----------------------------------------------------------------
 
 def main():
+    global LAYERS
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=DEFAULT_STEPS)
@@ -274,8 +275,12 @@ def main():
     ap.add_argument("--impl", default="lserve", choices=["lserve", "reference"])
     ap.add_argument("--no-prefill", action="store_true", help="skip the prefill stage")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--layers", type=int, default=LAYERS,
+                    help="layer replicas (fewer = a small case for profiling; < 32 may fit in L2)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
+    LAYERS = max(1, args.layers)
     if args.impl == "reference":
         return reference_arm(args)
 
@@ -405,16 +410,18 @@ def main():
             o_host[l].copy_(outs[l], non_blocking=True)
 
     e2e_steps = min(args.steps, 400)
-    with torch.cuda.stream(stream):
-        for t in range(args.warmup):
-            e2e_step(t)
-    t_e2e = timed(lambda: [e2e_step(t) for t in range(e2e_steps)])
-    t_e2e = max_over_ranks(t_e2e, ws, dev)
-    h2d = q_host.numel() * 2
-    d2h = o_host.numel() * 2
-    e2e = {"value": step_bytes * e2e_steps * ws / t_e2e / 1e9, "unit": "GB/s",
-           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-           "ms_per_step": t_e2e / e2e_steps * 1e3}
+    e2e = None
+    if not args.no_e2e:
+        with torch.cuda.stream(stream):
+            for t in range(args.warmup):
+                e2e_step(t)
+        t_e2e = timed(lambda: [e2e_step(t) for t in range(e2e_steps)])
+        t_e2e = max_over_ranks(t_e2e, ws, dev)
+        h2d = q_host.numel() * 2
+        d2h = o_host.numel() * 2
+        e2e = {"value": step_bytes * e2e_steps * ws / t_e2e / 1e9, "unit": "GB/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "ms_per_step": t_e2e / e2e_steps * 1e3}
 
     launches = args.steps * LAYERS * 2 + (-(-args.steps // REUSE)) * LAYERS * 2
     result = {

@@ -58,7 +58,7 @@ def library_path() -> str:
 
 def _load(path):
     if not os.path.exists(path):
-        raise ImportError(f"{path} not built: run `python -m block_sparse_attention_page_b200.build`")
+        raise ImportError(f"{path} not built: run `python block_sparse_attention_page_b200/build.py`")
     lib = ctypes.CDLL(path)
     vp, i32, sz, u64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t, ctypes.c_uint64
     P = ctypes.POINTER

@@ -1,6 +1,8 @@
 """Build liblserve.so in place (nvcc, sm_100a only).
 
-    python -m block_sparse_attention_page_b200.build [--force] [--verbose]
+    python block_sparse_attention_page_b200/build.py [--force] [--verbose]
+
+(run by path: importing the package loads the library this script builds)
 
 Objects go to block_sparse_attention_page_b200/_build/; the shared library is
 written next to this file so that it travels with the source tree.

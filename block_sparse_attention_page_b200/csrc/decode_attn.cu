@@ -391,8 +391,9 @@ decode_attn_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
 // whose tile ranges overlap the pair.  Lanes take one segment each (32 at a
 // time): the max and the weighted row sum are warp reductions, then every lane
 // accumulates its D/32 channels over the segments with independent loads.
+template <int D>
 __global__ void __launch_bounds__(128)
-decode_combine_kernel(const __grid_constant__ DecodeParams p, int G, int D) {
+decode_combine_kernel(const __grid_constant__ DecodeParams p, int G) {
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
   const int P = p.batch * p.num_kv_heads;
   if (warp >= P * G) return;
@@ -403,8 +404,10 @@ decode_combine_kernel(const __grid_constant__ DecodeParams p, int G, int D) {
   const int NW = p.num_warps;
   const float* po = p.partial;
   const float* pml = p.partial + (size_t)(NW + P) * G * D;
-  const int CPL = D / 32;
-  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  constexpr int CPL = D / 32;
+  float acc[CPL];
+#pragma unroll
+  for (int j = 0; j < CPL; ++j) acc[j] = 0.f;
   float M = -INFINITY, Lsum = 0.f;
   if (T1 > T0) {
     // first warp whose range holds tile T0: start(w) = floor(U*w/NW) <= T0 < start(w+1)
@@ -437,12 +440,24 @@ decode_combine_kernel(const __grid_constant__ DecodeParams p, int G, int D) {
       for (int j = 0; j < CPL; ++j) acc[j] *= rescale;
       M = Mn;
       const int nseg = (int)min(32ll, w1 - base + 1);
-#pragma unroll 4
-      for (int i = 0; i < nseg; ++i) {
+      const float* src0 = po + ((size_t)(base + pair) * G + g) * D + lane * CPL;
+      const size_t stride = (size_t)G * D;
+      // slots of empty-range warps were never written: their weight is 0 and the
+      // select below (not a multiply) keeps whatever they hold out of the sum
+#pragma unroll 8
+      for (int i = 0; i < 32; ++i) {
+        if (i >= nseg) break;
         const float wi = __shfl_sync(0xffffffffu, w_s, i);
-        if (wi == 0.f) continue;
-        const float* src = po + ((size_t)(base + i + pair) * G + g) * D + lane * CPL;
-        for (int j = 0; j < CPL; ++j) acc[j] = fmaf(wi, src[j], acc[j]);
+        float v[CPL];
+        if constexpr (CPL == 4) {
+          const float4 t4 = *reinterpret_cast<const float4*>(src0 + i * stride);
+          v[0] = t4.x; v[1] = t4.y; v[2] = t4.z; v[3] = t4.w;
+        } else {
+          const float2 t2 = *reinterpret_cast<const float2*>(src0 + i * stride);
+          v[0] = t2.x; v[1] = t2.y;
+        }
+#pragma unroll
+        for (int j = 0; j < CPL; ++j) acc[j] = wi != 0.f ? fmaf(wi, v[j], acc[j]) : acc[j];
       }
     }
   }
@@ -514,7 +529,10 @@ cudaError_t launch_decode(const DecodeParams& p_in, const CUtensorMap& kmap, con
   if (e != cudaSuccess) return e;
   const int P = p.batch * p.num_kv_heads;
   const int warps = P * G;
-  decode_combine_kernel<<<(warps + 3) / 4, 128, 0, stream>>>(p, G, D);
+  if (D == 128)
+    decode_combine_kernel<128><<<(warps + 3) / 4, 128, 0, stream>>>(p, G);
+  else
+    decode_combine_kernel<64><<<(warps + 3) / 4, 128, 0, stream>>>(p, G);
   return cudaGetLastError();
 }
 
