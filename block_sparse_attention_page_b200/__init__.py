@@ -30,7 +30,7 @@ EXPORTED = [
     "lserve_page_stats", "lserve_page_select", "lserve_sparse_decode_attn",
     "lserve_blocksparse_prefill", "lserve_workspace_size", "lserve_read_device_status",
     "lserve_set_wait_limit_cycles", "lserve_debug_wait_timeout", "lserve_status_string",
-    "lserve_bounds_checked",
+    "lserve_bounds_checked", "lserve_page_select_noalloc",
 ]
 
 
@@ -68,6 +68,8 @@ def _load(path):
                                               i32, ctypes.c_float, vp, vp, vp, sz, vp]
     lib.lserve_blocksparse_prefill.argtypes = [P(PrefillDesc), vp, vp, vp, vp, ctypes.c_float, vp, vp,
                                                vp, sz, vp]
+    lib.lserve_page_select_noalloc.argtypes = [P(PagedDesc), vp, vp, vp, vp, vp, i32, vp, vp, vp]
+    lib.lserve_page_select_noalloc.restype = ctypes.c_int
     lib.lserve_workspace_size.argtypes = [ctypes.c_int, vp, i32]
     lib.lserve_workspace_size.restype = sz
     lib.lserve_read_device_status.argtypes = [vp]
@@ -130,6 +132,15 @@ def page_select(desc, q, stats_pool, block_table, ctx_lens, head_kind, top_k, se
         ctypes.byref(desc), _ptr(q), _ptr(stats_pool), _ptr(block_table), _ptr(ctx_lens),
         _ptr(head_kind), top_k, _ptr(sel), _ptr(sel_count), _ptr(phys_scores), _ptr(workspace),
         ws_bytes, _stream(stream)))
+
+
+def page_select_noalloc(desc, q, stats_pool, block_table, ctx_lens, head_kind, top_k, sel, sel_count,
+                        stream=None):
+    """lserve_page_select with the scores kept in the library's static device
+    array instead of a caller workspace (for callers that cannot allocate)."""
+    _check("lserve_page_select_noalloc", lib.lserve_page_select_noalloc(
+        ctypes.byref(desc), _ptr(q), _ptr(stats_pool), _ptr(block_table), _ptr(ctx_lens),
+        _ptr(head_kind), top_k, _ptr(sel), _ptr(sel_count), _stream(stream)))
 
 
 def sparse_decode_attn(desc, q, k_pool, v_pool, block_table, ctx_lens, head_kind, sel, sel_count,

@@ -177,6 +177,29 @@ int lserve_blocksparse_prefill(const lserve_prefill_desc* desc, const void* q, c
                                void* out, float* lse, void* workspace, size_t workspace_bytes,
                                void* stream);
 
+/*
+ * lserve_page_select_noalloc -- lserve_page_select for callers that cannot
+ * allocate device memory.  (The LServe pages have no counterpart: this is a
+ * deployment convenience of this library.)
+ *
+ * Same arguments and results as lserve_page_select without phys_scores and
+ * workspace.  The physical-page scores go to a fixed 4 MiB array inside the
+ * library's device memory, so no cudaMalloc is needed -- useful where the
+ * caller runs inside a host callback or a plug-in whose host process owns all
+ * allocations.  Limits and caveats:
+ *   - B * H_kv * max_pages_per_seq must be <= 1,048,576, else
+ *     LSERVE_ERR_UNSUPPORTED is returned and nothing is launched;
+ *   - each GPU that loads the library holds the array until the process exits;
+ *   - every call on a device shares the array (the previous call's scores stay
+ *     there and are overwritten): calls that overlap on the GPU race;
+ *   - the first call on each device looks up the array's device address with
+ *     that device current; make that first call before any stream capture.
+ */
+int lserve_page_select_noalloc(const lserve_paged_desc* desc, const void* q, const void* stats_pool,
+                               const int32_t* block_table, const int32_t* ctx_lens,
+                               const uint8_t* head_kind, int32_t top_k, int32_t* sel,
+                               int32_t* sel_count, void* stream);
+
 /* Bytes of workspace `op` needs for these shapes on the CURRENT device
  * (desc points to lserve_paged_desc, or lserve_prefill_desc for PREFILL).
  * Returns 0 for invalid shapes. */
