@@ -175,5 +175,6 @@ def debug_wait_timeout(cycles: int, stream=None):
 
 
 def alloc_workspace(nbytes: int, device="cuda") -> torch.Tensor:
-    """Caller-owned workspace (256-byte aligned by the caching allocator)."""
-    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+    """Caller-owned workspace: 256-byte aligned (caching allocator) and
+    zero-filled, as lserve_sparse_decode_attn requires before its first use."""
+    return torch.zeros(max(int(nbytes), 256), dtype=torch.uint8, device=device)

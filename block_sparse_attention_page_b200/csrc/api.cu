@@ -154,7 +154,9 @@ int supported_paged(const lserve_paged_desc* d) {
   if (G != 1 && G != 2 && G != 4 && G != 8) return LSERVE_ERR_UNSUPPORTED;
   if (d->logical_page != 8 && d->logical_page != 16 && d->logical_page != 32 && d->logical_page != 64)
     return LSERVE_ERR_UNSUPPORTED;
-  if (d->physical_page % kDecodeTile || d->physical_page > 1024) return LSERVE_ERR_UNSUPPORTED;
+  // tiles of min(N_P, 64) tokens: N_P = 32, or a multiple of 64 up to 1024
+  if (!(d->physical_page == 32 || (d->physical_page % 64 == 0 && d->physical_page <= 1024)))
+    return LSERVE_ERR_UNSUPPORTED;
   const long long rows = (long long)d->num_pool_pages * d->num_kv_heads * d->physical_page;
   if (rows >= (1ll << 31)) return LSERVE_ERR_UNSUPPORTED;
   return LSERVE_OK;
@@ -168,10 +170,7 @@ size_t decode_ws(const lserve_paged_desc* d) {
   const int sms = current_sm_count();
   if (sms <= 0) return 0;
   const int G = d->num_q_heads / d->num_kv_heads;
-  const int wpc = decode_warps_per_cta(d->head_dim, G);
-  if (wpc <= 0) return 0;
-  return decode_workspace_bytes(d->batch * d->num_kv_heads, decode_num_ctas(sms) * wpc, G,
-                                d->head_dim);
+  return decode_workspace_bytes(d->batch * d->num_kv_heads, decode_grid(sms), G, d->head_dim);
 }
 
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? LSERVE_OK : LSERVE_ERR_CUDA; }
@@ -337,12 +336,15 @@ int lserve_sparse_decode_attn(const lserve_paged_desc* desc, const void* q, cons
   if (need == 0) return LSERVE_ERR_CUDA;
   if (!workspace || workspace_bytes < need || !aligned(workspace, 256)) return LSERVE_ERR_WORKSPACE;
   const int D = desc->head_dim, G = desc->num_q_heads / desc->num_kv_heads;
+  const int P = desc->batch * desc->num_kv_heads;
+  if (P > kDecodeMaxPairs) return LSERVE_ERR_UNSUPPORTED;
+  const int tile_rows = desc->physical_page < kDecodeTileMax ? desc->physical_page : kDecodeTileMax;
   const uint64_t rows = (uint64_t)desc->num_pool_pages * desc->num_kv_heads * desc->physical_page;
   CUtensorMap kmap, vmap;
-  if (!make_map_2d(&kmap, k_pool, rows, D, D, kDecodeTile) ||
-      !make_map_2d(&vmap, v_pool, rows, D, D, kDecodeTile))
+  if (!make_map_2d(&kmap, k_pool, rows, D, D, tile_rows) ||
+      !make_map_2d(&vmap, v_pool, rows, D, D, tile_rows))
     return LSERVE_ERR_CUDA;
-  const int P = desc->batch * desc->num_kv_heads;
+  const int grid = decode_grid(current_sm_count());
   DecodeParams p;
   p.q = static_cast<const __nv_bfloat16*>(q);
   p.block_table = block_table;
@@ -352,9 +354,13 @@ int lserve_sparse_decode_attn(const lserve_paged_desc* desc, const void* q, cons
   p.sel_count = sel_count;
   p.out = static_cast<__nv_bfloat16*>(out);
   p.lse = lse;
-  p.pair_tiles = static_cast<int32_t*>(workspace);
-  p.partial = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
-                                       ((size_t)(P + 1) * 4 + 255) / 256 * 256);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const size_t cnt_bytes = ((size_t)(P + 1) * 4 + 255) / 256 * 256;
+  const size_t slots = (size_t)grid + P;
+  const size_t o_bytes = (slots * G * D * 4 + 255) / 256 * 256;
+  p.counters = reinterpret_cast<uint32_t*>(ws);
+  p.part_o = reinterpret_cast<float*>(ws + cnt_bytes);
+  p.part_ml = reinterpret_cast<float*>(ws + cnt_bytes + o_bytes);
   p.batch = desc->batch;
   p.num_q_heads = desc->num_q_heads;
   p.num_kv_heads = desc->num_kv_heads;
@@ -364,14 +370,13 @@ int lserve_sparse_decode_attn(const lserve_paged_desc* desc, const void* q, cons
   p.top_k = top_k;
   p.sink = sink_tokens;
   p.local = local_tokens;
-  p.tiles_per_page = desc->physical_page / kDecodeTile;
-  p.num_warps = 0;  // set by launch_decode
+  p.tile_rows = tile_rows;
+  p.tiles_per_page = desc->physical_page / tile_rows;
   p.scale_log2 = softmax_scale * 1.4426950408889634f;
   p.wait_limit = wait_limit();
   p.status = device_status_word();
   if (!p.status) return LSERVE_ERR_CUDA;
-  return cuda_status(
-      launch_decode(p, kmap, vmap, D, G, decode_num_ctas(current_sm_count()), static_cast<cudaStream_t>(stream)));
+  return cuda_status(launch_decode(p, kmap, vmap, D, G, grid, static_cast<cudaStream_t>(stream)));
 }
 
 int lserve_blocksparse_prefill(const lserve_prefill_desc* desc, const void* q, const void* k,

@@ -39,11 +39,11 @@ struct SelectParams {
   int top_k;
 };
 
-// Decode split: the tiles of all (sequence, KV head) pairs are laid end to end
-// and cut into equal ranges, one per consumer warp of a persistent grid.
-constexpr int kDecodeTile = 32;       // tokens per tile
-constexpr int kDecodeWarps = 6;       // consumer warps per CTA
-constexpr int kDecodeStages = 2;      // tiles in flight per warp
+// Decode split: tiles of up to 64 tokens (a physical page, or a 64-token part of
+// a larger one); the tiles of all (sequence, KV head) pairs are laid end to end
+// and cut into equal contiguous ranges, one per CTA of a persistent grid.
+constexpr int kDecodeTileMax = 64;
+constexpr int kDecodeMaxPairs = 2048;   // B * H_kv
 
 struct DecodeParams {
   const __nv_bfloat16* q;
@@ -54,13 +54,14 @@ struct DecodeParams {
   const int32_t* sel_count;
   __nv_bfloat16* out;
   float* lse;
-  int32_t* pair_tiles;    // workspace [P + 1]: exclusive prefix of tiles per pair
-  float* partial;         // workspace: o [(num_warps + P)][G][D], then (m, l) [..][G][2]
+  uint32_t* counters;     // workspace [P]: segments finished per pair; zero between calls
+  float* part_o;          // workspace [(grid + P)][G][D]: unnormalised partial outputs
+  float* part_ml;         // workspace [(grid + P)][G][2]: (running max, row sum) per partial
   unsigned int* status;
   int batch, num_q_heads, num_kv_heads, physical_page, max_pages, num_pool_pages;
   int top_k, sink, local;
+  int tile_rows;          // tokens per tile: min(N_P, 64)
   int tiles_per_page;
-  int num_warps;          // consumer warps in the whole grid
   float scale_log2;       // softmax_scale * log2(e)
   uint64_t wait_limit;
 };
@@ -69,11 +70,9 @@ cudaError_t launch_page_stats(const StatsParams& p, int D, int max_logical_pages
                               cudaStream_t stream);
 cudaError_t launch_page_select(const SelectParams& p, int D, cudaStream_t stream);
 cudaError_t launch_decode(const DecodeParams& p, const CUtensorMap& kmap, const CUtensorMap& vmap,
-                          int D, int G, int num_ctas, cudaStream_t stream);
-size_t decode_workspace_bytes(int pairs, int num_warps, int G, int D);
-int decode_num_ctas(int sm_count);
-size_t decode_smem_bytes(int D, int G);
-int decode_warps_per_cta(int D, int G);
+                          int D, int G, int grid, cudaStream_t stream);
+size_t decode_workspace_bytes(int pairs, int grid, int G, int D);
+int decode_grid(int sm_count);
 
 cudaError_t launch_wait_timeout_probe(uint64_t cycles, unsigned int* status, cudaStream_t stream);
 

@@ -70,7 +70,7 @@ typedef struct {
   int32_t num_kv_heads;      /* H_kv >= 1; G = H_q / H_kv in {1, 2, 4, 8}           */
   int32_t head_dim;          /* D in {64, 128}                                      */
   int32_t logical_page;      /* N_L in {8, 16, 32, 64}                              */
-  int32_t physical_page;     /* N_P = g * N_L, g >= 1; N_P in {32, 64, 128, 256}    */
+  int32_t physical_page;     /* N_P = g * N_L; 32 or a multiple of 64, <= 1024      */
   int32_t max_pages_per_seq; /* row length of block_table                           */
   int32_t num_pool_pages;    /* first dimension of k_pool / v_pool / stats_pool     */
 } lserve_paged_desc;
@@ -146,7 +146,12 @@ int lserve_page_select(const lserve_paged_desc* desc, const void* q, const void*
  *   out  bf16 [B][H_q][D]
  *   lse  float [B][H_q] natural-log sum of exp(scale * q.k), or NULL.
  * A head with no token to attend (n_b = 0) gets out = 0, lse = -inf.
- * workspace: lserve_workspace_size(LSERVE_OP_DECODE, desc, top_k) bytes.
+ * workspace: lserve_workspace_size(LSERVE_OP_DECODE, desc, top_k) bytes,
+ * 256-byte aligned and ZERO-FILLED before its first use: besides the split
+ * partials it holds per-pair completion counters, which every successful call
+ * leaves at zero again (after an error, zero it again).  Calls that may run
+ * concurrently need separate workspaces.
+ * Limits: B * H_kv <= 2048; N_P = 32 or a multiple of 64.
  */
 int lserve_sparse_decode_attn(const lserve_paged_desc* desc, const void* q, const void* k_pool,
                               const void* v_pool, const int32_t* block_table, const int32_t* ctx_lens,
