@@ -340,9 +340,10 @@ int lserve_sparse_decode_attn(const lserve_paged_desc* desc, const void* q, cons
   if (P > kDecodeMaxPairs) return LSERVE_ERR_UNSUPPORTED;
   const int tile_rows = desc->physical_page < kDecodeTileMax ? desc->physical_page : kDecodeTileMax;
   const uint64_t rows = (uint64_t)desc->num_pool_pages * desc->num_kv_heads * desc->physical_page;
+  // [rows][D/64][64] view: a tile of tile_rows x D is one contiguous TMA copy
   CUtensorMap kmap, vmap;
-  if (!make_map_2d(&kmap, k_pool, rows, D, D, tile_rows) ||
-      !make_map_2d(&vmap, v_pool, rows, D, D, tile_rows))
+  if (!make_map_tiled(&kmap, k_pool, 3, 64, D / 64, rows, 64, D / 64, tile_rows) ||
+      !make_map_tiled(&vmap, v_pool, 3, 64, D / 64, rows, 64, D / 64, tile_rows))
     return LSERVE_ERR_CUDA;
   const int grid = decode_grid(current_sm_count());
   DecodeParams p;

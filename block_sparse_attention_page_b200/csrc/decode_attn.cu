@@ -246,11 +246,9 @@ decode_attn_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
     info[s] = make_int2(t.x, t.z);
     const int b = t.x / p.num_kv_heads, h = t.x - b * p.num_kv_heads;
     mbar_arrive_expect_tx(&full[s], 2 * TR * D * 2 + L::kStageQ);
-#pragma unroll
-    for (int bx = 0; bx < NBOX; ++bx) {
-      tma_load_2d(st + bx * TR * 128, &kmap, bx * 64, t.y, &full[s]);
-      tma_load_2d(st + L::kTileK + bx * TR * 128, &vmap, bx * 64, t.y, &full[s]);
-    }
+    // one contiguous TR x D tile each: 3-D view (64 channels, D/64 halves, rows)
+    tma_load_3d(st, &kmap, 0, 0, t.y, &full[s]);
+    tma_load_3d(st + L::kTileK, &vmap, 0, 0, t.y, &full[s]);
     bulk_load_1d(st + 2 * L::kTileK, p.q + ((size_t)b * p.num_q_heads + (size_t)h * G) * D,
                  L::kStageQ, &full[s]);
   };
@@ -271,16 +269,17 @@ decode_attn_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
   const int pv_t0 = warp * tpw + half * pv_n;
   // byte offsets inside a stage, fixed for the lane: its key chunks, and the
   // value words of its tokens
+  // (a token row is NBOX consecutive 128-byte swizzle rows: row NBOX*t + half)
   uint32_t koff[CPT / 8];
 #pragma unroll
   for (int ch = 0; ch < CPT / 8; ++ch) {
     const int c = (lane % LPT) * (CPT / 8) + ch;
-    koff[ch] = (c / 8) * TR * 128 + sw128_offset(warp * tpw + lane / LPT, c % 8);
+    koff[ch] = sw128_offset(NBOX * (warp * tpw + lane / LPT) + c / 8, c % 8);
   }
   uint32_t voff[pv_n];
 #pragma unroll
   for (int j = 0; j < pv_n; ++j)
-    voff[j] = L::kTileK + pv_box * TR * 128 + pv_byte + sw128_offset(pv_t0 + j, pv_cc);
+    voff[j] = L::kTileK + pv_byte + sw128_offset(NBOX * (pv_t0 + j) + pv_box, pv_cc);
   float2* ps = ps_all + warp * 2 * TPW_MAX * G;  // [tile 0/1][token][head]
   int cur_pair = -1;
   float m_w[G], l_part[NHB];
