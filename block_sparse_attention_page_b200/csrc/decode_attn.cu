@@ -9,26 +9,30 @@
 // SM).  Every SM therefore streams the same number of KV bytes, however unequal
 // the pairs are (64 selected pages next to ~10 sink + local pages).
 //
-// Per CTA: 16 warps (four per SM sub-partition to hide latency).  Every warp
-// owns 1/16 of each tile's tokens and keeps its own online-softmax state, so a
-// tile needs no CTA-wide barrier: warps run ahead of one another and overlap
-// their phases.
-//   feeding : all threads resolve up to 256 tiles at once (pair, page ordinal,
-//             block-table lookup); each stage of an S-deep ring is refilled by
-//             the last warp to finish with it -- K and V by TMA (128-byte
-//             swizzle), the pair's q by a 1-D bulk copy.
-//   QK      : 8 lanes per token, each an eighth of D with q of the heads in
-//             registers (from the stage's bf16 q); packed FFMA2; three shuffles
-//             join the eighths.
-//   softmax : base-2 online softmax in fp32 per warp (warp-uniform running max
-//             per head, row sums per lane).
-//   PV      : lane = channel quad, over the warp's tokens; o of all G heads in
-//             registers across tiles.
-// At a pair boundary the warps' states are merged in shared memory.  A pair
-// covered by one CTA is finalised there; otherwise each CTA writes an
-// unnormalised (o, m, l) partial and the last CTA to finish the pair (per-pair
-// counter in the workspace) merges the partials with log-sum-exp weights and
-// resets the counter to zero.
+// Per CTA: one producer warp and kConsumerWarps consumer warps.
+//   producer : its lanes resolve 32 tiles at a time (pair, page ordinal,
+//              block-table lookup); then, stage by stage of an S-deep ring, it
+//              waits until every consumer warp has released the stage and
+//              refills it -- K and V by TMA (128-byte swizzle), the pair's q by
+//              a 1-D bulk copy.
+//   consumers: every warp owns 1/kConsumerWarps of each tile's tokens and keeps
+//              its own online-softmax state, so a tile needs no CTA-wide
+//              barrier.  An iteration takes one tile, or two consecutive tiles
+//              of the same pair.
+//     QK     : 8 lanes per token, each an eighth of D with q in registers;
+//              packed FFMA2; the G x rows partial dots of a lane are joined by
+//              a reduce-scatter over the 8 lanes, so that afterwards every lane
+//              holds whole dots of ONE head.
+//     softmax: base-2 online softmax in fp32; running max per head shared by
+//              the warp, one exp2 per head and lane for the rescale.
+//     PV     : lane = channel quad, over the warp's tokens; o of all G heads in
+//              registers across tiles, rescaled only when a running max grew.
+// Pair boundaries come from the tile plan in shared memory, so all consumer
+// warps agree on them whatever the data.  At a boundary the warps' states are
+// merged in shared memory.  A pair covered by one CTA is finalised there;
+// otherwise each CTA writes an unnormalised (o, m, l) partial and the last CTA
+// to finish the pair (per-pair counter in the workspace) merges the partials
+// with log-sum-exp weights and resets the counter to zero.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -36,19 +40,22 @@ namespace lserve {
 
 namespace {
 
-constexpr int kWarps = 16;
-constexpr int kMergeWarps = 8;        // warps whose state fits the merge buffer at once
-constexpr int kThreads = kWarps * 32;
-constexpr int kTable = 256;            // tile descriptor slots
-constexpr int kRound = kTable - 8;     // descriptors resolved per round (8 slots of slack)
+constexpr int kConsumerWarps = 8;
+constexpr int kThreads = (kConsumerWarps + 1) * 32;  // + the producer warp
+constexpr int kConsumerThreads = kConsumerWarps * 32;
+constexpr int kBarConsumers = 1;       // named barrier of the consumer warps
+constexpr int kMaxGrid = 512;          // CTAs whose range starts the range table holds
+constexpr unsigned kFull = 0xffffffffu;
 
 // Pages the pair attends (retrieval: the selection; streaming: sink + local).
 __device__ __forceinline__ int pair_pages(const DecodeParams& p, int pair) {
   const int b = pair / p.num_kv_heads, h = pair - b * p.num_kv_heads;
   const int n = p.ctx_lens[b];
+  const int kind = p.head_kind[h];
+  const int nsel = p.sel_count[pair];  // loaded whatever the kind: one round trip
   const int NP = p.physical_page;
   const int npages = (n + NP - 1) / NP;
-  if (p.head_kind[h] == 0) return min(max(p.sel_count[pair], 0), min(p.top_k, npages));
+  if (kind == 0) return min(max(nsel, 0), min(p.top_k, npages));
   const int ns = min((p.sink + NP - 1) / NP, npages);
   const int ls = max(max(0, n - p.local) / NP, ns);
   return ns + max(0, npages - ls);
@@ -59,12 +66,13 @@ struct DecLayout {
   static constexpr int kTileK = kDecodeTileMax * D * 2;                  // K (or V) tile bytes
   static constexpr int kStageQ = G * D * 2;
   static constexpr int kStage = (2 * kTileK + kStageQ + 1023) / 1024 * 1024;
-  static constexpr int kPs = kWarps * 2 * (kDecodeTileMax / kWarps) * G * 8;  // two tiles
-  static constexpr int kOw = kMergeWarps * G * D * 4;
-  static constexpr int kMl = kMergeWarps * G * 2 * 4;
-  static constexpr int kOff = (kDecodeMaxPairs + 1) * 4;
-  static constexpr int kTab = kTable * 16;
-  static constexpr int kFixed = kPs + kOw + kMl + kOff + kTab + 512;
+  static constexpr int kPs = 2 * kDecodeTileMax * G * 8;                 // p of two tiles
+  static constexpr int kOw = kConsumerWarps * G * D * 4;                 // o per warp
+  static constexpr int kMl = kConsumerWarps * G * 2 * 4;                 // (m, l) per warp
+  static constexpr int kSc = (kConsumerWarps + 1) * G * 4;               // merge weights + max
+  static constexpr int kOff = ((kDecodeMaxPairs + 1) * 4 + 15) / 16 * 16;
+  static constexpr int kCst = ((kMaxGrid + 1) * 4 + 15) / 16 * 16;
+  static constexpr int kFixed = kPs + kOw + kMl + kSc + kOff + kCst + 1024;
   static constexpr int kBudget = 227 * 1024 - 1024;
   static constexpr int kStagesFit = (kBudget - kFixed) / kStage;
   static constexpr int kStages = kStagesFit > 8 ? 8 : kStagesFit;
@@ -72,25 +80,46 @@ struct DecLayout {
   static constexpr int oPs = kStages * kStage;
   static constexpr int oOw = oPs + kPs;
   static constexpr int oMl = oOw + kOw;
-  static constexpr int oOff = oMl + kMl;
-  static constexpr int oTab = (oOff + kOff + 15) / 16 * 16;
-  static constexpr int oInfo = oTab + kTab;
-  static constexpr int oBar = oInfo + kStages * 8;
-  static constexpr int oCnt = oBar + kStages * 8;
-  static constexpr int oMisc = oCnt + kStages * 4;
+  static constexpr int oSc = oMl + kMl;
+  static constexpr int oOff = (oSc + kSc + 15) / 16 * 16;
+  static constexpr int oCst = oOff + kOff;
+  static constexpr int oInfo = oCst + kCst;
+  static constexpr int oFull = (oInfo + kStages * 4 + 7) / 8 * 8;
+  static constexpr int oEmpty = oFull + kStages * 8;
+  static constexpr int oMisc = (oEmpty + kStages * 8 + 15) / 16 * 16;
   static constexpr int kBytes = oMisc + 128;
   static_assert(kStages >= 2, "decode ring needs two stages");
+  static_assert(oPs % 16 == 0 && oOw % 16 == 0 && oMl % 16 == 0 && oSc % 16 == 0 &&
+                    oOff % 16 == 0 && oCst % 16 == 0 && oInfo % 4 == 0 && oFull % 8 == 0 &&
+                    oEmpty % 8 == 0 && oMisc % 16 == 0,
+                "decode shared-memory arrays must keep their alignment");
   static_assert(kBytes <= kBudget, "decode shared memory over budget");
 };
 
-// CTA whose range holds tile u: largest c with floor(U*c/NC) <= u.
-__device__ __forceinline__ int cta_of(long long u, long long U, int NC) {
-  return (int)(((u + 1) * NC + U - 1) / U) - 1;
+// cst[c] = floor(U * c / NC) is the first tile of CTA c's range (cst[NC] = U).
+// CTA whose range holds tile u: the largest c < NC with cst[c] <= u (ranges
+// can be empty when U < NC; the largest such c is the one that owns u).
+__device__ __forceinline__ int cta_of(const int* cst, int u, int NC) {
+  int lo = 0, hi = NC - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (cst[mid] <= u) lo = mid; else hi = mid - 1;
+  }
+  return lo;
 }
 
-// CTA c has at least one tile (when U < NC some ranges are empty)
-__device__ __forceinline__ bool cta_busy(int c, long long U, int NC) {
-  return U * (c + 1) / NC > U * c / NC;
+// CTA c has at least one tile
+__device__ __forceinline__ bool cta_busy(const int* cst, int c) { return cst[c + 1] > cst[c]; }
+
+// Pair that tile u belongs to: the last pair with off[pair] <= u (pairs without
+// tiles share their offset with the next pair and are skipped).
+__device__ __forceinline__ int pair_of(const int* off, int u, int P) {
+  int lo = 0, hi = P - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (off[mid] <= u) lo = mid; else hi = mid - 1;
+  }
+  return lo;
 }
 
 // Bounded wait that gives up at once when another warp already timed out.
@@ -109,6 +138,56 @@ __device__ __forceinline__ bool stage_wait(uint64_t* bar, uint32_t parity, uint6
   return true;
 }
 
+// ---- QK join: a lane's V = G * R partial dots (index v = g * R + r, r the
+// row of 4 tokens) are summed over the 8 lanes of its token by halving the
+// list at lane strides 4, 2, 1: the lane keeps one half and sends the other.
+// A step whose half would be empty sums the single value instead.
+// first index a lane holds after the join, for lane bits (qtr) of the token
+__host__ __device__ constexpr int join_base(int V, int qtr) {
+  return ((qtr & 4) && V >= 2 ? V / 2 : 0) + ((qtr & 2) && V >= 4 ? V / 4 : 0) +
+         ((qtr & 1) && V >= 8 ? V / 8 : 0);
+}
+// the step at this lane stride split the list inside one head's R rows: the
+// two lanes hold different rows of the same head (a step that did not split
+// leaves both lanes with the same values)
+__host__ __device__ constexpr bool row_bit(int V, int R, int stride) {
+  return (V * stride / 8) >= 1 && (V * stride / 8) < R;
+}
+// lane (of the 8) that holds head g's first row after the join
+__host__ __device__ constexpr int head_src(int V, int R, int g) {
+  int src = 0;
+  for (int q = 7; q >= 0; --q)
+    if (join_base(V, q) == g * R) src = q;
+  return src;
+}
+
+template <int N, int STRIDE>
+__device__ __forceinline__ void join_step(const float (&in)[N], float (&out)[N >= 2 ? N / 2 : 1],
+                                          bool up) {
+  if constexpr (N >= 2) {
+#pragma unroll
+    for (int i = 0; i < N / 2; ++i) {
+      const float send = up ? in[i] : in[i + N / 2];
+      const float keep = up ? in[i + N / 2] : in[i];
+      out[i] = keep + __shfl_xor_sync(kFull, send, STRIDE);
+    }
+  } else {
+    out[0] = in[0] + __shfl_xor_sync(kFull, in[0], STRIDE);
+  }
+}
+
+template <int V>
+constexpr int join_out() { return V >= 8 ? V / 8 : 1; }
+
+template <int V>
+__device__ __forceinline__ void join_dots(const float (&d)[V], float (&out)[join_out<V>()], int qtr) {
+  constexpr int N1 = V >= 2 ? V / 2 : 1, N2 = N1 >= 2 ? N1 / 2 : 1;
+  float a[N1], b[N2];
+  join_step<V, 4>(d, a, (qtr & 4) != 0);
+  join_step<N1, 2>(a, b, (qtr & 2) != 0);
+  join_step<N2, 1>(b, out, (qtr & 1) != 0);
+}
+
 }  // namespace
 
 template <int D, int G, int TR>
@@ -116,28 +195,40 @@ __global__ void __launch_bounds__(kThreads, 1)
 decode_attn_kernel(const __grid_constant__ DecodeParams p, const __grid_constant__ CUtensorMap kmap,
                    const __grid_constant__ CUtensorMap vmap) {
   using L = DecLayout<D, G>;
+  constexpr int W = kConsumerWarps;
   constexpr int S = L::kStages;
   constexpr int HB = G < 4 ? G : 4;      // heads whose q a QK lane holds at a time
   constexpr int NHB = G / HB;            // head blocks (2 for G = 8)
   constexpr int LPT = 8;                 // QK lanes per token
   constexpr int CPT = D / LPT;           // channels per QK lane (an eighth of D)
-  constexpr int NOUT = (G * D + kThreads - 1) / kThreads;  // merged outputs per thread
+  constexpr int KCH = CPT / 8;           // 16-byte key chunks per QK lane
+  constexpr int TPW = TR / W;            // tokens of a tile per consumer warp
+  constexpr int R = TPW / 4;             // QK rows (4 tokens each) per warp and tile
+  constexpr int V = G * R;               // partial dots per lane and tile
+  constexpr int C = join_out<V>();       // dots per lane after the join
   constexpr int NQ = D / 4;              // PV channel quads
   constexpr int LPQ = 32 / NQ;           // PV lane groups per warp (1 at D=128, 2 at D=64)
+  constexpr int PVN = TPW / LPQ;         // tokens per PV lane and tile
   constexpr int NBOX = D / 64;
-  constexpr int TPW_MAX = kDecodeTileMax / kWarps;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  float2* ps_all = reinterpret_cast<float2*>(smem + L::oPs);
-  float* ow = reinterpret_cast<float*>(smem + L::oOw);
-  float* mlw = reinterpret_cast<float*>(smem + L::oMl);
+  constexpr int NOUT = (G * D + kConsumerThreads - 1) / kConsumerThreads;
+  static_assert(TPW % 4 == 0 && R >= 1, "a warp takes whole rows of 4 tokens");
+  static_assert(C <= R && R % C == 0, "after the join a lane holds rows of one head");
+
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  // 1024-byte aligned base, kept as an offset into the shared array
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  float2* ps = reinterpret_cast<float2*>(smem + L::oPs);   // [tile 0/1][token][head] (p, p)
+  float* ow = reinterpret_cast<float*>(smem + L::oOw);     // [warp][head][D]
+  float2* mlw = reinterpret_cast<float2*>(smem + L::oMl);  // [warp][head] (m, l)
+  float* msc = reinterpret_cast<float*>(smem + L::oSc);    // [warp][head] weights, [head] max
   int* off = reinterpret_cast<int*>(smem + L::oOff);
-  int4* tab = reinterpret_cast<int4*>(smem + L::oTab);
-  int2* info = reinterpret_cast<int2*>(smem + L::oInfo);
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::oBar);
-  int* done_cnt = reinterpret_cast<int*>(smem + L::oCnt);
+  int* cst = reinterpret_cast<int*>(smem + L::oCst);
+  int* info = reinterpret_cast<int*>(smem + L::oInfo);     // valid tokens of the stage's tile
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::oFull);
+  uint64_t* empty = reinterpret_cast<uint64_t*>(smem + L::oEmpty);
   int* misc = reinterpret_cast<int*>(smem + L::oMisc);  // [0..15] scan, [16] last flag, [18] abort
   volatile int* abort_flag = misc + 18;
+  const uint8_t* zero16 = reinterpret_cast<const uint8_t*>(misc + 24);  // 16 zero bytes
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int P = p.batch * p.num_kv_heads;
@@ -148,9 +239,10 @@ decode_attn_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
   if (tid == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(&full[s], 1);
-      done_cnt[s] = 0;
+      mbar_init(&empty[s], W);
     }
     misc[18] = 0;
+    misc[24] = misc[25] = misc[26] = misc[27] = 0;
     fence_mbar_init();
   }
   if (tid == 32) {
@@ -171,7 +263,7 @@ decode_attn_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
     int incl = sum;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-      const int t = __shfl_up_sync(0xffffffffu, incl, o);
+      const int t = __shfl_up_sync(kFull, incl, o);
       if (lane >= o) incl += t;
     }
     if (lane == 31) misc[warp] = incl;
@@ -188,6 +280,7 @@ decode_attn_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
     __syncthreads();
   }
   const long long U = off[P];
+  for (int c = tid; c <= NC; c += kThreads) cst[c] = (int)(U * c / NC);
   const int u0 = (int)(U * cta / NC), u1 = (int)(U * (cta + 1) / NC);
   const int ntiles = u1 - u0;
 
@@ -203,102 +296,117 @@ decode_attn_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
       }
     }
   }
+  __syncthreads();  // range table, barrier init and plan visible to every warp
 
-  // ---- tile descriptors: (pair, first row in the [pool rows][D] view, valid tokens)
-  auto lookup = [&](int u) -> int4 {
-    int lo = 0, hi = P - 1;  // last pair with off[pair] <= u
-    while (lo < hi) {
-      const int mid = (lo + hi + 1) >> 1;
-      if (off[mid] <= u) lo = mid; else hi = mid - 1;
+  // =========================== producer warp ===============================
+  if (warp == W) {
+    // descriptor of tile u: (pair, first row in the [pool rows][D] view, valid tokens)
+    auto lookup = [&](int u, int& pair, int& row, int& valid) {
+      pair = pair_of(off, u, P);
+      const int local = u - off[pair];
+      const int li = local / tpp, sub = local - li * tpp;
+      const int b = pair / p.num_kv_heads, h = pair - b * p.num_kv_heads;
+      const int n = p.ctx_lens[b];
+      const int NP = p.physical_page;
+      const int npages = (n + NP - 1) / NP;
+      int m;
+      if (p.head_kind[h] == 0) {
+        m = p.sel[(size_t)pair * p.top_k + li];
+      } else {
+        const int ns = min((p.sink + NP - 1) / NP, npages);
+        const int ls = max(max(0, n - p.local) / NP, ns);
+        m = li < ns ? li : ls + (li - ns);
+      }
+      int pid = -1;
+      if (m >= 0 && m < npages && m < p.max_pages) pid = p.block_table[(size_t)b * p.max_pages + m];
+      if (pid < 0 || pid >= p.num_pool_pages) {  // bad selection or block-table entry: skip the page
+        raise_status(p.status, LSERVE_ERR_BOUNDS);
+        row = 0;
+        valid = 0;
+        return;
+      }
+      row = (int)(((long long)pid * p.num_kv_heads + h) * NP + sub * TR);
+      valid = max(0, min(TR, n - m * NP - sub * TR));
+    };
+    int issued = 0;
+    bool alive = true;
+    for (int kb = 0; kb < ntiles && alive; kb += 32) {
+      int tp = 0, trow = 0, tval = 0;
+      if (kb + lane < ntiles) lookup(u0 + kb + lane, tp, trow, tval);
+      const int nb = min(32, ntiles - kb);
+      for (int j = 0; j < nb; ++j) {
+        const int k = kb + j, s = k % S;
+        const int pr = __shfl_sync(kFull, tp, j);
+        const int row = __shfl_sync(kFull, trow, j);
+        const int val = __shfl_sync(kFull, tval, j);
+        int ok = 1;
+        if (lane == 0) {
+          if (k >= S) ok = stage_wait(&empty[s], ((k / S) - 1) & 1, lim, p.status, abort_flag);
+          if (ok && !*abort_flag) {
+            fence_proxy_async_smem();  // the consumers' reads of the stage come first
+            info[s] = val;
+            const int b = pr / p.num_kv_heads, h = pr - b * p.num_kv_heads;
+            uint8_t* st = smem + s * L::kStage;
+            mbar_arrive_expect_tx(&full[s], 2 * TR * D * 2 + L::kStageQ);
+            // one contiguous TR x D tile each: 3-D view (64 channels, D/64 halves, rows)
+            tma_load_3d(st, &kmap, 0, 0, row, &full[s]);
+            tma_load_3d(st + L::kTileK, &vmap, 0, 0, row, &full[s]);
+            bulk_load_1d(st + 2 * L::kTileK, p.q + ((size_t)b * p.num_q_heads + (size_t)h * G) * D,
+                         L::kStageQ, &full[s]);
+          } else {
+            ok = 0;
+          }
+        }
+        if (!__shfl_sync(kFull, ok, 0)) {
+          alive = false;
+          break;
+        }
+        ++issued;
+      }
     }
-    const int pair = lo;
-    const int local = u - off[pair];
-    const int li = local / tpp, sub = local - li * tpp;
-    const int b = pair / p.num_kv_heads, h = pair - b * p.num_kv_heads;
-    const int n = p.ctx_lens[b];
-    const int NP = p.physical_page;
-    const int npages = (n + NP - 1) / NP;
-    int m;
-    if (p.head_kind[h] == 0) {
-      m = p.sel[(size_t)pair * p.top_k + li];
-    } else {
-      const int ns = min((p.sink + NP - 1) / NP, npages);
-      const int ls = max(max(0, n - p.local) / NP, ns);
-      m = li < ns ? li : ls + (li - ns);
-    }
-    int pid = -1;
-    if (m >= 0 && m < npages && m < p.max_pages) pid = p.block_table[(size_t)b * p.max_pages + m];
-    if (pid < 0 || pid >= p.num_pool_pages) {  // bad selection or block-table entry: skip the page
-      raise_status(p.status, LSERVE_ERR_BOUNDS);
-      return make_int4(pair, 0, 0, 0);
-    }
-    return make_int4(pair, (int)(((long long)pid * p.num_kv_heads + h) * NP + sub * TR),
-                     max(0, min(TR, n - m * NP - sub * TR)), 0);
-  };
-  auto lookup_round = [&](int k0) {
-    for (int i = tid; i < kRound && k0 + i < ntiles; i += kThreads) tab[(k0 + i) % kTable] = lookup(u0 + k0 + i);
-  };
-  // one thread: load tile k into stage k % S
-  auto issue = [&](int k) {
-    const int4 t = tab[k % kTable];
-    const int s = k % S;
-    uint8_t* st = smem + s * L::kStage;
-    info[s] = make_int2(t.x, t.z);
-    const int b = t.x / p.num_kv_heads, h = t.x - b * p.num_kv_heads;
-    mbar_arrive_expect_tx(&full[s], 2 * TR * D * 2 + L::kStageQ);
-    // one contiguous TR x D tile each: 3-D view (64 channels, D/64 halves, rows)
-    tma_load_3d(st, &kmap, 0, 0, t.y, &full[s]);
-    tma_load_3d(st + L::kTileK, &vmap, 0, 0, t.y, &full[s]);
-    bulk_load_1d(st + 2 * L::kTileK, p.q + ((size_t)b * p.num_q_heads + (size_t)h * G) * D,
-                 L::kStageQ, &full[s]);
-  };
-  lookup_round(0);
-  __syncthreads();
-  if (warp == 0 && lane < S && lane < ntiles) issue(lane);
-
-  // ---- per-warp mapping and state
-  constexpr int tpw = TR / kWarps;             // tokens of each tile this warp owns
-  const int tok_l = lane / LPT, qtr = lane % LPT;  // QK: (token, eighth of D)
-  const int tok = warp * tpw + tok_l;
-  const bool qk_lane = tok_l < tpw;
-  const int quad = lane % NQ, half = lane / NQ;  // PV: channel quad (+ token half at D=64)
-  const int pv_chunk = (4 * quad) / 8;
-  const int pv_box = pv_chunk / 8, pv_cc = pv_chunk % 8;
-  const int pv_byte = (quad & 1) * 8;
-  constexpr int pv_n = tpw / LPQ;
-  const int pv_t0 = warp * tpw + half * pv_n;
-  // byte offsets inside a stage, fixed for the lane: its key chunks, and the
-  // value words of its tokens
-  // (a token row is NBOX consecutive 128-byte swizzle rows: row NBOX*t + half)
-  uint32_t koff[CPT / 8];
-#pragma unroll
-  for (int ch = 0; ch < CPT / 8; ++ch) {
-    const int c = (lane % LPT) * (CPT / 8) + ch;
-    koff[ch] = sw128_offset(NBOX * (warp * tpw + lane / LPT) + c / 8, c % 8);
+    // after a timeout: let the copies still in flight land before the CTA exits
+    if (!alive && lane == 0)
+      for (int k = max(0, issued - S); k < issued; ++k) mbar_wait(&full[k % S], (k / S) & 1, lim, p.status);
+    return;
   }
-  uint32_t voff[pv_n];
+
+  // =========================== consumer warps ==============================
+  const int tok_l = lane / LPT, qtr = lane % LPT;  // QK: (token of the row, eighth of D)
+  const int jb = join_base(V, qtr);
+  const int my_g = jb / R, my_r0 = jb % R;         // head and first row of the joined dots
+  const int quad = lane % NQ, half = lane / NQ;    // PV: channel quad (+ token half at D=64)
+  const int wt0 = warp * TPW;                      // first token of this warp in a tile
+  const int pv_t0 = wt0 + half * PVN;
+  // byte offsets inside a stage, fixed for the lane (a token row is NBOX
+  // consecutive 128-byte swizzle rows)
+  uint32_t koff[R][KCH];
 #pragma unroll
-  for (int j = 0; j < pv_n; ++j)
-    voff[j] = L::kTileK + pv_byte + sw128_offset(NBOX * (pv_t0 + j) + pv_box, pv_cc);
-  float2* ps = ps_all + warp * 2 * TPW_MAX * G;  // [tile 0/1][token][head]
-  int cur_pair = -1;
-  float m_w[G], l_part[NHB];
-  float2 o_acc[G][2];
+  for (int r = 0; r < R; ++r)
+#pragma unroll
+    for (int ch = 0; ch < KCH; ++ch) {
+      const int c = qtr * KCH + ch;  // 16-byte chunk of the key row
+      koff[r][ch] = sw128_offset(NBOX * (wt0 + 4 * r + tok_l) + c / 8, c % 8);
+    }
+  uint32_t voff[PVN];
+  {
+    const int chunk = (4 * quad) / 8;
+#pragma unroll
+    for (int j = 0; j < PVN; ++j)
+      voff[j] = L::kTileK + (quad & 1) * 8 + sw128_offset(NBOX * (pv_t0 + j) + chunk / 8, chunk % 8);
+  }
+
   float2 qreg[HB][CPT / 2];
+  float m_run = -INFINITY, l_run = 0.f;  // this lane's head: running max, partial row sum
+  float2 o_acc[G][2];
 #pragma unroll
-  for (int g = 0; g < G; ++g) {
-    m_w[g] = -INFINITY;
-    o_acc[g][0] = o_acc[g][1] = make_float2(0.f, 0.f);
-  }
-#pragma unroll
-  for (int i = 0; i < NHB; ++i) l_part[i] = 0.f;
+  for (int g = 0; g < G; ++g) o_acc[g][0] = o_acc[g][1] = make_float2(0.f, 0.f);
 
-  auto load_q = [&](const uint8_t* st, int hb) {  // bf16 q of the stage -> this lane's quarter
+  auto load_q = [&](const uint8_t* st, int hb) {  // bf16 q of the stage -> this lane's eighth
 #pragma unroll
     for (int h = 0; h < HB; ++h) {
       const uint4* src = reinterpret_cast<const uint4*>(st + 2 * L::kTileK + ((hb * HB + h) * D + qtr * CPT) * 2);
 #pragma unroll
-      for (int i = 0; i < CPT / 8; ++i) {
+      for (int i = 0; i < KCH; ++i) {
         const uint4 w = src[i];
         qreg[h][4 * i + 0] = bf16x2_to_float2(w.x);
         qreg[h][4 * i + 1] = bf16x2_to_float2(w.y);
@@ -308,110 +416,142 @@ decode_attn_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
     }
   };
 
-  // End of a pair segment (every warp arrives here at the same tile index):
-  // merge the warps, then finalise or publish + maybe merge across CTAs.
-  auto flush = [&](int pair) {
-    float lw[NHB];  // this warp's row sum per head h, held by lane 2h
+  // partial dots of tile st for the rows of this lane: d[g * R + r]
+  auto qk_tile = [&](const uint8_t* st, float (&d)[V], int hb) {
 #pragma unroll
-    for (int hb = 0; hb < NHB; ++hb) {
-      float lv = l_part[hb];
+    for (int r = 0; r < R; ++r) {
+      float2 acc[HB];
 #pragma unroll
-      for (int o = LPT; o < 32; o <<= 1) lv += __shfl_xor_sync(0xffffffffu, lv, o);
-      lw[hb] = lv;
+      for (int h = 0; h < HB; ++h) acc[h] = make_float2(0.f, 0.f);
+#pragma unroll
+      for (int ch = 0; ch < KCH; ++ch) {
+        const uint4 kw = *reinterpret_cast<const uint4*>(st + koff[r][ch]);
+        const float2 k0 = bf16x2_to_float2(kw.x), k1 = bf16x2_to_float2(kw.y);
+        const float2 k2 = bf16x2_to_float2(kw.z), k3 = bf16x2_to_float2(kw.w);
+#pragma unroll
+        for (int h = 0; h < HB; ++h) {
+          acc[h] = __ffma2_rn(qreg[h][4 * ch + 0], k0, acc[h]);
+          acc[h] = __ffma2_rn(qreg[h][4 * ch + 1], k1, acc[h]);
+          acc[h] = __ffma2_rn(qreg[h][4 * ch + 2], k2, acc[h]);
+          acc[h] = __ffma2_rn(qreg[h][4 * ch + 3], k3, acc[h]);
+        }
+      }
+#pragma unroll
+      for (int h = 0; h < HB; ++h) d[(hb * HB + h) * R + r] = acc[h].x + acc[h].y;
     }
+  };
+
+  // o += p v over this lane's tokens of tile st (tokens past `valid` read zeros)
+  auto pv_tile = [&](const uint8_t* st, int i, int valid) {
+#pragma unroll
+    for (int j = 0; j < PVN; ++j) {
+      const int t = pv_t0 + j;
+      const uint8_t* vp = t < valid ? st + voff[j] : zero16;
+      const uint2 vw = *reinterpret_cast<const uint2*>(vp);
+      const float2 v01 = bf16x2_to_float2(vw.x), v23 = bf16x2_to_float2(vw.y);
+      const float2* pt = ps + (i * kDecodeTileMax + t) * G;
+      if constexpr (G >= 2) {
+#pragma unroll
+        for (int g2 = 0; g2 < G / 2; ++g2) {
+          const float4 pq = reinterpret_cast<const float4*>(pt)[g2];
+          const float2 pa = make_float2(pq.x, pq.y), pb = make_float2(pq.z, pq.w);
+          o_acc[2 * g2][0] = __ffma2_rn(pa, v01, o_acc[2 * g2][0]);
+          o_acc[2 * g2][1] = __ffma2_rn(pa, v23, o_acc[2 * g2][1]);
+          o_acc[2 * g2 + 1][0] = __ffma2_rn(pb, v01, o_acc[2 * g2 + 1][0]);
+          o_acc[2 * g2 + 1][1] = __ffma2_rn(pb, v23, o_acc[2 * g2 + 1][1]);
+        }
+      } else {
+        const float2 pa = pt[0];
+        o_acc[0][0] = __ffma2_rn(pa, v01, o_acc[0][0]);
+        o_acc[0][1] = __ffma2_rn(pa, v23, o_acc[0][1]);
+      }
+    }
+  };
+
+  // End of a pair segment (every consumer warp arrives here at the same tile):
+  // merge the warps, then finalise, or publish a partial and maybe merge the
+  // pair's partials across CTAs.
+  auto flush = [&](int pair) {
+    float lw = l_run;  // row sum of this lane's head over the warp's tokens
+    if constexpr (row_bit(V, R, 4)) lw += __shfl_xor_sync(kFull, lw, 4);
+    if constexpr (row_bit(V, R, 2)) lw += __shfl_xor_sync(kFull, lw, 2);
+    if constexpr (row_bit(V, R, 1)) lw += __shfl_xor_sync(kFull, lw, 1);
+    lw += __shfl_xor_sync(kFull, lw, 8);
+    lw += __shfl_xor_sync(kFull, lw, 16);
     if constexpr (LPQ == 2) {
 #pragma unroll
-      for (int g = 0; g < G; ++g) {
+      for (int g = 0; g < G; ++g)
 #pragma unroll
         for (int j = 0; j < 2; ++j) {
-          o_acc[g][j].x += __shfl_xor_sync(0xffffffffu, o_acc[g][j].x, 16);
-          o_acc[g][j].y += __shfl_xor_sync(0xffffffffu, o_acc[g][j].y, 16);
+          o_acc[g][j].x += __shfl_xor_sync(kFull, o_acc[g][j].x, 16);
+          o_acc[g][j].y += __shfl_xor_sync(kFull, o_acc[g][j].y, 16);
         }
-      }
-    }
-    // merge the warps, kMergeWarps at a time, into per-thread (M, o, l) of the outputs
-    float Mo[NOUT], Oo[NOUT], Lo[NOUT];
-#pragma unroll
-    for (int i = 0; i < NOUT; ++i) {
-      Mo[i] = -INFINITY;
-      Oo[i] = 0.f;
-      Lo[i] = 0.f;
     }
 #pragma unroll
-    for (int r = 0; r < kWarps / kMergeWarps; ++r) {
-      const int wl = warp - r * kMergeWarps;
-      if (wl >= 0 && wl < kMergeWarps) {
+    for (int g = 0; g < G; ++g)
+      if (lane == head_src(V, R, g)) mlw[warp * G + g] = make_float2(m_run, lw);
+    if (lane < NQ) {
 #pragma unroll
-        for (int hb = 0; hb < NHB; ++hb)
-          if (lane < 2 * HB && (lane & 1) == 0) mlw[(wl * G + hb * HB + (lane >> 1)) * 2 + 1] = lw[hb];
-#pragma unroll
-        for (int g = 0; g < G; ++g)
-          if (lane == g) mlw[(wl * G + g) * 2] = m_w[g];
-        if (lane < NQ) {
-#pragma unroll
-          for (int g = 0; g < G; ++g)
-            *reinterpret_cast<float4*>(ow + (wl * G + g) * D + 4 * quad) =
-                make_float4(o_acc[g][0].x, o_acc[g][0].y, o_acc[g][1].x, o_acc[g][1].y);
-        }
-      }
-      __syncthreads();
-#pragma unroll
-      for (int i = 0; i < NOUT; ++i) {
-        const int j = tid + i * kThreads;
-        if (j < G * D) {
-          const int g = j / D, c = j - g * D;
-#pragma unroll
-          for (int w = 0; w < kMergeWarps; ++w) {
-            const float mw = mlw[(w * G + g) * 2];
-            if (mw == -INFINITY) continue;
-            const float Mn = fmaxf(Mo[i], mw);
-            const float sc = exp2f(Mo[i] - Mn), wt = exp2f(mw - Mn);
-            Oo[i] = Oo[i] * sc + wt * ow[(w * G + g) * D + c];
-            Lo[i] = Lo[i] * sc + wt * mlw[(w * G + g) * 2 + 1];
-            Mo[i] = Mn;
-          }
-        }
-      }
-      __syncthreads();
+      for (int g = 0; g < G; ++g)
+        *reinterpret_cast<float4*>(ow + (warp * G + g) * D + 4 * quad) =
+            make_float4(o_acc[g][0].x, o_acc[g][0].y, o_acc[g][1].x, o_acc[g][1].y);
     }
-    const bool live = !*abort_flag;
+    const bool live = named_sync_and(kBarConsumers, kConsumerThreads, !*abort_flag);
+    if (tid < W * G) {  // weight of warp w's state for head g: 2^(m_w - max over warps)
+      const int g = tid % G;
+      float M = -INFINITY;
+#pragma unroll
+      for (int w = 0; w < W; ++w) M = fmaxf(M, mlw[w * G + g].x);
+      const float mw = mlw[tid].x;
+      msc[tid] = mw == -INFINITY ? 0.f : fast_ex2(mw - M);
+      if (tid < G) msc[W * G + g] = M;
+    }
+    named_sync(kBarConsumers, kConsumerThreads);
     const int b = pair / p.num_kv_heads, h = pair - b * p.num_kv_heads;
-    const int c_first = cta_of(off[pair], U, NC), c_last = cta_of(off[pair + 1] - 1, U, NC);
+    const int c_first = cta_of(cst, off[pair], NC), c_last = cta_of(cst, off[pair + 1] - 1, NC);
     int nseg = 0;  // CTAs with tiles of this pair (CTAs without tiles write nothing)
-    for (int cc = c_first; cc <= c_last; ++cc) nseg += cta_busy(cc, U, NC) ? 1 : 0;
+    for (int cc = c_first; cc <= c_last; ++cc) nseg += cta_busy(cst, cc) ? 1 : 0;
     const size_t slot = (size_t)cta + pair;
 #pragma unroll
     for (int i = 0; i < NOUT; ++i) {
-      const int j = tid + i * kThreads;
+      const int j = tid + i * kConsumerThreads;
       if (j >= G * D || !live) continue;
       const int g = j / D, c = j - g * D;
+      float o = 0.f, l = 0.f;
+#pragma unroll
+      for (int w = 0; w < W; ++w) {
+        const float wt = msc[w * G + g];
+        o += wt * ow[(w * G + g) * D + c];
+        l += wt * mlw[w * G + g].y;
+      }
+      const float M = msc[W * G + g];
       const size_t qh = (size_t)b * p.num_q_heads + (size_t)h * G + g;
       if (nseg == 1) {
-        const bool empty_row = !(Lo[i] > 0.f);
-        p.out[qh * D + c] = __float2bfloat16_rn(empty_row ? 0.f : Oo[i] / Lo[i]);
+        const bool empty_row = !(l > 0.f);
+        p.out[qh * D + c] = __float2bfloat16_rn(empty_row ? 0.f : o / l);
         if (c == 0 && p.lse)
-          p.lse[qh] = empty_row ? -INFINITY : (Mo[i] + __log2f(Lo[i])) * 0.69314718055994530942f;
+          p.lse[qh] = empty_row ? -INFINITY : (M + __log2f(l)) * 0.69314718055994530942f;
       } else {
-        p.part_o[(slot * G + g) * D + c] = Oo[i];
-        if (c == 0) *reinterpret_cast<float2*>(p.part_ml + (slot * G + g) * 2) = make_float2(Mo[i], Lo[i]);
+        p.part_o[(slot * G + g) * D + c] = o;
+        if (c == 0) *reinterpret_cast<float2*>(p.part_ml + (slot * G + g) * 2) = make_float2(M, l);
       }
     }
     if (nseg > 1 && live) {
       __threadfence();
-      __syncthreads();
+      named_sync(kBarConsumers, kConsumerThreads);
       if (tid == 0) misc[16] = (atomicAdd(&p.counters[pair], 1u) == (unsigned)(nseg - 1)) ? 1 : 0;
-      __syncthreads();
+      named_sync(kBarConsumers, kConsumerThreads);
       if (misc[16]) {  // last segment to finish: merge every partial of the pair
         __threadfence();
 #pragma unroll
         for (int i = 0; i < NOUT; ++i) {
-          const int j = tid + i * kThreads;
+          const int j = tid + i * kConsumerThreads;
           if (j >= G * D) continue;
           const int g = j / D, c = j - g * D;
           float M = -INFINITY, o = 0.f, lsum = 0.f;
 #pragma unroll 4
           for (int cc = c_first; cc <= c_last; ++cc) {
-            const bool busy = cta_busy(cc, U, NC);  // predicated, independent loads
+            const bool busy = cta_busy(cst, cc);  // predicated, independent loads
             const size_t sl = (size_t)cc + pair;
             const float2 ml = busy ? *reinterpret_cast<const float2*>(p.part_ml + (sl * G + g) * 2)
                                    : make_float2(-INFINITY, 0.f);
@@ -432,199 +572,110 @@ decode_attn_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
         if (tid == 0) p.counters[pair] = 0u;
       }
     }
-    __syncthreads();  // ow / mlw / misc free again
+    named_sync(kBarConsumers, kConsumerThreads);  // ow / mlw / msc / misc free again
   };
 
   // Each iteration takes one tile, or two consecutive tiles of the same pair:
-  // one softmax update per 128 tokens and two independent token chains per lane.
-  int next_round = kRound;
+  // one softmax update per 2 * TPW tokens of the warp.
+  int cur = -1, pend = 0;  // current pair, and the local index of its first tile after it
+  bool need_q = false;
   for (int k = 0; k < ntiles;) {
-    if (k + S + 1 >= next_round && next_round < ntiles) {  // next round of tile descriptors
-      __syncthreads();
-      lookup_round(next_round);
-      __syncthreads();
-      next_round += kRound;
+    if (k >= pend) {  // first tile of a new pair (same decision in every consumer warp)
+      if (cur >= 0) flush(cur);
+      cur = pair_of(off, u0 + k, P);
+      pend = off[cur + 1] - u0;
+      m_run = -INFINITY;
+      l_run = 0.f;
+#pragma unroll
+      for (int g = 0; g < G; ++g) o_acc[g][0] = o_acc[g][1] = make_float2(0.f, 0.f);
+      need_q = true;
     }
+    const int nt = (k + 1 < ntiles && k + 1 < pend) ? 2 : 1;
     const int s0 = k % S, s1 = (k + 1) % S;
-    const bool has1 = k + 1 < ntiles;
-    bool arrived = stage_wait(&full[s0], (k / S) & 1, lim, p.status, abort_flag);
-    if (has1) arrived = stage_wait(&full[s1], ((k + 1) / S) & 1, lim, p.status, abort_flag) && arrived;
-    const bool ok = __all_sync(0xffffffffu, arrived);
-    const int2 inf0 = info[s0];
-    const int2 inf1 = has1 ? info[s1] : make_int2(-1, 0);
+    const bool ok0 = __all_sync(kFull, stage_wait(&full[s0], (k / S) & 1, lim, p.status, abort_flag));
+    const bool ok1 =
+        nt == 2 && __all_sync(kFull, stage_wait(&full[s1], ((k + 1) / S) & 1, lim, p.status, abort_flag));
+    const int valid0 = ok0 ? info[s0] : 0;
+    const int valid1 = ok1 ? info[s1] : 0;
     const uint8_t* st0 = smem + s0 * L::kStage;
     const uint8_t* st1 = smem + s1 * L::kStage;
-    if (inf0.x != cur_pair) {  // same decision in every warp (stage info is shared)
-      if (cur_pair >= 0) flush(cur_pair);
-      cur_pair = inf0.x;
-#pragma unroll
-      for (int g = 0; g < G; ++g) {
-        m_w[g] = -INFINITY;
-        o_acc[g][0] = o_acc[g][1] = make_float2(0.f, 0.f);
-      }
-#pragma unroll
-      for (int i = 0; i < NHB; ++i) l_part[i] = 0.f;
-      if constexpr (NHB == 1) load_q(st0, 0);
+    if constexpr (NHB == 1) {
+      if (need_q) load_q(st0, 0);
     }
-    const int nt = (has1 && inf1.x == inf0.x) ? 2 : 1;
-    int valid[2];
-    valid[0] = ok ? inf0.y : 0;
-    valid[1] = (ok && nt == 2) ? inf1.y : 0;
-    const uint8_t* stg[2] = {st0, st1};
+    need_q = false;
 
-    // ---- QK: partial dots over this lane's eighth of D, joined by three shuffles
-    float x[2][NHB];
+    // ---- QK: partial dots over this lane's eighth of D, joined over the 8 lanes
+    float d0[V], d1[V];
 #pragma unroll
     for (int hb = 0; hb < NHB; ++hb) {
       if constexpr (NHB > 1) load_q(st0, hb);
-      float2 acc[2][HB];
-#pragma unroll
-      for (int i = 0; i < 2; ++i)
-#pragma unroll
-        for (int h = 0; h < HB; ++h) acc[i][h] = make_float2(0.f, 0.f);
-#pragma unroll
-      for (int i = 0; i < 2; ++i) {
-        if (qk_lane && tok < valid[i]) {
-#pragma unroll
-          for (int ch = 0; ch < CPT / 8; ++ch) {
-            const int c = qtr * (CPT / 8) + ch;  // 16-byte chunk of the key row
-            const uint4 kw = *reinterpret_cast<const uint4*>(stg[i] + koff[ch]);
-            (void)c;
-            const float2 k0 = bf16x2_to_float2(kw.x), k1 = bf16x2_to_float2(kw.y);
-            const float2 k2 = bf16x2_to_float2(kw.z), k3 = bf16x2_to_float2(kw.w);
-#pragma unroll
-            for (int h = 0; h < HB; ++h) {
-              acc[i][h] = __ffma2_rn(qreg[h][4 * ch + 0], k0, acc[i][h]);
-              acc[i][h] = __ffma2_rn(qreg[h][4 * ch + 1], k1, acc[i][h]);
-              acc[i][h] = __ffma2_rn(qreg[h][4 * ch + 2], k2, acc[i][h]);
-              acc[i][h] = __ffma2_rn(qreg[h][4 * ch + 3], k3, acc[i][h]);
-            }
-          }
-        }
-      }
-#pragma unroll
-      for (int i = 0; i < 2; ++i) {
-        // join the 8 eighths by reduce-scatter: after the xor-4 and xor-2 steps
-        // lane e holds head e % 4 summed over 4 lanes, the xor-1 step completes it
-        float d[4];
-#pragma unroll
-        for (int h = 0; h < 4; ++h) {
-          const int hh = h < HB ? h : 0;
-          d[h] = h < HB ? acc[i][hh].x + acc[i][hh].y : 0.f;
-        }
-        const bool up4 = (qtr & 4) != 0, up2 = (qtr & 2) != 0;
-        // step 1: keep heads {0,1} (low lanes) or {2,3} (high lanes), send the other two
-        const float s0 = up4 ? d[0] : d[2], s1 = up4 ? d[1] : d[3];
-        const float r0 = __shfl_xor_sync(0xffffffffu, s0, 4), r1 = __shfl_xor_sync(0xffffffffu, s1, 4);
-        const float k0 = (up4 ? d[2] : d[0]) + r0, k1 = (up4 ? d[3] : d[1]) + r1;
-        // step 2: keep one of the two
-        const float sx = up2 ? k0 : k1;
-        const float kx = (up2 ? k1 : k0) + __shfl_xor_sync(0xffffffffu, sx, 2);
-        const float dot = kx + __shfl_xor_sync(0xffffffffu, kx, 1);
-        // lane e now holds head ((e & 4) ? 2 : 0) + ((e & 2) ? 1 : 0) = (e >> 1) & 3
-        x[i][hb] = dot;
-      }
+      qk_tile(st0, d0, hb);
+      if (nt == 2) qk_tile(st1, d1, hb);
     }
-    // each lane's head after the reduce-scatter; lanes whose head is >= HB hold nothing
-    const int my_h = (qtr >> 1) & 3;
+    float x[2][C];
+    join_dots<V>(d0, x[0], qtr);
+    if (nt == 2) join_dots<V>(d1, x[1], qtr);
+#pragma unroll
+    for (int j = 0; j < C; ++j) {
+      const int tok = wt0 + 4 * (my_r0 + j) + tok_l;
+      x[0][j] = tok < valid0 ? x[0][j] * p.scale_log2 : -INFINITY;
+      x[1][j] = tok < valid1 ? x[1][j] * p.scale_log2 : -INFINITY;
+    }
+
+    // ---- online softmax of this lane's head: warp max over its rows and tokens
+    float mx = x[0][0];
 #pragma unroll
     for (int i = 0; i < 2; ++i)
 #pragma unroll
-      for (int hb = 0; hb < NHB; ++hb)
-        x[i][hb] = (qk_lane && tok < valid[i] && my_h < HB && (qtr & 1) == 0) ? x[i][hb] * p.scale_log2 : -INFINITY;
-    // ---- warp max per head over both tiles, new running max
-    float tmax[G];
+      for (int j = 0; j < C; ++j) mx = fmaxf(mx, x[i][j]);
+    if constexpr (row_bit(V, R, 4)) mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 4));
+    if constexpr (row_bit(V, R, 2)) mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 2));
+    if constexpr (row_bit(V, R, 1)) mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 1));
+    mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 8));
+    mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 16));
+    const float m_new = fmaxf(m_run, mx);
+    const float alpha = m_new == -INFINITY ? 1.f : fast_ex2(m_run - m_new);
+    const float m_use = m_new == -INFINITY ? 0.f : m_new;
+    m_run = m_new;
+    float lsum = l_run * alpha;
 #pragma unroll
-    for (int hb = 0; hb < NHB; ++hb) {
-      float mx = fmaxf(x[0][hb], x[1][hb]);
+    for (int i = 0; i < 2; ++i)
 #pragma unroll
-      for (int o = LPT; o < 32; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-#pragma unroll
-      for (int h = 0; h < HB; ++h) tmax[hb * HB + h] = __shfl_sync(0xffffffffu, mx, 2 * h);
-    }
-    float alpha[G];
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-      const float mnew = fmaxf(m_w[g], tmax[g]);
-      alpha[g] = mnew == -INFINITY ? 1.f : fast_ex2(m_w[g] - mnew);
-      m_w[g] = mnew;
-    }
-#pragma unroll
-    for (int hb = 0; hb < NHB; ++hb) {
-      float m_h = 0.f, a_h = 1.f;  // this lane's head, picked without dynamic indexing
-#pragma unroll
-      for (int g = 0; g < HB; ++g) {
-        if (g == my_h) {
-          m_h = m_w[hb * HB + g];
-          a_h = alpha[hb * HB + g];
-        }
-      }
-      float lsum = l_part[hb] * a_h;
-#pragma unroll
-      for (int i = 0; i < 2; ++i) {
-        const float pr = fast_ex2(x[i][hb] - m_h);  // x = -inf gives 0
+      for (int j = 0; j < C; ++j) {
+        const float pr = fast_ex2(x[i][j] - m_use);  // x = -inf gives 0
         lsum += pr;
-        if (qk_lane && (qtr & 1) == 0 && my_h < HB)
-          ps[(i * TPW_MAX + tok_l) * G + hb * HB + my_h] = make_float2(pr, pr);
+        const int tok = wt0 + 4 * (my_r0 + j) + tok_l;
+        if (i == 0 || nt == 2) ps[(i * kDecodeTileMax + tok) * G + my_g] = make_float2(pr, pr);
       }
-      l_part[hb] = lsum;
-    }
+    l_run = lsum;
     __syncwarp();
 
-    // ---- PV: lane = channel quad, over this warp's tokens of both tiles, all G heads
+    // ---- PV: rescale o only when some head's running max grew
+    float a[G];
+    bool grew = false;
 #pragma unroll
     for (int g = 0; g < G; ++g) {
+      a[g] = __shfl_sync(kFull, alpha, head_src(V, R, g));
+      grew |= a[g] != 1.f;
+    }
+    if (grew) {  // warp-uniform: a[] was broadcast
 #pragma unroll
-      for (int j = 0; j < 2; ++j) {
-        o_acc[g][j].x *= alpha[g];
-        o_acc[g][j].y *= alpha[g];
+      for (int g = 0; g < G; ++g) {
+        o_acc[g][0] = __fmul2_rn(o_acc[g][0], make_float2(a[g], a[g]));
+        o_acc[g][1] = __fmul2_rn(o_acc[g][1], make_float2(a[g], a[g]));
       }
     }
-#pragma unroll
-    for (int i = 0; i < 2; ++i) {
-#pragma unroll
-      for (int j = 0; j < pv_n; ++j) {
-        const int t = pv_t0 + j;
-        if (t < valid[i]) {
-          const uint2 vw = *reinterpret_cast<const uint2*>(stg[i] + voff[j]);
-          const float2 v01 = bf16x2_to_float2(vw.x), v23 = bf16x2_to_float2(vw.y);
-          const float2* pt = ps + (i * TPW_MAX + half * pv_n + j) * G;
-          if constexpr (G >= 2) {
-#pragma unroll
-            for (int g2 = 0; g2 < G / 2; ++g2) {
-              const float4 pq = reinterpret_cast<const float4*>(pt)[g2];
-              const float2 pa = make_float2(pq.x, pq.y), pb = make_float2(pq.z, pq.w);
-              o_acc[2 * g2][0] = __ffma2_rn(pa, v01, o_acc[2 * g2][0]);
-              o_acc[2 * g2][1] = __ffma2_rn(pa, v23, o_acc[2 * g2][1]);
-              o_acc[2 * g2 + 1][0] = __ffma2_rn(pb, v01, o_acc[2 * g2 + 1][0]);
-              o_acc[2 * g2 + 1][1] = __ffma2_rn(pb, v23, o_acc[2 * g2 + 1][1]);
-            }
-          } else {
-            const float2 pa = pt[0];
-            o_acc[0][0] = __ffma2_rn(pa, v01, o_acc[0][0]);
-            o_acc[0][1] = __ffma2_rn(pa, v23, o_acc[0][1]);
-          }
-        }
-      }
-    }
+    pv_tile(st0, 0, valid0);
+    if (nt == 2) pv_tile(st1, 1, valid1);
     __syncwarp();
-    // ---- release the stage(s); the last warp to finish one refills it
+    // ---- release the stage(s) to the producer
     if (lane == 0) {
-      __threadfence_block();
-      for (int i = 0; i < nt; ++i) {
-        const int kk = k + i, ss = kk % S;
-        if (atomicAdd(&done_cnt[ss], 1) == kWarps - 1) {
-          done_cnt[ss] = 0;
-          if (kk + S < ntiles && !*abort_flag) {
-            fence_proxy_async_smem();
-            issue(kk + S);
-          }
-        }
-      }
+      if (ok0) mbar_arrive(&empty[s0]);
+      if (ok1) mbar_arrive(&empty[s1]);
     }
     k += nt;
   }
-  if (cur_pair >= 0) flush(cur_pair);
+  if (cur >= 0) flush(cur);
 }
 
 size_t decode_workspace_bytes(int pairs, int grid, int G, int D) {
@@ -639,6 +690,7 @@ int decode_grid(int sm_count) { return sm_count; }
 cudaError_t launch_decode(const DecodeParams& p, const CUtensorMap& kmap, const CUtensorMap& vmap,
                           int D, int G, int grid, cudaStream_t stream) {
   cudaError_t e = cudaSuccess;
+  if (grid < 1 || grid > kMaxGrid) return cudaErrorInvalidValue;
 #define LSERVE_DECODE_CASE(DD, GG)                                                        \
   if (D == DD && G == GG) {                                                               \
     const int smem = DecLayout<DD, GG>::kBytes + 1024;                                    \
