@@ -226,7 +226,8 @@ decode_attn_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
   int* info = reinterpret_cast<int*>(smem + L::oInfo);     // valid tokens of the stage's tile
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::oFull);
   uint64_t* empty = reinterpret_cast<uint64_t*>(smem + L::oEmpty);
-  int* misc = reinterpret_cast<int*>(smem + L::oMisc);  // [0..15] scan, [16] last flag, [18] abort
+  // [0..15] scan, [18] abort, [20..21] pairs to merge, [24..27] zeros
+  int* misc = reinterpret_cast<int*>(smem + L::oMisc);
   volatile int* abort_flag = misc + 18;
   const uint8_t* zero16 = reinterpret_cast<const uint8_t*>(misc + 24);  // 16 zero bytes
 
@@ -242,6 +243,7 @@ decode_attn_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
       mbar_init(&empty[s], W);
     }
     misc[18] = 0;
+    misc[20] = misc[21] = -1;  // pairs to merge at the end (first, last of the range)
     misc[24] = misc[25] = misc[26] = misc[27] = 0;
     fence_mbar_init();
   }
@@ -468,6 +470,14 @@ decode_attn_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
     }
   };
 
+  // CTAs holding tiles of the pair (CTAs whose range is empty write nothing)
+  auto seg_count = [&](int pair) {
+    const int c_first = cta_of(cst, off[pair], NC), c_last = cta_of(cst, off[pair + 1] - 1, NC);
+    int nseg = 0;
+    for (int cc = c_first; cc <= c_last; ++cc) nseg += cta_busy(cst, cc) ? 1 : 0;
+    return nseg;
+  };
+
   // End of a pair segment (every consumer warp arrives here at the same tile):
   // merge the warps, then finalise, or publish a partial and maybe merge the
   // pair's partials across CTAs.
@@ -508,9 +518,8 @@ decode_attn_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
     }
     named_sync(kBarConsumers, kConsumerThreads);
     const int b = pair / p.num_kv_heads, h = pair - b * p.num_kv_heads;
-    const int c_first = cta_of(cst, off[pair], NC), c_last = cta_of(cst, off[pair + 1] - 1, NC);
-    int nseg = 0;  // CTAs with tiles of this pair (CTAs without tiles write nothing)
-    for (int cc = c_first; cc <= c_last; ++cc) nseg += cta_busy(cst, cc) ? 1 : 0;
+    // only the first and the last pair of a CTA's range can reach into other CTAs
+    const bool whole = off[pair] >= u0 && off[pair + 1] <= u1;
     const size_t slot = (size_t)cta + pair;
 #pragma unroll
     for (int i = 0; i < NOUT; ++i) {
@@ -526,7 +535,7 @@ decode_attn_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
       }
       const float M = msc[W * G + g];
       const size_t qh = (size_t)b * p.num_q_heads + (size_t)h * G + g;
-      if (nseg == 1) {
+      if (whole) {
         const bool empty_row = !(l > 0.f);
         p.out[qh * D + c] = __float2bfloat16_rn(empty_row ? 0.f : o / l);
         if (c == 0 && p.lse)
@@ -536,43 +545,50 @@ decode_attn_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
         if (c == 0) *reinterpret_cast<float2*>(p.part_ml + (slot * G + g) * 2) = make_float2(M, l);
       }
     }
-    if (nseg > 1 && live) {
+    named_sync(kBarConsumers, kConsumerThreads);  // ow / mlw / msc free again, partial written
+    // A partial: one thread publishes it (the barrier above ordered every
+    // thread's stores before its fence) and counts the pair's finished
+    // segments; the CTA that completes the count merges the pair at its end.
+    // Only warp 0 waits for the fence.
+    if (!whole && live && tid == 0) {
       __threadfence();
-      named_sync(kBarConsumers, kConsumerThreads);
-      if (tid == 0) misc[16] = (atomicAdd(&p.counters[pair], 1u) == (unsigned)(nseg - 1)) ? 1 : 0;
-      named_sync(kBarConsumers, kConsumerThreads);
-      if (misc[16]) {  // last segment to finish: merge every partial of the pair
-        __threadfence();
-#pragma unroll
-        for (int i = 0; i < NOUT; ++i) {
-          const int j = tid + i * kConsumerThreads;
-          if (j >= G * D) continue;
-          const int g = j / D, c = j - g * D;
-          float M = -INFINITY, o = 0.f, lsum = 0.f;
-#pragma unroll 4
-          for (int cc = c_first; cc <= c_last; ++cc) {
-            const bool busy = cta_busy(cst, cc);  // predicated, independent loads
-            const size_t sl = (size_t)cc + pair;
-            const float2 ml = busy ? *reinterpret_cast<const float2*>(p.part_ml + (sl * G + g) * 2)
-                                   : make_float2(-INFINITY, 0.f);
-            const float os = busy ? p.part_o[(sl * G + g) * D + c] : 0.f;
-            const float Mn = fmaxf(M, ml.x);
-            if (Mn == -INFINITY) continue;
-            const float sc = exp2f(M - Mn), wt = exp2f(ml.x - Mn);
-            o = o * sc + wt * os;
-            lsum = lsum * sc + wt * ml.y;
-            M = Mn;
-          }
-          const size_t qh = (size_t)b * p.num_q_heads + (size_t)h * G + g;
-          const bool empty_row = !(lsum > 0.f);
-          p.out[qh * D + c] = __float2bfloat16_rn(empty_row ? 0.f : o / lsum);
-          if (c == 0 && p.lse)
-            p.lse[qh] = empty_row ? -INFINITY : (M + __log2f(lsum)) * 0.69314718055994530942f;
-        }
-        if (tid == 0) p.counters[pair] = 0u;
-      }
+      if (atomicAdd(&p.counters[pair], 1u) == (unsigned)(seg_count(pair) - 1))
+        misc[20 + (off[pair] < u0 ? 0 : 1)] = pair;
     }
-    named_sync(kBarConsumers, kConsumerThreads);  // ow / mlw / msc / misc free again
+  };
+
+  // Merge every partial (o, m, l) of a pair with log-sum-exp weights; the
+  // counter goes back to zero for the next call.
+  auto merge_partials = [&](int pair) {
+    const int b = pair / p.num_kv_heads, h = pair - b * p.num_kv_heads;
+    const int c_first = cta_of(cst, off[pair], NC), c_last = cta_of(cst, off[pair + 1] - 1, NC);
+#pragma unroll
+    for (int i = 0; i < NOUT; ++i) {
+      const int j = tid + i * kConsumerThreads;
+      if (j >= G * D) continue;
+      const int g = j / D, c = j - g * D;
+      float M = -INFINITY, o = 0.f, lsum = 0.f;
+#pragma unroll 4
+      for (int cc = c_first; cc <= c_last; ++cc) {
+        const bool busy = cta_busy(cst, cc);  // predicated, independent loads
+        const size_t sl = (size_t)cc + pair;
+        const float2 ml = busy ? __ldcg(reinterpret_cast<const float2*>(p.part_ml + (sl * G + g) * 2))
+                               : make_float2(-INFINITY, 0.f);
+        const float os = busy ? __ldcg(p.part_o + (sl * G + g) * D + c) : 0.f;
+        const float Mn = fmaxf(M, ml.x);
+        if (Mn == -INFINITY) continue;
+        const float sc = exp2f(M - Mn), wt = exp2f(ml.x - Mn);
+        o = o * sc + wt * os;
+        lsum = lsum * sc + wt * ml.y;
+        M = Mn;
+      }
+      const size_t qh = (size_t)b * p.num_q_heads + (size_t)h * G + g;
+      const bool empty_row = !(lsum > 0.f);
+      p.out[qh * D + c] = __float2bfloat16_rn(empty_row ? 0.f : o / lsum);
+      if (c == 0 && p.lse)
+        p.lse[qh] = empty_row ? -INFINITY : (M + __log2f(lsum)) * 0.69314718055994530942f;
+    }
+    if (tid == 0) p.counters[pair] = 0u;
   };
 
   // Each iteration takes one tile, or two consecutive tiles of the same pair:
@@ -676,6 +692,10 @@ decode_attn_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
     k += nt;
   }
   if (cur >= 0) flush(cur);
+  // the pairs this CTA completed: merge their partials
+  named_sync(kBarConsumers, kConsumerThreads);
+  if (misc[20] >= 0) merge_partials(misc[20]);
+  if (misc[21] >= 0) merge_partials(misc[21]);
 }
 
 size_t decode_workspace_bytes(int pairs, int grid, int G, int D) {
