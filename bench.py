@@ -104,6 +104,28 @@ def stats_build_bytes(w):
     return rd + wr
 
 
+def decode_traffic():
+    """DRAM bytes (read + write) per decode-attention launch from the committed
+    ncu summary, provided the kernel source is still the one it measured."""
+    import hashlib
+    summ = os.path.join(ROOT, "profiles", "decode_attn_llama3_8b_decode.md")
+    src = os.path.join(ROOT, "block_sparse_attention_page_b200", "csrc", "decode_attn.cu")
+    try:
+        fields = {}
+        with open(summ) as f:
+            for line in f:
+                if line.startswith("- ") and ":" in line:
+                    k, v = line[2:].split(":", 1)
+                    fields[k.strip()] = v.strip().strip("`")
+        with open(src, "rb") as f:
+            digest = hashlib.sha256(f.read()).hexdigest()
+        if fields.get("decode_attn.cu sha256") != digest:
+            return None
+        return float(fields["traffic bytes per launch"])
+    except (OSError, KeyError, ValueError):
+        return None
+
+
 # --- clocks sampling ----------------------------------------------------------
 
 class ClockSampler:
@@ -278,6 +300,10 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--layers", type=int, default=LAYERS,
                     help="layer replicas (fewer = a small case for profiling; < 32 may fit in L2)")
+    ap.add_argument("--prefill-only", action="store_true",
+                    help="run only the prefill stage (profiling)")
+    ap.add_argument("--prefill-seq", type=int, default=None,
+                    help="prefill sequence length (default: the 128K workload)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
     LAYERS = max(1, args.layers)
@@ -299,6 +325,12 @@ def main():
     from synth.device import DecodeBuffers
 
     hbm_peak, tc_peak, tc_sustained, peak_src = peaks()
+    if args.prefill_only:
+        res = prefill_stage(lserve, synth, dev, torch.cuda.Stream(device=dev), tc_peak, None,
+                            args.prefill_seq)
+        if rank == 0:
+            print(json.dumps({"prefill": res}))
+        return 0
     w = synth.llama3_8b_decode()
     buf = DecodeBuffers(w, device=dev, layers=LAYERS)
     d = lserve.paged_desc(w.B, w.H_q, w.H_kv, w.D, w.N_L, w.N_P, w.max_pages, w.num_pool_pages)
@@ -343,9 +375,18 @@ def main():
     g_select_only = capture(lambda: [select(l) for l in range(LAYERS)])
     g_stats = capture(stats_all)
 
-    def run_steps(k0, k):
+    def run_steps(k0, k, ev=None):
+        # ev: event pairs recorded around the attention-only replays, so that the
+        # average attention launch is measured inside the timed region itself
         for t in range(k0, k0 + k):
-            (g_sel if t % REUSE == 0 else g_reuse).replay()
+            if t % REUSE == 0:
+                g_sel.replay()
+            elif ev is not None and t < len(ev):
+                ev[t][0].record(stream)
+                g_reuse.replay()
+                ev[t][1].record(stream)
+            else:
+                g_reuse.replay()
 
     def timed(fn, reps=1):
         e0 = torch.cuda.Event(enable_timing=True)
@@ -370,8 +411,12 @@ def main():
     sampler = ClockSampler(local, getattr(torch.cuda.get_device_properties(dev), "uuid", None))
     sampler.start() if rank == 0 else None
     time.sleep(0.3)
-    elapsed = timed(lambda: run_steps(0, args.steps))
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          if t % REUSE else None for t in range(args.steps)]
+    elapsed = timed(lambda: run_steps(0, args.steps, ev))
     clocks = sampler.stop() if rank == 0 else None
+    attn_in_region = [a.elapsed_time(b) / 1e3 for t, (a, b) in enumerate(e for e in ev if e)]
+    t_attn_region = float(np.mean(attn_in_region)) / LAYERS if attn_in_region else None
     elapsed = max_over_ranks(elapsed, ws, dev)
     step_bytes = acct["step"] * LAYERS
     value = step_bytes * args.steps * ws / elapsed / 1e9
@@ -380,6 +425,8 @@ def main():
     # stages, each alone (graph replays, CUDA events on the launching stream)
     reps = 20
     t_attn = timed(lambda: g_reuse.replay(), reps) / (reps * LAYERS)
+    if t_attn_region is not None:
+        t_attn = t_attn_region  # the launches of the timed region themselves
     t_sel = timed(lambda: g_select_only.replay(), reps) / (reps * LAYERS)
     t_stats = timed(lambda: g_stats.replay(), 3) / (3 * LAYERS)
     sb = stats_build_bytes(w)
@@ -423,17 +470,21 @@ def main():
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "ms_per_step": t_e2e / e2e_steps * 1e3}
 
-    launches = args.steps * LAYERS * 2 + (-(-args.steps // REUSE)) * LAYERS * 2
+    # one kernel per attention call, two per selection call (scores, top-K)
+    launches = args.steps * LAYERS + (-(-args.steps // REUSE)) * LAYERS * 2
     result = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": ws, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": elapsed / args.steps * 1e3,
         "us_per_layer_step": us_layer, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": workload_config(w),
-        "roofline": {"bound": "hbm", "kernel": "lserve_sparse_decode_attn (split + combine)",
+        "roofline": {"bound": "hbm", "kernel": "decode_attn_kernel (lserve_sparse_decode_attn)",
                      "achieved": attn_gbs, "peak": hbm_peak, "unit": "GB/s",
-                     "frac": attn_gbs / hbm_peak, "traffic": None,
-                     "peak_source": f"{peak_src} hbm_gbs (copy)"},
+                     "frac": attn_gbs / hbm_peak, "traffic": decode_traffic(),
+                     "algorithmic_bytes": acct["attn"],
+                     "peak_source": f"{peak_src} hbm_gbs (copy, burst); of {peak_src}",
+                     "timing": "mean attention launch inside the timed region (CUDA events "
+                               "around the attention-only graph replays)"},
         "stages": stages,
         "e2e": e2e,
         "gpu_launches": launches,
@@ -444,7 +495,8 @@ def main():
     torch.cuda.empty_cache()
 
     if not args.no_prefill:
-        result["stages"]["prefill"] = prefill_stage(lserve, synth, dev, stream, tc_peak, timed)
+        result["stages"]["prefill"] = prefill_stage(lserve, synth, dev, stream, tc_peak, timed,
+                                                    args.prefill_seq)
 
     if rank == 0 and not args.no_cpu_baseline:
         per_step, sample = oracle_step_sample(w, budget_s=15.0)
@@ -459,11 +511,25 @@ def main():
     return 0
 
 
-def prefill_stage(lserve, synth, dev, stream, tc_peak, timed):
-    """Block-sparse prefill on the 128K workload: TFLOP/s over computed blocks."""
+def prefill_stage(lserve, synth, dev, stream, tc_peak, timed, seq=None):
+    """Block-sparse prefill on the 128K workload (or `seq` tokens of the same
+    shape): TFLOP/s over computed blocks."""
     import torch
     import oracle
-    w = synth.prefill_128k()
+    w = synth.prefill_128k() if seq is None else synth.prefill_workload(
+        seq, 32, 8, 128, 128, 1004, name=f"prefill_{seq}")
+    if timed is None:
+        def timed(fn, reps=1):
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            torch.cuda.synchronize()
+            e0.record(stream)
+            with torch.cuda.stream(stream):
+                for _ in range(reps):
+                    fn()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            return e0.elapsed_time(e1) / 1e3
     d = lserve.prefill_desc(w.T, w.H_q, w.H_kv, w.D, w.block, w.sink_blocks, w.local_blocks)
     need = lserve.workspace_size(lserve.OP_PREFILL, d)
     try:
