@@ -10,9 +10,11 @@ namespace lserve {
 
 constexpr int kStatsWarps = 8;   // warps per CTA of the stats kernel
 constexpr int kScoreWarps = 8;   // warps per CTA of the score kernel
-constexpr int kScorePagesPerWarp = 2;
+constexpr int kScorePagesPerWarp = 4;
+constexpr int kScoreSteps = 2;        // warp steps (of 32 / (D/8) logical pages) loaded at once
 constexpr int kTopkThreads = 512;
 constexpr int kTopkMaxPages = 32768;
+constexpr int kTopkCand = 128;       // bucket size ranked pairwise
 
 struct StatsParams {
   const __nv_bfloat16* k_pool;

@@ -3,26 +3,37 @@
 // "Top-K物理ページ" node of the 統一ブロックスパースアテンション figure).
 //
 // 1. page_score_kernel: a stream over the statistics pool.  One warp scores
-//    physical pages; D/8 lanes share a logical page, each holding 8 channels
-//    of the G query heads (fp32) in registers.  Per channel the sign of q
-//    picks k_max or k_min (q*max(.)/q*min(.) without a second product: the
-//    larger of q*k_max and q*k_min is q times k_max when q >= 0, else times
-//    k_min; bf16 x bf16 products are exact in fp32).  Lanes reduce with
-//    shuffles, the max over the g logical pages gives the physical score.
+//    kScorePagesPerWarp physical pages, issuing all their stats loads before
+//    it reduces; D/8 lanes share a logical page, each holding 8 channels of
+//    the group-folded query Qp = sum_h max(q_h, 0), Qn = sum_h min(q_h, 0)
+//    (max(q*k_max, q*k_min) = max(q,0)*k_max + min(q,0)*k_min because
+//    k_max >= k_min).  Lanes reduce with shuffles, the max over the g logical
+//    pages gives the physical score.
 // 2. page_topk_kernel: one CTA per (sequence, retrieval head) finds the K-th
 //    largest score by an 8-bit radix select over order-preserving integer
-//    keys, then compacts the winners in ascending page order with one block
-//    scan; ties at the threshold go to the lowest page indices.
+//    keys, stopping once the bucket holding it has at most kTopkCand keys,
+//    which are ranked exactly by (score, page index); then it compacts the
+//    winners in ascending page order with one block scan.  Ties go to the
+//    lowest page indices.
 #include "common.cuh"
 #include "kernels.h"
 
 namespace lserve {
 
+// Scores of kScorePagesPerWarp physical pages per warp.  Every lane first issues
+// all its 16-byte stats loads for those pages (up to kScoreSteps warp steps of
+// LPI logical pages each, k_min and k_max), then reduces.  The sum over the G
+// query heads of the group is folded into q before the stream: since
+// k_max >= k_min, max(q*k_max, q*k_min) = max(q,0)*k_max + min(q,0)*k_min, so
+//   S^j = sum_i Qp[i] * k_max^j[i] + Qn[i] * k_min^j[i]
+// with Qp[i] = sum_h max(q_h[i], 0) and Qn[i] = sum_h min(q_h[i], 0).
 template <int D, int G>
-__global__ void __launch_bounds__(kScoreWarps * 32)
+__global__ void __launch_bounds__(kScoreWarps * 32, 2)
 page_score_kernel(SelectParams p) {
-  constexpr int LPR = D / 8;      // lanes per logical page
+  constexpr int LPR = D / 8;      // lanes per logical page (16 channels x 8 = 128)
   constexpr int LPI = 32 / LPR;   // logical pages per warp step
+  constexpr int PW = kScorePagesPerWarp;
+  constexpr int SB = kScoreSteps;  // warp steps per page loaded at once
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int b = blockIdx.z, h = blockIdx.y;
   if (p.head_kind[h] != 0) return;
@@ -30,12 +41,19 @@ page_score_kernel(SelectParams p) {
   const int NP = p.physical_page, NL = p.logical_page, g = NP / NL;
   const int npages = min((n + NP - 1) / NP, p.max_pages);
   const int nlog = (n + NL - 1) / NL;
-  const int m0 = (blockIdx.x * kScoreWarps + warp) * kScorePagesPerWarp;
+  const int m0 = (blockIdx.x * kScoreWarps + warp) * PW;
   if (m0 >= npages) return;
   const int c = (lane % LPR) * 8;
   const int slot = lane / LPR;
+  const size_t pair = (size_t)b * p.num_kv_heads + h;
 
-  float qf[G][8];
+  // block-table entries of the warp's pages: lane j holds page m0 + j
+  int pid_l = -1;
+  if (lane < PW && m0 + lane < npages) pid_l = p.block_table[(size_t)b * p.max_pages + m0 + lane];
+
+  float qp[8], qn[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) qp[k] = qn[k] = 0.f;
 #pragma unroll
   for (int hh = 0; hh < G; ++hh) {
     const uint4 w = *reinterpret_cast<const uint4*>(
@@ -43,53 +61,72 @@ page_score_kernel(SelectParams p) {
     const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
-      qf[hh][2 * k] = bf16_lo(ww[k]);
-      qf[hh][2 * k + 1] = bf16_hi(ww[k]);
+      const float lo = bf16_lo(ww[k]), hi = bf16_hi(ww[k]);
+      qp[2 * k] += fmaxf(lo, 0.f);
+      qn[2 * k] += fminf(lo, 0.f);
+      qp[2 * k + 1] += fmaxf(hi, 0.f);
+      qn[2 * k + 1] += fminf(hi, 0.f);
     }
   }
 
-  for (int mi = 0; mi < kScorePagesPerWarp; ++mi) {
-    const int m = m0 + mi;
-    if (m >= npages) break;
-    const int pid = p.block_table[(size_t)b * p.max_pages + m];
-    if (kCheckBounds && (pid < 0 || pid >= p.num_pool_pages)) {
-      raise_status(p.status, LSERVE_ERR_BOUNDS);
-      continue;
-    }
-    const __nv_bfloat16* st = p.stats_pool + (((size_t)pid * p.num_kv_heads + h) * g) * 2 * D + c;
-    float best = -INFINITY;
-    for (int s0 = 0; s0 < g; s0 += LPI) {
-      const int sub = s0 + slot;
-      const bool valid = sub < g && m * g + sub < nlog;
-      float part = 0.f;
-      if (valid) {
-        const uint4 mn = ldg_nc_v4(st + (size_t)sub * 2 * D);
-        const uint4 mx = ldg_nc_v4(st + (size_t)sub * 2 * D + D);
-        const uint32_t wn[4] = {mn.x, mn.y, mn.z, mn.w};
-        const uint32_t wx[4] = {mx.x, mx.y, mx.z, mx.w};
-        float kn[8], kx[8];
+  int pid[PW];
+  bool pok[PW];
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          kn[2 * k] = bf16_lo(wn[k]);
-          kn[2 * k + 1] = bf16_hi(wn[k]);
-          kx[2 * k] = bf16_lo(wx[k]);
-          kx[2 * k + 1] = bf16_hi(wx[k]);
-        }
+  for (int j = 0; j < PW; ++j) {
+    pid[j] = __shfl_sync(0xffffffffu, pid_l, j);
+    pok[j] = m0 + j < npages && pid[j] >= 0 && pid[j] < p.num_pool_pages;
+    if (kCheckBounds && m0 + j < npages && !pok[j] && lane == 0) raise_status(p.status, LSERVE_ERR_BOUNDS);
+  }
+  float best[PW];
 #pragma unroll
-        for (int hh = 0; hh < G; ++hh) {
+  for (int j = 0; j < PW; ++j) best[j] = -INFINITY;
+
+  const int steps = (g + LPI - 1) / LPI;
+  for (int s0 = 0; s0 < steps; s0 += SB) {
+    uint4 mn[PW][SB], mx[PW][SB];
+    bool ok[PW][SB];
 #pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            const float qq = qf[hh][k];
-            part = fmaf(qq, qq >= 0.f ? kx[k] : kn[k], part);
-          }
+    for (int j = 0; j < PW; ++j) {
+      const __nv_bfloat16* st = p.stats_pool + (((size_t)pid[j] * p.num_kv_heads + h) * g) * 2 * D + c;
+#pragma unroll
+      for (int t = 0; t < SB; ++t) {
+        const int sub = (s0 + t) * LPI + slot;
+        ok[j][t] = pok[j] && s0 + t < steps && sub < g && (m0 + j) * g + sub < nlog;
+        if (ok[j][t]) {
+          mn[j][t] = ldg_nc_v4(st + (size_t)sub * 2 * D);
+          mx[j][t] = ldg_nc_v4(st + (size_t)sub * 2 * D + D);
         }
       }
-#pragma unroll
-      for (int o = 1; o < LPR; o <<= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
-      if (valid) best = fmaxf(best, part);
     }
-    best = warp_max(best);
-    if (lane == 0) p.scores[((size_t)b * p.num_kv_heads + h) * p.max_pages + m] = best;
+#pragma unroll
+    for (int j = 0; j < PW; ++j) {
+#pragma unroll
+      for (int t = 0; t < SB; ++t) {
+        float part = 0.f;
+        if (ok[j][t]) {
+          const uint32_t wn[4] = {mn[j][t].x, mn[j][t].y, mn[j][t].z, mn[j][t].w};
+          const uint32_t wx[4] = {mx[j][t].x, mx[j][t].y, mx[j][t].z, mx[j][t].w};
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            part = fmaf(qp[2 * k], bf16_lo(wx[k]), part);
+            part = fmaf(qp[2 * k + 1], bf16_hi(wx[k]), part);
+            part = fmaf(qn[2 * k], bf16_lo(wn[k]), part);
+            part = fmaf(qn[2 * k + 1], bf16_hi(wn[k]), part);
+          }
+        }
+#pragma unroll
+        for (int o = 1; o < LPR; o <<= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+        if (ok[j][t]) best[j] = fmaxf(best[j], part);
+      }
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < PW; ++j) {
+    float v = best[j];
+#pragma unroll
+    for (int o = LPR; o < 32; o <<= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    // a page whose block-table entry is bad scores -inf (never chosen ahead of a valid one)
+    if (lane == 0 && m0 + j < npages) p.scores[pair * p.max_pages + m0 + j] = v;
   }
 }
 
@@ -102,7 +139,8 @@ __device__ __forceinline__ uint32_t order_key(float f) {
 __global__ void __launch_bounds__(kTopkThreads) page_topk_kernel(SelectParams p) {
   extern __shared__ uint32_t keys[];  // [npages]
   __shared__ int hist[256];
-  __shared__ int sh_digit, sh_above;
+  __shared__ int sh_digit, sh_above, sh_bucket, sh_ncand;
+  __shared__ int cand[kTopkCand];
   __shared__ uint32_t warp_tot[kTopkThreads / 32];
   const int b = blockIdx.y, h = blockIdx.x, tid = threadIdx.x;
   const int lane = tid & 31, warp = tid >> 5;
@@ -129,15 +167,23 @@ __global__ void __launch_bounds__(kTopkThreads) page_topk_kernel(SelectParams p)
   for (int m = tid; m < M; m += blockDim.x) keys[m] = order_key(sc[m]);
   __syncthreads();
 
-  // radix select of the K-th largest key, 8 bits at a time from the top
+  // Radix select of the K-th largest key, 8 bits at a time from the top, until
+  // the bucket that holds it has at most kTopkCand keys; those few are then
+  // ranked exactly by (key, page index).  `need` keys of the bucket are kept.
   uint32_t prefix = 0, mask = 0;
-  int need = K;
-  for (int shift = 24; shift >= 0; shift -= 8) {
+  int need = K, bucket = M;
+  for (int shift = 24; shift >= 0 && bucket > kTopkCand; shift -= 8) {
     for (int i = tid; i < 256; i += blockDim.x) hist[i] = 0;
     __syncthreads();
-    for (int m = tid; m < M; m += blockDim.x) {
-      const uint32_t k = keys[m];
-      if ((k & mask) == prefix) atomicAdd(&hist[(k >> shift) & 255u], 1);
+    // warp-aggregated: the lanes holding the same digit add their count once
+    // (most keys share their top digits, which would serialise plain atomics)
+    for (int base = 0; base < M; base += blockDim.x) {
+      const int m = base + tid;
+      const uint32_t k = m < M ? keys[m] : 0u;
+      const bool act = m < M && (k & mask) == prefix;
+      const uint32_t digit = act ? (k >> shift) & 255u : 256u;
+      const unsigned peers = __match_any_sync(0xffffffffu, digit);
+      if (act && lane == __ffs(peers) - 1) atomicAdd(&hist[digit], __popc(peers));
     }
     __syncthreads();
     if (warp == 0) {
@@ -161,6 +207,7 @@ __global__ void __launch_bounds__(kTopkThreads) page_topk_kernel(SelectParams p)
           if (above < need && need <= above + cnt[i]) {
             sh_digit = 255 - 8 * lane - i;
             sh_above = above;
+            sh_bucket = cnt[i];
           }
           above += cnt[i];
         }
@@ -170,19 +217,43 @@ __global__ void __launch_bounds__(kTopkThreads) page_topk_kernel(SelectParams p)
     need -= sh_above;
     prefix |= (uint32_t)sh_digit << shift;
     mask |= 255u << shift;
+    bucket = sh_bucket;
+  }
+  uint8_t* chosen = reinterpret_cast<uint8_t*>(keys + M);  // [M], valid for bucket members
+  const bool ranked = bucket <= kTopkCand;
+  if (ranked) {
+    if (tid == 0) sh_ncand = 0;
+    __syncthreads();
+    for (int m = tid; m < M; m += blockDim.x)
+      if ((keys[m] & mask) == prefix) cand[atomicAdd(&sh_ncand, 1)] = m;
+    __syncthreads();
+    for (int i = tid; i < bucket; i += blockDim.x) {
+      const int mi = cand[i];
+      const uint32_t ki = keys[mi];
+      int r = 0;  // bucket keys ahead of this one
+      for (int j = 0; j < bucket; ++j) {
+        const int mj = cand[j];
+        const uint32_t kj = keys[mj];
+        r += (kj > ki) || (kj == ki && mj < mi);
+      }
+      chosen[mi] = r < need;
+    }
     __syncthreads();
   }
-  const uint32_t T = prefix;  // the K-th largest key; `need` keys equal to it are kept
+  // Otherwise all four digits were used and the bucket's keys are all equal:
+  // the `need` lowest page indices among them are kept.
 
-  // block scan of (greater, equal) counts over contiguous per-thread chunks
+  // Compaction in ascending page order: one block scan of (above, kept) counts
+  // over contiguous per-thread chunks.
   const int per = (M + blockDim.x - 1) / blockDim.x;
   const int lo = min(M, tid * per), hi = min(M, lo + per);
-  uint32_t gt = 0, eq = 0;
+  uint32_t na = 0, nk = 0;
   for (int m = lo; m < hi; ++m) {
-    gt += keys[m] > T;
-    eq += keys[m] == T;
+    const uint32_t km = keys[m] & mask;
+    na += km > prefix;
+    nk += km == prefix && (!ranked || chosen[m]);
   }
-  uint32_t v = (gt << 16) | eq, incl = v;
+  uint32_t v = (na << 16) | nk, incl = v;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
     const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
@@ -202,15 +273,15 @@ __global__ void __launch_bounds__(kTopkThreads) page_topk_kernel(SelectParams p)
   }
   __syncthreads();
   const uint32_t before = warp_tot[warp] + incl - v;
-  uint32_t gt_before = before >> 16, eq_before = before & 0xFFFFu;
+  uint32_t a_before = before >> 16, k_before = before & 0xFFFFu;
   for (int m = lo; m < hi; ++m) {
-    const uint32_t k = keys[m];
-    if (k > T) {
-      sel[gt_before + min(eq_before, (uint32_t)need)] = m;
-      ++gt_before;
-    } else if (k == T) {
-      if (eq_before < (uint32_t)need) sel[gt_before + eq_before] = m;
-      ++eq_before;
+    const uint32_t km = keys[m] & mask;
+    if (km > prefix) {
+      sel[a_before + min(k_before, (uint32_t)need)] = m;
+      ++a_before;
+    } else if (km == prefix && (!ranked || chosen[m])) {
+      if (k_before < (uint32_t)need) sel[a_before + k_before] = m;
+      ++k_before;
     }
   }
   if (tid == 0) p.sel_count[pair] = K;
@@ -236,7 +307,7 @@ cudaError_t launch_page_select(const SelectParams& p, int D, cudaStream_t stream
 #undef LSERVE_SCORE_CASE
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  const size_t smem = (size_t)p.max_pages * sizeof(uint32_t);
+  const size_t smem = (size_t)p.max_pages * (sizeof(uint32_t) + 1);  // keys + kept flags
   if (smem > 48 * 1024) {
     e = set_smem_once((const void*)page_topk_kernel, (int)smem);
     if (e != cudaSuccess) return e;
