@@ -357,10 +357,14 @@ def main():
         lserve.page_select(d, qs[l], buf.stats[l], buf.block_table, buf.ctx_lens, buf.head_kind,
                            w.top_k, buf.sel[l], buf.sel_count[l], workspace=ws_sel)
 
-    def attn(l):
+    def attn(l, overlap=False):
+        # overlap: the kernel before this call is the previous layer's attention,
+        # which writes none of the selection / block-table inputs, so the split
+        # plan and first page lookups may run while it finishes (PDL)
         lserve.sparse_decode_attn(d, qs[l], buf.k_pools[l], buf.v_pools[l], buf.block_table,
                                   buf.ctx_lens, buf.head_kind, buf.sel[l], buf.sel_count[l], w.top_k,
-                                  w.sink, w.local, scale, outs[l], None, workspace=ws_dec)
+                                  w.sink, w.local, scale, outs[l], None, workspace=ws_dec,
+                                  overlap_prologue=overlap)
 
     with torch.cuda.stream(stream):
         stats_all()
@@ -377,7 +381,7 @@ def main():
         return g
 
     g_sel = capture(lambda: [(select(l), attn(l)) for l in range(LAYERS)])
-    g_reuse = capture(lambda: [attn(l) for l in range(LAYERS)])
+    g_reuse = capture(lambda: [attn(l, overlap=l > 0) for l in range(LAYERS)])
     g_select_only = capture(lambda: [select(l) for l in range(LAYERS)])
     g_stats = capture(stats_all)
 

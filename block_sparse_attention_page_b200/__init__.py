@@ -30,8 +30,9 @@ EXPORTED = [
     "lserve_page_stats", "lserve_page_select", "lserve_sparse_decode_attn",
     "lserve_blocksparse_prefill", "lserve_workspace_size", "lserve_read_device_status",
     "lserve_set_wait_limit_cycles", "lserve_debug_wait_timeout", "lserve_status_string",
-    "lserve_bounds_checked", "lserve_page_select_noalloc",
+    "lserve_bounds_checked", "lserve_page_select_noalloc", "lserve_sparse_decode_attn_ex",
 ]
+DECODE_OVERLAP_PROLOGUE = 1
 
 
 class LServeError(RuntimeError):
@@ -66,6 +67,9 @@ def _load(path):
     lib.lserve_page_select.argtypes = [P(PagedDesc), vp, vp, vp, vp, vp, i32, vp, vp, vp, vp, sz, vp]
     lib.lserve_sparse_decode_attn.argtypes = [P(PagedDesc), vp, vp, vp, vp, vp, vp, vp, vp, i32, i32,
                                               i32, ctypes.c_float, vp, vp, vp, sz, vp]
+    lib.lserve_sparse_decode_attn_ex.argtypes = [P(PagedDesc), vp, vp, vp, vp, vp, vp, vp, vp, i32,
+                                                 i32, i32, ctypes.c_float, vp, vp, ctypes.c_uint32,
+                                                 vp, sz, vp]
     lib.lserve_blocksparse_prefill.argtypes = [P(PrefillDesc), vp, vp, vp, vp, ctypes.c_float, vp, vp,
                                                vp, sz, vp]
     lib.lserve_page_select_noalloc.argtypes = [P(PagedDesc), vp, vp, vp, vp, vp, i32, vp, vp, vp]
@@ -145,8 +149,19 @@ def page_select_noalloc(desc, q, stats_pool, block_table, ctx_lens, head_kind, t
 
 def sparse_decode_attn(desc, q, k_pool, v_pool, block_table, ctx_lens, head_kind, sel, sel_count,
                        top_k, sink_tokens, local_tokens, softmax_scale, out, lse=None,
-                       workspace=None, stream=None):
+                       workspace=None, stream=None, overlap_prologue=False):
+    """lserve_sparse_decode_attn; overlap_prologue=True calls
+    lserve_sparse_decode_attn_ex with LSERVE_DECODE_OVERLAP_PROLOGUE (the caller
+    guarantees the previous kernel on the stream writes none of block_table,
+    ctx_lens, head_kind, sel, sel_count)."""
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    if overlap_prologue:
+        _check("lserve_sparse_decode_attn_ex", lib.lserve_sparse_decode_attn_ex(
+            ctypes.byref(desc), _ptr(q), _ptr(k_pool), _ptr(v_pool), _ptr(block_table),
+            _ptr(ctx_lens), _ptr(head_kind), _ptr(sel), _ptr(sel_count), top_k, sink_tokens,
+            local_tokens, float(softmax_scale), _ptr(out), _ptr(lse), DECODE_OVERLAP_PROLOGUE,
+            _ptr(workspace), ws_bytes, _stream(stream)))
+        return
     _check("lserve_sparse_decode_attn", lib.lserve_sparse_decode_attn(
         ctypes.byref(desc), _ptr(q), _ptr(k_pool), _ptr(v_pool), _ptr(block_table), _ptr(ctx_lens),
         _ptr(head_kind), _ptr(sel), _ptr(sel_count), top_k, sink_tokens, local_tokens,

@@ -321,7 +321,20 @@ int lserve_sparse_decode_attn(const lserve_paged_desc* desc, const void* q, cons
                               int32_t top_k, int32_t sink_tokens, int32_t local_tokens,
                               float softmax_scale, void* out, float* lse, void* workspace,
                               size_t workspace_bytes, void* stream) {
+  return lserve_sparse_decode_attn_ex(desc, q, k_pool, v_pool, block_table, ctx_lens, head_kind, sel,
+                                      sel_count, top_k, sink_tokens, local_tokens, softmax_scale, out,
+                                      lse, 0u, workspace, workspace_bytes, stream);
+}
+
+int lserve_sparse_decode_attn_ex(const lserve_paged_desc* desc, const void* q, const void* k_pool,
+                                 const void* v_pool, const int32_t* block_table,
+                                 const int32_t* ctx_lens, const uint8_t* head_kind,
+                                 const int32_t* sel, const int32_t* sel_count, int32_t top_k,
+                                 int32_t sink_tokens, int32_t local_tokens, float softmax_scale,
+                                 void* out, float* lse, uint32_t flags, void* workspace,
+                                 size_t workspace_bytes, void* stream) {
   if (!valid_paged(desc)) return LSERVE_ERR_INVALID_ARG;
+  if (flags & ~(uint32_t)LSERVE_DECODE_OVERLAP_PROLOGUE) return LSERVE_ERR_INVALID_ARG;
   if (!q || !k_pool || !v_pool || !block_table || !ctx_lens || !head_kind || !sel || !sel_count || !out)
     return LSERVE_ERR_INVALID_ARG;
   if (!aligned(q, 16) || !aligned(k_pool, 16) || !aligned(v_pool, 16) || !aligned(out, 16) ||
@@ -375,6 +388,7 @@ int lserve_sparse_decode_attn(const lserve_paged_desc* desc, const void* q, cons
   p.tiles_per_page = desc->physical_page / tile_rows;
   p.scale_log2 = softmax_scale * 1.4426950408889634f;
   p.wait_limit = wait_limit();
+  p.overlap_prologue = (flags & LSERVE_DECODE_OVERLAP_PROLOGUE) ? 1 : 0;
   p.status = device_status_word();
   if (!p.status) return LSERVE_ERR_CUDA;
   return cuda_status(launch_decode(p, kmap, vmap, D, G, grid, static_cast<cudaStream_t>(stream)));

@@ -129,6 +129,17 @@ __device__ __forceinline__ void bulk_load_1d(void* smem_dst, const void* gsrc, u
       : "memory");
 }
 
+// Programmatic dependent launch: let the next kernel on the stream start its
+// thread blocks (they still wait for this grid before touching its results),
+// and wait until the previous kernel has completed with its memory visible.
+// Both are no-ops for a kernel launched without the programmatic attribute.
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait_prior_grid() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 // barrier among `nthreads` threads (a multiple of 32) on hardware barrier `id`
 __device__ __forceinline__ void named_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");

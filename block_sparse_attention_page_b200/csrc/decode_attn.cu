@@ -237,6 +237,11 @@ decode_attn_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
   const int NC = gridDim.x, cta = blockIdx.x;
   const uint64_t lim = p.wait_limit;
 
+  // The next kernel may start as soon as SMs free up; without the prologue
+  // overlap, this grid reads nothing before the previous kernel completes.
+  pdl_launch_dependents();
+  if (!p.overlap_prologue) pdl_wait_prior_grid();
+
   if (tid == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(&full[s], 1);
@@ -286,18 +291,6 @@ decode_attn_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
   const int u0 = (int)(U * cta / NC), u1 = (int)(U * (cta + 1) / NC);
   const int ntiles = u1 - u0;
 
-  // pairs with nothing to attend (n = 0): zero output, lse = -inf
-  if (cta == 0) {
-    for (int pr = tid; pr < P; pr += kThreads) {
-      if (off[pr + 1] != off[pr]) continue;
-      const int b = pr / p.num_kv_heads, h = pr - b * p.num_kv_heads;
-      for (int g = 0; g < G; ++g) {
-        const size_t qh = (size_t)b * p.num_q_heads + (size_t)h * G + g;
-        for (int c = 0; c < D; ++c) p.out[qh * D + c] = __float2bfloat16_rn(0.f);
-        if (p.lse) p.lse[qh] = -INFINITY;
-      }
-    }
-  }
   __syncthreads();  // range table, barrier init and plan visible to every warp
 
   // =========================== producer warp ===============================
@@ -335,6 +328,7 @@ decode_attn_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
     for (int kb = 0; kb < ntiles && alive; kb += 32) {
       int tp = 0, trow = 0, tval = 0;
       if (kb + lane < ntiles) lookup(u0 + kb + lane, tp, trow, tval);
+      if (kb == 0) pdl_wait_prior_grid();  // q and the KV pools may come from the previous kernel
       const int nb = min(32, ntiles - kb);
       for (int j = 0; j < nb; ++j) {
         const int k = kb + j, s = k % S;
@@ -373,6 +367,19 @@ decode_attn_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
   }
 
   // =========================== consumer warps ==============================
+  pdl_wait_prior_grid();  // no global write before the previous kernel completes
+  // pairs with nothing to attend (n = 0): zero output, lse = -inf
+  if (cta == 0) {
+    for (int pr = tid; pr < P; pr += kConsumerThreads) {
+      if (off[pr + 1] != off[pr]) continue;
+      const int b = pr / p.num_kv_heads, h = pr - b * p.num_kv_heads;
+      for (int g = 0; g < G; ++g) {
+        const size_t qh = (size_t)b * p.num_q_heads + (size_t)h * G + g;
+        for (int c = 0; c < D; ++c) p.out[qh * D + c] = __float2bfloat16_rn(0.f);
+        if (p.lse) p.lse[qh] = -INFINITY;
+      }
+    }
+  }
   const int tok_l = lane / LPT, qtr = lane % LPT;  // QK: (token of the row, eighth of D)
   const int jb = join_base(V, qtr);
   const int my_g = jb / R, my_r0 = jb % R;         // head and first row of the joined dots
@@ -711,19 +718,27 @@ cudaError_t launch_decode(const DecodeParams& p, const CUtensorMap& kmap, const 
                           int D, int G, int grid, cudaStream_t stream) {
   cudaError_t e = cudaSuccess;
   if (grid < 1 || grid > kMaxGrid) return cudaErrorInvalidValue;
+  // launched as a programmatic dependent of the previous work on the stream
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
 #define LSERVE_DECODE_CASE(DD, GG)                                                        \
   if (D == DD && G == GG) {                                                               \
-    const int smem = DecLayout<DD, GG>::kBytes + 1024;                                    \
+    cfg.dynamicSmemBytes = DecLayout<DD, GG>::kBytes + 1024;                              \
     if (p.tile_rows == 64) {                                                              \
-      e = set_smem_once((const void*)decode_attn_kernel<DD, GG, 64>, smem);               \
+      e = set_smem_once((const void*)decode_attn_kernel<DD, GG, 64>, (int)cfg.dynamicSmemBytes); \
       if (e != cudaSuccess) return e;                                                     \
-      decode_attn_kernel<DD, GG, 64><<<grid, kThreads, smem, stream>>>(p, kmap, vmap);    \
-    } else {                                                                              \
-      e = set_smem_once((const void*)decode_attn_kernel<DD, GG, 32>, smem);               \
-      if (e != cudaSuccess) return e;                                                     \
-      decode_attn_kernel<DD, GG, 32><<<grid, kThreads, smem, stream>>>(p, kmap, vmap);    \
+      return cudaLaunchKernelEx(&cfg, decode_attn_kernel<DD, GG, 64>, p, kmap, vmap);     \
     }                                                                                     \
-    return cudaGetLastError();                                                            \
+    e = set_smem_once((const void*)decode_attn_kernel<DD, GG, 32>, (int)cfg.dynamicSmemBytes); \
+    if (e != cudaSuccess) return e;                                                       \
+    return cudaLaunchKernelEx(&cfg, decode_attn_kernel<DD, GG, 32>, p, kmap, vmap);       \
   }
   LSERVE_DECODE_CASE(64, 1)
   LSERVE_DECODE_CASE(64, 2)

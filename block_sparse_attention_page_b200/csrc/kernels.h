@@ -66,6 +66,7 @@ struct DecodeParams {
   int tiles_per_page;
   float scale_log2;       // softmax_scale * log2(e)
   uint64_t wait_limit;
+  int overlap_prologue;   // plan + first lookups may run before the preceding kernel ends
 };
 
 cudaError_t launch_page_stats(const StatsParams& p, int D, int max_logical_pages,

@@ -161,6 +161,36 @@ int lserve_sparse_decode_attn(const lserve_paged_desc* desc, const void* q, cons
                               size_t workspace_bytes, void* stream);
 
 /*
+ * lserve_sparse_decode_attn_ex -- lserve_sparse_decode_attn with launch flags.
+ * (No counterpart on the pages: a launch option of this library.)
+ *
+ * The kernel is launched as a programmatic dependent of the work before it on
+ * the stream: its thread blocks may start while that work is still finishing,
+ * and they wait for it to complete (with its memory visible) before reading
+ * q or the KV pools and before writing anything.  flags:
+ *   0                                  plan and page lookups also wait
+ *                                      (lserve_sparse_decode_attn does this).
+ *   LSERVE_DECODE_OVERLAP_PROLOGUE     the caller guarantees that the kernel
+ *                                      just before this call on the stream
+ *                                      writes none of block_table, ctx_lens,
+ *                                      head_kind, sel, sel_count: the split
+ *                                      plan and the first page lookups then
+ *                                      run before that kernel completes
+ *                                      (e.g. consecutive decode-attention
+ *                                      calls of different layers).
+ * Any other bit: LSERVE_ERR_INVALID_ARG.  Everything else as
+ * lserve_sparse_decode_attn.
+ */
+#define LSERVE_DECODE_OVERLAP_PROLOGUE 1u
+int lserve_sparse_decode_attn_ex(const lserve_paged_desc* desc, const void* q, const void* k_pool,
+                                 const void* v_pool, const int32_t* block_table,
+                                 const int32_t* ctx_lens, const uint8_t* head_kind,
+                                 const int32_t* sel, const int32_t* sel_count, int32_t top_k,
+                                 int32_t sink_tokens, int32_t local_tokens, float softmax_scale,
+                                 void* out, float* lse, uint32_t flags, void* workspace,
+                                 size_t workspace_bytes, void* stream);
+
+/*
  * lserve_blocksparse_prefill -- causal block-sparse flash attention for one
  * sequence.
  * [統一ブロックスパースアテンション: retrieval heads "block-sparse attention, static

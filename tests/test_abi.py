@@ -122,3 +122,18 @@ def test_workspace_size_of_select():
     d = _desc()
     assert lserve.workspace_size(lserve.OP_SELECT, d) >= 1 * 2 * 32 * 4
     assert lserve.workspace_size(99, d) == 0
+
+
+def test_decode_ex_rejects_unknown_flags():
+    d = _desc()
+    for flags in (2, 4, 0x80000000):
+        st = lserve.lib.lserve_sparse_decode_attn_ex(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, FAKE,
+                                                     FAKE, FAKE, FAKE, 8, 64, 256, 0.125, FAKE, None,
+                                                     flags, None, 0, None)
+        assert st == lserve.ERR_INVALID_ARG
+    # a known flag passes the flag check and fails later: on the missing
+    # workspace (GPU present) or on the device query (no GPU here)
+    st = lserve.lib.lserve_sparse_decode_attn_ex(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
+                                                 FAKE, FAKE, 8, 64, 256, 0.125, FAKE, None,
+                                                 lserve.DECODE_OVERLAP_PROLOGUE, None, 0, None)
+    assert st in (lserve.ERR_WORKSPACE, lserve.ERR_CUDA)

@@ -149,3 +149,39 @@ def test_workspace_too_small_is_rejected_on_device_shapes():
                                   buf.head_kind, buf.sel[0], buf.sel_count[0], w.top_k, w.sink,
                                   w.local, 0.1, buf.out, buf.lse, workspace=ws[:need - 512])
     assert e.value.status == lserve.ERR_WORKSPACE
+
+
+def test_overlapped_prologue_across_layers_is_bitwise_identical():
+    """Back-to-back decode calls of several layers, launched as programmatic
+    dependents with the prologue overlap (plan and lookups before the previous
+    layer's kernel ends), give exactly the outputs of plain calls."""
+    import math
+    w = synth.llama3_8b_decode()
+    layers = 3
+    buf = DecodeBuffers(w, layers=layers)
+    d = desc_of(w)
+    ws_sel = lserve.alloc_workspace(lserve.workspace_size(lserve.OP_SELECT, d, w.top_k))
+    for l in range(layers):
+        lserve.page_stats(d, buf.k_pools[l], buf.block_table, buf.ctx_lens, buf.head_kind, buf.stats[l])
+        lserve.page_select(d, buf.q, buf.stats[l], buf.block_table, buf.ctx_lens, buf.head_kind,
+                           w.top_k, buf.sel[l], buf.sel_count[l], workspace=ws_sel)
+    ws = lserve.alloc_workspace(lserve.workspace_size(lserve.OP_DECODE, d, w.top_k))
+    scale = 1.0 / math.sqrt(w.D)
+
+    def run(overlap):
+        outs = [torch.zeros_like(buf.out) for _ in range(layers)]
+        lses = [torch.zeros_like(buf.lse) for _ in range(layers)]
+        for rep in range(2):
+            for l in range(layers):
+                lserve.sparse_decode_attn(d, buf.q, buf.k_pools[l], buf.v_pools[l], buf.block_table,
+                                          buf.ctx_lens, buf.head_kind, buf.sel[l], buf.sel_count[l],
+                                          w.top_k, w.sink, w.local, scale, outs[l], lses[l],
+                                          workspace=ws, overlap_prologue=overlap)
+        torch.cuda.synchronize()
+        assert lserve.read_device_status() == lserve.OK
+        return outs, lses
+
+    plain_o, plain_l = run(False)
+    ov_o, ov_l = run(True)
+    for l in range(layers):
+        assert torch.equal(plain_o[l], ov_o[l]) and torch.equal(plain_l[l], ov_l[l])
