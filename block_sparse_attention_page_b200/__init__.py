@@ -31,6 +31,7 @@ EXPORTED = [
     "lserve_blocksparse_prefill", "lserve_workspace_size", "lserve_read_device_status",
     "lserve_set_wait_limit_cycles", "lserve_debug_wait_timeout", "lserve_status_string",
     "lserve_bounds_checked", "lserve_page_select_noalloc", "lserve_sparse_decode_attn_ex",
+    "lserve_decode_append",
 ]
 DECODE_OVERLAP_PROLOGUE = 1
 
@@ -70,6 +71,7 @@ def _load(path):
     lib.lserve_sparse_decode_attn_ex.argtypes = [P(PagedDesc), vp, vp, vp, vp, vp, vp, vp, vp, i32,
                                                  i32, i32, ctypes.c_float, vp, vp, ctypes.c_uint32,
                                                  vp, sz, vp]
+    lib.lserve_decode_append.argtypes = [P(PagedDesc), vp, vp, vp, vp, vp, vp, vp, vp, vp]
     lib.lserve_blocksparse_prefill.argtypes = [P(PrefillDesc), vp, vp, vp, vp, ctypes.c_float, vp, vp,
                                                vp, sz, vp]
     lib.lserve_page_select_noalloc.argtypes = [P(PagedDesc), vp, vp, vp, vp, vp, i32, vp, vp, vp]
@@ -166,6 +168,15 @@ def sparse_decode_attn(desc, q, k_pool, v_pool, block_table, ctx_lens, head_kind
         ctypes.byref(desc), _ptr(q), _ptr(k_pool), _ptr(v_pool), _ptr(block_table), _ptr(ctx_lens),
         _ptr(head_kind), _ptr(sel), _ptr(sel_count), top_k, sink_tokens, local_tokens,
         float(softmax_scale), _ptr(out), _ptr(lse), _ptr(workspace), ws_bytes, _stream(stream)))
+
+
+def decode_append(desc, k_new, v_new, block_table, ctx_lens, head_kind, k_pool, v_pool, stats_pool,
+                  stream=None):
+    """lserve_decode_append: write each sequence's new K/V row at position
+    ctx_lens[b] and update that logical page's k_min / k_max (retrieval heads)."""
+    _check("lserve_decode_append", lib.lserve_decode_append(
+        ctypes.byref(desc), _ptr(k_new), _ptr(v_new), _ptr(block_table), _ptr(ctx_lens),
+        _ptr(head_kind), _ptr(k_pool), _ptr(v_pool), _ptr(stats_pool), _stream(stream)))
 
 
 def blocksparse_prefill(desc, q, k, v, head_kind_host, softmax_scale, out, lse=None, workspace=None,

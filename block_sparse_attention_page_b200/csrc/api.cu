@@ -273,6 +273,38 @@ int lserve_page_stats(const lserve_paged_desc* desc, const void* k_pool, const i
   return cuda_status(launch_page_stats(p, desc->head_dim, (int)max_lp, static_cast<cudaStream_t>(stream)));
 }
 
+int lserve_decode_append(const lserve_paged_desc* desc, const void* k_new, const void* v_new,
+                         const int32_t* block_table, const int32_t* ctx_lens,
+                         const uint8_t* head_kind, void* k_pool, void* v_pool, void* stats_pool,
+                         void* stream) {
+  if (!valid_paged(desc)) return LSERVE_ERR_INVALID_ARG;
+  if (!k_new || !v_new || !block_table || !ctx_lens || !head_kind || !k_pool || !v_pool || !stats_pool)
+    return LSERVE_ERR_INVALID_ARG;
+  if (!aligned(k_new, 16) || !aligned(v_new, 16) || !aligned(k_pool, 16) || !aligned(v_pool, 16) ||
+      !aligned(stats_pool, 16) || !aligned(block_table, 4) || !aligned(ctx_lens, 4))
+    return LSERVE_ERR_INVALID_ARG;
+  const int st = supported_paged(desc);
+  if (st != LSERVE_OK) return st;
+  AppendParams p;
+  p.k_new = static_cast<const __nv_bfloat16*>(k_new);
+  p.v_new = static_cast<const __nv_bfloat16*>(v_new);
+  p.block_table = block_table;
+  p.ctx_lens = ctx_lens;
+  p.head_kind = head_kind;
+  p.k_pool = static_cast<__nv_bfloat16*>(k_pool);
+  p.v_pool = static_cast<__nv_bfloat16*>(v_pool);
+  p.stats_pool = static_cast<__nv_bfloat16*>(stats_pool);
+  p.batch = desc->batch;
+  p.num_kv_heads = desc->num_kv_heads;
+  p.logical_page = desc->logical_page;
+  p.physical_page = desc->physical_page;
+  p.max_pages = desc->max_pages_per_seq;
+  p.num_pool_pages = desc->num_pool_pages;
+  p.status = device_status_word();
+  if (!p.status) return LSERVE_ERR_CUDA;
+  return cuda_status(launch_decode_append(p, desc->head_dim, static_cast<cudaStream_t>(stream)));
+}
+
 int lserve_page_select(const lserve_paged_desc* desc, const void* q, const void* stats_pool,
                        const int32_t* block_table, const int32_t* ctx_lens, const uint8_t* head_kind,
                        int32_t top_k, int32_t* sel, int32_t* sel_count, float* phys_scores,

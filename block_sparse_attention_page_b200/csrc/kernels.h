@@ -69,6 +69,22 @@ struct DecodeParams {
   int overlap_prologue;   // plan + first lookups may run before the preceding kernel ends
 };
 
+// lserve_decode_append: one warp per (sequence, KV head)
+constexpr int kAppendWarps = 8;
+struct AppendParams {
+  const __nv_bfloat16* k_new;   // [B][H_kv][D]
+  const __nv_bfloat16* v_new;   // [B][H_kv][D]
+  const int32_t* block_table;
+  const int32_t* ctx_lens;      // position of the new token of each sequence
+  const uint8_t* head_kind;
+  __nv_bfloat16* k_pool;
+  __nv_bfloat16* v_pool;
+  __nv_bfloat16* stats_pool;
+  unsigned int* status;
+  int batch, num_kv_heads, logical_page, physical_page, max_pages, num_pool_pages;
+};
+cudaError_t launch_decode_append(const AppendParams& p, int D, cudaStream_t stream);
+
 cudaError_t launch_page_stats(const StatsParams& p, int D, int max_logical_pages,
                               cudaStream_t stream);
 cudaError_t launch_page_select(const SelectParams& p, int D, cudaStream_t stream);

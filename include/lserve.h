@@ -106,6 +106,32 @@ int lserve_page_stats(const lserve_paged_desc* desc, const void* k_pool, const i
                       int32_t first_logical_page, void* stream);
 
 /*
+ * lserve_decode_append -- cache maintenance of one decode step: append each
+ * sequence's new token to the paged KV pools and keep the page statistics.
+ * [技術的詳細 › 動的スパーシティ: the k_min / k_max statistics of logical page j;
+ *  階層的ページング: logical pages of N_L tokens inside physical pages.  The pages
+ *  describe the statistics, not how they are kept during decode: here a page's
+ *  statistics after an append equal those lserve_page_stats would build.]
+ *
+ * For every sequence b and KV head h the token at position pos = ctx_lens[b]
+ * (the length BEFORE this step; the caller advances ctx_lens afterwards) is
+ * written: k_new[b][h][:] into k_pool at pool id block_table[b][pos / N_P],
+ * row pos % N_P, and v_new likewise into v_pool.  For retrieval heads the
+ * statistics of logical page pos / N_L (sub-page (pos % N_P) / N_L of that
+ * pool page) become k_min = k_max = k_new when pos % N_L == 0, else the
+ * elementwise min / max of the stored values and k_new (exact in bf16).
+ * Streaming heads' statistics are not touched.
+ *   k_new, v_new  bf16 [B][H_kv][D], 16-byte aligned.
+ * The block table must already hold the page of pos.  A position outside
+ * [0, max_pages_per_seq * N_P) or a bad pool id skips that sequence and sets
+ * LSERVE_ERR_BOUNDS (lserve_read_device_status).  No workspace.
+ */
+int lserve_decode_append(const lserve_paged_desc* desc, const void* k_new, const void* v_new,
+                         const int32_t* block_table, const int32_t* ctx_lens,
+                         const uint8_t* head_kind, void* k_pool, void* v_pool, void* stats_pool,
+                         void* stream);
+
+/*
  * lserve_page_select -- query-centric page scores and top-K physical pages.
  * [技術的詳細 › 動的スパーシティ, the equation
  *    S^j = sum_{i=1..D} max(q[i] * k_max^j[i], q[i] * k_min^j[i]);
