@@ -126,6 +126,15 @@ def decode_traffic():
         return None
 
 
+def append_bytes(w):
+    """lserve_decode_append: read k_new / v_new and write one K and V row per
+    (sequence, KV head); read + write the two statistics rows of the retrieval
+    heads' current logical page."""
+    rows = w.B * w.H_kv * w.D * 2
+    retrieval = int(sum(1 for h in range(w.H_kv) if w.head_kind[h] == 0)) * w.B
+    return 2 * 2 * rows + retrieval * 2 * w.D * 2 * 2
+
+
 # --- clocks sampling ----------------------------------------------------------
 
 class ClockSampler:
@@ -306,6 +315,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--layers", type=int, default=LAYERS,
                     help="layer replicas (fewer = a small case for profiling; < 32 may fit in L2)")
+    ap.add_argument("--no-mha", action="store_true", help="skip the MHA decode stage")
     ap.add_argument("--prefill-only", action="store_true",
                     help="run only the prefill stage (profiling)")
     ap.add_argument("--prefill-seq", type=int, default=None,
@@ -385,6 +395,27 @@ def main():
     g_select_only = capture(lambda: [select(l) for l in range(LAYERS)])
     g_stats = capture(stats_all)
 
+    # decode-time cache maintenance (lserve_decode_append), timed alone: each
+    # sequence's last token is written again with its own K/V (position n - 1,
+    # inside the block table), which leaves the cache and statistics unchanged
+    lens_last = (buf.ctx_lens - 1).to(torch.int32)
+    last = [(int(w.block_table[b, (int(w.ctx_lens[b]) - 1) // w.N_P]),
+             (int(w.ctx_lens[b]) - 1) % w.N_P) for b in range(w.B)]
+    k_last = [torch.stack([buf.k_pools[l][pid, :, r] for pid, r in last]).contiguous()
+              for l in range(LAYERS)]
+    v_last = [torch.stack([buf.v_pools[l][pid, :, r] for pid, r in last]).contiguous()
+              for l in range(LAYERS)]
+
+    def append_all():
+        for l in range(LAYERS):
+            lserve.decode_append(d, k_last[l], v_last[l], buf.block_table, lens_last, buf.head_kind,
+                                 buf.k_pools[l], buf.v_pools[l], buf.stats[l])
+    with torch.cuda.stream(stream):
+        append_all()
+    torch.cuda.synchronize()
+    assert lserve.read_device_status(stream) == lserve.OK
+    g_append = capture(append_all)
+
     def run_steps(k0, k, ev=None):
         # ev: event pairs recorded around the attention-only replays, so that the
         # average attention launch is measured inside the timed region itself
@@ -439,6 +470,8 @@ def main():
         t_attn = t_attn_region  # the launches of the timed region themselves
     t_sel = timed(lambda: g_select_only.replay(), reps) / (reps * LAYERS)
     t_stats = timed(lambda: g_stats.replay(), 3) / (3 * LAYERS)
+    t_app = timed(lambda: g_append.replay(), reps) / (reps * LAYERS)
+    app_bytes = append_bytes(w)
     sb = stats_build_bytes(w)
     attn_gbs = acct["attn"] / t_attn / 1e9
     stages = {
@@ -448,8 +481,10 @@ def main():
                       "frac": acct["select"] / t_sel / 1e9 / hbm_peak, "bytes": acct["select"]},
         "stats_build": {"us": t_stats * 1e6, "GB/s": sb / t_stats / 1e9,
                         "frac": sb / t_stats / 1e9 / hbm_peak, "bytes": sb},
+        "append": {"us": t_app * 1e6, "GB/s": app_bytes / t_app / 1e9, "bytes": app_bytes,
+                   "note": "lserve_decode_append per layer; launch-latency bound (16 KB of K/V)"},
     }
-    del g_stats
+    del g_stats, g_append
 
     # e2e: per step, copy the step's q (all layers) host->device from pinned memory,
     # run the step, read every layer's output back to pinned host memory
@@ -504,6 +539,8 @@ def main():
     buf = None
     torch.cuda.empty_cache()
 
+    if not args.no_mha:
+        result["stages"]["attention_mha"] = mha_stage(lserve, synth, dev, stream, hbm_peak, timed)
     if not args.no_prefill:
         result["stages"]["prefill"] = prefill_stage(lserve, synth, dev, stream, tc_peak, timed,
                                                     args.prefill_seq)
@@ -519,6 +556,52 @@ def main():
         torch.distributed.barrier()
         torch.distributed.destroy_process_group()
     return 0
+
+
+def mha_stage(lserve, synth, dev, stream, hbm_peak, timed, layers=8):
+    """Decode attention on the Llama-2-7B-shaped MHA layer (G = 1), alone:
+    `layers` replicas back to back (each touches ~155 MB, more than L2)."""
+    import torch
+    from synth.device import DecodeBuffers
+    w = synth.llama2_7b_mha_decode()
+    buf = DecodeBuffers(w, device=dev, layers=layers)
+    d = lserve.paged_desc(w.B, w.H_q, w.H_kv, w.D, w.N_L, w.N_P, w.max_pages, w.num_pool_pages)
+    wss = lserve.alloc_workspace(lserve.workspace_size(lserve.OP_SELECT, d, w.top_k), device=dev)
+    wsd = lserve.alloc_workspace(lserve.workspace_size(lserve.OP_DECODE, d, w.top_k), device=dev)
+    outs = [torch.empty_like(buf.out) for _ in range(layers)]
+    scale = 1.0 / math.sqrt(w.D)
+    with torch.cuda.stream(stream):
+        for l in range(layers):
+            lserve.page_stats(d, buf.k_pools[l], buf.block_table, buf.ctx_lens, buf.head_kind,
+                              buf.stats[l])
+            lserve.page_select(d, buf.q, buf.stats[l], buf.block_table, buf.ctx_lens, buf.head_kind,
+                               w.top_k, buf.sel[l], buf.sel_count[l], workspace=wss)
+    torch.cuda.synchronize()
+
+    def attn_all():
+        for l in range(layers):
+            lserve.sparse_decode_attn(d, buf.q, buf.k_pools[l], buf.v_pools[l], buf.block_table,
+                                      buf.ctx_lens, buf.head_kind, buf.sel[l], buf.sel_count[l],
+                                      w.top_k, w.sink, w.local, scale, outs[l], None, workspace=wsd,
+                                      overlap_prologue=l > 0)
+    with torch.cuda.stream(stream):
+        attn_all()
+    torch.cuda.synchronize()
+    assert lserve.read_device_status(stream) == lserve.OK
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        attn_all()
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            g.replay()
+    reps = 20
+    t = timed(lambda: g.replay(), reps) / (reps * layers)
+    bts = decode_bytes(w)["attn"]
+    del g
+    return {"us": t * 1e6, "GB/s": bts / t / 1e9, "frac": bts / t / 1e9 / hbm_peak, "bytes": bts,
+            "workload": f"{w.name}: B={w.B} n={int(w.ctx_lens[0])} H_q={w.H_q} H_kv={w.H_kv} "
+                        f"D={w.D} N_L={w.N_L} N_P={w.N_P} top_k={w.top_k} sink={w.sink} "
+                        f"local={w.local}"}
 
 
 def prefill_stage(lserve, synth, dev, stream, tc_peak, timed, seq=None):

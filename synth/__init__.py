@@ -340,6 +340,20 @@ def long_decode_256k() -> DecodeWorkload:
     return w
 
 
+def llama2_7b_mha_decode() -> DecodeWorkload:
+    """Llama-2-7B-shaped (MHA, G = 1) decode layer: B=4, n=32K, 32 query = 32 KV
+    heads, D=128, N_L=16, N_P=64, top-K 64 pages (4K tokens), sink 128 + local
+    512 for the streaming half; K/V ~ N(0,1) * s_c, s_c ~ U[0.5, 2] per
+    (KV head, channel)."""
+    seed = 1006
+    w = decode_workload(4, 32, 32, 128, 16, 64, 64, 128, 512, [32768] * 4, seed,
+                        name="llama2_7b_mha_decode")
+    H, D = w.H_kv, w.D
+    w.k_scale = 0.5 + 1.5 * uniform_array(tensor_key(seed, TAG_KSCALE), H * D).reshape(H, D)
+    w.v_scale = 0.5 + 1.5 * uniform_array(tensor_key(seed, TAG_VSCALE), H * D).reshape(H, D)
+    return w
+
+
 def mixed_batch_decode() -> DecodeWorkload:
     """Batched mixed-length decode: B=32, n_b ~ U{8192..131072}, 32 q / 8 KV
     heads, D=128, N_L=16, N_P=64, pages shuffled through the block table,
@@ -407,5 +421,6 @@ DECODE_CONFIGS = {
     "llama3_8b_decode": llama3_8b_decode,
     "long_decode_256k": long_decode_256k,
     "mixed_batch_decode": mixed_batch_decode,
+    "llama2_7b_mha_decode": llama2_7b_mha_decode,
 }
 PREFILL_CONFIGS = {"tiny": tiny_prefill, "prefill_128k": prefill_128k}

@@ -92,6 +92,19 @@ def test_mixed_batch_decode_sampled_pairs():
     assert np.all(np.isfinite(res["out"]))
 
 
+def test_llama2_7b_mha_decode_sampled_pairs():
+    """The MHA (G = 1) shape of the pages' second model: every KV head has one
+    query head; retrieval heads 0-15, streaming 16-31."""
+    w = synth.llama2_7b_mha_decode()
+    res = run_decode_path(DecodeBuffers(w))
+    rng = np.random.default_rng(6)
+    pairs = [(int(b), int(h)) for b, h in zip(rng.integers(0, w.B, 16), rng.integers(0, w.H_kv, 16))]
+    pairs += [(0, 0), (w.B - 1, w.H_kv - 1), (1, 15), (2, 16)]
+    for b, h in pairs:
+        check_pair(w, res, b, h)
+    assert np.all(np.isfinite(res["out"]))
+
+
 def test_shuffled_pool_equals_identity_layout():
     a = synth.decode_workload(4, 8, 2, 128, 16, 64, 8, 64, 256, [3000, 5000, 64, 9000], seed=99)
     b = synth.decode_workload(4, 8, 2, 128, 16, 64, 8, 64, 256, [3000, 5000, 64, 9000], seed=99,
