@@ -638,12 +638,35 @@ def prefill_stage(lserve, synth, dev, stream, tc_peak, timed, seq=None):
             run()
         torch.cuda.synchronize()
         t = timed(run, 3) / 3
+        # the prefilled sequence handed to the paged decode cache: K/V into the
+        # pools and the retrieval heads' page statistics in one pass
+        N_L, N_P = 16, 64
+        npages = -(-w.T // N_P)
+        pd = lserve.paged_desc(1, w.H_q, w.H_kv, w.D, N_L, N_P, npages, npages)
+        kp = torch.empty((npages, w.H_kv, N_P, w.D), dtype=torch.bfloat16, device=dev)
+        vp = torch.empty_like(kp)
+        sp = torch.empty((npages, w.H_kv, N_P // N_L, 2, w.D), dtype=torch.bfloat16, device=dev)
+        bt = torch.randperm(npages, generator=torch.Generator().manual_seed(5)).to(torch.int32).to(dev)
+        hk = torch.from_numpy(np.ascontiguousarray(w.head_kind)).to(dev)
+
+        def to_pages():
+            lserve.prefill_to_pages(pd, w.T, pb.k, pb.v, bt, hk, kp, vp, sp, stream=stream)
+        with torch.cuda.stream(stream):
+            to_pages()
+        torch.cuda.synchronize()
+        t_tp = timed(to_pages, 3) / 3
+        retr = int(sum(1 for h in range(w.H_kv) if w.head_kind[h] == 0))
+        tp_bytes = 2 * 2 * w.T * w.H_kv * w.D * 2 + retr * (-(-w.T // N_L)) * 2 * w.D * 2
+        del kp, vp, sp
     except lserve.LServeError as e:
         return {"unavailable": str(e)}
     flops = oracle.prefill_flops(w.T, w.H_q, w.H_kv, w.D, w.block, w.head_kind, w.sink_blocks,
                                  w.local_blocks)
     tf = flops / t / 1e12
     return {"ms": t * 1e3, "TFLOP/s": tf, "frac": tf / tc_peak, "flops": flops,
+            "to_pages": {"us": t_tp * 1e6, "GB/s": tp_bytes / t_tp / 1e9, "bytes": tp_bytes,
+                         "what": "lserve_prefill_to_pages: K/V into the paged pools (N_P=64) "
+                                 "+ page statistics (N_L=16), one pass"},
             "workload": f"{w.name}: T={w.T} H_q={w.H_q} H_kv={w.H_kv} D={w.D} block={w.block} "
                         f"Lambda({w.sink_blocks},{w.local_blocks}) on KV heads 4-7"}
 

@@ -31,7 +31,7 @@ EXPORTED = [
     "lserve_blocksparse_prefill", "lserve_workspace_size", "lserve_read_device_status",
     "lserve_set_wait_limit_cycles", "lserve_debug_wait_timeout", "lserve_status_string",
     "lserve_bounds_checked", "lserve_page_select_noalloc", "lserve_sparse_decode_attn_ex",
-    "lserve_decode_append",
+    "lserve_decode_append", "lserve_prefill_to_pages",
 ]
 DECODE_OVERLAP_PROLOGUE = 1
 
@@ -72,6 +72,7 @@ def _load(path):
                                                  i32, i32, ctypes.c_float, vp, vp, ctypes.c_uint32,
                                                  vp, sz, vp]
     lib.lserve_decode_append.argtypes = [P(PagedDesc), vp, vp, vp, vp, vp, vp, vp, vp, vp]
+    lib.lserve_prefill_to_pages.argtypes = [P(PagedDesc), i32, vp, vp, vp, vp, vp, vp, vp, vp]
     lib.lserve_blocksparse_prefill.argtypes = [P(PrefillDesc), vp, vp, vp, vp, ctypes.c_float, vp, vp,
                                                vp, sz, vp]
     lib.lserve_page_select_noalloc.argtypes = [P(PagedDesc), vp, vp, vp, vp, vp, i32, vp, vp, vp]
@@ -177,6 +178,15 @@ def decode_append(desc, k_new, v_new, block_table, ctx_lens, head_kind, k_pool, 
     _check("lserve_decode_append", lib.lserve_decode_append(
         ctypes.byref(desc), _ptr(k_new), _ptr(v_new), _ptr(block_table), _ptr(ctx_lens),
         _ptr(head_kind), _ptr(k_pool), _ptr(v_pool), _ptr(stats_pool), _stream(stream)))
+
+
+def prefill_to_pages(desc, seq_len, k, v, block_table, head_kind, k_pool, v_pool, stats_pool,
+                     stream=None):
+    """lserve_prefill_to_pages: one sequence's prefill K/V ([T][H_kv][D]) into the
+    paged pools, with the retrieval heads' page statistics, in one pass."""
+    _check("lserve_prefill_to_pages", lib.lserve_prefill_to_pages(
+        ctypes.byref(desc), int(seq_len), _ptr(k), _ptr(v), _ptr(block_table), _ptr(head_kind),
+        _ptr(k_pool), _ptr(v_pool), _ptr(stats_pool), _stream(stream)))
 
 
 def blocksparse_prefill(desc, q, k, v, head_kind_host, softmax_scale, out, lse=None, workspace=None,

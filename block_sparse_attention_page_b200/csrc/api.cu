@@ -273,6 +273,40 @@ int lserve_page_stats(const lserve_paged_desc* desc, const void* k_pool, const i
   return cuda_status(launch_page_stats(p, desc->head_dim, (int)max_lp, static_cast<cudaStream_t>(stream)));
 }
 
+int lserve_prefill_to_pages(const lserve_paged_desc* desc, int32_t seq_len, const void* k,
+                            const void* v, const int32_t* block_table, const uint8_t* head_kind,
+                            void* k_pool, void* v_pool, void* stats_pool, void* stream) {
+  if (!valid_paged(desc)) return LSERVE_ERR_INVALID_ARG;
+  if (seq_len < 0) return LSERVE_ERR_INVALID_ARG;
+  if (!k || !v || !block_table || !head_kind || !k_pool || !v_pool || !stats_pool)
+    return LSERVE_ERR_INVALID_ARG;
+  if (!aligned(k, 16) || !aligned(v, 16) || !aligned(k_pool, 16) || !aligned(v_pool, 16) ||
+      !aligned(stats_pool, 16) || !aligned(block_table, 4))
+    return LSERVE_ERR_INVALID_ARG;
+  const int st = supported_paged(desc);
+  if (st != LSERVE_OK) return st;
+  if ((long long)seq_len > (long long)desc->max_pages_per_seq * desc->physical_page)
+    return LSERVE_ERR_INVALID_ARG;
+  if (seq_len == 0) return LSERVE_OK;
+  ToPagesParams p;
+  p.k = static_cast<const __nv_bfloat16*>(k);
+  p.v = static_cast<const __nv_bfloat16*>(v);
+  p.block_table = block_table;
+  p.head_kind = head_kind;
+  p.k_pool = static_cast<__nv_bfloat16*>(k_pool);
+  p.v_pool = static_cast<__nv_bfloat16*>(v_pool);
+  p.stats_pool = static_cast<__nv_bfloat16*>(stats_pool);
+  p.seq_len = seq_len;
+  p.num_kv_heads = desc->num_kv_heads;
+  p.logical_page = desc->logical_page;
+  p.physical_page = desc->physical_page;
+  p.max_pages = desc->max_pages_per_seq;
+  p.num_pool_pages = desc->num_pool_pages;
+  p.status = device_status_word();
+  if (!p.status) return LSERVE_ERR_CUDA;
+  return cuda_status(launch_prefill_to_pages(p, desc->head_dim, static_cast<cudaStream_t>(stream)));
+}
+
 int lserve_decode_append(const lserve_paged_desc* desc, const void* k_new, const void* v_new,
                          const int32_t* block_table, const int32_t* ctx_lens,
                          const uint8_t* head_kind, void* k_pool, void* v_pool, void* stats_pool,

@@ -85,6 +85,21 @@ struct AppendParams {
 };
 cudaError_t launch_decode_append(const AppendParams& p, int D, cudaStream_t stream);
 
+// lserve_prefill_to_pages: one warp per (logical page, KV head)
+constexpr int kToPagesWarps = 8;
+struct ToPagesParams {
+  const __nv_bfloat16* k;      // [T][H_kv][D]
+  const __nv_bfloat16* v;      // [T][H_kv][D]
+  const int32_t* block_table;  // [max_pages] of this sequence
+  const uint8_t* head_kind;
+  __nv_bfloat16* k_pool;
+  __nv_bfloat16* v_pool;
+  __nv_bfloat16* stats_pool;
+  unsigned int* status;
+  int seq_len, num_kv_heads, logical_page, physical_page, max_pages, num_pool_pages;
+};
+cudaError_t launch_prefill_to_pages(const ToPagesParams& p, int D, cudaStream_t stream);
+
 cudaError_t launch_page_stats(const StatsParams& p, int D, int max_logical_pages,
                               cudaStream_t stream);
 cudaError_t launch_page_select(const SelectParams& p, int D, cudaStream_t stream);

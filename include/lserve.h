@@ -106,6 +106,28 @@ int lserve_page_stats(const lserve_paged_desc* desc, const void* k_pool, const i
                       int32_t first_logical_page, void* stream);
 
 /*
+ * lserve_prefill_to_pages -- hand a prefilled sequence to the paged decode
+ * cache: K / V into the pools and the page statistics, in one pass over K.
+ * [技術的詳細 › 動的スパーシティ: k_min^j / k_max^j of logical page j; 階層的ページング:
+ *  logical pages of N_L tokens inside physical pages of N_P tokens.  The pages
+ *  do not say where the statistics are built; building them while K is read
+ *  once saves lserve_page_stats' separate pass over the cache.]
+ *
+ * One sequence of seq_len tokens: k, v bf16 [seq_len][H_kv][D] (the layout
+ * lserve_blocksparse_prefill reads), block_table int32 [max_pages_per_seq]
+ * (this sequence's page ordinal -> pool id; must cover seq_len tokens).
+ * Token t of head h goes to pool id block_table[t / N_P], row t % N_P, of
+ * k_pool / v_pool; for retrieval heads every logical page j of the sequence
+ * gets k_min / k_max over its valid tokens in stats_pool (pool id
+ * block_table[j / g], sub-page j % g) -- exactly what lserve_page_stats writes.
+ * desc->batch is not used.  A bad pool id skips that page and sets
+ * LSERVE_ERR_BOUNDS.  seq_len = 0 does nothing.  No workspace.
+ */
+int lserve_prefill_to_pages(const lserve_paged_desc* desc, int32_t seq_len, const void* k,
+                            const void* v, const int32_t* block_table, const uint8_t* head_kind,
+                            void* k_pool, void* v_pool, void* stats_pool, void* stream);
+
+/*
  * lserve_decode_append -- cache maintenance of one decode step: append each
  * sequence's new token to the paged KV pools and keep the page statistics.
  * [技術的詳細 › 動的スパーシティ: the k_min / k_max statistics of logical page j;
