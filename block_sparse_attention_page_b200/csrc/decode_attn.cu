@@ -565,35 +565,97 @@ decode_attn_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
   };
 
   // Merge every partial (o, m, l) of a pair with log-sum-exp weights; the
-  // counter goes back to zero for the next call.
+  // counter goes back to zero for the next call.  The (m, l) of all segments
+  // are loaded at once into the (now free) merge buffer, the weights
+  // 2^(m_s - M) computed once per (segment, head), and each output sums its
+  // segments with independent loads -- a couple of L2 round trips, however
+  // many CTAs the pair spans.
   auto merge_partials = [&](int pair) {
     const int b = pair / p.num_kv_heads, h = pair - b * p.num_kv_heads;
     const int c_first = cta_of(cst, off[pair], NC), c_last = cta_of(cst, off[pair + 1] - 1, NC);
-#pragma unroll
-    for (int i = 0; i < NOUT; ++i) {
-      const int j = tid + i * kConsumerThreads;
-      if (j >= G * D) continue;
-      const int g = j / D, c = j - g * D;
-      float M = -INFINITY, o = 0.f, lsum = 0.f;
-#pragma unroll 4
-      for (int cc = c_first; cc <= c_last; ++cc) {
-        const bool busy = cta_busy(cst, cc);  // predicated, independent loads
-        const size_t sl = (size_t)cc + pair;
-        const float2 ml = busy ? __ldcg(reinterpret_cast<const float2*>(p.part_ml + (sl * G + g) * 2))
-                               : make_float2(-INFINITY, 0.f);
-        const float os = busy ? __ldcg(p.part_o + (sl * G + g) * D + c) : 0.f;
-        const float Mn = fmaxf(M, ml.x);
-        if (Mn == -INFINITY) continue;
-        const float sc = exp2f(M - Mn), wt = exp2f(ml.x - Mn);
-        o = o * sc + wt * os;
-        lsum = lsum * sc + wt * ml.y;
-        M = Mn;
+    const int nc = c_last - c_first + 1;
+    constexpr int kCap = L::kOw / 8;  // float2 slots of the merge buffer
+    float2* wml = reinterpret_cast<float2*>(ow);  // [segment][head]: (m, l), then (weight, l)
+    float* hm = msc;                              // [head] max, [G + head] sum of weights * l
+    if (nc * G <= kCap) {
+      for (int i = tid; i < nc * G; i += kConsumerThreads) {
+        const int cc = c_first + i / G, g = i - (i / G) * G;
+        wml[i] = cta_busy(cst, cc)
+                     ? __ldcg(reinterpret_cast<const float2*>(p.part_ml + (((size_t)cc + pair) * G + g) * 2))
+                     : make_float2(-INFINITY, 0.f);
       }
-      const size_t qh = (size_t)b * p.num_q_heads + (size_t)h * G + g;
-      const bool empty_row = !(lsum > 0.f);
-      p.out[qh * D + c] = __float2bfloat16_rn(empty_row ? 0.f : o / lsum);
-      if (c == 0 && p.lse)
-        p.lse[qh] = empty_row ? -INFINITY : (M + __log2f(lsum)) * 0.69314718055994530942f;
+      named_sync(kBarConsumers, kConsumerThreads);
+      if (tid < G) {
+        float M = -INFINITY;
+        for (int sgi = 0; sgi < nc; ++sgi) M = fmaxf(M, wml[sgi * G + tid].x);
+        hm[tid] = M;
+      }
+      named_sync(kBarConsumers, kConsumerThreads);
+      for (int i = tid; i < nc * G; i += kConsumerThreads) {
+        const float M = hm[i % G], m = wml[i].x;
+        wml[i].x = (m == -INFINITY) ? 0.f : exp2f(m - M);
+      }
+      named_sync(kBarConsumers, kConsumerThreads);
+      if (tid < G) {
+        float l = 0.f;
+        for (int sgi = 0; sgi < nc; ++sgi) l += wml[sgi * G + tid].x * wml[sgi * G + tid].y;
+        hm[G + tid] = l;
+      }
+      named_sync(kBarConsumers, kConsumerThreads);
+#pragma unroll
+      for (int i = 0; i < NOUT; ++i) {
+        const int j = tid + i * kConsumerThreads;
+        if (j >= G * D) continue;
+        const int g = j / D, c = j - g * D;
+        float o = 0.f;
+        constexpr int kBatch = 8;  // independent loads in flight per thread
+        for (int s0 = 0; s0 < nc; s0 += kBatch) {
+          float os[kBatch];
+#pragma unroll
+          for (int u = 0; u < kBatch; ++u) {
+            const int sgi = s0 + u;
+            os[u] = (sgi < nc && wml[min(sgi, nc - 1) * G + g].x != 0.f)
+                        ? __ldcg(p.part_o + (((size_t)(c_first + sgi) + pair) * G + g) * D + c)
+                        : 0.f;
+          }
+#pragma unroll
+          for (int u = 0; u < kBatch; ++u)
+            if (s0 + u < nc) o += wml[(s0 + u) * G + g].x * os[u];
+        }
+        const float lsum = hm[G + g], M = hm[g];
+        const size_t qh = (size_t)b * p.num_q_heads + (size_t)h * G + g;
+        const bool empty_row = !(lsum > 0.f);
+        p.out[qh * D + c] = __float2bfloat16_rn(empty_row ? 0.f : o / lsum);
+        if (c == 0 && p.lse)
+          p.lse[qh] = empty_row ? -INFINITY : (M + __log2f(lsum)) * 0.69314718055994530942f;
+      }
+      named_sync(kBarConsumers, kConsumerThreads);  // the buffer is free for the next merge
+    } else {  // more segments than the buffer holds: one segment at a time
+#pragma unroll
+      for (int i = 0; i < NOUT; ++i) {
+        const int j = tid + i * kConsumerThreads;
+        if (j >= G * D) continue;
+        const int g = j / D, c = j - g * D;
+        float M = -INFINITY, o = 0.f, lsum = 0.f;
+        for (int cc = c_first; cc <= c_last; ++cc) {
+          const bool busy = cta_busy(cst, cc);
+          const size_t sl = (size_t)cc + pair;
+          const float2 ml = busy ? __ldcg(reinterpret_cast<const float2*>(p.part_ml + (sl * G + g) * 2))
+                                 : make_float2(-INFINITY, 0.f);
+          const float os = busy ? __ldcg(p.part_o + (sl * G + g) * D + c) : 0.f;
+          const float Mn = fmaxf(M, ml.x);
+          if (Mn == -INFINITY) continue;
+          const float sc = exp2f(M - Mn), wt = exp2f(ml.x - Mn);
+          o = o * sc + wt * os;
+          lsum = lsum * sc + wt * ml.y;
+          M = Mn;
+        }
+        const size_t qh = (size_t)b * p.num_q_heads + (size_t)h * G + g;
+        const bool empty_row = !(lsum > 0.f);
+        p.out[qh * D + c] = __float2bfloat16_rn(empty_row ? 0.f : o / lsum);
+        if (c == 0 && p.lse)
+          p.lse[qh] = empty_row ? -INFINITY : (M + __log2f(lsum)) * 0.69314718055994530942f;
+      }
     }
     if (tid == 0) p.counters[pair] = 0u;
   };
