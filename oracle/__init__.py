@@ -31,6 +31,10 @@ Readings where the pages are silent (each is listed in the design notes):
      [i - local + 1, i] (the diagonal counts as local).   (parity unpinned)
   R7 retrieval heads in prefill are dense causal.
   R8 softmax scale is a parameter (1/sqrt(D) in the harness); scores unscaled.
+  R15 quantized KV cache (row f3): symmetric int8, one float32 scale per
+     (pool page, KV head, channel) over the page's valid tokens, codes decided
+     in float32 (quantize_kv8); attention reads bf16(code * scale).
+     (parity unpinned by the pages: they name KV quantization, not a scheme)
 """
 from .lserve import (  # noqa: F401
     widen_bf16,
@@ -49,4 +53,7 @@ from .lserve import (  # noqa: F401
     theoretical_speedup,
     prefill_rows,
     prefill_flops,
+    quantize_kv8,
+    dequantize_kv8,
+    dequantized_seq,
 )

@@ -203,3 +203,52 @@ def prefill_rows(q: np.ndarray, k: np.ndarray, v: np.ndarray, kind: int, block: 
         o[r] = (e @ v[keys]) / lsum
         lse[r] = zmax + math.log(lsum)
     return o, lse
+
+
+# --- quantized KV cache (row f3) [R15] -----------------------------------------
+# The pages name KV-cache quantization (QServe KV4, "orthogonal integration" in
+# the abstract of the explainer) but give no scheme.  R15 reading: symmetric
+# int8 with one scale per (pool page, KV head, channel) over the page's valid
+# tokens; the integer codes are decided in float32 exactly as written below so
+# that both sides take the same decision, and the attention reads the
+# dequantized values rounded to bf16 (the decode compute type).
+
+def quantize_kv8(x_bits: np.ndarray):
+    """Codes and scales of one page of one KV head.
+
+    x_bits: bf16 bits [t][D] of the page's valid tokens (t >= 1).
+    amax_c = max_t |x[t][c]| (exact in float32); inv_c = float32(127) /
+    float32(amax_c); code = rint(float32(x) * inv_c) (float32 product, round
+    half to even), clamped to [-127, 127]; scale_c = float32(amax_c) /
+    float32(127).  A channel with amax 0 gets codes 0 and scale 0.
+    Returns (codes int8 [t][D], scale float32 [D]).
+    """
+    x = widen_bf16(x_bits).astype(np.float32)
+    amax = np.max(np.abs(x), axis=0).astype(np.float32)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        inv = np.where(amax > 0, np.float32(127.0) / amax, np.float32(0.0)).astype(np.float32)
+    prod = (x * inv[None, :]).astype(np.float32)
+    codes = np.clip(np.rint(prod), -127, 127).astype(np.int8)
+    scale = (amax / np.float32(127.0)).astype(np.float32)
+    return codes, scale
+
+
+def dequantize_kv8(codes: np.ndarray, scale: np.ndarray) -> np.ndarray:
+    """bf16 bits of float32(code) * scale (float32 product), rounded to bf16
+    (round to nearest even) -- the values the quantized decode attends."""
+    prod = (codes.astype(np.float32) * scale.astype(np.float32)[None, :]).astype(np.float32)
+    u = prod.view(np.uint32).astype(np.uint64)
+    u = u + 0x7FFF + ((u >> 16) & 1)
+    return (u >> 16).astype(np.uint16)
+
+
+def dequantized_seq(x_bits: np.ndarray, N_P: int) -> np.ndarray:
+    """A sequence's K or V ([n][D] bf16 bits) as the quantized cache holds it:
+    each physical page of N_P tokens quantized on its own valid tokens and
+    dequantized (bf16 bits [n][D])."""
+    n = x_bits.shape[0]
+    out = np.empty_like(x_bits)
+    for t0 in range(0, n, N_P):
+        c, s = quantize_kv8(x_bits[t0:t0 + N_P])
+        out[t0:t0 + N_P] = dequantize_kv8(c, s)
+    return out

@@ -358,3 +358,53 @@ def test_method_constants_in_workloads():
         assert w.N_L == c["logical_page"] and w.N_P % w.N_L == 0
         assert c["physical_page_range"][0] <= w.N_P <= c["physical_page_range"][1]
         assert np.mean(w.head_kind) == c["streaming_fraction"]
+
+
+# --- quantized KV (R15) ---------------------------------------------------------
+
+def _bits(x):
+    return synth.to_bf16(np.asarray(x, dtype=np.float64))
+
+
+def test_kv8_hand_example():
+    # channel 0: amax 2 -> inv 63.5; 1 -> 63.5 -> 64 (half to even), -2 -> -127, 0.5 -> 31.75 -> 32
+    x = _bits([[1.0, 0.0], [-2.0, 0.0], [0.5, 0.0]])
+    codes, scale = oracle.quantize_kv8(x)
+    assert codes[:, 0].tolist() == [64, -127, 32]
+    assert codes[:, 1].tolist() == [0, 0, 0] and scale[1] == 0.0   # all-zero channel
+    assert scale[0] == np.float32(2.0) / np.float32(127.0)
+
+
+def test_kv8_round_trip_error_and_range():
+    rng = np.random.default_rng(11)
+    x = _bits(rng.normal(size=(64, 128)) * rng.uniform(0.5, 8, size=128))
+    codes, scale = oracle.quantize_kv8(x)
+    assert codes.min() >= -127 and codes.max() <= 127
+    xf = oracle.widen_bf16(x)
+    amax = np.abs(xf).max(axis=0)
+    # the largest magnitude of each channel maps to +-127
+    j = np.abs(xf).argmax(axis=0)
+    assert np.all(np.abs(codes[j, np.arange(128)]) == 127)
+    back = oracle.widen_bf16(oracle.dequantize_kv8(codes, scale))
+    # quantization error <= half a step, plus the final bf16 rounding
+    bound = amax / 127 / 2 * (1 + 1e-6) + np.abs(back) * 2.0 ** -8
+    assert np.all(np.abs(back - xf) <= bound[None, :] + 1e-30)
+
+
+def test_kv8_is_odd_and_scale_invariant():
+    rng = np.random.default_rng(12)
+    x = _bits(rng.normal(size=(16, 64)))
+    c1, s1 = oracle.quantize_kv8(x)
+    c2, s2 = oracle.quantize_kv8(x ^ np.uint16(0x8000))          # negate every value
+    assert np.array_equal(c2, -c1) and np.array_equal(s1, s2)
+    c4, s4 = oracle.quantize_kv8(_bits(oracle.widen_bf16(x) * 4))  # exact power-of-two scaling
+    assert np.array_equal(c4, c1) and np.allclose(s4, 4 * s1, rtol=0, atol=0)
+
+
+def test_dequantized_seq_pages_are_independent():
+    rng = np.random.default_rng(13)
+    x = _bits(rng.normal(size=(150, 32)))
+    whole = oracle.dequantized_seq(x, 64)
+    for t0 in (0, 64, 128):
+        c, s = oracle.quantize_kv8(x[t0:t0 + 64])
+        assert np.array_equal(whole[t0:t0 + 64], oracle.dequantize_kv8(c, s))
