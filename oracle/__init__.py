@@ -33,7 +33,7 @@ Readings where the pages are silent (each is listed in the design notes):
   R8 softmax scale is a parameter (1/sqrt(D) in the harness); scores unscaled.
   R15 quantized KV cache (row f3): symmetric int8, one float32 scale per
      (pool page, KV head, channel) over the page's valid tokens, codes decided
-     in float32 (quantize_kv8); attention reads bf16(code * scale).
+     in float32 (quantize_kv8); attention attends code * scale.
      (parity unpinned by the pages: they name KV quantization, not a scheme)
 """
 from .lserve import (  # noqa: F401

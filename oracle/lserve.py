@@ -205,13 +205,14 @@ def prefill_rows(q: np.ndarray, k: np.ndarray, v: np.ndarray, kind: int, block: 
     return o, lse
 
 
-# --- quantized KV cache (row f3) [R15] -----------------------------------------
-# The pages name KV-cache quantization (QServe KV4, "orthogonal integration" in
-# the abstract of the explainer) but give no scheme.  R15 reading: symmetric
+# --- quantized KV cache [R15] ------------------------------------------------
+# The pages name KV-cache quantization (QServe KV4, combined with LServe's
+# sparsity in the abstract page) but give no scheme.  R15 reading: symmetric
 # int8 with one scale per (pool page, KV head, channel) over the page's valid
 # tokens; the integer codes are decided in float32 exactly as written below so
-# that both sides take the same decision, and the attention reads the
-# dequantized values rounded to bf16 (the decode compute type).
+# that both sides take the same decision; the attention attends the value
+# code * scale (a real number, exact in float64 here; each side rounds it as
+# its own arithmetic does).
 
 def quantize_kv8(x_bits: np.ndarray):
     """Codes and scales of one page of one KV head.
@@ -234,20 +235,16 @@ def quantize_kv8(x_bits: np.ndarray):
 
 
 def dequantize_kv8(codes: np.ndarray, scale: np.ndarray) -> np.ndarray:
-    """bf16 bits of float32(code) * scale (float32 product), rounded to bf16
-    (round to nearest even) -- the values the quantized decode attends."""
-    prod = (codes.astype(np.float32) * scale.astype(np.float32)[None, :]).astype(np.float32)
-    u = prod.view(np.uint32).astype(np.uint64)
-    u = u + 0x7FFF + ((u >> 16) & 1)
-    return (u >> 16).astype(np.uint16)
+    """code * scale per element, float64 (exact: 8-bit times 24-bit)."""
+    return codes.astype(np.float64) * scale.astype(np.float64)[None, :]
 
 
 def dequantized_seq(x_bits: np.ndarray, N_P: int) -> np.ndarray:
     """A sequence's K or V ([n][D] bf16 bits) as the quantized cache holds it:
-    each physical page of N_P tokens quantized on its own valid tokens and
-    dequantized (bf16 bits [n][D])."""
+    each physical page of N_P tokens quantized on its own valid tokens, then
+    dequantized (float64 [n][D])."""
     n = x_bits.shape[0]
-    out = np.empty_like(x_bits)
+    out = np.empty(x_bits.shape, dtype=np.float64)
     for t0 in range(0, n, N_P):
         c, s = quantize_kv8(x_bits[t0:t0 + N_P])
         out[t0:t0 + N_P] = dequantize_kv8(c, s)

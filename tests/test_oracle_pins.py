@@ -385,10 +385,11 @@ def test_kv8_round_trip_error_and_range():
     # the largest magnitude of each channel maps to +-127
     j = np.abs(xf).argmax(axis=0)
     assert np.all(np.abs(codes[j, np.arange(128)]) == 127)
-    back = oracle.widen_bf16(oracle.dequantize_kv8(codes, scale))
-    # quantization error <= half a step, plus the final bf16 rounding
-    bound = amax / 127 / 2 * (1 + 1e-6) + np.abs(back) * 2.0 ** -8
-    assert np.all(np.abs(back - xf) <= bound[None, :] + 1e-30)
+    back = oracle.dequantize_kv8(codes, scale)
+    # quantization error <= half a step (plus the float32 rounding of the
+    # scale and of the product that decided the code)
+    bound = amax / 127 / 2 * (1 + 1e-5)
+    assert np.all(np.abs(back - xf) <= bound[None, :])
 
 
 def test_kv8_is_odd_and_scale_invariant():
@@ -408,3 +409,18 @@ def test_dequantized_seq_pages_are_independent():
     for t0 in (0, 64, 128):
         c, s = oracle.quantize_kv8(x[t0:t0 + 64])
         assert np.array_equal(whole[t0:t0 + 64], oracle.dequantize_kv8(c, s))
+
+
+def test_kv8_lossless_on_grid_values():
+    # integers in [-127, 127] times a per-channel power of two, each channel
+    # reaching +-127: the codes are the integers and the round trip is exact
+    rng = np.random.default_rng(14)
+    ints = rng.integers(-127, 128, size=(40, 16))
+    ints[3] = 127
+    ints[7, ::2] = -127
+    step = 2.0 ** rng.integers(-6, 3, size=16)
+    x = _bits(ints * step)
+    codes, scale = oracle.quantize_kv8(x)
+    assert np.array_equal(np.abs(codes.astype(np.int64)), np.abs(ints))
+    assert np.array_equal(codes.astype(np.int64), ints)
+    assert np.array_equal(oracle.dequantize_kv8(codes, scale), oracle.widen_bf16(x))
