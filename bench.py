@@ -92,6 +92,39 @@ def decode_bytes(w):
     return dict(attn=attn, select=select, step=attn + select / REUSE, kv=kv, stats=stats)
 
 
+def decode_bytes_kv8(w):
+    """Bytes one decode-attention call over the int8 cache moves: the codes of
+    the attended pages (K and V, D bytes per token each), the two float32
+    channel-scale rows of every attended (page, head), q and the output."""
+    import oracle
+    D, NP = w.D, w.N_P
+    kv = 0
+    for b in range(w.B):
+        n = int(w.ctx_lens[b])
+        npages = -(-n // NP)
+        for h in range(w.H_kv):
+            if w.head_kind[h] == 0:
+                k = min(w.top_k, npages)
+                kv += k * NP * D * 2 + k * 2 * D * 4
+            else:
+                pages = oracle.streaming_pages(n, NP, w.sink, w.local)
+                toks = len(oracle.page_tokens(pages, n, NP))
+                kv += toks * D * 2 + len(pages) * 2 * D * 4
+    return kv + 2 * w.B * w.H_q * D * 2
+
+
+def quantize_bytes(w):
+    """lserve_quantize_pages_kv8: read the valid bf16 K/V rows of every page,
+    write the int8 codes (whole pages) and the float32 scales."""
+    rd = wr = 0
+    for b in range(w.B):
+        n = int(w.ctx_lens[b])
+        npages = -(-n // w.N_P)
+        rd += 2 * n * w.H_kv * w.D * 2
+        wr += 2 * npages * w.H_kv * (w.N_P * w.D + w.D * 4)
+    return rd + wr
+
+
 def stats_build_bytes(w):
     """lserve_page_stats full build: read K of the retrieval heads, write stats."""
     rd = wr = 0
@@ -316,6 +349,7 @@ def main():
     ap.add_argument("--layers", type=int, default=LAYERS,
                     help="layer replicas (fewer = a small case for profiling; < 32 may fit in L2)")
     ap.add_argument("--no-mha", action="store_true", help="skip the MHA decode stage")
+    ap.add_argument("--no-kv8", action="store_true", help="skip the int8-cache decode stages")
     ap.add_argument("--prefill-only", action="store_true",
                     help="run only the prefill stage (profiling)")
     ap.add_argument("--prefill-seq", type=int, default=None,
@@ -541,6 +575,14 @@ def main():
 
     if not args.no_mha:
         result["stages"]["attention_mha"] = mha_stage(lserve, synth, dev, stream, hbm_peak, timed)
+    if not args.no_kv8:
+        result["stages"]["attention_kv8"] = kv8_stage(lserve, synth, dev, stream, hbm_peak, timed,
+                                                      synth.llama3_8b_decode, 16,
+                                                      stages["attention"]["us"])
+        if not args.no_mha:
+            result["stages"]["attention_mha_kv8"] = kv8_stage(
+                lserve, synth, dev, stream, hbm_peak, timed, synth.llama2_7b_mha_decode, 8,
+                result["stages"]["attention_mha"]["us"])
     if not args.no_prefill:
         result["stages"]["prefill"] = prefill_stage(lserve, synth, dev, stream, tc_peak, timed,
                                                     args.prefill_seq)
@@ -602,6 +644,71 @@ def mha_stage(lserve, synth, dev, stream, hbm_peak, timed, layers=8):
             "workload": f"{w.name}: B={w.B} n={int(w.ctx_lens[0])} H_q={w.H_q} H_kv={w.H_kv} "
                         f"D={w.D} N_L={w.N_L} N_P={w.N_P} top_k={w.top_k} sink={w.sink} "
                         f"local={w.local}"}
+
+
+def kv8_stage(lserve, synth, dev, stream, hbm_peak, timed, make, layers, bf16_us):
+    """Decode attention over the int8 cache (lserve_sparse_decode_attn_kv8),
+    alone: the workload's pools quantized once (lserve_quantize_pages_kv8,
+    timed too), then `layers` replicas of the int8 pools attended back to back
+    (more bytes than L2 holds), the selection being the bf16 statistics'."""
+    import torch
+    from synth.device import DecodeBuffers
+    w = make()
+    buf = DecodeBuffers(w, device=dev, layers=1)
+    d = lserve.paged_desc(w.B, w.H_q, w.H_kv, w.D, w.N_L, w.N_P, w.max_pages, w.num_pool_pages)
+    wss = lserve.alloc_workspace(lserve.workspace_size(lserve.OP_SELECT, d, w.top_k), device=dev)
+    wsd = lserve.alloc_workspace(lserve.workspace_size(lserve.OP_DECODE, d, w.top_k), device=dev)
+    k8 = torch.empty(w.pool_shape(), dtype=torch.int8, device=dev)
+    v8 = torch.empty_like(k8)
+    ks = torch.empty((w.num_pool_pages, w.H_kv, w.D), dtype=torch.float32, device=dev)
+    vs = torch.empty_like(ks)
+
+    def quantize():
+        lserve.quantize_pages_kv8(d, buf.k_pool, buf.v_pool, buf.block_table, buf.ctx_lens, k8, v8,
+                                  ks, vs, stream=stream)
+    with torch.cuda.stream(stream):
+        lserve.page_stats(d, buf.k_pool, buf.block_table, buf.ctx_lens, buf.head_kind, buf.stats[0])
+        lserve.page_select(d, buf.q, buf.stats[0], buf.block_table, buf.ctx_lens, buf.head_kind,
+                           w.top_k, buf.sel[0], buf.sel_count[0], workspace=wss)
+        quantize()
+    torch.cuda.synchronize()
+    assert lserve.read_device_status(stream) == lserve.OK
+    t_q = timed(quantize, 3) / 3
+    qb = quantize_bytes(w)
+    buf.k_pools = buf.v_pools = None  # the bf16 pools are not read below
+    torch.cuda.empty_cache()
+    pools = [(k8, v8, ks, vs)] + [(k8.clone(), v8.clone(), ks.clone(), vs.clone())
+                                  for _ in range(layers - 1)]
+    outs = [torch.empty_like(buf.out) for _ in range(layers)]
+    scale = 1.0 / math.sqrt(w.D)
+
+    def attn_all():
+        for l, (a, b, c, e) in enumerate(pools):
+            lserve.sparse_decode_attn_kv8(d, buf.q, a, b, c, e, buf.block_table, buf.ctx_lens,
+                                          buf.head_kind, buf.sel[0], buf.sel_count[0], w.top_k,
+                                          w.sink, w.local, scale, outs[l], None, workspace=wsd,
+                                          overlap_prologue=l > 0)
+    with torch.cuda.stream(stream):
+        attn_all()
+    torch.cuda.synchronize()
+    assert lserve.read_device_status(stream) == lserve.OK
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        attn_all()
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            g.replay()
+    reps = 20
+    t = timed(lambda: g.replay(), reps) / (reps * layers)
+    bts = decode_bytes_kv8(w)
+    del g, pools
+    torch.cuda.empty_cache()
+    return {"us": t * 1e6, "GB/s": bts / t / 1e9, "frac": bts / t / 1e9 / hbm_peak, "bytes": bts,
+            "speedup_vs_bf16_cache": bf16_us / (t * 1e6),
+            "quantize": {"us": t_q * 1e6, "GB/s": qb / t_q / 1e9, "frac": qb / t_q / 1e9 / hbm_peak,
+                         "bytes": qb, "what": "lserve_quantize_pages_kv8 of the whole cache"},
+            "workload": f"{w.name} (int8 cache): B={w.B} n={int(w.ctx_lens[0])} H_q={w.H_q} "
+                        f"H_kv={w.H_kv} D={w.D} N_P={w.N_P} top_k={w.top_k}"}
 
 
 def prefill_stage(lserve, synth, dev, stream, tc_peak, timed, seq=None):

@@ -31,7 +31,8 @@ EXPORTED = [
     "lserve_blocksparse_prefill", "lserve_workspace_size", "lserve_read_device_status",
     "lserve_set_wait_limit_cycles", "lserve_debug_wait_timeout", "lserve_status_string",
     "lserve_bounds_checked", "lserve_page_select_noalloc", "lserve_sparse_decode_attn_ex",
-    "lserve_decode_append", "lserve_prefill_to_pages",
+    "lserve_decode_append", "lserve_prefill_to_pages", "lserve_quantize_pages_kv8",
+    "lserve_sparse_decode_attn_kv8",
 ]
 DECODE_OVERLAP_PROLOGUE = 1
 
@@ -75,6 +76,10 @@ def _load(path):
     lib.lserve_prefill_to_pages.argtypes = [P(PagedDesc), i32, vp, vp, vp, vp, vp, vp, vp, vp]
     lib.lserve_blocksparse_prefill.argtypes = [P(PrefillDesc), vp, vp, vp, vp, ctypes.c_float, vp, vp,
                                                vp, sz, vp]
+    lib.lserve_quantize_pages_kv8.argtypes = [P(PagedDesc), vp, vp, vp, vp, vp, vp, vp, vp, vp]
+    lib.lserve_sparse_decode_attn_kv8.argtypes = [P(PagedDesc), vp, vp, vp, vp, vp, vp, vp, vp, vp,
+                                                  vp, i32, i32, i32, ctypes.c_float, vp, vp,
+                                                  ctypes.c_uint32, vp, sz, vp]
     lib.lserve_page_select_noalloc.argtypes = [P(PagedDesc), vp, vp, vp, vp, vp, i32, vp, vp, vp]
     lib.lserve_page_select_noalloc.restype = ctypes.c_int
     lib.lserve_workspace_size.argtypes = [ctypes.c_int, vp, i32]
@@ -87,7 +92,9 @@ def _load(path):
     lib.lserve_status_string.restype = ctypes.c_char_p
     for name in ("lserve_page_stats", "lserve_page_select", "lserve_sparse_decode_attn",
                  "lserve_blocksparse_prefill", "lserve_read_device_status", "lserve_debug_wait_timeout",
-                 "lserve_bounds_checked"):
+                 "lserve_bounds_checked", "lserve_quantize_pages_kv8",
+                 "lserve_sparse_decode_attn_kv8", "lserve_sparse_decode_attn_ex",
+                 "lserve_decode_append", "lserve_prefill_to_pages"):
         getattr(lib, name).restype = ctypes.c_int
     return lib
 
@@ -187,6 +194,30 @@ def prefill_to_pages(desc, seq_len, k, v, block_table, head_kind, k_pool, v_pool
     _check("lserve_prefill_to_pages", lib.lserve_prefill_to_pages(
         ctypes.byref(desc), int(seq_len), _ptr(k), _ptr(v), _ptr(block_table), _ptr(head_kind),
         _ptr(k_pool), _ptr(v_pool), _ptr(stats_pool), _stream(stream)))
+
+
+def quantize_pages_kv8(desc, k_pool, v_pool, block_table, ctx_lens, k_pool8, v_pool8, k_scale,
+                       v_scale, stream=None):
+    """lserve_quantize_pages_kv8: int8 codes (int8 tensors shaped like the
+    pools) and float32 per-(page, head, channel) scales ([pool pages][H_kv][D])
+    of every page the block table references."""
+    _check("lserve_quantize_pages_kv8", lib.lserve_quantize_pages_kv8(
+        ctypes.byref(desc), _ptr(k_pool), _ptr(v_pool), _ptr(block_table), _ptr(ctx_lens),
+        _ptr(k_pool8), _ptr(v_pool8), _ptr(k_scale), _ptr(v_scale), _stream(stream)))
+
+
+def sparse_decode_attn_kv8(desc, q, k_pool8, v_pool8, k_scale, v_scale, block_table, ctx_lens,
+                           head_kind, sel, sel_count, top_k, sink_tokens, local_tokens,
+                           softmax_scale, out, lse=None, workspace=None, stream=None,
+                           overlap_prologue=False):
+    """lserve_sparse_decode_attn_kv8: sparse decode attention over the int8 cache."""
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    flags = DECODE_OVERLAP_PROLOGUE if overlap_prologue else 0
+    _check("lserve_sparse_decode_attn_kv8", lib.lserve_sparse_decode_attn_kv8(
+        ctypes.byref(desc), _ptr(q), _ptr(k_pool8), _ptr(v_pool8), _ptr(k_scale), _ptr(v_scale),
+        _ptr(block_table), _ptr(ctx_lens), _ptr(head_kind), _ptr(sel), _ptr(sel_count), top_k,
+        sink_tokens, local_tokens, float(softmax_scale), _ptr(out), _ptr(lse), flags,
+        _ptr(workspace), ws_bytes, _stream(stream)))
 
 
 def blocksparse_prefill(desc, q, k, v, head_kind_host, softmax_scale, out, lse=None, workspace=None,

@@ -19,7 +19,8 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 ROOT = os.path.dirname(HERE)
 SOURCES = ["api.cu", "page_stats.cu", "page_select.cu", "decode_attn.cu", "decode_append.cu",
-           "prefill.cu", "prefill_to_pages.cu", "select_noalloc.cu"]
+           "prefill.cu", "prefill_to_pages.cu", "select_noalloc.cu",
+           "quantize_kv8.cu"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
          "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr", "-I", os.path.join(ROOT, "include")]

@@ -392,20 +392,23 @@ int lserve_sparse_decode_attn(const lserve_paged_desc* desc, const void* q, cons
                                       lse, 0u, workspace, workspace_bytes, stream);
 }
 
-int lserve_sparse_decode_attn_ex(const lserve_paged_desc* desc, const void* q, const void* k_pool,
-                                 const void* v_pool, const int32_t* block_table,
-                                 const int32_t* ctx_lens, const uint8_t* head_kind,
-                                 const int32_t* sel, const int32_t* sel_count, int32_t top_k,
-                                 int32_t sink_tokens, int32_t local_tokens, float softmax_scale,
-                                 void* out, float* lse, uint32_t flags, void* workspace,
-                                 size_t workspace_bytes, void* stream) {
+}  // extern "C"
+
+namespace {
+
+// Validation and parameters shared by the bf16 and int8 decode entry points
+// (everything except the KV pools).
+int decode_params(const lserve_paged_desc* desc, const void* q, const int32_t* block_table,
+                  const int32_t* ctx_lens, const uint8_t* head_kind, const int32_t* sel,
+                  const int32_t* sel_count, int32_t top_k, int32_t sink_tokens, int32_t local_tokens,
+                  float softmax_scale, void* out, float* lse, uint32_t flags, void* workspace,
+                  size_t workspace_bytes, DecodeParams& p, int& grid) {
   if (!valid_paged(desc)) return LSERVE_ERR_INVALID_ARG;
   if (flags & ~(uint32_t)LSERVE_DECODE_OVERLAP_PROLOGUE) return LSERVE_ERR_INVALID_ARG;
-  if (!q || !k_pool || !v_pool || !block_table || !ctx_lens || !head_kind || !sel || !sel_count || !out)
+  if (!q || !block_table || !ctx_lens || !head_kind || !sel || !sel_count || !out)
     return LSERVE_ERR_INVALID_ARG;
-  if (!aligned(q, 16) || !aligned(k_pool, 16) || !aligned(v_pool, 16) || !aligned(out, 16) ||
-      !aligned(block_table, 4) || !aligned(ctx_lens, 4) || !aligned(sel, 4) || !aligned(sel_count, 4) ||
-      (lse && !aligned(lse, 4)))
+  if (!aligned(q, 16) || !aligned(out, 16) || !aligned(block_table, 4) || !aligned(ctx_lens, 4) ||
+      !aligned(sel, 4) || !aligned(sel_count, 4) || (lse && !aligned(lse, 4)))
     return LSERVE_ERR_INVALID_ARG;
   if (top_k < 1 || top_k > desc->max_pages_per_seq) return LSERVE_ERR_INVALID_ARG;
   if (sink_tokens < 0 || local_tokens < 0 || !std::isfinite(softmax_scale)) return LSERVE_ERR_INVALID_ARG;
@@ -418,14 +421,8 @@ int lserve_sparse_decode_attn_ex(const lserve_paged_desc* desc, const void* q, c
   const int P = desc->batch * desc->num_kv_heads;
   if (P > kDecodeMaxPairs) return LSERVE_ERR_UNSUPPORTED;
   const int tile_rows = desc->physical_page < kDecodeTileMax ? desc->physical_page : kDecodeTileMax;
-  const uint64_t rows = (uint64_t)desc->num_pool_pages * desc->num_kv_heads * desc->physical_page;
-  // [rows][D/64][64] view: a tile of tile_rows x D is one contiguous TMA copy
-  CUtensorMap kmap, vmap;
-  if (!make_map_tiled(&kmap, k_pool, 3, 64, D / 64, rows, 64, D / 64, tile_rows) ||
-      !make_map_tiled(&vmap, v_pool, 3, 64, D / 64, rows, 64, D / 64, tile_rows))
-    return LSERVE_ERR_CUDA;
-  const int grid = decode_grid(current_sm_count());
-  DecodeParams p;
+  grid = decode_grid(current_sm_count());
+  p = DecodeParams{};
   p.q = static_cast<const __nv_bfloat16*>(q);
   p.block_table = block_table;
   p.ctx_lens = ctx_lens;
@@ -457,7 +454,93 @@ int lserve_sparse_decode_attn_ex(const lserve_paged_desc* desc, const void* q, c
   p.overlap_prologue = (flags & LSERVE_DECODE_OVERLAP_PROLOGUE) ? 1 : 0;
   p.status = device_status_word();
   if (!p.status) return LSERVE_ERR_CUDA;
+  return LSERVE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int lserve_sparse_decode_attn_ex(const lserve_paged_desc* desc, const void* q, const void* k_pool,
+                                 const void* v_pool, const int32_t* block_table,
+                                 const int32_t* ctx_lens, const uint8_t* head_kind,
+                                 const int32_t* sel, const int32_t* sel_count, int32_t top_k,
+                                 int32_t sink_tokens, int32_t local_tokens, float softmax_scale,
+                                 void* out, float* lse, uint32_t flags, void* workspace,
+                                 size_t workspace_bytes, void* stream) {
+  if (!k_pool || !v_pool || !aligned(k_pool, 16) || !aligned(v_pool, 16)) return LSERVE_ERR_INVALID_ARG;
+  DecodeParams p;
+  int grid = 0;
+  const int st = decode_params(desc, q, block_table, ctx_lens, head_kind, sel, sel_count, top_k,
+                               sink_tokens, local_tokens, softmax_scale, out, lse, flags, workspace,
+                               workspace_bytes, p, grid);
+  if (st != LSERVE_OK) return st;
+  const int D = desc->head_dim, G = desc->num_q_heads / desc->num_kv_heads;
+  const uint64_t rows = (uint64_t)desc->num_pool_pages * desc->num_kv_heads * desc->physical_page;
+  // [rows][D/64][64] view: a tile of tile_rows x D is one contiguous TMA copy
+  CUtensorMap kmap, vmap;
+  if (!make_map_tiled(&kmap, k_pool, 3, 64, D / 64, rows, 64, D / 64, p.tile_rows) ||
+      !make_map_tiled(&vmap, v_pool, 3, 64, D / 64, rows, 64, D / 64, p.tile_rows))
+    return LSERVE_ERR_CUDA;
   return cuda_status(launch_decode(p, kmap, vmap, D, G, grid, static_cast<cudaStream_t>(stream)));
+}
+
+int lserve_sparse_decode_attn_kv8(const lserve_paged_desc* desc, const void* q, const void* k_pool8,
+                                  const void* v_pool8, const float* k_scale, const float* v_scale,
+                                  const int32_t* block_table, const int32_t* ctx_lens,
+                                  const uint8_t* head_kind, const int32_t* sel,
+                                  const int32_t* sel_count, int32_t top_k, int32_t sink_tokens,
+                                  int32_t local_tokens, float softmax_scale, void* out, float* lse,
+                                  uint32_t flags, void* workspace, size_t workspace_bytes,
+                                  void* stream) {
+  if (!k_pool8 || !v_pool8 || !k_scale || !v_scale) return LSERVE_ERR_INVALID_ARG;
+  if (!aligned(k_pool8, 16) || !aligned(v_pool8, 16) || !aligned(k_scale, 16) || !aligned(v_scale, 16))
+    return LSERVE_ERR_INVALID_ARG;
+  DecodeParams p;
+  int grid = 0;
+  const int st = decode_params(desc, q, block_table, ctx_lens, head_kind, sel, sel_count, top_k,
+                               sink_tokens, local_tokens, softmax_scale, out, lse, flags, workspace,
+                               workspace_bytes, p, grid);
+  if (st != LSERVE_OK) return st;
+  p.k8 = static_cast<const int8_t*>(k_pool8);
+  p.v8 = static_cast<const int8_t*>(v_pool8);
+  p.k_scale = k_scale;
+  p.v_scale = v_scale;
+  const int D = desc->head_dim, G = desc->num_q_heads / desc->num_kv_heads;
+  return cuda_status(launch_decode_kv8(p, D, G, grid, static_cast<cudaStream_t>(stream)));
+}
+
+int lserve_quantize_pages_kv8(const lserve_paged_desc* desc, const void* k_pool, const void* v_pool,
+                              const int32_t* block_table, const int32_t* ctx_lens, void* k_pool8,
+                              void* v_pool8, float* k_scale, float* v_scale, void* stream) {
+  if (!valid_paged(desc)) return LSERVE_ERR_INVALID_ARG;
+  if (!k_pool || !v_pool || !block_table || !ctx_lens || !k_pool8 || !v_pool8 || !k_scale || !v_scale)
+    return LSERVE_ERR_INVALID_ARG;
+  if (!aligned(k_pool, 16) || !aligned(v_pool, 16) || !aligned(k_pool8, 16) || !aligned(v_pool8, 16) ||
+      !aligned(k_scale, 16) || !aligned(v_scale, 16) || !aligned(block_table, 4) ||
+      !aligned(ctx_lens, 4))
+    return LSERVE_ERR_INVALID_ARG;
+  const int st = supported_paged(desc);
+  if (st != LSERVE_OK) return st;
+  if ((long long)desc->batch * desc->max_pages_per_seq > 0x7fffffffll || desc->num_kv_heads > 65535)
+    return LSERVE_ERR_UNSUPPORTED;
+  QuantParams p;
+  p.k_pool = static_cast<const __nv_bfloat16*>(k_pool);
+  p.v_pool = static_cast<const __nv_bfloat16*>(v_pool);
+  p.block_table = block_table;
+  p.ctx_lens = ctx_lens;
+  p.k_pool8 = static_cast<int8_t*>(k_pool8);
+  p.v_pool8 = static_cast<int8_t*>(v_pool8);
+  p.k_scale = k_scale;
+  p.v_scale = v_scale;
+  p.batch = desc->batch;
+  p.num_kv_heads = desc->num_kv_heads;
+  p.physical_page = desc->physical_page;
+  p.max_pages = desc->max_pages_per_seq;
+  p.num_pool_pages = desc->num_pool_pages;
+  p.status = device_status_word();
+  if (!p.status) return LSERVE_ERR_CUDA;
+  return cuda_status(launch_quantize_kv8(p, desc->head_dim, static_cast<cudaStream_t>(stream)));
 }
 
 int lserve_blocksparse_prefill(const lserve_prefill_desc* desc, const void* q, const void* k,

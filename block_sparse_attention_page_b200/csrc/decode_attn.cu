@@ -33,6 +33,8 @@
 // otherwise each CTA writes an unnormalised (o, m, l) partial and the last CTA
 // to finish the pair (per-pair counter in the workspace) merges the partials
 // with log-sum-exp weights and resets the counter to zero.
+#include <cstring>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -61,11 +63,16 @@ __device__ __forceinline__ int pair_pages(const DecodeParams& p, int pair) {
   return ns + max(0, npages - ls);
 }
 
-template <int D, int G>
+// Q8: the int8 cache -- K / V tiles of 1-byte codes followed by the page's
+// K and V channel scales (float32 [D] each); otherwise bf16 tiles.
+template <int D, int G, bool Q8 = false>
 struct DecLayout {
-  static constexpr int kTileK = kDecodeTileMax * D * 2;                  // K (or V) tile bytes
+  static constexpr int kTileK = kDecodeTileMax * D * (Q8 ? 1 : 2);       // K (or V) tile bytes
+  static constexpr int kScales = Q8 ? 2 * D * 4 : 0;                     // K, V channel scales
+  static constexpr int oScale = 2 * kTileK;                              // stage offsets
+  static constexpr int oQ = oScale + kScales;
   static constexpr int kStageQ = G * D * 2;
-  static constexpr int kStage = (2 * kTileK + kStageQ + 1023) / 1024 * 1024;
+  static constexpr int kStage = (oQ + kStageQ + 1023) / 1024 * 1024;
   static constexpr int kPs = 2 * kDecodeTileMax * G * 8;                 // p of two tiles
   static constexpr int kOw = kConsumerWarps * G * D * 4;                 // o per warp
   static constexpr int kMl = kConsumerWarps * G * 2 * 4;                 // (m, l) per warp
@@ -179,6 +186,21 @@ __device__ __forceinline__ void join_step(const float (&in)[N], float (&out)[N >
 template <int V>
 constexpr int join_out() { return V >= 8 ? V / 8 : 1; }
 
+// Four int8 codes (one 32-bit word, lowest byte first) times their channel
+// scales.  A code c becomes the float 2^23 + (c + 128) by placing the byte
+// c ^ 0x80 in the mantissa of 2^23; subtracting 2^23 + 128 leaves c exactly.
+__device__ __forceinline__ void dequant4_s8(uint32_t w, float2 s01, float2 s23, float2& x01,
+                                            float2& x23) {
+  const uint32_t u = w ^ 0x80808080u;
+  const float2 bias = make_float2(-8388736.f, -8388736.f);
+  const float2 f01 = make_float2(__uint_as_float(__byte_perm(u, 0x4B000000u, 0x7440)),
+                                 __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7441)));
+  const float2 f23 = make_float2(__uint_as_float(__byte_perm(u, 0x4B000000u, 0x7442)),
+                                 __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7443)));
+  x01 = __fmul2_rn(__fadd2_rn(f01, bias), s01);
+  x23 = __fmul2_rn(__fadd2_rn(f23, bias), s23);
+}
+
 template <int V>
 __device__ __forceinline__ void join_dots(const float (&d)[V], float (&out)[join_out<V>()], int qtr) {
   constexpr int N1 = V >= 2 ? V / 2 : 1, N2 = N1 >= 2 ? N1 / 2 : 1;
@@ -190,11 +212,11 @@ __device__ __forceinline__ void join_dots(const float (&d)[V], float (&out)[join
 
 }  // namespace
 
-template <int D, int G, int TR>
+template <int D, int G, int TR, bool Q8>
 __global__ void __launch_bounds__(kThreads, 1)
 decode_attn_kernel(const __grid_constant__ DecodeParams p, const __grid_constant__ CUtensorMap kmap,
                    const __grid_constant__ CUtensorMap vmap) {
-  using L = DecLayout<D, G>;
+  using L = DecLayout<D, G, Q8>;
   constexpr int W = kConsumerWarps;
   constexpr int S = L::kStages;
   constexpr int HB = G < 4 ? G : 4;      // heads whose q a QK lane holds at a time
@@ -252,9 +274,11 @@ decode_attn_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
     misc[24] = misc[25] = misc[26] = misc[27] = 0;
     fence_mbar_init();
   }
-  if (tid == 32) {
-    tma_prefetch_desc(&kmap);
-    tma_prefetch_desc(&vmap);
+  if constexpr (!Q8) {
+    if (tid == 32) {
+      tma_prefetch_desc(&kmap);
+      tma_prefetch_desc(&vmap);
+    }
   }
 
   // ---- plan: tiles per pair -> exclusive prefix off[0..P] in shared memory
@@ -343,11 +367,21 @@ decode_attn_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
             info[s] = val;
             const int b = pr / p.num_kv_heads, h = pr - b * p.num_kv_heads;
             uint8_t* st = smem + s * L::kStage;
-            mbar_arrive_expect_tx(&full[s], 2 * TR * D * 2 + L::kStageQ);
-            // one contiguous TR x D tile each: 3-D view (64 channels, D/64 halves, rows)
-            tma_load_3d(st, &kmap, 0, 0, row, &full[s]);
-            tma_load_3d(st + L::kTileK, &vmap, 0, 0, row, &full[s]);
-            bulk_load_1d(st + 2 * L::kTileK, p.q + ((size_t)b * p.num_q_heads + (size_t)h * G) * D,
+            if constexpr (Q8) {
+              // codes: one contiguous TR x D byte tile each; then the page's scales
+              const size_t ph = (size_t)row / p.physical_page;  // pool page * H_kv + head
+              mbar_arrive_expect_tx(&full[s], 2 * TR * D + L::kScales + L::kStageQ);
+              bulk_load_1d(st, p.k8 + (size_t)row * D, TR * D, &full[s]);
+              bulk_load_1d(st + L::kTileK, p.v8 + (size_t)row * D, TR * D, &full[s]);
+              bulk_load_1d(st + L::oScale, p.k_scale + ph * D, D * 4, &full[s]);
+              bulk_load_1d(st + L::oScale + D * 4, p.v_scale + ph * D, D * 4, &full[s]);
+            } else {
+              mbar_arrive_expect_tx(&full[s], 2 * TR * D * 2 + L::kStageQ);
+              // one contiguous TR x D tile each: 3-D view (64 channels, D/64 halves, rows)
+              tma_load_3d(st, &kmap, 0, 0, row, &full[s]);
+              tma_load_3d(st + L::kTileK, &vmap, 0, 0, row, &full[s]);
+            }
+            bulk_load_1d(st + L::oQ, p.q + ((size_t)b * p.num_q_heads + (size_t)h * G) * D,
                          L::kStageQ, &full[s]);
           } else {
             ok = 0;
@@ -389,15 +423,20 @@ decode_attn_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
   // byte offsets inside a stage, fixed for the lane (a token row is NBOX
   // consecutive 128-byte swizzle rows)
   uint32_t koff[R][KCH];
-#pragma unroll
-  for (int r = 0; r < R; ++r)
-#pragma unroll
-    for (int ch = 0; ch < KCH; ++ch) {
-      const int c = qtr * KCH + ch;  // 16-byte chunk of the key row
-      koff[r][ch] = sw128_offset(NBOX * (wt0 + 4 * r + tok_l) + c / 8, c % 8);
-    }
   uint32_t voff[PVN];
-  {
+  if constexpr (Q8) {  // unswizzled byte rows of D codes
+#pragma unroll
+    for (int r = 0; r < R; ++r) koff[r][0] = (wt0 + 4 * r + tok_l) * D + qtr * CPT;
+#pragma unroll
+    for (int j = 0; j < PVN; ++j) voff[j] = L::kTileK + (pv_t0 + j) * D + 4 * quad;
+  } else {
+#pragma unroll
+    for (int r = 0; r < R; ++r)
+#pragma unroll
+      for (int ch = 0; ch < KCH; ++ch) {
+        const int c = qtr * KCH + ch;  // 16-byte chunk of the key row
+        koff[r][ch] = sw128_offset(NBOX * (wt0 + 4 * r + tok_l) + c / 8, c % 8);
+      }
     const int chunk = (4 * quad) / 8;
 #pragma unroll
     for (int j = 0; j < PVN; ++j)
@@ -413,7 +452,7 @@ decode_attn_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
   auto load_q = [&](const uint8_t* st, int hb) {  // bf16 q of the stage -> this lane's eighth
 #pragma unroll
     for (int h = 0; h < HB; ++h) {
-      const uint4* src = reinterpret_cast<const uint4*>(st + 2 * L::kTileK + ((hb * HB + h) * D + qtr * CPT) * 2);
+      const uint4* src = reinterpret_cast<const uint4*>(st + L::oQ + ((hb * HB + h) * D + qtr * CPT) * 2);
 #pragma unroll
       for (int i = 0; i < KCH; ++i) {
         const uint4 w = src[i];
@@ -427,37 +466,87 @@ decode_attn_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
 
   // partial dots of tile st for the rows of this lane: d[g * R + r]
   auto qk_tile = [&](const uint8_t* st, float (&d)[V], int hb) {
+    if constexpr (Q8) {
+      // this lane's CPT channel scales of the tile's page
+      float2 sk[CPT / 2];
+      const float4* skp = reinterpret_cast<const float4*>(st + L::oScale) + qtr * (CPT / 4);
 #pragma unroll
-    for (int r = 0; r < R; ++r) {
-      float2 acc[HB];
-#pragma unroll
-      for (int h = 0; h < HB; ++h) acc[h] = make_float2(0.f, 0.f);
-#pragma unroll
-      for (int ch = 0; ch < KCH; ++ch) {
-        const uint4 kw = *reinterpret_cast<const uint4*>(st + koff[r][ch]);
-        const float2 k0 = bf16x2_to_float2(kw.x), k1 = bf16x2_to_float2(kw.y);
-        const float2 k2 = bf16x2_to_float2(kw.z), k3 = bf16x2_to_float2(kw.w);
-#pragma unroll
-        for (int h = 0; h < HB; ++h) {
-          acc[h] = __ffma2_rn(qreg[h][4 * ch + 0], k0, acc[h]);
-          acc[h] = __ffma2_rn(qreg[h][4 * ch + 1], k1, acc[h]);
-          acc[h] = __ffma2_rn(qreg[h][4 * ch + 2], k2, acc[h]);
-          acc[h] = __ffma2_rn(qreg[h][4 * ch + 3], k3, acc[h]);
-        }
+      for (int i = 0; i < CPT / 4; ++i) {
+        const float4 s4 = skp[i];
+        sk[2 * i] = make_float2(s4.x, s4.y);
+        sk[2 * i + 1] = make_float2(s4.z, s4.w);
       }
 #pragma unroll
-      for (int h = 0; h < HB; ++h) d[(hb * HB + h) * R + r] = acc[h].x + acc[h].y;
+      for (int r = 0; r < R; ++r) {
+        uint32_t cw[CPT / 4];
+        if constexpr (CPT == 16) {
+          const uint4 w = *reinterpret_cast<const uint4*>(st + koff[r][0]);
+          cw[0] = w.x; cw[1] = w.y; cw[2] = w.z; cw[3] = w.w;
+        } else {
+          const uint2 w = *reinterpret_cast<const uint2*>(st + koff[r][0]);
+          cw[0] = w.x; cw[1] = w.y;
+        }
+        float2 acc[HB];
+#pragma unroll
+        for (int h = 0; h < HB; ++h) acc[h] = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int i = 0; i < CPT / 4; ++i) {
+          float2 k01, k23;
+          dequant4_s8(cw[i], sk[2 * i], sk[2 * i + 1], k01, k23);
+#pragma unroll
+          for (int h = 0; h < HB; ++h) {
+            acc[h] = __ffma2_rn(qreg[h][2 * i + 0], k01, acc[h]);
+            acc[h] = __ffma2_rn(qreg[h][2 * i + 1], k23, acc[h]);
+          }
+        }
+#pragma unroll
+        for (int h = 0; h < HB; ++h) d[(hb * HB + h) * R + r] = acc[h].x + acc[h].y;
+      }
+    } else {
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        float2 acc[HB];
+#pragma unroll
+        for (int h = 0; h < HB; ++h) acc[h] = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int ch = 0; ch < KCH; ++ch) {
+          const uint4 kw = *reinterpret_cast<const uint4*>(st + koff[r][ch]);
+          const float2 k0 = bf16x2_to_float2(kw.x), k1 = bf16x2_to_float2(kw.y);
+          const float2 k2 = bf16x2_to_float2(kw.z), k3 = bf16x2_to_float2(kw.w);
+#pragma unroll
+          for (int h = 0; h < HB; ++h) {
+            acc[h] = __ffma2_rn(qreg[h][4 * ch + 0], k0, acc[h]);
+            acc[h] = __ffma2_rn(qreg[h][4 * ch + 1], k1, acc[h]);
+            acc[h] = __ffma2_rn(qreg[h][4 * ch + 2], k2, acc[h]);
+            acc[h] = __ffma2_rn(qreg[h][4 * ch + 3], k3, acc[h]);
+          }
+        }
+#pragma unroll
+        for (int h = 0; h < HB; ++h) d[(hb * HB + h) * R + r] = acc[h].x + acc[h].y;
+      }
     }
   };
 
   // o += p v over this lane's tokens of tile st (tokens past `valid` read zeros)
   auto pv_tile = [&](const uint8_t* st, int i, int valid) {
+    float2 sv01, sv23;  // Q8: this lane's four channel scales of V
+    if constexpr (Q8) {
+      const float4 s4 = reinterpret_cast<const float4*>(st + L::oScale + D * 4)[quad];
+      sv01 = make_float2(s4.x, s4.y);
+      sv23 = make_float2(s4.z, s4.w);
+    }
 #pragma unroll
     for (int j = 0; j < PVN; ++j) {
       const int t = pv_t0 + j;
       const uint8_t* vp = t < valid ? st + voff[j] : zero16;
-      const uint2 vw = *reinterpret_cast<const uint2*>(vp);
-      const float2 v01 = bf16x2_to_float2(vw.x), v23 = bf16x2_to_float2(vw.y);
+      float2 v01, v23;
+      if constexpr (Q8) {
+        dequant4_s8(*reinterpret_cast<const uint32_t*>(vp), sv01, sv23, v01, v23);
+      } else {
+        const uint2 vw = *reinterpret_cast<const uint2*>(vp);
+        v01 = bf16x2_to_float2(vw.x);
+        v23 = bf16x2_to_float2(vw.y);
+      }
       const float2* pt = ps + (i * kDecodeTileMax + t) * G;
       if constexpr (G >= 2) {
 #pragma unroll
@@ -776,11 +865,11 @@ size_t decode_workspace_bytes(int pairs, int grid, int G, int D) {
 
 int decode_grid(int sm_count) { return sm_count; }
 
-cudaError_t launch_decode(const DecodeParams& p, const CUtensorMap& kmap, const CUtensorMap& vmap,
-                          int D, int G, int grid, cudaStream_t stream) {
-  cudaError_t e = cudaSuccess;
-  if (grid < 1 || grid > kMaxGrid) return cudaErrorInvalidValue;
-  // launched as a programmatic dependent of the previous work on the stream
+namespace {
+// launched as a programmatic dependent of the previous work on the stream
+template <int D, int G, bool Q8>
+cudaError_t launch_decode_t(const DecodeParams& p, const CUtensorMap& kmap, const CUtensorMap& vmap,
+                            int grid, cudaStream_t stream) {
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
@@ -790,18 +879,20 @@ cudaError_t launch_decode(const DecodeParams& p, const CUtensorMap& kmap, const 
   cfg.stream = stream;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-#define LSERVE_DECODE_CASE(DD, GG)                                                        \
-  if (D == DD && G == GG) {                                                               \
-    cfg.dynamicSmemBytes = DecLayout<DD, GG>::kBytes + 1024;                              \
-    if (p.tile_rows == 64) {                                                              \
-      e = set_smem_once((const void*)decode_attn_kernel<DD, GG, 64>, (int)cfg.dynamicSmemBytes); \
-      if (e != cudaSuccess) return e;                                                     \
-      return cudaLaunchKernelEx(&cfg, decode_attn_kernel<DD, GG, 64>, p, kmap, vmap);     \
-    }                                                                                     \
-    e = set_smem_once((const void*)decode_attn_kernel<DD, GG, 32>, (int)cfg.dynamicSmemBytes); \
-    if (e != cudaSuccess) return e;                                                       \
-    return cudaLaunchKernelEx(&cfg, decode_attn_kernel<DD, GG, 32>, p, kmap, vmap);       \
-  }
+  cfg.dynamicSmemBytes = DecLayout<D, G, Q8>::kBytes + 1024;
+  auto kern = p.tile_rows == 64 ? decode_attn_kernel<D, G, 64, Q8> : decode_attn_kernel<D, G, 32, Q8>;
+  const cudaError_t e = set_smem_once((const void*)kern, (int)cfg.dynamicSmemBytes);
+  if (e != cudaSuccess) return e;
+  return cudaLaunchKernelEx(&cfg, kern, p, kmap, vmap);
+}
+
+template <bool Q8>
+cudaError_t launch_decode_any(const DecodeParams& p, const CUtensorMap& kmap, const CUtensorMap& vmap,
+                              int D, int G, int grid, cudaStream_t stream) {
+  if (grid < 1 || grid > kMaxGrid) return cudaErrorInvalidValue;
+  if (p.tile_rows != 64 && p.tile_rows != 32) return cudaErrorInvalidValue;
+#define LSERVE_DECODE_CASE(DD, GG) \
+  if (D == DD && G == GG) return launch_decode_t<DD, GG, Q8>(p, kmap, vmap, grid, stream);
   LSERVE_DECODE_CASE(64, 1)
   LSERVE_DECODE_CASE(64, 2)
   LSERVE_DECODE_CASE(64, 4)
@@ -811,8 +902,19 @@ cudaError_t launch_decode(const DecodeParams& p, const CUtensorMap& kmap, const 
   LSERVE_DECODE_CASE(128, 4)
   LSERVE_DECODE_CASE(128, 8)
 #undef LSERVE_DECODE_CASE
-  (void)e;
   return cudaErrorInvalidValue;
+}
+}  // namespace
+
+cudaError_t launch_decode(const DecodeParams& p, const CUtensorMap& kmap, const CUtensorMap& vmap,
+                          int D, int G, int grid, cudaStream_t stream) {
+  return launch_decode_any<false>(p, kmap, vmap, D, G, grid, stream);
+}
+
+cudaError_t launch_decode_kv8(const DecodeParams& p, int D, int G, int grid, cudaStream_t stream) {
+  CUtensorMap unused;  // the int8 tiles are plain bulk copies: no tensor map
+  memset(&unused, 0, sizeof(unused));
+  return launch_decode_any<true>(p, unused, unused, D, G, grid, stream);
 }
 
 }  // namespace lserve

@@ -67,6 +67,12 @@ struct DecodeParams {
   float scale_log2;       // softmax_scale * log2(e)
   uint64_t wait_limit;
   int overlap_prologue;   // plan + first lookups may run before the preceding kernel ends
+  // int8 cache (lserve_sparse_decode_attn_kv8): codes [pool rows][D] and
+  // float scales [num_pool_pages][H_kv][D]; null for the bf16 cache
+  const int8_t* k8;
+  const int8_t* v8;
+  const float* k_scale;
+  const float* v_scale;
 };
 
 // lserve_decode_append: one warp per (sequence, KV head)
@@ -100,11 +106,28 @@ struct ToPagesParams {
 };
 cudaError_t launch_prefill_to_pages(const ToPagesParams& p, int D, cudaStream_t stream);
 
+// lserve_quantize_pages_kv8: one CTA per (page of a sequence, KV head, K or V)
+struct QuantParams {
+  const __nv_bfloat16* k_pool;
+  const __nv_bfloat16* v_pool;
+  const int32_t* block_table;
+  const int32_t* ctx_lens;
+  int8_t* k_pool8;
+  int8_t* v_pool8;
+  float* k_scale;   // [num_pool_pages][H_kv][D]
+  float* v_scale;
+  unsigned int* status;
+  int batch, num_kv_heads, physical_page, max_pages, num_pool_pages;
+};
+cudaError_t launch_quantize_kv8(const QuantParams& p, int D, cudaStream_t stream);
+
 cudaError_t launch_page_stats(const StatsParams& p, int D, int max_logical_pages,
                               cudaStream_t stream);
 cudaError_t launch_page_select(const SelectParams& p, int D, cudaStream_t stream);
 cudaError_t launch_decode(const DecodeParams& p, const CUtensorMap& kmap, const CUtensorMap& vmap,
                           int D, int G, int grid, cudaStream_t stream);
+// the int8-cache variant (p.k8 / p.v8 / p.k_scale / p.v_scale set; no tensor maps)
+cudaError_t launch_decode_kv8(const DecodeParams& p, int D, int G, int grid, cudaStream_t stream);
 size_t decode_workspace_bytes(int pairs, int grid, int G, int D);
 int decode_grid(int sm_count);
 

@@ -239,6 +239,56 @@ int lserve_sparse_decode_attn_ex(const lserve_paged_desc* desc, const void* q, c
                                  size_t workspace_bytes, void* stream);
 
 /*
+ * lserve_quantize_pages_kv8 -- an int8 copy of the paged K / V cache.
+ * [LServe abstract page: the unified sparse attention is combined with a
+ *  quantized KV cache (QServe's KV4 in the end-to-end results); the pages give
+ *  no quantization scheme.  This library's scheme: symmetric int8, one float32
+ *  scale per (pool page, KV head, channel) over the page's valid tokens.]
+ *
+ * For every sequence b, page ordinal m < ceil(n_b / N_P) and KV head h, with
+ * pool id pid = block_table[b][m] and valid = min(N_P, n_b - m*N_P) tokens,
+ * and separately for K and V:
+ *   amax_c  = max over the valid rows of |x[row][c]|
+ *   code    = rint(x * (127 / amax_c)) clamped to [-127, 127]  (float32,
+ *             IEEE-rounded quotient and product, ties to even; 0 if amax_c = 0)
+ *   scale_c = amax_c / 127                                      (float32)
+ *   k_pool8 / v_pool8  int8 [num_pool_pages][H_kv][N_P][D]: the codes; rows
+ *                      past `valid` are written as 0;
+ *   k_scale / v_scale  float [num_pool_pages][H_kv][D]: the scales.
+ * The value the cache holds is code * scale_c.  Inputs k_pool / v_pool are the
+ * bf16 pools (layout above); they are only read, so the page statistics built
+ * from them (lserve_page_stats, lserve_prefill_to_pages) stay the selection's
+ * input.  Pool pages no sequence references are not touched.  A bad pool id
+ * skips that page and sets LSERVE_ERR_BOUNDS.  No workspace.  All pointers
+ * 16-byte aligned.
+ */
+int lserve_quantize_pages_kv8(const lserve_paged_desc* desc, const void* k_pool, const void* v_pool,
+                              const int32_t* block_table, const int32_t* ctx_lens, void* k_pool8,
+                              void* v_pool8, float* k_scale, float* v_scale, void* stream);
+
+/*
+ * lserve_sparse_decode_attn_kv8 -- lserve_sparse_decode_attn_ex over the int8
+ * cache that lserve_quantize_pages_kv8 writes.
+ * [Same pages as lserve_sparse_decode_attn; the quantized cache as above.]
+ *
+ * Every attended token contributes k = code_k * k_scale and v = code_v *
+ * v_scale of its page (fp32 arithmetic); pages, softmax, outputs, lse,
+ * flags and workspace are exactly those of lserve_sparse_decode_attn_ex with
+ * the same arguments.  k_pool8 / v_pool8 int8 [num_pool_pages][H_kv][N_P][D],
+ * k_scale / v_scale float [num_pool_pages][H_kv][D], all 16-byte aligned.
+ * Each attended page moves N_P*D bytes of K codes and of V codes plus 2*D*4
+ * bytes of scales: about half the bf16 call's traffic.
+ */
+int lserve_sparse_decode_attn_kv8(const lserve_paged_desc* desc, const void* q, const void* k_pool8,
+                                  const void* v_pool8, const float* k_scale, const float* v_scale,
+                                  const int32_t* block_table, const int32_t* ctx_lens,
+                                  const uint8_t* head_kind, const int32_t* sel,
+                                  const int32_t* sel_count, int32_t top_k, int32_t sink_tokens,
+                                  int32_t local_tokens, float softmax_scale, void* out, float* lse,
+                                  uint32_t flags, void* workspace, size_t workspace_bytes,
+                                  void* stream);
+
+/*
  * lserve_blocksparse_prefill -- causal block-sparse flash attention for one
  * sequence.
  * [統一ブロックスパースアテンション: retrieval heads "block-sparse attention, static

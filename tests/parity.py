@@ -57,6 +57,63 @@ def run_decode_path(buf: DecodeBuffers, layer: int = 0, scale=None):
     )
 
 
+def run_decode_path_kv8(buf: DecodeBuffers, layer: int = 0, scale=None, overlap=False):
+    """stats -> select on the bf16 cache, then quantize the pools to int8 and
+    decode over the int8 cache; returns host copies (plus codes and scales)."""
+    w = buf.w
+    d = desc_of(w)
+    scale = 1.0 / math.sqrt(w.D) if scale is None else scale
+    lserve.page_stats(d, buf.k_pools[layer], buf.block_table, buf.ctx_lens, buf.head_kind,
+                      buf.stats[layer])
+    lserve.page_select(d, buf.q, buf.stats[layer], buf.block_table, buf.ctx_lens, buf.head_kind,
+                       w.top_k, buf.sel[layer], buf.sel_count[layer], phys_scores=buf.scores)
+    k8 = torch.full(w.pool_shape(), 99, dtype=torch.int8, device=buf.device)
+    v8 = torch.full(w.pool_shape(), -99, dtype=torch.int8, device=buf.device)
+    ks = torch.full((w.num_pool_pages, w.H_kv, w.D), float("nan"), dtype=torch.float32,
+                    device=buf.device)
+    vs = torch.full_like(ks, float("nan"))
+    lserve.quantize_pages_kv8(d, buf.k_pools[layer], buf.v_pools[layer], buf.block_table,
+                              buf.ctx_lens, k8, v8, ks, vs)
+    ws = lserve.alloc_workspace(lserve.workspace_size(lserve.OP_DECODE, d, w.top_k))
+    lserve.sparse_decode_attn_kv8(d, buf.q, k8, v8, ks, vs, buf.block_table, buf.ctx_lens,
+                                  buf.head_kind, buf.sel[layer], buf.sel_count[layer], w.top_k,
+                                  w.sink, w.local, scale, buf.out, buf.lse, workspace=ws,
+                                  overlap_prologue=overlap)
+    torch.cuda.synchronize()
+    st = lserve.read_device_status()
+    assert st == lserve.OK, lserve.status_string(st)
+    return dict(
+        stats=bf16_bits(buf.stats[layer]),
+        scores=buf.scores.cpu().numpy(),
+        sel=buf.sel[layer].cpu().numpy(),
+        sel_count=buf.sel_count[layer].cpu().numpy(),
+        out=oracle.widen_bf16(bf16_bits(buf.out)),
+        lse=buf.lse.cpu().numpy().astype(np.float64),
+        scale=scale,
+        k8=k8, v8=v8, k_scale=ks, v_scale=vs,
+    )
+
+
+def check_quantized_pages(w, res, b, h):
+    """Codes and scales of every page of (b, h), K and V, bit for bit against
+    the oracle's quantize_kv8; rows past the valid tokens hold code 0."""
+    n = int(w.ctx_lens[b])
+    for key in ("k8", "v8", "k_scale", "v_scale"):   # one device -> host copy per call
+        if key + "_np" not in res:
+            res[key + "_np"] = res[key].cpu().numpy()
+    for name, bits, codes_all, scale_all in (("K", w.k_seq(b, h), res["k8_np"], res["k_scale_np"]),
+                                             ("V", w.v_seq(b, h), res["v8_np"], res["v_scale_np"])):
+        for m in range(-(-n // w.N_P)):
+            pid = int(w.block_table[b, m])
+            t0, t1 = m * w.N_P, min((m + 1) * w.N_P, n)
+            codes, sc = oracle.quantize_kv8(bits[t0:t1])
+            got_c = codes_all[pid, h]
+            got_s = scale_all[pid, h]
+            assert np.array_equal(got_c[:t1 - t0], codes), (name, b, h, m)
+            assert np.all(got_c[t1 - t0:] == 0), (name, b, h, m)
+            assert np.array_equal(got_s.view(np.uint32), sc.view(np.uint32)), (name, b, h, m)
+
+
 def check_stats(w, res, b, h, k):
     """Bit-exact k_min/k_max of every logical page of (b, h) against the oracle."""
     n = int(w.ctx_lens[b])
@@ -122,13 +179,21 @@ def check_outputs(w, res, b, h, q, k, v, pages, stats_out=None):
         assert np.max(np.abs(gl - lse)) <= LSE_ABS, (b, h, gl, lse)
 
 
-def check_pair(w, res, b, h, errs=None, check_stats_bits=True):
-    """Full parity of one (sequence, KV head): stats, scores, selection, output."""
+def check_pair(w, res, b, h, errs=None, check_stats_bits=True, kv8=False):
+    """Full parity of one (sequence, KV head): stats, scores, selection, output.
+    kv8: the attention read the int8 cache, so the oracle attends the
+    dequantized keys and values (pages and statistics stay those of bf16 K)."""
     G = w.G
     n = int(w.ctx_lens[b])
     q = oracle.widen_bf16(w.q[b, h * G:(h + 1) * G])
-    k = oracle.widen_bf16(w.k_seq(b, h))
-    v = oracle.widen_bf16(w.v_seq(b, h))
+    k_bits = w.k_seq(b, h)
+    v_bits = w.v_seq(b, h)
+    k = oracle.widen_bf16(k_bits)
+    v = oracle.widen_bf16(v_bits)
+    k_att, v_att = k, v
+    if kv8:
+        k_att = oracle.dequantized_seq(k_bits, w.N_P)
+        v_att = oracle.dequantized_seq(v_bits, w.N_P)
     if w.head_kind[h] == 0:
         if n > 0:
             if check_stats_bits:
@@ -143,5 +208,5 @@ def check_pair(w, res, b, h, errs=None, check_stats_bits=True):
     else:
         assert int(res["sel_count"][b, h]) == 0 and np.all(res["sel"][b, h] == -1)
         pages = oracle.streaming_pages(n, w.N_P, w.sink, w.local)
-    check_outputs(w, res, b, h, q, k, v, pages, errs)
+    check_outputs(w, res, b, h, q, k_att, v_att, pages, errs)
     return pages

@@ -137,3 +137,43 @@ def test_decode_ex_rejects_unknown_flags():
                                                  FAKE, FAKE, 8, 64, 256, 0.125, FAKE, None,
                                                  lserve.DECODE_OVERLAP_PROLOGUE, None, 0, None)
     assert st in (lserve.ERR_WORKSPACE, lserve.ERR_CUDA)
+
+
+def _quant(desc, k=FAKE, k8=FAKE, scale=FAKE):
+    return lserve.lib.lserve_quantize_pages_kv8(ctypes.byref(desc), k, FAKE, FAKE, FAKE, k8, FAKE, scale,
+                                                FAKE, None)
+
+
+def _decode8(desc, top_k=8, k8=FAKE, scale=FAKE, flags=0, out=FAKE):
+    return lserve.lib.lserve_sparse_decode_attn_kv8(ctypes.byref(desc), FAKE, k8, FAKE, scale, FAKE, FAKE,
+                                                    FAKE, FAKE, FAKE, FAKE, top_k, 64, 256, 0.125, out,
+                                                    None, flags, None, 0, None)
+
+
+@pytest.mark.parametrize("bad", [dict(B=0), dict(H_kv=0), dict(H_q=3), dict(N_P=40), dict(N_L=0),
+                                 dict(max_pages=0), dict(num_pool_pages=0)])
+def test_kv8_calls_reject_invalid_shapes(bad):
+    d = _desc(**bad)
+    assert _quant(d) == lserve.ERR_INVALID_ARG
+    assert _decode8(d) == lserve.ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("bad", [dict(D=96), dict(H_q=6, H_kv=2), dict(N_P=48, N_L=16)])
+def test_kv8_calls_reject_unsupported_shapes(bad):
+    d = _desc(**bad)
+    assert _quant(d) == lserve.ERR_UNSUPPORTED
+    assert _decode8(d) == lserve.ERR_UNSUPPORTED
+
+
+def test_kv8_calls_reject_null_misaligned_and_bad_scalars():
+    d = _desc()
+    assert _quant(d, k=None) == lserve.ERR_INVALID_ARG
+    assert _quant(d, k8=MISALIGNED) == lserve.ERR_INVALID_ARG
+    assert _quant(d, scale=None) == lserve.ERR_INVALID_ARG
+    assert _decode8(d, k8=None) == lserve.ERR_INVALID_ARG
+    assert _decode8(d, k8=MISALIGNED) == lserve.ERR_INVALID_ARG
+    assert _decode8(d, scale=MISALIGNED) == lserve.ERR_INVALID_ARG
+    assert _decode8(d, out=None) == lserve.ERR_INVALID_ARG
+    assert _decode8(d, top_k=0) == lserve.ERR_INVALID_ARG
+    assert _decode8(d, top_k=33) == lserve.ERR_INVALID_ARG
+    assert _decode8(d, flags=2) == lserve.ERR_INVALID_ARG
