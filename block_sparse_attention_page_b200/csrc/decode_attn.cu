@@ -201,6 +201,32 @@ __device__ __forceinline__ void dequant4_s8(uint32_t w, float2 s01, float2 s23, 
   x23 = __fmul2_rn(__fadd2_rn(f23, bias), s23);
 }
 
+// Warp-level tensor-core tiles (mma.sync, bf16 in, fp32 accumulate).  The
+// fragment layouts are those of the PTX ISA for m16n8k16 / m16n8k8 row.col:
+// lane L holds rows L/4 (and L/4 + 8) of A and C, columns 2*(L%4) + {0,1}.
+__device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a2, uint32_t b0,
+                                          uint32_t b1) {
+  // rows 8..15 of A are zero (at most 8 query heads per KV head)
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9},"
+      " {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ void mma_1688(float (&d)[4], uint32_t a0, uint32_t b0) {
+  asm("mma.sync.aligned.m16n8k8.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5}, {%6},"
+      " {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(0u), "r"(b0));
+}
+// four 8x8 bf16 matrices, transposed, from shared memory (lane L gives the
+// address of row L%8 of matrix L/8)
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr)
+               : "memory");
+}
+
 template <int V>
 __device__ __forceinline__ void join_dots(const float (&d)[V], float (&out)[join_out<V>()], int qtr) {
   constexpr int N1 = V >= 2 ? V / 2 : 1, N2 = N1 >= 2 ? N1 / 2 : 1;
@@ -349,6 +375,7 @@ decode_attn_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
     };
     int issued = 0;
     bool alive = true;
+    const uint64_t pol = l2_policy_evict_first();  // KV tiles: read once
     for (int kb = 0; kb < ntiles && alive; kb += 32) {
       int tp = 0, trow = 0, tval = 0;
       if (kb + lane < ntiles) lookup(u0 + kb + lane, tp, trow, tval);
@@ -371,15 +398,15 @@ decode_attn_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
               // codes: one contiguous TR x D byte tile each; then the page's scales
               const size_t ph = (size_t)row / p.physical_page;  // pool page * H_kv + head
               mbar_arrive_expect_tx(&full[s], 2 * TR * D + L::kScales + L::kStageQ);
-              bulk_load_1d(st, p.k8 + (size_t)row * D, TR * D, &full[s]);
-              bulk_load_1d(st + L::kTileK, p.v8 + (size_t)row * D, TR * D, &full[s]);
+              bulk_load_1d_hint(st, p.k8 + (size_t)row * D, TR * D, &full[s], pol);
+              bulk_load_1d_hint(st + L::kTileK, p.v8 + (size_t)row * D, TR * D, &full[s], pol);
               bulk_load_1d(st + L::oScale, p.k_scale + ph * D, D * 4, &full[s]);
               bulk_load_1d(st + L::oScale + D * 4, p.v_scale + ph * D, D * 4, &full[s]);
             } else {
               mbar_arrive_expect_tx(&full[s], 2 * TR * D * 2 + L::kStageQ);
               // one contiguous TR x D tile each: 3-D view (64 channels, D/64 halves, rows)
-              tma_load_3d(st, &kmap, 0, 0, row, &full[s]);
-              tma_load_3d(st + L::kTileK, &vmap, 0, 0, row, &full[s]);
+              tma_load_3d_hint(st, &kmap, 0, 0, row, &full[s], pol);
+              tma_load_3d_hint(st + L::kTileK, &vmap, 0, 0, row, &full[s], pol);
             }
             bulk_load_1d(st + L::oQ, p.q + ((size_t)b * p.num_q_heads + (size_t)h * G) * D,
                          L::kStageQ, &full[s]);
@@ -448,6 +475,120 @@ decode_attn_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
   float2 o_acc[G][2];
 #pragma unroll
   for (int g = 0; g < G; ++g) o_acc[g][0] = o_acc[g][1] = make_float2(0.f, 0.f);
+
+  // ---- tensor-core consumer (bf16 cache, G >= 4).  Each warp owns 8 tokens of every
+  // tile.  S = q K^T is one m16n8k16 row block per tile: the rows are the G
+  // query heads of the pair (rows G..15 zero), the 8 columns the warp's
+  // tokens, k over D in D/16 steps.  The reduction over channels is order-free,
+  // so k-step ks, lane quad position qq takes channels CPL*qq + 4*ks + {0..3}:
+  // each lane reads its CPL contiguous channels of q and of its token's key
+  // with 16-byte loads (no transpose).  O += P V with P (fp32 softmax weights
+  // split into bf16 hi + lo parts, so the product keeps ~16 bits) as the A
+  // operand straight from the S accumulator layout and V^T fragments by
+  // ldmatrix.trans; O (rows = heads, 8 channels per n-tile) stays in
+  // registers across the pair's tiles.
+  constexpr bool kMma = !Q8 && G >= 4;  // G < 4: most MMA rows would be padding
+  constexpr int KS = D / 16;   // QK k-steps
+  constexpr int CPL = D / 4;   // channels per lane in the QK operands
+  constexpr int NTl = D / 8;   // PV n-tiles (8 channels each)
+  const int hr = lane >> 2, qq = lane & 3;  // fragment row (head) and quad position
+  const bool real_row = hr < G;
+  const int mt0 = warp * 8;                  // the warp's 8 tokens of a tile
+  const bool has_tok = mt0 < TR;             // 32-token tiles: warps 4..7 hold none
+  uint32_t kof[CPL / 8];                     // this lane's key chunks (token mt0 + hr)
+  uint32_t vof[NTl / 4];                     // ldmatrix row addresses of V, per 4 n-tiles
+#pragma unroll
+  for (int i = 0; i < CPL / 8; ++i) {
+    const int c = (CPL * qq) / 8 + i;
+    kof[i] = sw128_offset(NBOX * (mt0 + hr) + c / 8, c % 8);
+  }
+#pragma unroll
+  for (int j = 0; j < NTl / 4; ++j) {
+    const int c = 4 * j + (lane >> 3);
+    vof[j] = L::kTileK + sw128_offset(NBOX * (mt0 + (lane & 7)) + c / 8, c % 8);
+  }
+  uint32_t qa[KS][2];   // A fragments of q: (a0, a2) per k-step
+  float om[NTl][4];     // O fragments (only [0], [1] are real rows)
+#pragma unroll
+  for (int n = 0; n < NTl; ++n) om[n][0] = om[n][1] = om[n][2] = om[n][3] = 0.f;
+  const uint32_t smem_base = smem_u32(smem);
+
+  auto load_q_mma = [&](const uint8_t* st) {
+#pragma unroll
+    for (int i = 0; i < CPL / 8; ++i) {
+      uint4 w = make_uint4(0u, 0u, 0u, 0u);
+      if (real_row) w = reinterpret_cast<const uint4*>(st + L::oQ + (hr * D + CPL * qq) * 2)[i];
+      qa[2 * i][0] = w.x;
+      qa[2 * i][1] = w.y;
+      qa[2 * i + 1][0] = w.z;
+      qa[2 * i + 1][1] = w.w;
+    }
+  };
+  // S of the warp's 8 tokens of tile st (two accumulators: even / odd k-steps)
+  auto qk_mma = [&](const uint8_t* st, float (&sa)[4], float (&sb)[4]) {
+    uint32_t kw[CPL / 2];
+#pragma unroll
+    for (int i = 0; i < CPL / 8; ++i) {
+      const uint4 w = *reinterpret_cast<const uint4*>(st + kof[i]);
+      kw[4 * i] = w.x;
+      kw[4 * i + 1] = w.y;
+      kw[4 * i + 2] = w.z;
+      kw[4 * i + 3] = w.w;
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) sa[i] = sb[i] = 0.f;
+#pragma unroll
+    for (int ks = 0; ks < KS; ++ks) {
+      if (ks & 1) mma_16816(sb, qa[ks][0], qa[ks][1], kw[2 * ks], kw[2 * ks + 1]);
+      else mma_16816(sa, qa[ks][0], qa[ks][1], kw[2 * ks], kw[2 * ks + 1]);
+    }
+  };
+  // bf16 halves of V rows mt0 + 2*qq + {0,1} that lie past `valid` -> 0 (the
+  // cache may hold anything there; p is 0 for them but 0 * NaN is not)
+  auto vmask = [&](int valid) -> uint32_t {
+    const int t = mt0 + 2 * qq;
+    return (t < valid ? 0x0000FFFFu : 0u) | (t + 1 < valid ? 0xFFFF0000u : 0u);
+  };
+  // O += P V over the warp's tokens of one or two tiles
+  auto pv_mma = [&](int s0, int s1, int nt, const float (&pr)[2][2], int valid0, int valid1) {
+    uint32_t ah[2], al[2];
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      ah[i] = float2_to_bf16x2(pr[i][0], pr[i][1]);
+      al[i] = float2_to_bf16x2(pr[i][0] - bf16_lo(ah[i]), pr[i][1] - bf16_hi(ah[i]));
+    }
+    const bool part0 = mt0 + 8 > valid0, part1 = nt == 2 && mt0 + 8 > valid1;  // warp-uniform
+    const uint32_t mk0 = vmask(valid0), mk1 = vmask(valid1);
+    const uint32_t b0 = smem_base + s0 * L::kStage, b1 = smem_base + s1 * L::kStage;
+#pragma unroll
+    for (int j = 0; j < NTl / 4; ++j) {
+      uint32_t v0[4];
+      ldsm_x4_trans(v0, b0 + vof[j]);
+      if (part0) {
+#pragma unroll
+        for (int r = 0; r < 4; ++r) v0[r] &= mk0;
+      }
+      if (nt == 2) {
+        uint32_t v1[4];
+        ldsm_x4_trans(v1, b1 + vof[j]);
+        if (part1) {
+#pragma unroll
+          for (int r = 0; r < 4; ++r) v1[r] &= mk1;
+        }
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          mma_16816(om[4 * j + r], ah[0], ah[1], v0[r], v1[r]);
+          mma_16816(om[4 * j + r], al[0], al[1], v0[r], v1[r]);
+        }
+      } else {
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          mma_1688(om[4 * j + r], ah[0], v0[r]);
+          mma_1688(om[4 * j + r], al[0], v0[r]);
+        }
+      }
+    }
+  };
 
   auto load_q = [&](const uint8_t* st, int hb) {  // bf16 q of the stage -> this lane's eighth
 #pragma unroll
@@ -578,6 +719,18 @@ decode_attn_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
   // merge the warps, then finalise, or publish a partial and maybe merge the
   // pair's partials across CTAs.
   auto flush = [&](int pair) {
+    if constexpr (kMma) {
+      float lw = l_run;  // row sum of head hr over the warp's tokens: the row's 4 lanes
+      lw += __shfl_xor_sync(kFull, lw, 1);
+      lw += __shfl_xor_sync(kFull, lw, 2);
+      if (real_row) {
+        if (qq == 0) mlw[warp * G + hr] = make_float2(m_run, lw);
+#pragma unroll
+        for (int n = 0; n < NTl; ++n)
+          *reinterpret_cast<float2*>(ow + (warp * G + hr) * D + 8 * n + 2 * qq) =
+              make_float2(om[n][0], om[n][1]);
+      }
+    } else {
     float lw = l_run;  // row sum of this lane's head over the warp's tokens
     if constexpr (row_bit(V, R, 4)) lw += __shfl_xor_sync(kFull, lw, 4);
     if constexpr (row_bit(V, R, 2)) lw += __shfl_xor_sync(kFull, lw, 2);
@@ -601,6 +754,7 @@ decode_attn_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
       for (int g = 0; g < G; ++g)
         *reinterpret_cast<float4*>(ow + (warp * G + g) * D + 4 * quad) =
             make_float4(o_acc[g][0].x, o_acc[g][0].y, o_acc[g][1].x, o_acc[g][1].y);
+    }
     }
     const bool live = named_sync_and(kBarConsumers, kConsumerThreads, !*abort_flag);
     if (tid < W * G) {  // weight of warp w's state for head g: 2^(m_w - max over warps)
@@ -645,7 +799,8 @@ decode_attn_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
     // A partial: one thread publishes it (the barrier above ordered every
     // thread's stores before its fence) and counts the pair's finished
     // segments; the CTA that completes the count merges the pair at its end.
-    // Only warp 0 waits for the fence.
+    // Only warp 0 waits for the fence (counting at the kernel's end instead
+    // measured slower: the merges then start later).
     if (!whole && live && tid == 0) {
       __threadfence();
       if (atomicAdd(&p.counters[pair], 1u) == (unsigned)(seg_count(pair) - 1))
@@ -664,9 +819,22 @@ decode_attn_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
     const int c_first = cta_of(cst, off[pair], NC), c_last = cta_of(cst, off[pair + 1] - 1, NC);
     const int nc = c_last - c_first + 1;
     constexpr int kCap = L::kOw / 8;  // float2 slots of the merge buffer
-    float2* wml = reinterpret_cast<float2*>(ow);  // [segment][head]: (m, l), then (weight, l)
-    float* hm = msc;                              // [head] max, [G + head] sum of weights * l
+    float2* wml = reinterpret_cast<float2*>(ow);  // [segment][head]: (m, l)
+    constexpr int kPre = 12;  // o partials of the first segments, loaded with the (m, l)
     if (nc * G <= kCap) {
+      // one round of loads: every (m, l) into shared memory and the first
+      // kPre segments' o of this thread's outputs into registers
+      float opre[NOUT][kPre];
+#pragma unroll
+      for (int i = 0; i < NOUT; ++i) {
+        const int j = min(tid + i * kConsumerThreads, G * D - 1);
+        const int g = j / D, c = j - g * D;
+#pragma unroll
+        for (int u = 0; u < kPre; ++u)
+          opre[i][u] = (u < nc && cta_busy(cst, c_first + u))
+                           ? __ldcg(p.part_o + (((size_t)(c_first + u) + pair) * G + g) * D + c)
+                           : 0.f;
+      }
       for (int i = tid; i < nc * G; i += kConsumerThreads) {
         const int cc = c_first + i / G, g = i - (i / G) * G;
         wml[i] = cta_busy(cst, cc)
@@ -674,44 +842,44 @@ decode_attn_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
                      : make_float2(-INFINITY, 0.f);
       }
       named_sync(kBarConsumers, kConsumerThreads);
-      if (tid < G) {
-        float M = -INFINITY;
-        for (int sgi = 0; sgi < nc; ++sgi) M = fmaxf(M, wml[sgi * G + tid].x);
-        hm[tid] = M;
-      }
-      named_sync(kBarConsumers, kConsumerThreads);
-      for (int i = tid; i < nc * G; i += kConsumerThreads) {
-        const float M = hm[i % G], m = wml[i].x;
-        wml[i].x = (m == -INFINITY) ? 0.f : exp2f(m - M);
-      }
-      named_sync(kBarConsumers, kConsumerThreads);
-      if (tid < G) {
-        float l = 0.f;
-        for (int sgi = 0; sgi < nc; ++sgi) l += wml[sgi * G + tid].x * wml[sgi * G + tid].y;
-        hm[G + tid] = l;
-      }
-      named_sync(kBarConsumers, kConsumerThreads);
+      // each output: M over the segments, weights 2^(m_s - M), weighted sums
 #pragma unroll
       for (int i = 0; i < NOUT; ++i) {
         const int j = tid + i * kConsumerThreads;
         if (j >= G * D) continue;
         const int g = j / D, c = j - g * D;
-        float o = 0.f;
+        float M = -INFINITY;
+        for (int sgi = 0; sgi < nc; ++sgi) M = fmaxf(M, wml[sgi * G + g].x);
+        float o = 0.f, lsum = 0.f;
+#pragma unroll
+        for (int u = 0; u < kPre; ++u) {
+          if (u < nc) {
+            const float2 ml = wml[u * G + g];
+            const float wt = ml.x == -INFINITY ? 0.f : exp2f(ml.x - M);
+            o += wt * opre[i][u];
+            lsum += wt * ml.y;
+          }
+        }
         constexpr int kBatch = 8;  // independent loads in flight per thread
-        for (int s0 = 0; s0 < nc; s0 += kBatch) {
+        for (int s0 = kPre; s0 < nc; s0 += kBatch) {
           float os[kBatch];
 #pragma unroll
           for (int u = 0; u < kBatch; ++u) {
             const int sgi = s0 + u;
-            os[u] = (sgi < nc && wml[min(sgi, nc - 1) * G + g].x != 0.f)
+            os[u] = (sgi < nc && cta_busy(cst, c_first + sgi))
                         ? __ldcg(p.part_o + (((size_t)(c_first + sgi) + pair) * G + g) * D + c)
                         : 0.f;
           }
 #pragma unroll
-          for (int u = 0; u < kBatch; ++u)
-            if (s0 + u < nc) o += wml[(s0 + u) * G + g].x * os[u];
+          for (int u = 0; u < kBatch; ++u) {
+            if (s0 + u < nc) {
+              const float2 ml = wml[(s0 + u) * G + g];
+              const float wt = ml.x == -INFINITY ? 0.f : exp2f(ml.x - M);
+              o += wt * os[u];
+              lsum += wt * ml.y;
+            }
+          }
         }
-        const float lsum = hm[G + g], M = hm[g];
         const size_t qh = (size_t)b * p.num_q_heads + (size_t)h * G + g;
         const bool empty_row = !(lsum > 0.f);
         p.out[qh * D + c] = __float2bfloat16_rn(empty_row ? 0.f : o / lsum);
@@ -760,8 +928,13 @@ decode_attn_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
       pend = off[cur + 1] - u0;
       m_run = -INFINITY;
       l_run = 0.f;
+      if constexpr (kMma) {
 #pragma unroll
-      for (int g = 0; g < G; ++g) o_acc[g][0] = o_acc[g][1] = make_float2(0.f, 0.f);
+        for (int n = 0; n < NTl; ++n) om[n][0] = om[n][1] = 0.f;
+      } else {
+#pragma unroll
+        for (int g = 0; g < G; ++g) o_acc[g][0] = o_acc[g][1] = make_float2(0.f, 0.f);
+      }
       need_q = true;
     }
     const int nt = (k + 1 < ntiles && k + 1 < pend) ? 2 : 1;
@@ -773,6 +946,49 @@ decode_attn_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
     const int valid1 = ok1 ? info[s1] : 0;
     const uint8_t* st0 = smem + s0 * L::kStage;
     const uint8_t* st1 = smem + s1 * L::kStage;
+    if constexpr (kMma) {
+      if (need_q) load_q_mma(st0);
+      need_q = false;
+      if (has_tok) {
+        float sa[2][4], sb[2][4];
+        qk_mma(st0, sa[0], sb[0]);
+        if (nt == 2) qk_mma(st1, sa[1], sb[1]);
+        float x[2][2];
+#pragma unroll
+        for (int i = 0; i < 2; ++i)
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            const int tok = mt0 + 2 * qq + j;
+            const bool ok = i == 0 ? tok < valid0 : (nt == 2 && tok < valid1);
+            x[i][j] = ok ? (sa[i][j] + sb[i][j]) * p.scale_log2 : -INFINITY;
+          }
+        float mx = fmaxf(fmaxf(x[0][0], x[0][1]), fmaxf(x[1][0], x[1][1]));
+        mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 1));
+        mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 2));
+        const float m_new = fmaxf(m_run, mx);
+        const float alpha = m_new == -INFINITY ? 1.f : fast_ex2(m_run - m_new);
+        const float m_use = m_new == -INFINITY ? 0.f : m_new;
+        m_run = m_new;
+        float pr[2][2];
+        float lsum = l_run * alpha;
+#pragma unroll
+        for (int i = 0; i < 2; ++i)
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            pr[i][j] = fast_ex2(x[i][j] - m_use);  // x = -inf gives 0
+            lsum += pr[i][j];
+          }
+        l_run = lsum;
+        if (__any_sync(kFull, alpha != 1.f)) {
+#pragma unroll
+          for (int n = 0; n < NTl; ++n) {
+            om[n][0] *= alpha;
+            om[n][1] *= alpha;
+          }
+        }
+        pv_mma(s0, s1, nt, pr, valid0, valid1);
+      }
+    } else {
     if constexpr (NHB == 1) {
       if (need_q) load_q(st0, 0);
     }
@@ -841,6 +1057,7 @@ decode_attn_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
     }
     pv_tile(st0, 0, valid0);
     if (nt == 2) pv_tile(st1, 1, valid1);
+    }
     __syncwarp();
     // ---- release the stage(s) to the producer
     if (lane == 0) {

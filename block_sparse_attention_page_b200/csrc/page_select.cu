@@ -36,6 +36,10 @@ page_score_kernel(SelectParams p) {
   constexpr int SB = kScoreSteps;  // warp steps per page loaded at once
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int b = blockIdx.z, h = blockIdx.y;
+  // launched as a programmatic dependent: q and the statistics may come from
+  // the kernel before, so nothing is read before it has completed
+  pdl_launch_dependents();
+  pdl_wait_prior_grid();
   if (p.head_kind[h] != 0) return;
   const int n = p.ctx_lens[b];
   const int NP = p.physical_page, NL = p.logical_page, g = NP / NL;
@@ -146,6 +150,8 @@ __global__ void __launch_bounds__(kTopkThreads) page_topk_kernel(SelectParams p)
   const int lane = tid & 31, warp = tid >> 5;
   const size_t pair = (size_t)b * p.num_kv_heads + h;
   int32_t* sel = p.sel + pair * p.top_k;
+  pdl_launch_dependents();
+  pdl_wait_prior_grid();  // the scores come from the kernel before
   const int K = p.top_k;
   if (p.head_kind[h] != 0) {
     for (int i = tid; i < K; i += blockDim.x) sel[i] = -1;
@@ -287,13 +293,33 @@ __global__ void __launch_bounds__(kTopkThreads) page_topk_kernel(SelectParams p)
   if (tid == 0) p.sel_count[pair] = K;
 }
 
+// Both kernels are launched as programmatic dependents of the work before
+// them on the stream: their blocks may be scheduled while that work drains
+// and wait (griddepcontrol.wait) before reading anything it may write.
+template <typename Kern>
+static cudaError_t launch_dependent(Kern kern, dim3 grid, int threads, size_t smem,
+                                    cudaStream_t stream, const SelectParams& p) {
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(threads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, p);
+}
+
 cudaError_t launch_page_select(const SelectParams& p, int D, cudaStream_t stream) {
   const int per_cta = kScoreWarps * kScorePagesPerWarp;
   dim3 grid((p.max_pages + per_cta - 1) / per_cta, p.num_kv_heads, p.batch);
   const int G = p.num_q_heads / p.num_kv_heads;
-#define LSERVE_SCORE_CASE(DD, GG)                                          \
-  if (D == DD && G == GG) {                                                \
-    page_score_kernel<DD, GG><<<grid, kScoreWarps * 32, 0, stream>>>(p);   \
+  cudaError_t e = cudaSuccess;
+#define LSERVE_SCORE_CASE(DD, GG)                                                          \
+  if (D == DD && G == GG) {                                                                \
+    e = launch_dependent(page_score_kernel<DD, GG>, grid, kScoreWarps * 32, 0, stream, p); \
   } else
   LSERVE_SCORE_CASE(64, 1)
   LSERVE_SCORE_CASE(64, 2)
@@ -305,15 +331,14 @@ cudaError_t launch_page_select(const SelectParams& p, int D, cudaStream_t stream
   LSERVE_SCORE_CASE(128, 8)
   return cudaErrorInvalidValue;
 #undef LSERVE_SCORE_CASE
-  cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const size_t smem = (size_t)p.max_pages * (sizeof(uint32_t) + 1);  // keys + kept flags
   if (smem > 48 * 1024) {
     e = set_smem_once((const void*)page_topk_kernel, (int)smem);
     if (e != cudaSuccess) return e;
   }
-  page_topk_kernel<<<dim3(p.num_kv_heads, p.batch), kTopkThreads, smem, stream>>>(p);
-  return cudaGetLastError();
+  return launch_dependent(page_topk_kernel, dim3(p.num_kv_heads, p.batch), kTopkThreads, smem, stream,
+                          p);
 }
 
 }  // namespace lserve
