@@ -39,6 +39,9 @@ CASES = [
     (1, 8, 2, 128, 64, 128, 2, 64, 64, [9000], False),          # N_L=64
     (4, 4, 2, 128, 16, 64, 64, 64, 256, [1, 17, 63, 4095], False),  # all selected, tiny n
     (2, 8, 4, 128, 16, 64, 8, 4096, 4096, [3000, 8000], False),  # n <= sink + local
+    (2, 16, 4, 64, 8, 32, 6, 32, 100, [777, 3001], True),       # G=4, D=64, 32-token tiles
+    (2, 16, 2, 64, 16, 64, 5, 64, 200, [1500, 4097], False),    # G=8, D=64
+    (2, 8, 2, 128, 16, 32, 7, 32, 64, [2000, 333], True),       # G=4, D=128, 32-token tiles
 ]
 
 

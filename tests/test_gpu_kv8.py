@@ -21,6 +21,7 @@ CASES = [
     (2, 16, 2, 128, 16, 128, 6, 128, 1024, [129, 20000], False),  # G=8, N_P=128
     (2, 8, 4, 64, 32, 256, 3, 300, 600, [2500, 513], True),       # D=64, N_P=256
     (4, 4, 2, 128, 16, 64, 64, 64, 256, [1, 17, 63, 4095], False),  # all selected, tiny n
+    (2, 16, 4, 64, 8, 32, 6, 32, 100, [777, 3001], True),         # G=4, D=64, N_P=32
 ]
 
 
