@@ -312,9 +312,16 @@ prefill_kernel(const __grid_constant__ PrefillParams p, const __grid_constant__ 
             if (!allowed) x[i] = -INFINITY;
           }
         }
-        float mt = -INFINITY;
+        // row max and (below) row sum as 8 independent partial chains: one
+        // softmax warp per SM sub-partition leaves no other warp to hide a
+        // 128-long dependent chain
+        float mt8[8];
 #pragma unroll
-        for (int i = 0; i < kBN; ++i) mt = fmaxf(mt, x[i]);
+        for (int i = 0; i < 8; ++i) mt8[i] = x[i];
+#pragma unroll
+        for (int i = 8; i < kBN; ++i) mt8[i & 7] = fmaxf(mt8[i & 7], x[i]);
+        const float mt = fmaxf(fmaxf(fmaxf(mt8[0], mt8[1]), fmaxf(mt8[2], mt8[3])),
+                               fmaxf(fmaxf(mt8[4], mt8[5]), fmaxf(mt8[6], mt8[7])));
         const float m_new = fmaxf(m, mt * p.scale_log2);
         float alpha = 1.f;
         bool rescale = false;
@@ -326,12 +333,15 @@ prefill_kernel(const __grid_constant__ PrefillParams p, const __grid_constant__ 
           rescale = true;
         }
         const float mu = (m == -INFINITY) ? 0.f : m;
-        float rs = 0.f;
+        float rs8[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) rs8[i] = 0.f;
 #pragma unroll
         for (int i = 0; i < kBN; ++i) {
           x[i] = tc::ex2(fmaf(x[i], p.scale_log2, -mu));
-          rs += x[i];
+          rs8[i & 7] += x[i];
         }
+        const float rs = ((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) + ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7]));
         l = l * alpha + rs;
         // P_j may overwrite P_{j-1} (and O may be rescaled) once PV_{j-1} is done
         if (pv_count > 0 && !warp_wait(p_free, (pv_count - 1) & 1, lim, p.status)) { ok = false; break; }
