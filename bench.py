@@ -350,6 +350,8 @@ def main():
                     help="layer replicas (fewer = a small case for profiling; < 32 may fit in L2)")
     ap.add_argument("--no-mha", action="store_true", help="skip the MHA decode stage")
     ap.add_argument("--no-kv8", action="store_true", help="skip the int8-cache decode stages")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the long-decode and mixed-batch decode stages")
     ap.add_argument("--prefill-only", action="store_true",
                     help="run only the prefill stage (profiling)")
     ap.add_argument("--prefill-seq", type=int, default=None,
@@ -575,6 +577,11 @@ def main():
 
     if not args.no_mha:
         result["stages"]["attention_mha"] = mha_stage(lserve, synth, dev, stream, hbm_peak, timed)
+    if not args.no_configs:
+        result["stages"]["long_decode_256k"] = decode_config_stage(
+            lserve, synth, dev, stream, hbm_peak, timed, synth.long_decode_256k, 16)
+        result["stages"]["mixed_batch_decode"] = decode_config_stage(
+            lserve, synth, dev, stream, hbm_peak, timed, synth.mixed_batch_decode, 3)
     if not args.no_kv8:
         result["stages"]["attention_kv8"] = kv8_stage(lserve, synth, dev, stream, hbm_peak, timed,
                                                       synth.llama3_8b_decode, 16,
@@ -644,6 +651,66 @@ def mha_stage(lserve, synth, dev, stream, hbm_peak, timed, layers=8):
             "workload": f"{w.name}: B={w.B} n={int(w.ctx_lens[0])} H_q={w.H_q} H_kv={w.H_kv} "
                         f"D={w.D} N_L={w.N_L} N_P={w.N_P} top_k={w.top_k} sink={w.sink} "
                         f"local={w.local}"}
+
+
+def decode_config_stage(lserve, synth, dev, stream, hbm_peak, timed, make, layers):
+    """Selection and decode attention of another decode workload, each timed
+    alone: `layers` replicas of its KV / stats / selection (together more bytes
+    than L2 holds), graph replays, attention launched as in the main step."""
+    import torch
+    from synth.device import DecodeBuffers
+    w = make()
+    buf = DecodeBuffers(w, device=dev, layers=layers)
+    d = lserve.paged_desc(w.B, w.H_q, w.H_kv, w.D, w.N_L, w.N_P, w.max_pages, w.num_pool_pages)
+    wss = lserve.alloc_workspace(lserve.workspace_size(lserve.OP_SELECT, d, w.top_k), device=dev)
+    wsd = lserve.alloc_workspace(lserve.workspace_size(lserve.OP_DECODE, d, w.top_k), device=dev)
+    outs = [torch.empty_like(buf.out) for _ in range(layers)]
+    scale = 1.0 / math.sqrt(w.D)
+
+    def select_all():
+        for l in range(layers):
+            lserve.page_select(d, buf.q, buf.stats[l], buf.block_table, buf.ctx_lens, buf.head_kind,
+                               w.top_k, buf.sel[l], buf.sel_count[l], workspace=wss)
+
+    def attn_all():
+        for l in range(layers):
+            lserve.sparse_decode_attn(d, buf.q, buf.k_pools[l], buf.v_pools[l], buf.block_table,
+                                      buf.ctx_lens, buf.head_kind, buf.sel[l], buf.sel_count[l],
+                                      w.top_k, w.sink, w.local, scale, outs[l], None, workspace=wsd,
+                                      overlap_prologue=l > 0)
+    with torch.cuda.stream(stream):
+        for l in range(layers):
+            lserve.page_stats(d, buf.k_pools[l], buf.block_table, buf.ctx_lens, buf.head_kind,
+                              buf.stats[l])
+        select_all()
+        attn_all()
+    torch.cuda.synchronize()
+    assert lserve.read_device_status(stream) == lserve.OK
+    graphs = []
+    for fn in (select_all, attn_all):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            fn()
+        with torch.cuda.stream(stream):
+            for _ in range(3):
+                g.replay()
+        graphs.append(g)
+    reps = 20
+    t_sel = timed(lambda: graphs[0].replay(), reps) / (reps * layers)
+    t_att = timed(lambda: graphs[1].replay(), reps) / (reps * layers)
+    acct = decode_bytes(w)
+    del graphs, buf
+    torch.cuda.empty_cache()
+    step = t_att + t_sel / REUSE
+    return {"attention": {"us": t_att * 1e6, "GB/s": acct["attn"] / t_att / 1e9,
+                          "frac": acct["attn"] / t_att / 1e9 / hbm_peak, "bytes": acct["attn"]},
+            "selection": {"us": t_sel * 1e6, "GB/s": acct["select"] / t_sel / 1e9,
+                          "frac": acct["select"] / t_sel / 1e9 / hbm_peak, "bytes": acct["select"]},
+            "us_per_layer_step": step * 1e6, "GB/s_per_step": acct["step"] / step / 1e9,
+            "layers": layers,
+            "workload": f"{w.name}: B={w.B} n={int(w.ctx_lens.min())}..{int(w.ctx_lens.max())} "
+                        f"H_q={w.H_q} H_kv={w.H_kv} D={w.D} N_L={w.N_L} N_P={w.N_P} "
+                        f"top_k={w.top_k} sink={w.sink} local={w.local} reuse={REUSE}"}
 
 
 def kv8_stage(lserve, synth, dev, stream, hbm_peak, timed, make, layers, bf16_us):
