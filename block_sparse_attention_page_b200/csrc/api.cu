@@ -422,6 +422,20 @@ int decode_params(const lserve_paged_desc* desc, const void* q, const int32_t* b
   if (P > kDecodeMaxPairs) return LSERVE_ERR_UNSUPPORTED;
   const int tile_rows = desc->physical_page < kDecodeTileMax ? desc->physical_page : kDecodeTileMax;
   grid = decode_grid(current_sm_count());
+  {
+    // Small calls use fewer CTAs: from the host-side shapes, a pair attends at
+    // most max(top_k, sink + local pages) pages, which bounds the tiles of the
+    // call; at least kDecodeMinTiles tiles per CTA keeps each pair split over
+    // fewer CTAs (fewer partials to merge) while large calls still fill the GPU.
+    const long long NP = desc->physical_page;
+    const long long stream_pages = (sink_tokens + NP - 1) / NP + (local_tokens + NP - 1) / NP + 1;
+    const long long sel_pages = top_k < desc->max_pages_per_seq ? top_k : desc->max_pages_per_seq;
+    long long per_pair = sel_pages > stream_pages ? sel_pages : stream_pages;
+    if (per_pair > desc->max_pages_per_seq) per_pair = desc->max_pages_per_seq;
+    const long long tiles_ub = (long long)P * per_pair * (desc->physical_page / tile_rows);
+    const long long want = (tiles_ub + kDecodeMinTiles - 1) / kDecodeMinTiles;
+    if (want < grid) grid = want < 1 ? 1 : (int)want;
+  }
   p = DecodeParams{};
   p.q = static_cast<const __nv_bfloat16*>(q);
   p.block_table = block_table;

@@ -46,6 +46,10 @@ struct SelectParams {
 // and cut into equal contiguous ranges, one per CTA of a persistent grid.
 constexpr int kDecodeTileMax = 64;
 constexpr int kDecodeMaxPairs = 2048;   // B * H_kv
+#ifndef LSERVE_DECODE_MIN_TILES
+#define LSERVE_DECODE_MIN_TILES 4
+#endif
+constexpr int kDecodeMinTiles = LSERVE_DECODE_MIN_TILES;  // tiles per CTA the grid aims at, at least
 
 struct DecodeParams {
   const __nv_bfloat16* q;
