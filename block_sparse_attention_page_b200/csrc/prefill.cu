@@ -56,6 +56,10 @@ struct PrefillParams {
   uint8_t dense_heads[kMaxHeads];
   uint8_t stream_heads[kMaxHeads];
   uint8_t kv_kind[kMaxHeads];
+  // the paired kernel: first query head of each pair (two heads of one KV head)
+  int n_dense_pairs, n_stream_pairs;
+  uint8_t dense_pairs[kMaxHeads / 2];
+  uint8_t stream_pairs[kMaxHeads / 2];
 };
 
 template <int D>
@@ -409,6 +413,344 @@ prefill_kernel(const __grid_constant__ PrefillParams p, const __grid_constant__ 
   }
 }
 
+// --- the paired kernel ------------------------------------------------------------
+// Two query heads of the same KV head and the same query tile form one work
+// tile: their key-tile ranges are identical and they read the same K and V
+// tiles.  Each head has its own softmax warpgroup, S and O in tensor memory,
+// and its P written over the first half of its own S (bf16 pairs, the A operand
+// of PV read from TMEM).  The tensor core alternates between the heads
+// (S_A0 S_B0 PV_A0 S_A1 PV_B0 S_B1 PV_A1 ...), so one head's softmax always
+// overlaps the other head's matrix products -- the single-tile kernel above
+// leaves the tensor core waiting for its one softmax warpgroup.
+//   warp 0        TMA producer: Q of both heads, K and V into two-stage rings
+//   warp 1        tensor-memory owner (all 512 columns) and MMA issuer
+//   warps 2, 3    idle (they only lend their registers)
+//   warps 4-7     softmax of head A (thread r: query row r = TMEM lane r)
+//   warps 8-11    softmax of head B
+// An S commit also covers the PV issued before it: when a softmax warpgroup
+// sees S_j, the PV that read its P_{j-1} (the same columns) has completed and
+// O may be rescaled.
+namespace {
+constexpr int kPairThreads = 384;
+constexpr int kPairRegsCtl = 88;    // warpgroup 0 after setmaxnreg
+constexpr int kPairRegsSoft = 208;  // softmax warpgroups: 128*88 + 256*208 = 384*168
+
+template <int D>
+struct PairLayout {
+  static constexpr int kBox = kBM * 128;
+  static constexpr int kTile = kBox * (D / 64);
+  static constexpr int kQ = 0;                  // Q_A, Q_B
+  static constexpr int kK = kQ + 2 * kTile;     // 2 stages
+  static constexpr int kV = kK + 2 * kTile;     // 2 stages
+  static constexpr int kBar = kV + 2 * kTile;
+  static constexpr int kNumBars = 19;
+  static constexpr int kBytes = kBar + kNumBars * 8 + 16;
+};
+
+__device__ __forceinline__ TileRef pair_tile_at(const PrefillParams& p, int idx) {
+  const int nd = p.n_dense_pairs * p.n_qt;
+  if (idx < nd) return {p.dense_pairs[idx % p.n_dense_pairs], p.n_qt - 1 - idx / p.n_dense_pairs};
+  idx -= nd;
+  return {p.stream_pairs[idx % p.n_stream_pairs], p.n_qt - 1 - idx / p.n_stream_pairs};
+}
+}  // namespace
+
+template <int D>
+__global__ void __launch_bounds__(kPairThreads, 1)
+prefill_pair_kernel(const __grid_constant__ PrefillParams p, const __grid_constant__ CUtensorMap qmap,
+                    const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap) {
+  using L = PairLayout<D>;
+  constexpr int NBOX = D / 64;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
+  uint64_t* q_full = bars + 0;
+  uint64_t* q_empty = bars + 1;
+  uint64_t* k_full = bars + 2;    // [2]
+  uint64_t* k_empty = bars + 4;   // [2]
+  uint64_t* v_full = bars + 6;    // [2]
+  uint64_t* v_empty = bars + 8;   // [2]
+  uint64_t* s_full = bars + 10;   // [head]
+  uint64_t* p_full = bars + 12;   // [head]
+  uint64_t* pv_done = bars + 14;  // [head]: the tile's last PV has completed
+  uint64_t* o_free = bars + 16;   // [head]: the epilogue has read O
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::kBar + L::kNumBars * 8);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&k_full[s], 1);
+      mbar_init(&k_empty[s], 1);
+      mbar_init(&v_full[s], 1);
+      mbar_init(&v_empty[s], 1);
+      mbar_init(&s_full[s], 1);
+      mbar_init(&p_full[s], 128);
+      mbar_init(&pv_done[s], 1);
+      mbar_init(&o_free[s], 128);
+    }
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tc::alloc(tmem_holder, 512);
+    tc::relinquish();
+  }
+  tc::fence_before();
+  __syncthreads();
+  tc::fence_after();
+  const uint32_t tmem = *tmem_holder;
+  // columns: S_A [0, 128), S_B [128, 256), O_A [256, 256 + D), O_B [256 + D, 256 + 2D);
+  // P_X over the first 64 columns of S_X
+  auto tmem_s = [&](int x) { return tmem + x * kBN; };
+  auto tmem_o = [&](int x) { return tmem + 2 * kBN + x * D; };
+
+  const int total = (p.n_dense_pairs + p.n_stream_pairs) * p.n_qt;
+  const int grid = gridDim.x;
+  const uint64_t lim = p.wait_limit;
+
+  if (warp < 4) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kPairRegsCtl));
+    if (warp == 0 && lane == 0) {
+      // ------------------------------------------------------------ TMA producer
+      tma_prefetch_desc(&qmap);
+      tma_prefetch_desc(&kmap);
+      tma_prefetch_desc(&vmap);
+      int q_use = 0, kv_use = 0;
+      for (int r = 0;; ++r) {
+        const int idx = cta_tile(r, blockIdx.x, grid);
+        if (idx >= total) break;
+        const TileRef t = pair_tile_at(p, idx);  // t.hq: head A, head B = t.hq + 1
+        const int hkv = t.hq / p.G;
+        const KvRange kr = kv_range(p, p.kv_kind[hkv], t.qt);
+        if (q_use > 0 && !mbar_wait(q_empty, (q_use - 1) & 1, lim, p.status)) break;
+        mbar_arrive_expect_tx(q_full, 2 * L::kTile);
+        for (int x = 0; x < 2; ++x)
+          for (int bx = 0; bx < NBOX; ++bx)
+            tma_load_3d(smem + L::kQ + x * L::kTile + bx * L::kBox, &qmap, bx * 64, t.hq + x,
+                        t.qt * kBM, q_full);
+        ++q_use;
+        bool ok = true;
+        const int nkv = kr.count();
+        for (int j = 0; j < nkv && ok; ++j) {
+          const int kt = kr.at(j);
+          const int s = kv_use & 1, n = kv_use >> 1;
+          if (n > 0 && !mbar_wait(&k_empty[s], (n - 1) & 1, lim, p.status)) { ok = false; break; }
+          mbar_arrive_expect_tx(&k_full[s], L::kTile);
+          for (int bx = 0; bx < NBOX; ++bx)
+            tma_load_3d(smem + L::kK + s * L::kTile + bx * L::kBox, &kmap, bx * 64, hkv, kt * kBN,
+                        &k_full[s]);
+          if (n > 0 && !mbar_wait(&v_empty[s], (n - 1) & 1, lim, p.status)) { ok = false; break; }
+          mbar_arrive_expect_tx(&v_full[s], L::kTile);
+          for (int bx = 0; bx < NBOX; ++bx)
+            tma_load_3d(smem + L::kV + s * L::kTile + bx * L::kBox, &vmap, bx * 64, hkv, kt * kBN,
+                        &v_full[s]);
+          ++kv_use;
+        }
+        if (!ok) break;
+      }
+    } else if (warp == 1 && lane == 0) {
+      // ------------------------------------------------------------ MMA issuer
+      constexpr uint32_t idesc_s = tc::idesc_bf16_f32(kBM, kBN, false, false);
+      constexpr uint32_t idesc_pv = tc::idesc_bf16_f32(kBM, D, false, true);
+      const uint32_t q_addr = smem_u32(smem + L::kQ);
+      int q_use = 0, kv_base = 0, pcount = 0, tile_count = 0;
+      bool ok = true;
+      for (int r = 0; ok; ++r) {
+        const int idx = cta_tile(r, blockIdx.x, grid);
+        if (idx >= total) break;
+        const TileRef t = pair_tile_at(p, idx);
+        const KvRange kr = kv_range(p, p.kv_kind[t.hq / p.G], t.qt);
+        const int nkv = kr.count();
+        if (!mbar_wait(q_full, q_use & 1, lim, p.status)) break;
+        ++q_use;
+        tc::fence_after();
+        // S_x(j) = Q_x K_j^T; K_j is released after head B's product
+        auto issue_s = [&](int x, int j) -> bool {
+          const int kvi = kv_base + j, s = kvi & 1, n = kvi >> 1;
+          if (x == 0) {
+            if (!mbar_wait(&k_full[s], n & 1, lim, p.status)) return false;
+            tc::fence_after();
+          }
+          const uint32_t k_addr = smem_u32(smem + L::kK + s * L::kTile);
+          const uint32_t qa = q_addr + x * L::kTile;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk / 4) * L::kBox + (kk % 4) * 32;
+            tc::mma_ss(tmem_s(x), tc::smem_desc_sw128(qa + off, 16, 1024),
+                       tc::smem_desc_sw128(k_addr + off, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
+          }
+          tc::commit(&s_full[x]);
+          if (x == 1) {
+            tc::commit(&k_empty[s]);
+            if (j == nkv - 1) tc::commit(q_empty);
+          }
+          return true;
+        };
+        // O_x += P_x(j) V_j, P from tensor memory; V_j is released after head B's product
+        auto issue_pv = [&](int x, int j) -> bool {
+          const int kvi = kv_base + j, s = kvi & 1, n = kvi >> 1;
+          if (!mbar_wait(&p_full[x], pcount & 1, lim, p.status)) return false;
+          if (j == 0 && tile_count > 0 && !mbar_wait(&o_free[x], (tile_count - 1) & 1, lim, p.status))
+            return false;
+          if (x == 0 && !mbar_wait(&v_full[s], n & 1, lim, p.status)) return false;
+          tc::fence_after();
+          const uint32_t v_addr = smem_u32(smem + L::kV + s * L::kTile);
+#pragma unroll
+          for (int kk = 0; kk < kBN / 16; ++kk)  // 16 keys = 8 columns of P per step
+            tc::mma_ts(tmem_o(x), tmem_s(x) + kk * 8,
+                       tc::smem_desc_sw128(v_addr + kk * 16 * 128, L::kBox, 1024), idesc_pv,
+                       (j > 0 || kk > 0) ? 1u : 0u);
+          if (x == 1) tc::commit(&v_empty[s]);
+          if (j == nkv - 1) tc::commit(&pv_done[x]);
+          return true;
+        };
+        ok = issue_s(0, 0) && issue_s(1, 0);
+        for (int j = 0; j < nkv && ok; ++j) {
+          ok = issue_pv(0, j);
+          if (ok && j + 1 < nkv) ok = issue_s(0, j + 1);
+          if (ok) ok = issue_pv(1, j);
+          if (ok && j + 1 < nkv) ok = issue_s(1, j + 1);
+          ++pcount;
+        }
+        kv_base += nkv;
+        ++tile_count;
+      }
+    }
+  } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kPairRegsSoft));
+    // ------------------------------------------------------------ softmax
+    const int x = (warp - 4) >> 2;             // head of the pair
+    const int quad = warp & 3;                 // TMEM lane quarter of this warp
+    const int row = quad * 32 + lane;          // query row within the tile
+    const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+    int jcount = 0, tile_count = 0;
+    bool ok = true;
+    for (int r = 0; ok; ++r) {
+      const int idx = cta_tile(r, blockIdx.x, grid);
+      if (idx >= total) break;
+      const TileRef t = pair_tile_at(p, idx);
+      const int hq = t.hq + x;
+      const int kind = p.kv_kind[t.hq / p.G];
+      const KvRange kr = kv_range(p, kind, t.qt);
+      const int nkv = kr.count();
+      const int q = t.qt * kBM + row;
+      float m = -INFINITY, l = 0.f;
+      for (int j = 0; j < nkv; ++j) {
+        const int kt = kr.at(j);
+        // S_j (its commit also covers PV_{j-1}: P's columns and O are free)
+        if (!warp_wait(&s_full[x], jcount & 1, lim, p.status)) { ok = false; break; }
+        tc::fence_after();
+        float xs[kBN];
+#pragma unroll
+        for (int c = 0; c < kBN / 32; ++c) {
+          uint32_t u[32];
+          tc::ld32(tmem_s(x) + lane_off + c * 32, u);
+          tc::wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) xs[c * 32 + i] = __uint_as_float(u[i]);
+        }
+        const bool need_mask = kt == t.qt || (kt + 1) * kBN > p.T || (kind == 1 && p.mask_block < kBN);
+        if (need_mask) {
+          const int qb = q / p.mask_block;
+#pragma unroll
+          for (int i = 0; i < kBN; ++i) {
+            const int k = kt * kBN + i;
+            const int kb = k / p.mask_block;
+            const bool allowed = k <= q && k < p.T &&
+                                 (kind == 0 || kb < p.sink_blocks || qb - kb < p.local_blocks);
+            if (!allowed) xs[i] = -INFINITY;
+          }
+        }
+        float mt8[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) mt8[i] = xs[i];
+#pragma unroll
+        for (int i = 8; i < kBN; ++i) mt8[i & 7] = fmaxf(mt8[i & 7], xs[i]);
+        const float mt = fmaxf(fmaxf(fmaxf(mt8[0], mt8[1]), fmaxf(mt8[2], mt8[3])),
+                               fmaxf(fmaxf(mt8[4], mt8[5]), fmaxf(mt8[6], mt8[7])));
+        const float m_new = fmaxf(m, mt * p.scale_log2);
+        float alpha = 1.f;
+        bool rescale = false;
+        if (j == 0) {
+          m = m_new;
+        } else if (m_new > m + kRescaleLog2) {
+          alpha = tc::ex2(m - m_new);
+          m = m_new;
+          rescale = true;
+        }
+        const float mu = (m == -INFINITY) ? 0.f : m;
+        float rs8[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) rs8[i] = 0.f;
+#pragma unroll
+        for (int i = 0; i < kBN; ++i) {
+          xs[i] = tc::ex2(fmaf(xs[i], p.scale_log2, -mu));
+          rs8[i & 7] += xs[i];
+        }
+        l = l * alpha + (((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) + ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7])));
+        if (rescale) {  // PV_{j-1} has completed (see above): O may be rescaled
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t u[32];
+            tc::ld32(tmem_o(x) + lane_off + c * 32, u);
+            tc::wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) u[i] = __float_as_uint(__uint_as_float(u[i]) * alpha);
+            tc::st32(tmem_o(x) + lane_off + c * 32, u);
+          }
+        }
+        // P_j over the first kBN / 2 columns of S_j (S_j is in registers now)
+#pragma unroll
+        for (int c = 0; c < kBN / 64; ++c) {
+          uint32_t u[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) u[i] = float2_to_bf16x2(xs[c * 64 + 2 * i], xs[c * 64 + 2 * i + 1]);
+          tc::st32(tmem_s(x) + lane_off + c * 32, u);
+        }
+        tc::wait_st();
+        tc::fence_before();
+        mbar_arrive(&p_full[x]);
+        ++jcount;
+      }
+      if (!ok) break;
+      // ---- epilogue: O / l -> bf16, log-sum-exp
+      if (!warp_wait(&pv_done[x], tile_count & 1, lim, p.status)) break;
+      tc::fence_after();
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+      __nv_bfloat16* orow = p.out + ((size_t)q * p.H_q + hq) * D;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t u[32];
+        tc::ld32(tmem_o(x) + lane_off + c * 32, u);
+        tc::wait_ld();
+        if (q < p.T) {
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            uint4 w;
+            w.x = float2_to_bf16x2(__uint_as_float(u[v * 8 + 0]) * inv, __uint_as_float(u[v * 8 + 1]) * inv);
+            w.y = float2_to_bf16x2(__uint_as_float(u[v * 8 + 2]) * inv, __uint_as_float(u[v * 8 + 3]) * inv);
+            w.z = float2_to_bf16x2(__uint_as_float(u[v * 8 + 4]) * inv, __uint_as_float(u[v * 8 + 5]) * inv);
+            w.w = float2_to_bf16x2(__uint_as_float(u[v * 8 + 6]) * inv, __uint_as_float(u[v * 8 + 7]) * inv);
+            *reinterpret_cast<uint4*>(orow + c * 32 + v * 8) = w;
+          }
+        }
+      }
+      if (p.lse != nullptr && q < p.T)
+        p.lse[(size_t)hq * p.T + q] = l > 0.f ? (m + __log2f(l)) * 0.69314718055994530942f : -INFINITY;
+      tc::fence_before();
+      mbar_arrive(&o_free[x]);
+      ++tile_count;
+    }
+  }
+  tc::fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc::fence_after();
+    tc::dealloc(tmem, 512);
+  }
+}
+
 // --- host side ------------------------------------------------------------------
 
 static bool make_map_3d(CUtensorMap* m, const void* base, uint64_t T, uint64_t H, uint64_t D) {
@@ -465,6 +807,15 @@ int prefill_entry(const lserve_prefill_desc* d, const void* q, const void* k, co
     else
       p.stream_heads[p.n_stream++] = (uint8_t)hq;
   }
+  const bool paired = p.G % 2 == 0;  // two query heads of one KV head per work tile
+  if (paired) {
+    for (int hq = 0; hq < d->num_q_heads; hq += 2) {
+      if (head_kind_host[hq / p.G] == 0)
+        p.dense_pairs[p.n_dense_pairs++] = (uint8_t)hq;
+      else
+        p.stream_pairs[p.n_stream_pairs++] = (uint8_t)hq;
+    }
+  }
   CUtensorMap qm, km, vm;
   if (!make_map_3d(&qm, q, d->seq_len, d->num_q_heads, d->head_dim) ||
       !make_map_3d(&km, k, d->seq_len, d->num_kv_heads, d->head_dim) ||
@@ -472,13 +823,26 @@ int prefill_entry(const lserve_prefill_desc* d, const void* q, const void* k, co
     return LSERVE_ERR_CUDA;
   const int sms = current_sm_count();
   if (sms <= 0) return LSERVE_ERR_CUDA;
-  const int tiles = d->num_q_heads * p.n_qt;
+  const int tiles = (paired ? d->num_q_heads / 2 : d->num_q_heads) * p.n_qt;
   const int grid = tiles < sms ? tiles : sms;
   cudaError_t e;
   // more than half of the SM's shared memory: one CTA per SM, so the 512-column
   // tensor-memory allocation never waits on a co-resident CTA
   const int kOneCtaSmem = 118 * 1024;
-  if (d->head_dim == 128) {
+  if (paired) {
+    // 512 tensor-memory columns: one CTA per SM (its shared memory alone guarantees that)
+    if (d->head_dim == 128) {
+      const int smem = std::max(PairLayout<128>::kBytes + 1024, kOneCtaSmem);
+      e = set_smem_once((const void*)prefill_pair_kernel<128>, smem);
+      if (e != cudaSuccess) return LSERVE_ERR_CUDA;
+      prefill_pair_kernel<128><<<grid, kPairThreads, smem, stream>>>(p, qm, km, vm);
+    } else {
+      const int smem = std::max(PairLayout<64>::kBytes + 1024, kOneCtaSmem);
+      e = set_smem_once((const void*)prefill_pair_kernel<64>, smem);
+      if (e != cudaSuccess) return LSERVE_ERR_CUDA;
+      prefill_pair_kernel<64><<<grid, kPairThreads, smem, stream>>>(p, qm, km, vm);
+    }
+  } else if (d->head_dim == 128) {
     const int smem = std::max(Layout<128>::kBytes + 1024, kOneCtaSmem);
     e = set_smem_once((const void*)prefill_kernel<128>, smem);
     if (e != cudaSuccess) return LSERVE_ERR_CUDA;
