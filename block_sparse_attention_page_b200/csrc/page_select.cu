@@ -3,8 +3,8 @@
 // "Top-K物理ページ" node of the 統一ブロックスパースアテンション figure).
 //
 // 1. page_score_kernel: a stream over the statistics pool.  One warp scores
-//    kScorePagesPerWarp physical pages, issuing all their stats loads before
-//    it reduces; D/8 lanes share a logical page, each holding 8 channels of
+//    kScorePagesPerWarp physical pages, issuing all their stats loads (into
+//    shared memory, by cp.async) before it reduces; D/8 lanes share a logical page, each holding 8 channels of
 //    the group-folded query Qp = sum_h max(q_h, 0), Qn = sum_h min(q_h, 0)
 //    (max(q*k_max, q*k_min) = max(q,0)*k_max + min(q,0)*k_min because
 //    k_max >= k_min).  Lanes reduce with shuffles, the max over the g logical
@@ -27,8 +27,15 @@ namespace lserve {
 // k_max >= k_min, max(q*k_max, q*k_min) = max(q,0)*k_max + min(q,0)*k_min, so
 //   S^j = sum_i Qp[i] * k_max^j[i] + Qn[i] * k_min^j[i]
 // with Qp[i] = sum_h max(q_h[i], 0) and Qn[i] = sum_h min(q_h[i], 0).
+// The stats loads go to shared memory by cp.async (16 bytes per lane and
+// load, each lane to its own slots), not to registers: with 71 registers
+// three blocks fit per SM and ~192 KB of statistics are in flight per SM --
+// staged in registers (127 of them) the kernel held two blocks per SM and
+// reached half the HBM bandwidth.
+constexpr int kScoreSmem = kScoreWarps * kScorePagesPerWarp * kScoreSteps * 2 * 32 * 16;
+
 template <int D, int G>
-__global__ void __launch_bounds__(kScoreWarps * 32, 2)
+__global__ void __launch_bounds__(kScoreWarps * 32, 3)
 page_score_kernel(SelectParams p) {
   constexpr int LPR = D / 8;      // lanes per logical page (16 channels x 8 = 128)
   constexpr int LPI = 32 / LPR;   // logical pages per warp step
@@ -87,7 +94,8 @@ page_score_kernel(SelectParams p) {
 
   const int steps = (g + LPI - 1) / LPI;
   for (int s0 = 0; s0 < steps; s0 += SB) {
-    uint4 mn[PW][SB], mx[PW][SB];
+    extern __shared__ uint4 sbuf[];  // [warp][PW][SB][k_min, k_max][lane]
+    uint4* mine = sbuf + (size_t)warp * PW * SB * 2 * 32;
     bool ok[PW][SB];
 #pragma unroll
     for (int j = 0; j < PW; ++j) {
@@ -97,19 +105,22 @@ page_score_kernel(SelectParams p) {
         const int sub = (s0 + t) * LPI + slot;
         ok[j][t] = pok[j] && s0 + t < steps && sub < g && (m0 + j) * g + sub < nlog;
         if (ok[j][t]) {
-          mn[j][t] = ldg_nc_v4(st + (size_t)sub * 2 * D);
-          mx[j][t] = ldg_nc_v4(st + (size_t)sub * 2 * D + D);
+          cp_async_16(mine + ((j * SB + t) * 2 + 0) * 32 + lane, st + (size_t)sub * 2 * D);
+          cp_async_16(mine + ((j * SB + t) * 2 + 1) * 32 + lane, st + (size_t)sub * 2 * D + D);
         }
       }
     }
+    cp_async_wait_all();  // this lane's copies have landed (each lane reads only its own slots)
 #pragma unroll
     for (int j = 0; j < PW; ++j) {
 #pragma unroll
       for (int t = 0; t < SB; ++t) {
         float part = 0.f;
         if (ok[j][t]) {
-          const uint32_t wn[4] = {mn[j][t].x, mn[j][t].y, mn[j][t].z, mn[j][t].w};
-          const uint32_t wx[4] = {mx[j][t].x, mx[j][t].y, mx[j][t].z, mx[j][t].w};
+          const uint4 vn = mine[((j * SB + t) * 2 + 0) * 32 + lane];
+          const uint4 vx = mine[((j * SB + t) * 2 + 1) * 32 + lane];
+          const uint32_t wn[4] = {vn.x, vn.y, vn.z, vn.w};
+          const uint32_t wx[4] = {vx.x, vx.y, vx.z, vx.w};
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
             part = fmaf(qp[2 * k], bf16_lo(wx[k]), part);
@@ -319,7 +330,9 @@ cudaError_t launch_page_select(const SelectParams& p, int D, cudaStream_t stream
   cudaError_t e = cudaSuccess;
 #define LSERVE_SCORE_CASE(DD, GG)                                                          \
   if (D == DD && G == GG) {                                                                \
-    e = launch_dependent(page_score_kernel<DD, GG>, grid, kScoreWarps * 32, 0, stream, p); \
+    e = set_smem_once((const void*)page_score_kernel<DD, GG>, kScoreSmem);                 \
+    if (e == cudaSuccess)                                                                  \
+      e = launch_dependent(page_score_kernel<DD, GG>, grid, kScoreWarps * 32, kScoreSmem, stream, p); \
   } else
   LSERVE_SCORE_CASE(64, 1)
   LSERVE_SCORE_CASE(64, 2)

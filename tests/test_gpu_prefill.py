@@ -62,6 +62,9 @@ SHAPES = [
     (640, 4, 1, 128, 64, 1, 4, [1]),             # streaming only, block 64
     (129, 2, 1, 128, 128, 1, 4, [0]),            # two query tiles, 1 row in the second
     (64, 4, 2, 64, 64, 1, 4, [0, 1]),            # shorter than one tile
+    (640, 12, 2, 64, 64, 1, 4, [0, 1]),          # G=6: three head pairs per KV head
+    (300, 16, 2, 128, 128, 1, 4, [1, 0]),        # G=8, ragged second tile
+    (450, 6, 3, 64, 128, 2, 2, [0, 1, 0]),       # G=2, D=64, two sink blocks
 ]
 
 
