@@ -35,6 +35,11 @@ Readings where the pages are silent (each is listed in the design notes):
      (pool page, KV head, channel) over the page's valid tokens, codes decided
      in float32 (quantize_kv8); attention attends code * scale.
      (parity unpinned by the pages: they name KV quantization, not a scheme)
+  R17 sequence-sharded decode (row f4): shard r of N holds the contiguous
+     physical pages [floor(M*r/N), floor(M*(r+1)/N)); each shard proposes its
+     own top-K, the global top-K is re-made from the proposals, and the
+     shards' attention results are merged by their log-sum-exp.  Pinned to the
+     unsharded selection and attention (the split changes no result).
 """
 from .lserve import (  # noqa: F401
     widen_bf16,
@@ -48,6 +53,11 @@ from .lserve import (  # noqa: F401
     page_tokens,
     decode_attention,
     decode_pair,
+    shard_bounds,
+    shard_candidates,
+    merge_candidates,
+    shard_streaming_pages,
+    lse_combine,
     kv_blocks,
     computed_blocks,
     theoretical_speedup,

@@ -139,6 +139,62 @@ def decode_pair(q, k, v, n, kind, N_L, N_P, K, sink, local, scale):
     return o, lse, pages
 
 
+# --- sequence-sharded decode (one long sequence over N GPUs) -------------------
+# Reading R17: the pages leave the multi-GPU split of one sequence open.  Shard
+# r of N holds the contiguous physical pages [floor(M*r/N), floor(M*(r+1)/N))
+# of a sequence of M pages; each shard scores its own pages, proposes its own
+# top-K, the proposals are exchanged, and the global choice is re-made from
+# them.  Attention runs per shard over the chosen pages it holds; the shards'
+# (o, lse) are then merged by their softmax normalisers.
+
+def shard_bounds(M: int, N: int) -> list:
+    """[P_0, ..., P_N] with P_r = floor(M * r / N): shard r holds pages [P_r, P_{r+1})."""
+    return [(M * r) // N for r in range(N + 1)]
+
+
+def shard_candidates(P_shard: np.ndarray, K: int, first_page: int) -> list:
+    """A shard's proposals: its own top-K pages (select_top_k on its scores),
+    as (score, global page index) pairs."""
+    return [(float(P_shard[m]), first_page + m) for m in select_top_k(P_shard, K)]
+
+
+def merge_candidates(cands, K: int, M: int) -> list:
+    """The global top-K re-made from every shard's proposals: the same order as
+    select_top_k -- score descending, then global page index ascending -- and
+    min(K, M) pages, returned ascending."""
+    order = sorted(cands, key=lambda c: (-c[0], c[1]))
+    return sorted(c[1] for c in order[:min(K, M)])
+
+
+def shard_streaming_pages(n: int, N_P: int, sink: int, local: int, lo: int, hi: int) -> list:
+    """A streaming head's pages (R5) that fall in shard pages [lo, hi), as shard-local ordinals."""
+    return [m - lo for m in streaming_pages(n, N_P, sink, local) if lo <= m < hi]
+
+
+def lse_combine(o_parts, lse_parts):
+    """Attention over disjoint token sets merged into attention over their union.
+
+    With o_r the softmax-weighted mean of v over set r and lse_r the natural log
+    of that set's sum of exp(logit): M = max_r lse_r, w_r = exp(lse_r - M),
+    o = sum_r w_r o_r / sum_r w_r and lse = M + log(sum_r w_r).  Sets with
+    lse_r = -inf weigh nothing; if every set is empty, o = 0 and lse = -inf.
+    o_parts [N][G][D], lse_parts [N][G]; returns (o [G][D], lse [G]).
+    """
+    o_parts = np.asarray(o_parts, dtype=np.float64)
+    lse_parts = np.asarray(lse_parts, dtype=np.float64)
+    N, G, D = o_parts.shape
+    o = np.zeros((G, D))
+    lse = np.full(G, -np.inf)
+    for g in range(G):
+        M = lse_parts[:, g].max()
+        if M == -np.inf:
+            continue
+        w = np.exp(lse_parts[:, g] - M)
+        o[g] = (w[:, None] * o_parts[:, g]).sum(axis=0) / w.sum()
+        lse[g] = M + math.log(w.sum())
+    return o, lse
+
+
 # --- prefill: block iterator [TD-static, TD-unified] ---------------------------
 
 def kv_blocks(i: int, kind: int, sink_blocks: int, local_blocks: int) -> list:
