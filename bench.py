@@ -579,7 +579,7 @@ def main():
         result["stages"]["attention_mha"] = mha_stage(lserve, synth, dev, stream, hbm_peak, timed)
     if not args.no_configs:
         result["stages"]["long_decode_256k"] = decode_config_stage(
-            lserve, synth, dev, stream, hbm_peak, timed, synth.long_decode_256k, 16)
+            lserve, synth, dev, stream, hbm_peak, timed, synth.long_decode_256k, 16, shards=4)
         result["stages"]["mixed_batch_decode"] = decode_config_stage(
             lserve, synth, dev, stream, hbm_peak, timed, synth.mixed_batch_decode, 3)
     if not args.no_kv8:
@@ -653,7 +653,7 @@ def mha_stage(lserve, synth, dev, stream, hbm_peak, timed, layers=8):
                         f"local={w.local}"}
 
 
-def decode_config_stage(lserve, synth, dev, stream, hbm_peak, timed, make, layers):
+def decode_config_stage(lserve, synth, dev, stream, hbm_peak, timed, make, layers, shards=1):
     """Selection and decode attention of another decode workload, each timed
     alone: `layers` replicas of its KV / stats / selection (together more bytes
     than L2 holds), graph replays, attention launched as in the main step."""
@@ -699,10 +699,15 @@ def decode_config_stage(lserve, synth, dev, stream, hbm_peak, timed, make, layer
     t_sel = timed(lambda: graphs[0].replay(), reps) / (reps * layers)
     t_att = timed(lambda: graphs[1].replay(), reps) / (reps * layers)
     acct = decode_bytes(w)
+    extra = {}
+    if shards > 1:
+        extra["seq_sharded"] = seqshard_timing(lserve, w, buf, d, dev, stream, timed, layers, shards,
+                                               scale)
     del graphs, buf
     torch.cuda.empty_cache()
     step = t_att + t_sel / REUSE
-    return {"attention": {"us": t_att * 1e6, "GB/s": acct["attn"] / t_att / 1e9,
+    return {**extra,
+            "attention": {"us": t_att * 1e6, "GB/s": acct["attn"] / t_att / 1e9,
                           "frac": acct["attn"] / t_att / 1e9 / hbm_peak, "bytes": acct["attn"]},
             "selection": {"us": t_sel * 1e6, "GB/s": acct["select"] / t_sel / 1e9,
                           "frac": acct["select"] / t_sel / 1e9 / hbm_peak, "bytes": acct["select"]},
@@ -711,6 +716,96 @@ def decode_config_stage(lserve, synth, dev, stream, hbm_peak, timed, make, layer
             "workload": f"{w.name}: B={w.B} n={int(w.ctx_lens.min())}..{int(w.ctx_lens.max())} "
                         f"H_q={w.H_q} H_kv={w.H_kv} D={w.D} N_L={w.N_L} N_P={w.N_P} "
                         f"top_k={w.top_k} sink={w.sink} local={w.local} reuse={REUSE}"}
+
+
+def seqshard_timing(lserve, w, buf, d, dev, stream, timed, layers, N, scale):
+    """Shard 0's part of an N-way sequence-sharded step of the same workload:
+    the selection part (its own pages' scores and top-K, its proposals, the
+    merge) and the attention part (attention over its chosen pages with float
+    partials, the combine), per layer, graph replays over the layer replicas.
+    Every shard's proposals and partials are computed once beforehand; the two
+    all-gathers between the parts cross GPUs and are not timed here."""
+    import torch
+    K, B, H_kv, H_q, D = w.top_k, w.B, w.H_kv, w.H_q, w.D
+    stride = lserve.seqshard_sel_stride(d, K, w.sink, w.local)
+    views = []
+    for r in range(N):
+        bounds = [lserve.seqshard_bounds(int(w.ctx_lens[b]), w.N_P, r, N) for b in range(B)]
+        ml = max([stride, 1] + [hi - lo for lo, hi, _ in bounds])
+        bt = np.full((B, ml), -1, dtype=np.int32)
+        for b, (lo, hi, _) in enumerate(bounds):
+            bt[b, :hi - lo] = w.block_table[b, lo:hi]
+        views.append((lserve.paged_desc(B, H_q, H_kv, D, w.N_L, w.N_P, ml, w.num_pool_pages),
+                      torch.from_numpy(bt).to(dev),
+                      torch.tensor([n for _, _, n in bounds], dtype=torch.int32, device=dev)))
+    i32, f32 = torch.int32, torch.float32
+    all_s = torch.empty((N, B, H_kv, K), dtype=f32, device=dev)
+    all_p = torch.empty((N, B, H_kv, K), dtype=i32, device=dev)
+    all_o = torch.empty((N, B * H_q, D), dtype=f32, device=dev)
+    all_l = torch.empty((N, B * H_q), dtype=f32, device=dev)
+    every_head = torch.zeros(H_kv, dtype=torch.uint8, device=dev)
+    sel = [torch.empty((B, H_kv, K), dtype=i32, device=dev) for _ in range(N)]
+    cnt = [torch.empty((B, H_kv), dtype=i32, device=dev) for _ in range(N)]
+    sc = [torch.empty((B, H_kv, v[0].max_pages_per_seq), dtype=f32, device=dev) for v in views]
+    sel_m = [torch.empty((B, H_kv, stride), dtype=i32, device=dev) for _ in range(N)]
+    cnt_m = [torch.empty((B, H_kv), dtype=i32, device=dev) for _ in range(N)]
+    wsd = [lserve.alloc_workspace(lserve.workspace_size(lserve.OP_DECODE, v[0], stride), device=dev)
+           for v in views]
+    outs = [torch.empty((B * H_q, D), dtype=torch.bfloat16, device=dev) for _ in range(layers)]
+
+    def select_part(r, l):
+        dr, bt, ctx = views[r]
+        lserve.page_select(dr, buf.q, buf.stats[l], bt, ctx, buf.head_kind, K, sel[r], cnt[r],
+                           phys_scores=sc[r])
+        lserve.seqshard_candidates(dr, r, N, buf.ctx_lens, buf.head_kind, sel[r], cnt[r], sc[r], K,
+                                   all_s[r], all_p[r])
+
+    def merge_part(r):
+        lserve.seqshard_merge(views[r][0], r, N, buf.ctx_lens, buf.head_kind, all_s, all_p, K, w.sink,
+                              w.local, sel_m[r], cnt_m[r])
+
+    def attend_part(r, l):
+        dr, bt, ctx = views[r]
+        lserve.sparse_decode_attn(dr, buf.q, buf.k_pools[l], buf.v_pools[l], bt, ctx, every_head,
+                                  sel_m[r], cnt_m[r], stride, w.sink, w.local, scale, all_o[r], all_l[r],
+                                  workspace=wsd[r], out_f32=True)
+
+    with torch.cuda.stream(stream):
+        for r in range(N):
+            select_part(r, 0)
+        for r in range(N):
+            merge_part(r)
+            attend_part(r, 0)
+    torch.cuda.synchronize()
+    assert lserve.read_device_status(stream) == lserve.OK
+
+    def sel0():
+        for l in range(layers):
+            select_part(0, l)
+            merge_part(0)
+
+    def att0():
+        for l in range(layers):
+            attend_part(0, l)
+            lserve.seqshard_combine(all_o, all_l, outs[l])
+    graphs = []
+    for fn in (sel0, att0):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            fn()
+        with torch.cuda.stream(stream):
+            for _ in range(3):
+                g.replay()
+        graphs.append(g)
+    reps = 20
+    t_sel = timed(lambda: graphs[0].replay(), reps) / (reps * layers)
+    t_att = timed(lambda: graphs[1].replay(), reps) / (reps * layers)
+    assert lserve.read_device_status(stream) == lserve.OK
+    del graphs
+    return {"shards": N, "timed_shard": 0, "selection_us": t_sel * 1e6, "attention_us": t_att * 1e6,
+            "us_per_layer_step": (t_att + t_sel / REUSE) * 1e6,
+            "not_timed": f"two all-gathers per step across GPUs: proposals {8 * B * H_kv * K} B and "
+                         f"partials {4 * B * H_q * (D + 1)} B per shard"}
 
 
 def kv8_stage(lserve, synth, dev, stream, hbm_peak, timed, make, layers, bf16_us):

@@ -32,9 +32,11 @@ EXPORTED = [
     "lserve_set_wait_limit_cycles", "lserve_debug_wait_timeout", "lserve_status_string",
     "lserve_bounds_checked", "lserve_page_select_noalloc", "lserve_sparse_decode_attn_ex",
     "lserve_decode_append", "lserve_prefill_to_pages", "lserve_quantize_pages_kv8",
-    "lserve_sparse_decode_attn_kv8",
+    "lserve_sparse_decode_attn_kv8", "lserve_seqshard_bounds", "lserve_seqshard_sel_stride",
+    "lserve_seqshard_candidates", "lserve_seqshard_merge", "lserve_seqshard_combine",
 ]
 DECODE_OVERLAP_PROLOGUE = 1
+DECODE_OUT_F32 = 2
 
 
 class LServeError(RuntimeError):
@@ -81,6 +83,15 @@ def _load(path):
                                                   vp, i32, i32, i32, ctypes.c_float, vp, vp,
                                                   ctypes.c_uint32, vp, sz, vp]
     lib.lserve_page_select_noalloc.argtypes = [P(PagedDesc), vp, vp, vp, vp, vp, i32, vp, vp, vp]
+    pi32 = P(i32)
+    lib.lserve_seqshard_bounds.argtypes = [i32, i32, i32, i32, pi32, pi32, pi32]
+    lib.lserve_seqshard_sel_stride.argtypes = [P(PagedDesc), i32, i32, i32]
+    lib.lserve_seqshard_sel_stride.restype = i32
+    lib.lserve_seqshard_candidates.argtypes = [P(PagedDesc), i32, i32, vp, vp, vp, vp, i32, vp, i32,
+                                               vp, vp, vp]
+    lib.lserve_seqshard_merge.argtypes = [P(PagedDesc), i32, i32, vp, vp, vp, vp, i32, i32, i32, vp,
+                                          vp, i32, vp]
+    lib.lserve_seqshard_combine.argtypes = [i32, i32, i32, vp, vp, vp, vp, vp]
     lib.lserve_page_select_noalloc.restype = ctypes.c_int
     lib.lserve_workspace_size.argtypes = [ctypes.c_int, vp, i32]
     lib.lserve_workspace_size.restype = sz
@@ -94,7 +105,8 @@ def _load(path):
                  "lserve_blocksparse_prefill", "lserve_read_device_status", "lserve_debug_wait_timeout",
                  "lserve_bounds_checked", "lserve_quantize_pages_kv8",
                  "lserve_sparse_decode_attn_kv8", "lserve_sparse_decode_attn_ex",
-                 "lserve_decode_append", "lserve_prefill_to_pages"):
+                 "lserve_decode_append", "lserve_prefill_to_pages", "lserve_seqshard_bounds",
+                 "lserve_seqshard_candidates", "lserve_seqshard_merge", "lserve_seqshard_combine"):
         getattr(lib, name).restype = ctypes.c_int
     return lib
 
@@ -159,17 +171,19 @@ def page_select_noalloc(desc, q, stats_pool, block_table, ctx_lens, head_kind, t
 
 def sparse_decode_attn(desc, q, k_pool, v_pool, block_table, ctx_lens, head_kind, sel, sel_count,
                        top_k, sink_tokens, local_tokens, softmax_scale, out, lse=None,
-                       workspace=None, stream=None, overlap_prologue=False):
-    """lserve_sparse_decode_attn; overlap_prologue=True calls
+                       workspace=None, stream=None, overlap_prologue=False, out_f32=False):
+    """lserve_sparse_decode_attn; overlap_prologue=True or out_f32=True call
     lserve_sparse_decode_attn_ex with LSERVE_DECODE_OVERLAP_PROLOGUE (the caller
     guarantees the previous kernel on the stream writes none of block_table,
-    ctx_lens, head_kind, sel, sel_count)."""
+    ctx_lens, head_kind, sel, sel_count) or LSERVE_DECODE_OUT_F32 (`out` is a
+    float32 tensor)."""
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    if overlap_prologue:
+    flags = (DECODE_OVERLAP_PROLOGUE if overlap_prologue else 0) | (DECODE_OUT_F32 if out_f32 else 0)
+    if flags:
         _check("lserve_sparse_decode_attn_ex", lib.lserve_sparse_decode_attn_ex(
             ctypes.byref(desc), _ptr(q), _ptr(k_pool), _ptr(v_pool), _ptr(block_table),
             _ptr(ctx_lens), _ptr(head_kind), _ptr(sel), _ptr(sel_count), top_k, sink_tokens,
-            local_tokens, float(softmax_scale), _ptr(out), _ptr(lse), DECODE_OVERLAP_PROLOGUE,
+            local_tokens, float(softmax_scale), _ptr(out), _ptr(lse), flags,
             _ptr(workspace), ws_bytes, _stream(stream)))
         return
     _check("lserve_sparse_decode_attn", lib.lserve_sparse_decode_attn(
@@ -227,6 +241,118 @@ def blocksparse_prefill(desc, q, k, v, head_kind_host, softmax_scale, out, lse=N
     _check("lserve_blocksparse_prefill", lib.lserve_blocksparse_prefill(
         ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), ctypes.cast(hk, ctypes.c_void_p),
         float(softmax_scale), _ptr(out), _ptr(lse), _ptr(workspace), ws_bytes, _stream(stream)))
+
+
+# --- sequence-sharded decode (one long sequence over several GPUs) -------------
+
+def seqshard_bounds(ctx_len: int, physical_page: int, rank: int, num_shards: int):
+    """(first page, end page, shard-local length) of shard `rank` (host only)."""
+    a, b, n = ctypes.c_int32(), ctypes.c_int32(), ctypes.c_int32()
+    _check("lserve_seqshard_bounds", lib.lserve_seqshard_bounds(
+        ctx_len, physical_page, rank, num_shards, ctypes.byref(a), ctypes.byref(b), ctypes.byref(n)))
+    return a.value, b.value, n.value
+
+
+def seqshard_sel_stride(desc, top_k: int, sink_tokens: int, local_tokens: int) -> int:
+    v = lib.lserve_seqshard_sel_stride(ctypes.byref(desc), top_k, sink_tokens, local_tokens)
+    if v <= 0:
+        raise LServeError("lserve_seqshard_sel_stride", ERR_INVALID_ARG, "invalid argument")
+    return v
+
+
+def seqshard_candidates(desc, rank, num_shards, ctx_lens_global, head_kind, sel, sel_count,
+                        phys_scores, top_k, cand_score, cand_page, stream=None):
+    """This shard's proposals from its own lserve_page_select result (`sel`'s
+    last dimension is the top_k that call used)."""
+    _check("lserve_seqshard_candidates", lib.lserve_seqshard_candidates(
+        ctypes.byref(desc), rank, num_shards, _ptr(ctx_lens_global), _ptr(head_kind), _ptr(sel),
+        _ptr(sel_count), sel.shape[-1], _ptr(phys_scores), top_k, _ptr(cand_score), _ptr(cand_page),
+        _stream(stream)))
+
+
+def seqshard_merge(desc, rank, num_shards, ctx_lens_global, head_kind, cand_score_all, cand_page_all,
+                   top_k, sink_tokens, local_tokens, sel_out, sel_count_out, stream=None):
+    """This shard's part of the global choice (`sel_out`'s last dimension is
+    the row length, at least seqshard_sel_stride)."""
+    _check("lserve_seqshard_merge", lib.lserve_seqshard_merge(
+        ctypes.byref(desc), rank, num_shards, _ptr(ctx_lens_global), _ptr(head_kind),
+        _ptr(cand_score_all), _ptr(cand_page_all), top_k, sink_tokens, local_tokens, _ptr(sel_out),
+        _ptr(sel_count_out), sel_out.shape[-1], _stream(stream)))
+
+
+def seqshard_combine(o_parts, lse_parts, out, lse=None, stream=None):
+    """o_parts float [N][rows][D], lse_parts float [N][rows] -> out bf16 [rows][D]."""
+    N, rows, D = o_parts.shape
+    _check("lserve_seqshard_combine", lib.lserve_seqshard_combine(
+        N, rows, D, _ptr(o_parts), _ptr(lse_parts), _ptr(out), _ptr(lse), _stream(stream)))
+
+
+class SeqShardStep:
+    """One shard's buffers and steps of a sequence-sharded decode step.
+
+    desc describes this shard's own paged cache (block-table rows of
+    max_pages_per_seq shard-local pages).  `all_gather(dst, src)` fills dst
+    [N, *src.shape] with every shard's src in shard order; the default is
+    torch.distributed.all_gather_into_tensor on `group` (NCCL between GPUs).
+    """
+
+    def __init__(self, desc, rank, num_shards, top_k, sink_tokens, local_tokens, device="cuda",
+                 group=None, all_gather=None):
+        B, H_q, H_kv, D = desc.batch, desc.num_q_heads, desc.num_kv_heads, desc.head_dim
+        self.desc, self.rank, self.N = desc, rank, num_shards
+        self.top_k, self.sink, self.local = top_k, sink_tokens, local_tokens
+        self.k_local = min(top_k, desc.max_pages_per_seq)
+        self.stride = seqshard_sel_stride(desc, top_k, sink_tokens, local_tokens)
+        if self.stride > desc.max_pages_per_seq:
+            raise LServeError("SeqShardStep", ERR_INVALID_ARG,
+                              "merged selection row longer than the shard's block-table row")
+        i32, f32 = torch.int32, torch.float32
+        self.sel = torch.empty((B, H_kv, self.k_local), dtype=i32, device=device)
+        self.cnt = torch.empty((B, H_kv), dtype=i32, device=device)
+        self.scores = torch.empty((B, H_kv, desc.max_pages_per_seq), dtype=f32, device=device)
+        self.cand_s = torch.empty((B, H_kv, top_k), dtype=f32, device=device)
+        self.cand_p = torch.empty((B, H_kv, top_k), dtype=i32, device=device)
+        self.all_s = torch.empty((num_shards, B, H_kv, top_k), dtype=f32, device=device)
+        self.all_p = torch.empty((num_shards, B, H_kv, top_k), dtype=i32, device=device)
+        self.sel_m = torch.empty((B, H_kv, self.stride), dtype=i32, device=device)
+        self.cnt_m = torch.empty((B, H_kv), dtype=i32, device=device)
+        self.all_heads = torch.zeros(H_kv, dtype=torch.uint8, device=device)
+        self.o = torch.empty((B * H_q, D), dtype=f32, device=device)
+        self.lse = torch.empty(B * H_q, dtype=f32, device=device)
+        self.all_o = torch.empty((num_shards, B * H_q, D), dtype=f32, device=device)
+        self.all_lse = torch.empty((num_shards, B * H_q), dtype=f32, device=device)
+        self.ws_dec = alloc_workspace(workspace_size(OP_DECODE, desc, self.stride), device)
+        if all_gather is None:
+            import torch.distributed as dist
+
+            def all_gather(dst, src):
+                dist.all_gather_into_tensor(dst, src, group=group)
+        self.all_gather = all_gather
+
+    def select(self, q, stats_pool, block_table, ctx_lens_local, ctx_lens_global, head_kind, stream=None):
+        """Steps 1-4: the shard's scores and own top-K, its proposals, their
+        exchange and the merge.  The result (sel_m, cnt_m) may be reused for
+        several decode steps."""
+        page_select(self.desc, q, stats_pool, block_table, ctx_lens_local, head_kind, self.k_local,
+                    self.sel, self.cnt, phys_scores=self.scores, stream=stream)
+        seqshard_candidates(self.desc, self.rank, self.N, ctx_lens_global, head_kind, self.sel, self.cnt,
+                            self.scores, self.top_k, self.cand_s, self.cand_p, stream=stream)
+        self.all_gather(self.all_s, self.cand_s)
+        self.all_gather(self.all_p, self.cand_p)
+        seqshard_merge(self.desc, self.rank, self.N, ctx_lens_global, head_kind, self.all_s, self.all_p,
+                       self.top_k, self.sink, self.local, self.sel_m, self.cnt_m, stream=stream)
+
+    def attend(self, q, k_pool, v_pool, block_table, ctx_lens_local, softmax_scale, out, lse=None,
+               stream=None):
+        """Steps 5-7: attention over the shard's chosen pages (float partials),
+        their exchange and the log-sum-exp combine into out bf16 [B][H_q][D]."""
+        sparse_decode_attn(self.desc, q, k_pool, v_pool, block_table, ctx_lens_local, self.all_heads,
+                           self.sel_m, self.cnt_m, self.stride, self.sink, self.local, softmax_scale,
+                           self.o, self.lse, workspace=self.ws_dec, stream=stream, out_f32=True)
+        self.all_gather(self.all_o, self.o)
+        self.all_gather(self.all_lse, self.lse)
+        seqshard_combine(self.all_o, self.all_lse, out.view(-1, out.shape[-1]),
+                         None if lse is None else lse.view(-1), stream=stream)
 
 
 def read_device_status(stream=None) -> int:

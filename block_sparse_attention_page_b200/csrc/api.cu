@@ -404,7 +404,8 @@ int decode_params(const lserve_paged_desc* desc, const void* q, const int32_t* b
                   float softmax_scale, void* out, float* lse, uint32_t flags, void* workspace,
                   size_t workspace_bytes, DecodeParams& p, int& grid) {
   if (!valid_paged(desc)) return LSERVE_ERR_INVALID_ARG;
-  if (flags & ~(uint32_t)LSERVE_DECODE_OVERLAP_PROLOGUE) return LSERVE_ERR_INVALID_ARG;
+  if (flags & ~(uint32_t)(LSERVE_DECODE_OVERLAP_PROLOGUE | LSERVE_DECODE_OUT_F32))
+    return LSERVE_ERR_INVALID_ARG;
   if (!q || !block_table || !ctx_lens || !head_kind || !sel || !sel_count || !out)
     return LSERVE_ERR_INVALID_ARG;
   if (!aligned(q, 16) || !aligned(out, 16) || !aligned(block_table, 4) || !aligned(ctx_lens, 4) ||
@@ -443,7 +444,8 @@ int decode_params(const lserve_paged_desc* desc, const void* q, const int32_t* b
   p.head_kind = head_kind;
   p.sel = sel;
   p.sel_count = sel_count;
-  p.out = static_cast<__nv_bfloat16*>(out);
+  if (flags & LSERVE_DECODE_OUT_F32) p.out_f32 = static_cast<float*>(out);
+  else p.out = static_cast<__nv_bfloat16*>(out);
   p.lse = lse;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   const size_t cnt_bytes = ((size_t)(P + 1) * 4 + 255) / 256 * 256;
@@ -555,6 +557,121 @@ int lserve_quantize_pages_kv8(const lserve_paged_desc* desc, const void* k_pool,
   p.status = device_status_word();
   if (!p.status) return LSERVE_ERR_CUDA;
   return cuda_status(launch_quantize_kv8(p, desc->head_dim, static_cast<cudaStream_t>(stream)));
+}
+
+int lserve_seqshard_bounds(int32_t ctx_len, int32_t physical_page, int32_t rank,
+                           int32_t num_shards, int32_t* first_page, int32_t* end_page,
+                           int32_t* local_len) {
+  if (ctx_len < 0 || physical_page < 1 || num_shards < 1 || rank < 0 || rank >= num_shards ||
+      !first_page || !end_page || !local_len)
+    return LSERVE_ERR_INVALID_ARG;
+  const long long M = ((long long)ctx_len + physical_page - 1) / physical_page;
+  const long long lo = M * rank / num_shards, hi = M * (rank + 1) / num_shards;
+  long long n = (long long)ctx_len - lo * physical_page;
+  const long long cap = (hi - lo) * physical_page;
+  n = n < 0 ? 0 : (n > cap ? cap : n);
+  *first_page = (int32_t)lo;
+  *end_page = (int32_t)hi;
+  *local_len = (int32_t)n;
+  return LSERVE_OK;
+}
+
+int32_t lserve_seqshard_sel_stride(const lserve_paged_desc* desc, int32_t top_k, int32_t sink_tokens,
+                                   int32_t local_tokens) {
+  if (!valid_paged(desc) || top_k < 1 || sink_tokens < 0 || local_tokens < 0) return 0;
+  const long long NP = desc->physical_page;
+  const long long stream = (sink_tokens + NP - 1) / NP + (local_tokens + NP - 1) / NP + 1;
+  const long long s = stream > top_k ? stream : top_k;
+  return s > 0x7fffffffll ? 0 : (int32_t)s;
+}
+
+int lserve_seqshard_candidates(const lserve_paged_desc* desc, int32_t rank, int32_t num_shards,
+                               const int32_t* ctx_lens_global, const uint8_t* head_kind,
+                               const int32_t* sel, const int32_t* sel_count, int32_t sel_top_k,
+                               const float* phys_scores, int32_t top_k, float* cand_score,
+                               int32_t* cand_page, void* stream) {
+  if (!valid_paged(desc)) return LSERVE_ERR_INVALID_ARG;
+  if (num_shards < 1 || rank < 0 || rank >= num_shards || top_k < 1 || sel_top_k < 1 ||
+      sel_top_k > desc->max_pages_per_seq)
+    return LSERVE_ERR_INVALID_ARG;
+  if (!ctx_lens_global || !head_kind || !sel || !sel_count || !phys_scores || !cand_score || !cand_page)
+    return LSERVE_ERR_INVALID_ARG;
+  if (!aligned(ctx_lens_global, 4) || !aligned(sel, 4) || !aligned(sel_count, 4) ||
+      !aligned(phys_scores, 4) || !aligned(cand_score, 4) || !aligned(cand_page, 4))
+    return LSERVE_ERR_INVALID_ARG;
+  ShardParams p = {};
+  p.ctx_lens = ctx_lens_global;
+  p.head_kind = head_kind;
+  p.sel = sel;
+  p.sel_count = sel_count;
+  p.scores = phys_scores;
+  p.cand_score = cand_score;
+  p.cand_page = cand_page;
+  p.batch = desc->batch;
+  p.num_kv_heads = desc->num_kv_heads;
+  p.physical_page = desc->physical_page;
+  p.max_pages = desc->max_pages_per_seq;
+  p.top_k = top_k;
+  p.sel_stride = sel_top_k;
+  p.rank = rank;
+  p.num_shards = num_shards;
+  p.status = device_status_word();
+  if (!p.status) return LSERVE_ERR_CUDA;
+  return cuda_status(launch_seqshard_candidates(p, static_cast<cudaStream_t>(stream)));
+}
+
+int lserve_seqshard_merge(const lserve_paged_desc* desc, int32_t rank, int32_t num_shards,
+                          const int32_t* ctx_lens_global, const uint8_t* head_kind,
+                          const float* cand_score_all, const int32_t* cand_page_all, int32_t top_k,
+                          int32_t sink_tokens, int32_t local_tokens, int32_t* sel_out,
+                          int32_t* sel_count_out, int32_t sel_stride, void* stream) {
+  if (!valid_paged(desc)) return LSERVE_ERR_INVALID_ARG;
+  if (num_shards < 1 || rank < 0 || rank >= num_shards || top_k < 1) return LSERVE_ERR_INVALID_ARG;
+  if (!ctx_lens_global || !head_kind || !cand_score_all || !cand_page_all || !sel_out || !sel_count_out)
+    return LSERVE_ERR_INVALID_ARG;
+  if (!aligned(ctx_lens_global, 4) || !aligned(cand_score_all, 4) || !aligned(cand_page_all, 4) ||
+      !aligned(sel_out, 4) || !aligned(sel_count_out, 4))
+    return LSERVE_ERR_INVALID_ARG;
+  const int32_t need = lserve_seqshard_sel_stride(desc, top_k, sink_tokens, local_tokens);
+  if (need == 0 || sel_stride < need) return LSERVE_ERR_INVALID_ARG;
+  if ((long long)num_shards * top_k * 8 > 200 * 1024) return LSERVE_ERR_UNSUPPORTED;
+  ShardParams p = {};
+  p.ctx_lens = ctx_lens_global;
+  p.head_kind = head_kind;
+  p.cand_score = const_cast<float*>(cand_score_all);
+  p.cand_page = const_cast<int32_t*>(cand_page_all);
+  p.out_sel = sel_out;
+  p.out_count = sel_count_out;
+  p.batch = desc->batch;
+  p.num_kv_heads = desc->num_kv_heads;
+  p.physical_page = desc->physical_page;
+  p.max_pages = desc->max_pages_per_seq;
+  p.top_k = top_k;
+  p.out_stride = sel_stride;
+  p.rank = rank;
+  p.num_shards = num_shards;
+  p.sink = sink_tokens;
+  p.local = local_tokens;
+  p.status = device_status_word();
+  if (!p.status) return LSERVE_ERR_CUDA;
+  return cuda_status(launch_seqshard_merge(p, static_cast<cudaStream_t>(stream)));
+}
+
+int lserve_seqshard_combine(int32_t num_shards, int32_t rows, int32_t head_dim, const float* o_parts,
+                            const float* lse_parts, void* out, float* lse, void* stream) {
+  if (num_shards < 1 || rows < 1 || (head_dim != 64 && head_dim != 128)) return LSERVE_ERR_INVALID_ARG;
+  if (!o_parts || !lse_parts || !out) return LSERVE_ERR_INVALID_ARG;
+  if (!aligned(o_parts, 4) || !aligned(lse_parts, 4) || !aligned(out, 2) || (lse && !aligned(lse, 4)))
+    return LSERVE_ERR_INVALID_ARG;
+  CombineParams p;
+  p.o_parts = o_parts;
+  p.lse_parts = lse_parts;
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.lse = lse;
+  p.num_shards = num_shards;
+  p.rows = rows;
+  p.head_dim = head_dim;
+  return cuda_status(launch_seqshard_combine(p, static_cast<cudaStream_t>(stream)));
 }
 
 int lserve_blocksparse_prefill(const lserve_prefill_desc* desc, const void* q, const void* k,

@@ -27,6 +27,13 @@ __device__ __forceinline__ void raise_status(unsigned int* word, int s) {
 // counts against max_pages) are always on: they cost a compare per page.
 constexpr bool kCheckBounds = true;
 
+// order-preserving map float -> uint32 for ranking page scores: a > b as
+// floats iff key(a) > key(b) as unsigned integers (-0 and +0 share one key)
+__device__ __forceinline__ uint32_t order_key(float f) {
+  uint32_t u = __float_as_uint(f == 0.f ? 0.f : f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
 // ---------------------------------------------------------------------------
 // bf16 helpers (storage is uint16; widening is exact)
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }

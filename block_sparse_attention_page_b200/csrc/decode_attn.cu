@@ -49,6 +49,12 @@ constexpr int kBarConsumers = 1;       // named barrier of the consumer warps
 constexpr int kMaxGrid = 512;          // CTAs whose range starts the range table holds
 constexpr unsigned kFull = 0xffffffffu;
 
+// One output element: bf16 by default, float with LSERVE_DECODE_OUT_F32.
+__device__ __forceinline__ void store_out(const DecodeParams& p, size_t i, float v) {
+  if (p.out_f32) p.out_f32[i] = v;
+  else p.out[i] = __float2bfloat16_rn(v);
+}
+
 // Pages the pair attends (retrieval: the selection; streaming: sink + local).
 __device__ __forceinline__ int pair_pages(const DecodeParams& p, int pair) {
   const int b = pair / p.num_kv_heads, h = pair - b * p.num_kv_heads;
@@ -436,7 +442,7 @@ decode_attn_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
       const int b = pr / p.num_kv_heads, h = pr - b * p.num_kv_heads;
       for (int g = 0; g < G; ++g) {
         const size_t qh = (size_t)b * p.num_q_heads + (size_t)h * G + g;
-        for (int c = 0; c < D; ++c) p.out[qh * D + c] = __float2bfloat16_rn(0.f);
+        for (int c = 0; c < D; ++c) store_out(p, qh * D + c, 0.f);
         if (p.lse) p.lse[qh] = -INFINITY;
       }
     }
@@ -787,7 +793,7 @@ decode_attn_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
       const size_t qh = (size_t)b * p.num_q_heads + (size_t)h * G + g;
       if (whole) {
         const bool empty_row = !(l > 0.f);
-        p.out[qh * D + c] = __float2bfloat16_rn(empty_row ? 0.f : o / l);
+        store_out(p, qh * D + c, empty_row ? 0.f : o / l);
         if (c == 0 && p.lse)
           p.lse[qh] = empty_row ? -INFINITY : (M + __log2f(l)) * 0.69314718055994530942f;
       } else {
@@ -882,7 +888,7 @@ decode_attn_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
         }
         const size_t qh = (size_t)b * p.num_q_heads + (size_t)h * G + g;
         const bool empty_row = !(lsum > 0.f);
-        p.out[qh * D + c] = __float2bfloat16_rn(empty_row ? 0.f : o / lsum);
+        store_out(p, qh * D + c, empty_row ? 0.f : o / lsum);
         if (c == 0 && p.lse)
           p.lse[qh] = empty_row ? -INFINITY : (M + __log2f(lsum)) * 0.69314718055994530942f;
       }
@@ -909,7 +915,7 @@ decode_attn_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
         }
         const size_t qh = (size_t)b * p.num_q_heads + (size_t)h * G + g;
         const bool empty_row = !(lsum > 0.f);
-        p.out[qh * D + c] = __float2bfloat16_rn(empty_row ? 0.f : o / lsum);
+        store_out(p, qh * D + c, empty_row ? 0.f : o / lsum);
         if (c == 0 && p.lse)
           p.lse[qh] = empty_row ? -INFINITY : (M + __log2f(lsum)) * 0.69314718055994530942f;
       }

@@ -58,7 +58,8 @@ struct DecodeParams {
   const uint8_t* head_kind;
   const int32_t* sel;
   const int32_t* sel_count;
-  __nv_bfloat16* out;
+  __nv_bfloat16* out;     // bf16 [B][H_q][D], or null when out_f32 is set
+  float* out_f32;         // float [B][H_q][D] instead (LSERVE_DECODE_OUT_F32)
   float* lse;
   uint32_t* counters;     // workspace [P]: segments finished per pair; zero between calls
   float* part_o;          // workspace [(grid + P)][G][D]: unnormalised partial outputs
@@ -124,6 +125,35 @@ struct QuantParams {
   int batch, num_kv_heads, physical_page, max_pages, num_pool_pages;
 };
 cudaError_t launch_quantize_kv8(const QuantParams& p, int D, cudaStream_t stream);
+
+// Sequence-sharded decode (seq_shard.cu): shard `rank` of `num_shards` holds
+// pages [floor(M*rank/N), floor(M*(rank+1)/N)) of each sequence.
+struct ShardParams {
+  const int32_t* ctx_lens;     // GLOBAL sequence lengths [B]
+  const uint8_t* head_kind;    // [H_kv]
+  // candidates: the shard's own selection
+  const int32_t* sel;          // [B][H_kv][sel_stride] shard-local page ordinals
+  const int32_t* sel_count;    // [B][H_kv]
+  const float* scores;         // [B][H_kv][max_pages] shard-local physical scores
+  float* cand_score;           // [B][H_kv][top_k] (candidates) / [N][B][H_kv][top_k] (merge)
+  int32_t* cand_page;          // global page ordinals, -1 = none
+  // merge: the shard's pages of the global choice
+  int32_t* out_sel;            // [B][H_kv][out_stride] shard-local ordinals, ascending, -1 padded
+  int32_t* out_count;          // [B][H_kv]
+  unsigned int* status;
+  int batch, num_kv_heads, physical_page, max_pages, top_k, sel_stride, out_stride;
+  int rank, num_shards, sink, local;
+};
+struct CombineParams {
+  const float* o_parts;        // [N][rows][D]
+  const float* lse_parts;      // [N][rows]
+  __nv_bfloat16* out;          // [rows][D]
+  float* lse;                  // [rows] or null
+  int num_shards, rows, head_dim;
+};
+cudaError_t launch_seqshard_candidates(const ShardParams& p, cudaStream_t stream);
+cudaError_t launch_seqshard_merge(const ShardParams& p, cudaStream_t stream);
+cudaError_t launch_seqshard_combine(const CombineParams& p, cudaStream_t stream);
 
 cudaError_t launch_page_stats(const StatsParams& p, int D, int max_logical_pages,
                               cudaStream_t stream);

@@ -145,12 +145,6 @@ page_score_kernel(SelectParams p) {
   }
 }
 
-// order-preserving map float -> uint32 (-0 and +0 map to the same key)
-__device__ __forceinline__ uint32_t order_key(float f) {
-  uint32_t u = __float_as_uint(f == 0.f ? 0.f : f);
-  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-}
-
 __global__ void __launch_bounds__(kTopkThreads) page_topk_kernel(SelectParams p) {
   extern __shared__ uint32_t keys[];  // [npages]
   __shared__ int hist[256];

@@ -226,10 +226,15 @@ int lserve_sparse_decode_attn(const lserve_paged_desc* desc, const void* q, cons
  *                                      run before that kernel completes
  *                                      (e.g. consecutive decode-attention
  *                                      calls of different layers).
+ *   LSERVE_DECODE_OUT_F32              `out` is float [B][H_q][D] (the
+ *                                      normalised output before bf16
+ *                                      rounding), e.g. a shard's partial
+ *                                      for lserve_seqshard_combine.
  * Any other bit: LSERVE_ERR_INVALID_ARG.  Everything else as
  * lserve_sparse_decode_attn.
  */
 #define LSERVE_DECODE_OVERLAP_PROLOGUE 1u
+#define LSERVE_DECODE_OUT_F32 2u
 int lserve_sparse_decode_attn_ex(const lserve_paged_desc* desc, const void* q, const void* k_pool,
                                  const void* v_pool, const int32_t* block_table,
                                  const int32_t* ctx_lens, const uint8_t* head_kind,
@@ -336,6 +341,93 @@ int lserve_page_select_noalloc(const lserve_paged_desc* desc, const void* q, con
 /* Bytes of workspace `op` needs for these shapes on the CURRENT device
  * (desc points to lserve_paged_desc, or lserve_prefill_desc for PREFILL).
  * Returns 0 for invalid shapes. */
+/*
+ * Sequence-sharded decode: one long sequence over N GPUs (one process each).
+ * [LServe explainer, 技術的詳細 › 動的スパーシティ / 階層的ページング: page scores
+ *  and the top-K; the split across GPUs is this library's reading -- the
+ *  pages leave it open.]
+ *
+ * Shard r of N holds the contiguous physical pages [P_r, P_{r+1}) of each
+ * sequence, P_r = floor(M * r / N), M = ceil(n / N_P) with n the GLOBAL
+ * length; its own paged cache holds them as shard-local ordinals 0.. with a
+ * shard-local length (lserve_seqshard_bounds).  One decode step per shard:
+ *   1. lserve_page_select(shard desc, local lengths, phys_scores non-NULL);
+ *   2. lserve_seqshard_candidates -> this shard's proposals [B][H_kv][top_k];
+ *   3. all-gather the proposals over the N shards (caller: NCCL) into
+ *      [N][B][H_kv][top_k], shard order;
+ *   4. lserve_seqshard_merge -> this shard's part of the global choice;
+ *   5. lserve_sparse_decode_attn_ex(shard desc, local lengths, head_kind all
+ *      0 (every head reads the merged selection), top_k = sel_stride,
+ *      flags LSERVE_DECODE_OUT_F32, lse non-NULL) -> float o, lse;
+ *   6. all-gather o [N][B*H_q][D] and lse [N][B*H_q] (caller);
+ *   7. lserve_seqshard_combine -> out bf16 [B][H_q][D].
+ * The choice equals the unsharded lserve_page_select bit for bit (the scores
+ * of a page do not depend on the shard; every page of the global top-K is in
+ * its own shard's top-K); out differs from the unsharded call only by
+ * rounding.  All calls are asynchronous on `stream`, allocate nothing, and
+ * set LSERVE_ERR_BOUNDS in the device status for out-of-range ordinals.
+ */
+
+/* Host only: this shard's page range [*first_page, *end_page) and its
+ * shard-local length (tokens of the sequence in those pages). */
+int lserve_seqshard_bounds(int32_t ctx_len, int32_t physical_page, int32_t rank,
+                           int32_t num_shards, int32_t* first_page, int32_t* end_page,
+                           int32_t* local_len);
+
+/* Host only: the row length of the merged selection, max(top_k,
+ * ceil(sink/N_P) + ceil(local/N_P) + 1); 0 on invalid arguments. */
+int32_t lserve_seqshard_sel_stride(const lserve_paged_desc* desc, int32_t top_k,
+                                   int32_t sink_tokens, int32_t local_tokens);
+
+/*
+ * lserve_seqshard_candidates -- this shard's proposals.  desc is the SHARD's
+ * descriptor (max_pages_per_seq = its block-table row length).  For each
+ * (b, h), proposal i < sel_count[b][h] (retrieval heads) is
+ *   cand_page  = P_r(b) + sel[b][h][i]          (global page ordinal)
+ *   cand_score = phys_scores[b][h][sel[b][h][i]]
+ * and the rest up to top_k are (-inf, -1); streaming heads propose nothing.
+ * sel / sel_count / phys_scores as lserve_page_select wrote them with top_k =
+ * sel_top_k (the row length of sel).  ctx_lens_global: int32 [B] device.
+ * Outputs float / int32 [B][H_kv][top_k], device.
+ */
+int lserve_seqshard_candidates(const lserve_paged_desc* desc, int32_t rank, int32_t num_shards,
+                               const int32_t* ctx_lens_global, const uint8_t* head_kind,
+                               const int32_t* sel, const int32_t* sel_count, int32_t sel_top_k,
+                               const float* phys_scores, int32_t top_k, float* cand_score,
+                               int32_t* cand_page, void* stream);
+
+/*
+ * lserve_seqshard_merge -- this shard's part of the global page choice.
+ * cand_score_all / cand_page_all: the all-gathered proposals [N][B][H_kv][top_k].
+ * Retrieval heads: the min(top_k, M) proposals first in (score descending,
+ * page ascending) order -- the unsharded top-K; those in [P_r, P_{r+1}) are
+ * written as shard-local ordinals, ascending.  Streaming heads: the sink
+ * pages [0, ceil(sink_tokens/N_P)) and every page holding one of the last
+ * local_tokens tokens (global positions), those in the shard, shard-local.
+ *   sel_out        int32 [B][H_kv][sel_stride], -1 padded;
+ *   sel_count_out  int32 [B][H_kv].
+ * sel_stride >= lserve_seqshard_sel_stride(desc, top_k, sink, local), else
+ * LSERVE_ERR_INVALID_ARG; N * top_k * 8 bytes must fit in shared memory
+ * (<= 200 KiB, else LSERVE_ERR_UNSUPPORTED).
+ */
+int lserve_seqshard_merge(const lserve_paged_desc* desc, int32_t rank, int32_t num_shards,
+                          const int32_t* ctx_lens_global, const uint8_t* head_kind,
+                          const float* cand_score_all, const int32_t* cand_page_all, int32_t top_k,
+                          int32_t sink_tokens, int32_t local_tokens, int32_t* sel_out,
+                          int32_t* sel_count_out, int32_t sel_stride, void* stream);
+
+/*
+ * lserve_seqshard_combine -- attention over disjoint token sets merged into
+ * attention over their union (log-sum-exp weights), per row (query head):
+ *   M = max_r lse[r], w_r = exp(lse[r] - M),
+ *   out = sum_r w_r o[r] / sum_r w_r   (bf16),   lse_out = M + log(sum_r w_r).
+ * Rows with every lse = -inf get out = 0, lse_out = -inf.
+ *   o_parts float [N][rows][head_dim], lse_parts float [N][rows] (natural log),
+ *   out bf16 [rows][head_dim], lse float [rows] or NULL; head_dim 64 or 128.
+ */
+int lserve_seqshard_combine(int32_t num_shards, int32_t rows, int32_t head_dim, const float* o_parts,
+                            const float* lse_parts, void* out, float* lse, void* stream);
+
 size_t lserve_workspace_size(int op, const void* desc, int32_t top_k);
 
 /* Synchronises `stream`, returns the first device-side error flag raised since
