@@ -634,7 +634,7 @@ int lserve_seqshard_merge(const lserve_paged_desc* desc, int32_t rank, int32_t n
     return LSERVE_ERR_INVALID_ARG;
   const int32_t need = lserve_seqshard_sel_stride(desc, top_k, sink_tokens, local_tokens);
   if (need == 0 || sel_stride < need) return LSERVE_ERR_INVALID_ARG;
-  if ((long long)num_shards * top_k * 8 > 200 * 1024) return LSERVE_ERR_UNSUPPORTED;
+  if ((long long)num_shards * top_k * 9 > 200 * 1024) return LSERVE_ERR_UNSUPPORTED;
   ShardParams p = {};
   p.ctx_lens = ctx_lens_global;
   p.head_kind = head_kind;

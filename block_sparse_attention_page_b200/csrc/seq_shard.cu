@@ -32,6 +32,7 @@ __device__ __forceinline__ int shard_first_page(int M, int r, int N) {
 
 constexpr int kMergeThreads = 256;
 constexpr int kMergeWarps = kMergeThreads / 32;
+constexpr int kRankMax = 512;  // up to this many proposals: ranked directly, no bisection
 
 // Sum of v over the block.  Two alternating slot rows make one barrier per
 // call enough: a row is written again only two calls later, after every
@@ -60,8 +61,8 @@ __global__ void seqshard_candidates_kernel(ShardParams p) {
   const int lo = shard_first_page(M, p.rank, p.num_shards);
   const int hi = shard_first_page(M, p.rank + 1, p.num_shards);
   const int own = min(hi - lo, p.max_pages);
-  int cnt = p.head_kind[h] == 0 ? p.sel_count[pair] : 0;
-  cnt = max(0, min(cnt, min(p.sel_stride, p.top_k)));
+  const int kind = p.head_kind[h], cnt_in = p.sel_count[pair];  // independent loads, issued together
+  const int cnt = kind == 0 ? max(0, min(cnt_in, min(p.sel_stride, p.top_k))) : 0;
   for (int i = threadIdx.x; i < p.top_k; i += blockDim.x) {
     float s = -INFINITY;
     int pg = -1;
@@ -80,14 +81,17 @@ __global__ void seqshard_candidates_kernel(ShardParams p) {
 }
 
 // One CTA per (sequence, KV head).  Retrieval heads: the global top-K of the
-// N * top_k proposals in shared memory, found without sorting -- the K-th
+// N * top_k proposals in shared memory, found without sorting.  Up to
+// kRankMax proposals, each one's rank is counted directly (the proposals that
+// come before it in (score descending, page ascending) order; pages are
+// unique, so ranks are too) -- no barrier inside.  Beyond that, the K-th
 // largest score key T by bisection over the 32-bit key space (each step one
 // block-wide count of keys >= the midpoint), then, among the proposals whose
 // key equals T, the lowest pages by a bisection over the page index.
 // Streaming heads: the sink pages [0, ceil(sink / N_P)) and the pages holding
 // the last local_tokens tokens, those in this shard.
 __global__ void __launch_bounds__(kMergeThreads) seqshard_merge_kernel(ShardParams p) {
-  extern __shared__ uint32_t smem[];  // keys [C], then pages [C]
+  extern __shared__ uint32_t smem[];  // keys [C], pages [C], chosen flags [C]
   __shared__ int red[2 * kMergeWarps];
   __shared__ int scan[kMergeWarps];
   const int h = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
@@ -121,6 +125,7 @@ __global__ void __launch_bounds__(kMergeThreads) seqshard_merge_kernel(ShardPara
   const int C = p.num_shards * K;
   uint32_t* key = smem;
   int* page = reinterpret_cast<int*>(smem + C);
+  uint8_t* chosen = reinterpret_cast<uint8_t*>(smem + 2 * C);
   int nvalid = 0;
   for (int c = tid; c < C; c += blockDim.x) {
     const int r = c / K, i = c - r * K;
@@ -138,37 +143,55 @@ __global__ void __launch_bounds__(kMergeThreads) seqshard_merge_kernel(ShardPara
   nvalid = block_sum(nvalid, red, phase);  // its barrier also publishes key / page
   const int keff = min(min(K, M), nvalid);
 
-  // T = the largest t with #{key >= t} >= keff (keff >= 1); every valid key >= 0
-  uint32_t T = 0;
-  int gt = 0;
-  uint32_t pstar = 0;
-  if (keff > 0) {
-    uint32_t tl = 0, th = 0xFFFFFFFFu;
-    while (tl < th) {
-      const uint32_t mid = tl + (uint32_t)(((uint64_t)th - tl + 1) >> 1);
-      int c_ge = 0;
-      for (int c = tid; c < C; c += blockDim.x) c_ge += page[c] >= 0 && key[c] >= mid;
-      if (block_sum(c_ge, red, phase) >= keff) tl = mid;
-      else th = mid - 1;
+  if (C <= kRankMax) {
+    for (int c = tid; c < C; c += blockDim.x) {
+      const int pg = page[c];
+      const uint32_t kc = key[c];
+      int r = 0;  // proposals ahead of this one (the same j for all threads: broadcast reads)
+      for (int j = 0; j < C; ++j) {
+        const int pj = page[j];
+        const uint32_t kj = key[j];
+        r += pj >= 0 && (kj > kc || (kj == kc && pj < pg));
+      }
+      chosen[c] = pg >= 0 && r < keff;
     }
-    T = tl;
-    int c_gt = 0;
-    for (int c = tid; c < C; c += blockDim.x) c_gt += page[c] >= 0 && key[c] > T;
-    gt = block_sum(c_gt, red, phase);
-    // the need = keff - gt lowest pages among key == T: P* = the smallest
-    // page bound with #{key == T, page <= P*} >= need
-    const int need = keff - gt;
-    uint32_t pl = 0, ph = (uint32_t)max(M - 1, 0);
-    while (pl < ph) {
-      const uint32_t mid = (pl + ph) >> 1;
-      int c_le = 0;
-      for (int c = tid; c < C; c += blockDim.x)
-        c_le += page[c] >= 0 && key[c] == T && (uint32_t)page[c] <= mid;
-      if (block_sum(c_le, red, phase) >= need) ph = mid;
-      else pl = mid + 1;
+  } else {
+    // T = the largest t with #{key >= t} >= keff (keff >= 1); every valid key >= 0
+    uint32_t T = 0;
+    uint32_t pstar = 0;
+    if (keff > 0) {
+      uint32_t tl = 0, th = 0xFFFFFFFFu;
+      while (tl < th) {
+        const uint32_t mid = tl + (uint32_t)(((uint64_t)th - tl + 1) >> 1);
+        int c_ge = 0;
+        for (int c = tid; c < C; c += blockDim.x) c_ge += page[c] >= 0 && key[c] >= mid;
+        if (block_sum(c_ge, red, phase) >= keff) tl = mid;
+        else th = mid - 1;
+      }
+      T = tl;
+      int c_gt = 0;
+      for (int c = tid; c < C; c += blockDim.x) c_gt += page[c] >= 0 && key[c] > T;
+      const int gt = block_sum(c_gt, red, phase);
+      // the need = keff - gt lowest pages among key == T: P* = the smallest
+      // page bound with #{key == T, page <= P*} >= need
+      const int need = keff - gt;
+      uint32_t pl = 0, ph = (uint32_t)max(M - 1, 0);
+      while (pl < ph) {
+        const uint32_t mid = (pl + ph) >> 1;
+        int c_le = 0;
+        for (int c = tid; c < C; c += blockDim.x)
+          c_le += page[c] >= 0 && key[c] == T && (uint32_t)page[c] <= mid;
+        if (block_sum(c_le, red, phase) >= need) ph = mid;
+        else pl = mid + 1;
+      }
+      pstar = pl;
     }
-    pstar = pl;
+    for (int c = tid; c < C; c += blockDim.x) {
+      const int pg = page[c];
+      chosen[c] = keff > 0 && pg >= 0 && (key[c] > T || (key[c] == T && (uint32_t)pg <= pstar));
+    }
   }
+  __syncthreads();
 
   // This shard's own proposals, slots [rank*K, rank*K + K), are its pages in
   // ascending order: the chosen ones are compacted in place by one block scan
@@ -176,12 +199,8 @@ __global__ void __launch_bounds__(kMergeThreads) seqshard_merge_kernel(ShardPara
   const int base = p.rank * K;
   const int per = (K + blockDim.x - 1) / blockDim.x;
   const int i0 = min(K, tid * per), i1 = min(K, i0 + per);
-  auto chosen = [&](int c) {
-    const int pg = page[c];
-    return keff > 0 && pg >= 0 && (key[c] > T || (key[c] == T && (uint32_t)pg <= pstar));
-  };
   int mine = 0;
-  for (int i = i0; i < i1; ++i) mine += chosen(base + i);
+  for (int i = i0; i < i1; ++i) mine += chosen[base + i];
   int incl = mine;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
@@ -198,7 +217,7 @@ __global__ void __launch_bounds__(kMergeThreads) seqshard_merge_kernel(ShardPara
     total += t;
   }
   for (int i = i0; i < i1; ++i)
-    if (chosen(base + i)) {
+    if (chosen[base + i]) {
       const int local = page[base + i] - lo;
       if (before < p.out_stride && local >= 0 && local < hi - lo) out[before] = local;
       ++before;
@@ -212,30 +231,42 @@ __global__ void __launch_bounds__(kMergeThreads) seqshard_merge_kernel(ShardPara
 }
 
 // One warp per output row (query head of a sequence): the N shards' (o, lse)
-// merged by their softmax normalisers.
+// merged by their softmax normalisers.  A lane holds D/32 channels; the
+// partials of four shards are loaded together (independent loads) before they
+// are summed.
 __global__ void seqshard_combine_kernel(CombineParams p) {
+  constexpr int kCpl = 4;  // channels per lane, D <= 128
+  constexpr int kBatch = 4;  // shards whose partials are in flight at once
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int row = blockIdx.x * (blockDim.x >> 5) + warp;
   if (row >= p.rows) return;
+  const int cpl = p.head_dim / 32;
   float M = -INFINITY;
   for (int r = 0; r < p.num_shards; ++r) M = fmaxf(M, p.lse_parts[(size_t)r * p.rows + row]);
   float wsum = 0.f;
-  for (int r = 0; r < p.num_shards; ++r) {
-    const float l = p.lse_parts[(size_t)r * p.rows + row];
-    wsum += (M == -INFINITY || l == -INFINITY) ? 0.f : expf(l - M);
-  }
-  for (int c = lane; c < p.head_dim; c += 32) {
-    float o = 0.f;
-    if (wsum > 0.f) {
-      for (int r = 0; r < p.num_shards; ++r) {
-        const float l = p.lse_parts[(size_t)r * p.rows + row];
-        if (l == -INFINITY) continue;
-        o += expf(l - M) * p.o_parts[((size_t)r * p.rows + row) * p.head_dim + c];
-      }
-      o /= wsum;
+  float acc[kCpl] = {0.f, 0.f, 0.f, 0.f};
+  for (int r0 = 0; r0 < p.num_shards; r0 += kBatch) {
+    float w[kBatch], v[kBatch][kCpl];
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int r = r0 + u;
+      const float l = r < p.num_shards ? p.lse_parts[(size_t)r * p.rows + row] : -INFINITY;
+      w[u] = (M == -INFINITY || l == -INFINITY) ? 0.f : expf(l - M);
+      const float* src = p.o_parts + ((size_t)r * p.rows + row) * p.head_dim + lane;
+#pragma unroll
+      for (int j = 0; j < kCpl; ++j) v[u][j] = (r < p.num_shards && j < cpl) ? src[32 * j] : 0.f;
     }
-    p.out[(size_t)row * p.head_dim + c] = __float2bfloat16_rn(o);
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      wsum += w[u];
+#pragma unroll
+      for (int j = 0; j < kCpl; ++j) acc[j] += w[u] * v[u][j];
+    }
   }
+#pragma unroll
+  for (int j = 0; j < kCpl; ++j)
+    if (j < cpl)
+      p.out[(size_t)row * p.head_dim + lane + 32 * j] = __float2bfloat16_rn(wsum > 0.f ? acc[j] / wsum : 0.f);
   if (lane == 0 && p.lse) p.lse[row] = wsum > 0.f ? M + logf(wsum) : -INFINITY;
 }
 
@@ -245,7 +276,7 @@ cudaError_t launch_seqshard_candidates(const ShardParams& p, cudaStream_t stream
 }
 
 cudaError_t launch_seqshard_merge(const ShardParams& p, cudaStream_t stream) {
-  const size_t smem = (size_t)p.num_shards * p.top_k * 8;
+  const size_t smem = ((size_t)p.num_shards * p.top_k * 9 + 15) / 16 * 16;
   if (smem > 48 * 1024) {
     const cudaError_t e = set_smem_once((const void*)seqshard_merge_kernel, (int)smem);
     if (e != cudaSuccess) return e;

@@ -407,7 +407,7 @@ int lserve_seqshard_candidates(const lserve_paged_desc* desc, int32_t rank, int3
  *   sel_out        int32 [B][H_kv][sel_stride], -1 padded;
  *   sel_count_out  int32 [B][H_kv].
  * sel_stride >= lserve_seqshard_sel_stride(desc, top_k, sink, local), else
- * LSERVE_ERR_INVALID_ARG; N * top_k * 8 bytes must fit in shared memory
+ * LSERVE_ERR_INVALID_ARG; N * top_k * 9 bytes must fit in shared memory
  * (<= 200 KiB, else LSERVE_ERR_UNSUPPORTED).
  */
 int lserve_seqshard_merge(const lserve_paged_desc* desc, int32_t rank, int32_t num_shards,
