@@ -638,8 +638,8 @@ int lserve_seqshard_merge(const lserve_paged_desc* desc, int32_t rank, int32_t n
   ShardParams p = {};
   p.ctx_lens = ctx_lens_global;
   p.head_kind = head_kind;
-  p.cand_score = const_cast<float*>(cand_score_all);
-  p.cand_page = const_cast<int32_t*>(cand_page_all);
+  p.all_score = cand_score_all;
+  p.all_page = cand_page_all;
   p.out_sel = sel_out;
   p.out_count = sel_count_out;
   p.batch = desc->batch;

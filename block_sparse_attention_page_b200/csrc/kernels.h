@@ -135,8 +135,10 @@ struct ShardParams {
   const int32_t* sel;          // [B][H_kv][sel_stride] shard-local page ordinals
   const int32_t* sel_count;    // [B][H_kv]
   const float* scores;         // [B][H_kv][max_pages] shard-local physical scores
-  float* cand_score;           // [B][H_kv][top_k] (candidates) / [N][B][H_kv][top_k] (merge)
+  float* cand_score;           // candidates' output [B][H_kv][top_k]
   int32_t* cand_page;          // global page ordinals, -1 = none
+  const float* all_score;      // merge's input: the gathered proposals [N][B][H_kv][top_k]
+  const int32_t* all_page;
   // merge: the shard's pages of the global choice
   int32_t* out_sel;            // [B][H_kv][out_stride] shard-local ordinals, ascending, -1 padded
   int32_t* out_count;          // [B][H_kv]

@@ -130,13 +130,13 @@ __global__ void __launch_bounds__(kMergeThreads) seqshard_merge_kernel(ShardPara
   for (int c = tid; c < C; c += blockDim.x) {
     const int r = c / K, i = c - r * K;
     const size_t idx = (((size_t)r * p.batch + b) * p.num_kv_heads + h) * K + i;
-    int pg = p.cand_page[idx];
+    int pg = p.all_page[idx];
     if (pg >= M) {  // a proposal past the sequence: ignored
       raise_status(p.status, LSERVE_ERR_BOUNDS);
       pg = -1;
     }
     page[c] = pg;
-    key[c] = pg >= 0 ? order_key(p.cand_score[idx]) : 0u;
+    key[c] = pg >= 0 ? order_key(p.all_score[idx]) : 0u;
     nvalid += pg >= 0;
   }
   int phase = 0;

@@ -139,6 +139,15 @@ def test_sharded_decode_shapes(G, D, N_P, K):
     _check_against_unsharded(w, res, run_sharded(w, buf, 3))
 
 
+def test_sharded_decode_many_proposals():
+    """4 shards x top-136 = 544 proposals: more than the merge ranks directly,
+    so the global choice comes from its bisection over score keys and pages."""
+    w = synth.decode_workload(2, 8, 2, 128, 16, 64, 136, 64, 256, [20000, 9000], seed=53)
+    buf = DecodeBuffers(w)
+    res = run_decode_path(buf)
+    _check_against_unsharded(w, res, run_sharded(w, buf, 4))
+
+
 @pytest.mark.parametrize("N", [4, 8])
 def test_long_decode_256k_sharded(N):
     w = synth.long_decode_256k()
