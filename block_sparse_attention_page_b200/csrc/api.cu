@@ -199,13 +199,11 @@ void lserve_set_wait_limit_cycles(uint64_t cycles) {
 }
 
 size_t lserve_workspace_size(int op, const void* desc, int32_t top_k) {
-  (void)top_k;
+  (void)top_k;  // no workspace depends on it
   if (!desc) return 0;
   switch (op) {
-    case LSERVE_OP_STATS: {
-      const auto* d = static_cast<const lserve_paged_desc*>(desc);
-      return valid_paged(d) ? 0 : 0;
-    }
+    case LSERVE_OP_STATS:  // the statistics kernel needs no workspace
+      return 0;
     case LSERVE_OP_SELECT: {
       const auto* d = static_cast<const lserve_paged_desc*>(desc);
       return valid_paged(d) ? select_ws(d) : 0;
