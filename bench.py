@@ -389,8 +389,12 @@ def main():
     scale = 1.0 / math.sqrt(w.D)
     ws_dec = lserve.alloc_workspace(lserve.workspace_size(lserve.OP_DECODE, d, w.top_k), device=dev)
     ws_sel = lserve.alloc_workspace(lserve.workspace_size(lserve.OP_SELECT, d, w.top_k), device=dev)
-    outs = [torch.empty_like(buf.out) for _ in range(LAYERS)]
-    qs = [buf.q.clone() for _ in range(LAYERS)]
+    # every layer's q and output are slices of one tensor each, so that a step's
+    # inputs and results cross the host link as one copy each (e2e below)
+    q_all = buf.q.unsqueeze(0).repeat(LAYERS, 1, 1, 1).contiguous()
+    out_all = torch.empty((LAYERS,) + tuple(buf.out.shape), dtype=buf.out.dtype, device=dev)
+    qs = [q_all[l] for l in range(LAYERS)]
+    outs = [out_all[l] for l in range(LAYERS)]
     stream = torch.cuda.Stream(device=dev)
     acct = decode_bytes(w)
 
@@ -522,20 +526,17 @@ def main():
     }
     del g_stats, g_append
 
-    # e2e: per step, copy the step's q (all layers) host->device from pinned memory,
-    # run the step, read every layer's output back to pinned host memory
-    q_host = torch.empty((LAYERS,) + tuple(buf.q.shape), dtype=torch.bfloat16).pin_memory()
-    o_host = torch.empty((LAYERS,) + tuple(buf.out.shape), dtype=torch.bfloat16).pin_memory()
-    q_host.copy_(torch.stack([q.cpu() for q in qs]))
-    q_dev = torch.empty_like(q_host, device=dev)
+    # e2e: per step, copy the step's q (all layers, one pinned buffer) host->device
+    # straight into the layers' q slices, run the step, read every layer's output
+    # back to pinned host memory in one copy
+    q_host = torch.empty(tuple(q_all.shape), dtype=torch.bfloat16).pin_memory()
+    o_host = torch.empty(tuple(out_all.shape), dtype=torch.bfloat16).pin_memory()
+    q_host.copy_(q_all.cpu())
 
     def e2e_step(t):
-        q_dev.copy_(q_host, non_blocking=True)
-        for l in range(LAYERS):
-            qs[l].copy_(q_dev[l], non_blocking=True)
+        q_all.copy_(q_host, non_blocking=True)
         (g_sel if t % REUSE == 0 else g_reuse).replay()
-        for l in range(LAYERS):
-            o_host[l].copy_(outs[l], non_blocking=True)
+        o_host.copy_(out_all, non_blocking=True)
 
     e2e_steps = min(args.steps, 400)
     e2e = None
