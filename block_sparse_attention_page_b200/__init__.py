@@ -294,6 +294,7 @@ class SeqShardStep:
     max_pages_per_seq shard-local pages).  `all_gather(dst, src)` fills dst
     [N, *src.shape] with every shard's src in shard order; the default is
     torch.distributed.all_gather_into_tensor on `group` (NCCL between GPUs).
+    Kernels and exchanges run on the current CUDA stream, in call order.
     """
 
     def __init__(self, desc, rank, num_shards, top_k, sink_tokens, local_tokens, device="cuda",
@@ -329,30 +330,29 @@ class SeqShardStep:
                 dist.all_gather_into_tensor(dst, src, group=group)
         self.all_gather = all_gather
 
-    def select(self, q, stats_pool, block_table, ctx_lens_local, ctx_lens_global, head_kind, stream=None):
+    def select(self, q, stats_pool, block_table, ctx_lens_local, ctx_lens_global, head_kind):
         """Steps 1-4: the shard's scores and own top-K, its proposals, their
         exchange and the merge.  The result (sel_m, cnt_m) may be reused for
         several decode steps."""
         page_select(self.desc, q, stats_pool, block_table, ctx_lens_local, head_kind, self.k_local,
-                    self.sel, self.cnt, phys_scores=self.scores, stream=stream)
+                    self.sel, self.cnt, phys_scores=self.scores)
         seqshard_candidates(self.desc, self.rank, self.N, ctx_lens_global, head_kind, self.sel, self.cnt,
-                            self.scores, self.top_k, self.cand_s, self.cand_p, stream=stream)
+                            self.scores, self.top_k, self.cand_s, self.cand_p)
         self.all_gather(self.all_s, self.cand_s)
         self.all_gather(self.all_p, self.cand_p)
         seqshard_merge(self.desc, self.rank, self.N, ctx_lens_global, head_kind, self.all_s, self.all_p,
-                       self.top_k, self.sink, self.local, self.sel_m, self.cnt_m, stream=stream)
+                       self.top_k, self.sink, self.local, self.sel_m, self.cnt_m)
 
-    def attend(self, q, k_pool, v_pool, block_table, ctx_lens_local, softmax_scale, out, lse=None,
-               stream=None):
+    def attend(self, q, k_pool, v_pool, block_table, ctx_lens_local, softmax_scale, out, lse=None):
         """Steps 5-7: attention over the shard's chosen pages (float partials),
         their exchange and the log-sum-exp combine into out bf16 [B][H_q][D]."""
         sparse_decode_attn(self.desc, q, k_pool, v_pool, block_table, ctx_lens_local, self.all_heads,
                            self.sel_m, self.cnt_m, self.stride, self.sink, self.local, softmax_scale,
-                           self.o, self.lse, workspace=self.ws_dec, stream=stream, out_f32=True)
+                           self.o, self.lse, workspace=self.ws_dec, out_f32=True)
         self.all_gather(self.all_o, self.o)
         self.all_gather(self.all_lse, self.lse)
         seqshard_combine(self.all_o, self.all_lse, out.view(-1, out.shape[-1]),
-                         None if lse is None else lse.view(-1), stream=stream)
+                         None if lse is None else lse.view(-1))
 
 
 def read_device_status(stream=None) -> int:
