@@ -96,9 +96,24 @@ def test_output_does_not_depend_on_the_split():
     assert lserve.read_device_status() == lserve.OK
     a = res["out"]
     bb = oracle.widen_bf16(bf16_bits(out2))
-    # at most one bf16 unit in the last place apart (the fp32 merge order differs)
+    # The fp32 sums are merged in another order: apart by at most one bf16 unit
+    # in the last place of the larger value, plus the fp32 rounding of the sums'
+    # terms (|p v| up to ~0.1 here, p carried as bf16 hi + lo: ~2^-16 of a term)
+    # for outputs that cancel to near zero.
     mag = np.maximum(np.maximum(np.abs(a), np.abs(bb)), 1e-30)
     ulp = 2.0 ** (np.floor(np.log2(mag)) - 7)
-    assert np.all(np.abs(a - bb) <= ulp)
+    d = np.abs(a - bb)
+    assert np.all(d <= ulp + 2e-5), (d.max(), (d / ulp).max(), int((d > ulp).sum()))
     l2 = lse2.cpu().numpy().astype(np.float64)
     assert np.allclose(l2, res["lse"], rtol=1e-5, atol=1e-5)
+    # and the second split meets the oracle on every pair
+    res2 = dict(res, out=bb, lse=l2)
+    G = w.G
+    for h in range(w.H_kv):
+        n = int(w.ctx_lens[0])
+        q = oracle.widen_bf16(w.q[0, h * G:(h + 1) * G])
+        k = oracle.widen_bf16(w.k_seq(0, h))
+        v = oracle.widen_bf16(w.v_seq(0, h))
+        pages = ([int(x) for x in res["sel"][0, h, :int(res["sel_count"][0, h])]] if w.head_kind[h] == 0
+                 else oracle.streaming_pages(n, w.N_P, w.sink, w.local))
+        check_outputs(w, res2, 0, h, q, k, v, pages)
