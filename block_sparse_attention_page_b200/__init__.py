@@ -287,6 +287,18 @@ def seqshard_combine(o_parts, lse_parts, out, lse=None, stream=None):
         N, rows, D, _ptr(o_parts), _ptr(lse_parts), _ptr(out), _ptr(lse), _stream(stream)))
 
 
+def process_group_all_gather(group=None):
+    """all_gather(dst, src) over a torch.distributed process group: dst[r] of
+    shape src.shape receives rank r's src (NCCL between GPUs; gloo too).  The
+    output is handed over as the concatenation along the first dimension (the
+    same memory as the [N, *src.shape] stack), the form every backend takes."""
+    import torch.distributed as dist
+
+    def all_gather(dst, src):
+        dist.all_gather_into_tensor(dst.view((-1,) + tuple(src.shape[1:])), src, group=group)
+    return all_gather
+
+
 class SeqShardStep:
     """One shard's buffers and steps of a sequence-sharded decode step.
 
@@ -323,12 +335,7 @@ class SeqShardStep:
         self.all_o = torch.empty((num_shards, B * H_q, D), dtype=f32, device=device)
         self.all_lse = torch.empty((num_shards, B * H_q), dtype=f32, device=device)
         self.ws_dec = alloc_workspace(workspace_size(OP_DECODE, desc, self.stride), device)
-        if all_gather is None:
-            import torch.distributed as dist
-
-            def all_gather(dst, src):
-                dist.all_gather_into_tensor(dst, src, group=group)
-        self.all_gather = all_gather
+        self.all_gather = all_gather if all_gather is not None else process_group_all_gather(group)
 
     def select(self, q, stats_pool, block_table, ctx_lens_local, ctx_lens_global, head_kind):
         """Steps 1-4: the shard's scores and own top-K, its proposals, their

@@ -190,3 +190,45 @@ def test_two_gloo_ranks_exchange_proposals_and_partials():
     for rank, same_sel, err_o, err_l in res:
         assert same_sel, rank
         assert err_o < 1e-12 and err_l < 1e-12, (rank, err_o, err_l)
+
+
+# --- the exchange SeqShardStep uses by default, as two gloo ranks ---------------------
+
+def _gather_main(rank, ws, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=ws)
+    try:
+        import block_sparse_attention_page_b200 as lserve
+        ag = lserve.process_group_all_gather()
+        # a rank's proposals (score, page) and partials, tagged by the rank
+        score = torch.full((2, 3, 4), float(rank) + 0.5)
+        page = torch.arange(24, dtype=torch.int32).reshape(2, 3, 4) + 100 * rank
+        all_s = torch.empty((ws, 2, 3, 4))
+        all_p = torch.empty((ws, 2, 3, 4), dtype=torch.int32)
+        ag(all_s, score)
+        ag(all_p, page)
+        lse = torch.arange(5, dtype=torch.float32) - rank       # 1-D, like the lse partials
+        all_l = torch.empty((ws, 5))
+        ag(all_l, lse)
+        ok = all(torch.all(all_s[r] == r + 0.5) and
+                 torch.equal(all_p[r], torch.arange(24, dtype=torch.int32).reshape(2, 3, 4) + 100 * r) and
+                 torch.equal(all_l[r], torch.arange(5, dtype=torch.float32) - r)
+                 for r in range(ws))
+        q.put((rank, bool(ok)))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_default_exchange_places_every_shard_in_order():
+    ws = 2
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_gather_main, args=(r, ws, port, q)) for r in range(ws)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=120) for _ in range(ws))
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert res == [(0, True), (1, True)]
