@@ -81,8 +81,8 @@ def test_reference_arm_prints_one_json_line_on_rank0(monkeypatch):
     import bench
     monkeypatch.setenv("RANK", "0")
     monkeypatch.setenv("WORLD_SIZE", "1")
-    monkeypatch.setattr(bench, "oracle_step_sample",
-                        lambda w, budget_s=0, max_pairs=None: (1e-3, "stub sample"))
+    monkeypatch.setattr(bench, "reference_steps",
+                        lambda w, steps, warmup: (1e-3 * steps, steps / 32, "stub sample"))
 
     class A:
         gpus, warmup, steps = 1, 3, 1
