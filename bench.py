@@ -643,7 +643,7 @@ def main():
         result["stages"]["prefill"] = prefill_stage(lserve, synth, dev, stream, tc_peak, timed,
                                                     args.prefill_seq)
 
-    if rank == 0 and not args.no_cpu_baseline:
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:  # the oracle baseline: one GPU runs only
         per_step, sample = oracle_step_sample(w, budget_s=15.0)
         cpu_val = acct["step"] / per_step / 1e9
         result["cpu_baseline"] = {"value": cpu_val, "unit": "GB/s", "cores": 1, "kind": "oracle",
