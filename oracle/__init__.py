@@ -62,6 +62,7 @@ from .lserve import (  # noqa: F401
     computed_blocks,
     theoretical_speedup,
     prefill_rows,
+    prefill_block_rows,
     prefill_flops,
     quantize_kv8,
     dequantize_kv8,

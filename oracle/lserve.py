@@ -261,6 +261,43 @@ def prefill_rows(q: np.ndarray, k: np.ndarray, v: np.ndarray, kind: int, block: 
     return o, lse
 
 
+def prefill_block_rows(q: np.ndarray, k: np.ndarray, v: np.ndarray, kind: int, block: int,
+                       sink_blocks: int, local_blocks: int, scale: float, rows):
+    """The same attention as prefill_rows for rows that all lie in ONE query
+    block i [TD-unified; TD-static]: every such row may see the same key blocks
+    kv_blocks(i), so their logits are one matrix product over those blocks
+    (keys s > t masked out of row t), followed by each row's softmax.  Used for
+    the long-sequence checks, where a row-by-row gather of up to T keys would
+    dominate the run time.
+
+    q [rows][D]; k, v [T][D] (one head).  Returns (o [rows][D], lse [rows]).
+    """
+    rows = np.asarray(rows, dtype=np.int64)
+    T, D = k.shape
+    i = int(rows[0]) // block
+    assert np.all(rows // block == i), "rows of one query block only"
+    blocks = kv_blocks(i, kind, sink_blocks, local_blocks)
+    keys = np.concatenate([np.arange(j * block, min((j + 1) * block, T)) for j in blocks])
+    # the allowed blocks are ascending and their union is a few contiguous runs:
+    # gather them as slices (views) rather than by index
+    runs, start = [], keys[0]
+    for a, b in zip(keys[:-1], keys[1:]):
+        if b != a + 1:
+            runs.append((start, a + 1))
+            start = b
+    runs.append((start, keys[-1] + 1))
+    ks = k[runs[0][0]:runs[0][1]] if len(runs) == 1 else np.concatenate([k[a:b] for a, b in runs])
+    vs = v[runs[0][0]:runs[0][1]] if len(runs) == 1 else np.concatenate([v[a:b] for a, b in runs])
+    z = scale * (q @ ks.T)                      # [rows][keys]
+    z[keys[None, :] > rows[:, None]] = -np.inf  # causal: keys s <= t only
+    zmax = z.max(axis=1, keepdims=True)
+    e = np.exp(z - zmax)
+    lsum = e.sum(axis=1)
+    o = (e @ vs) / lsum[:, None]
+    lse = zmax[:, 0] + np.log(lsum)
+    return o, lse
+
+
 # --- quantized KV cache [R15] ------------------------------------------------
 # The pages name KV-cache quantization (QServe KV4, combined with LServe's
 # sparsity in the abstract page) but give no scheme.  R15 reading: symmetric

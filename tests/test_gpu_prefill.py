@@ -1,7 +1,9 @@
 """GPU parity of the block-sparse prefill (tcgen05 kernel) against the fp64
 oracle: every row on small shapes (several query/key tiles, ragged tails, both
-head kinds, 64- and 128-token mask blocks, D = 64 and 128), and sampled rows on
-the 128K-token workload."""
+head kinds, 64- and 128-token mask blocks, D = 64 and 128), every row of 18 of
+the 32 query heads of a 16K-token sequence (many work units per CTA), and the
+128K-token workload's stratified sample (per query head: the first two and the
+last two query blocks, 8 random blocks and 256 random rows)."""
 import math
 
 import numpy as np
@@ -98,19 +100,85 @@ def test_prefill_repeated_calls_are_bitwise_identical():
     assert np.array_equal(a, b) and np.array_equal(la, lb)
 
 
-def test_prefill_128k_sampled_rows():
+def check_blocks(w, out, lse, plan, K=None, V=None):
+    """Compare the kernel's rows with the oracle's block-at-a-time form.
+
+    plan: {query head: {query block: row positions inside that block}}.  The
+    oracle reads each KV head's keys and values once (contiguous copies) and
+    each query block's rows of Q only.  Returns (worst |err|, rows checked)."""
+    K = oracle.widen_bf16(w.k()) if K is None else K
+    V = oracle.widen_bf16(w.v()) if V is None else V
+    scale = 1.0 / math.sqrt(w.D)
+    worst, checked, errs_sum = 0.0, 0, 0.0
+    for hk in range(w.H_kv):
+        heads = [hq for hq in plan if hq // w.G == hk]
+        if not heads:
+            continue
+        kh = np.ascontiguousarray(K[:, hk])
+        vh = np.ascontiguousarray(V[:, hk])
+        for i in sorted(set(b for hq in heads for b in plan[hq])):
+            t0, t1 = i * w.block, min((i + 1) * w.block, w.T)
+            q_blk = oracle.widen_bf16(w.q_rows(t0, t1))
+            # the rows the group's query heads need from this block, stacked into
+            # one call (they see the same key blocks)
+            parts = [(hq, np.asarray(sorted(plan[hq][i]), dtype=np.int64))
+                     for hq in heads if i in plan[hq]]
+            rows = np.concatenate([r for _, r in parts])
+            qs = np.concatenate([q_blk[r - t0, hq] for hq, r in parts])
+            o_all, ls_all = oracle.prefill_block_rows(qs, kh, vh, int(w.head_kind[hk]), w.block,
+                                                      w.sink_blocks, w.local_blocks, scale, rows)
+            at = 0
+            for hq, r in parts:
+                o, ls = o_all[at:at + len(r)], ls_all[at:at + len(r)]
+                at += len(r)
+                err = np.abs(out[r, hq] - o)
+                worst = max(worst, float(err.max()))
+                errs_sum += float(err.sum())
+                checked += len(r)
+                assert err.max() <= OUT_MAX_ABS, (hq, i, err.max())
+                assert err.mean() <= OUT_MEAN_ABS, (hq, i, err.mean())
+                assert np.max(np.abs(lse[hq, r] - ls)) <= LSE_ABS, (hq, i)
+    return worst, checked, errs_sum / max(1, checked * w.D)
+
+
+def test_prefill_16k_all_rows_multi_round():
+    """More (query head, 128-row tile) work units than the GPU has SMs
+    (16,384 tokens x 32 query heads = 4,096 units, 2,048 head pairs), so every
+    CTA of the persistent grid runs many rounds: all rows of all 16 Lambda
+    query heads and of two dense query heads are checked."""
+    w = synth.prefill_workload(16384, 32, 8, 128, 128, 1004, name="prefill_16k")
+    out, lse = run_prefill(w)
+    nb = -(-w.T // w.block)
+    full = {i: np.arange(i * w.block, min((i + 1) * w.block, w.T)) for i in range(nb)}
+    heads = [0, 13] + [hq for hq in range(w.H_q) if w.head_kind[hq // w.G] == 1]
+    worst, checked, mean = check_blocks(w, out, lse, {hq: full for hq in heads})
+    assert checked == len(heads) * w.T
+    print(f"16K prefill: {checked} rows, worst |err| = {worst:.4g}, mean |err| = {mean:.3g}")
+
+
+def test_prefill_128k_stratified_rows():
+    """The 128K workload, per query head: the first two and the last two
+    query blocks in full, 8 seeded-random blocks in full and 256 seeded-random
+    rows (drawn per KV head and checked for each of its query heads; all 32
+    query heads, dense and Lambda)."""
     w = synth.prefill_128k()
     out, lse = run_prefill(w)
-    Q, K, V = (oracle.widen_bf16(x) for x in (w.q(), w.k(), w.v()))
-    rng = np.random.default_rng(4)
-    T = w.T
-    fixed = np.array([0, 1, 127, 128, 129, 511, 512, 640, T // 2, T - 129, T - 128, T - 2, T - 1])
-
-    def rows(hq):
-        extra = rng.integers(0, T, 12)
-        return np.unique(np.concatenate([fixed, extra]))
-    worst = check_rows(w, out, lse, rows, Q, K, V)
-    print("128K prefill: worst sampled |err| =", worst)
+    K, V = oracle.widen_bf16(w.k()), oracle.widen_bf16(w.v())
+    nb = -(-w.T // w.block)
+    rng = np.random.default_rng(20250214)
+    plan = {}
+    for hk in range(w.H_kv):
+        # 256 random rows per KV head, checked for each of its query heads
+        rows = rng.choice(w.T, 256, replace=False)
+        for hq in range(hk * w.G, (hk + 1) * w.G):
+            blocks = {0, 1, nb - 2, nb - 1}
+            blocks |= set(int(x) for x in rng.choice(np.arange(2, nb - 2), 8, replace=False))
+            rows_of = {i: set(range(i * w.block, min((i + 1) * w.block, w.T))) for i in blocks}
+            for t in rows:
+                rows_of.setdefault(int(t) // w.block, set()).add(int(t))
+            plan[hq] = rows_of
+    worst, checked, mean = check_blocks(w, out, lse, plan, K, V)
+    print(f"128K prefill: {checked} rows, worst |err| = {worst:.4g}, mean |err| = {mean:.3g}")
     assert np.all(np.isfinite(out[::997]))
 
 

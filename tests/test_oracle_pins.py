@@ -349,6 +349,53 @@ def test_prefill_lambda_matches_masked_attention():
     assert np.allclose(o, _sdpa(q, k, v, 0.3, mask=visible), rtol=1e-12, atol=1e-12)
 
 
+@pytest.mark.parametrize("kind", [0, 1])
+def test_prefill_block_rows_match_masked_attention(kind):
+    """The block-at-a-time form against torch SDPA with the causal mask (dense
+    heads) or the R6 Lambda mask (streaming heads), every block of a ragged
+    sequence in full, and lse against scipy's logsumexp of the masked logits."""
+    from scipy.special import logsumexp
+    rng = _rng(26 + kind)
+    T, D, B = 16 * 11 + 5, 8, 16
+    q, k, v = (_bf16_values(rng, (T, D)) for _ in range(3))
+    t_idx = np.arange(T)
+    bt, bs = t_idx[:, None] // B, t_idx[None, :] // B
+    visible = t_idx[None, :] <= t_idx[:, None]
+    if kind == 1:
+        visible &= (bs == 0) | (bt - bs < 4)
+    want = _sdpa(q, k, v, 0.3, mask=visible)
+    z = 0.3 * q @ k.T
+    z[~visible] = -np.inf
+    want_lse = logsumexp(z, axis=1)
+    for i in range(-(-T // B)):
+        rows = np.arange(i * B, min((i + 1) * B, T))
+        o, lse = oracle.prefill_block_rows(q[rows], k, v, kind, B, 1, 4, 0.3, rows)
+        assert np.allclose(o, want[rows], rtol=1e-12, atol=1e-12), i
+        assert np.allclose(lse, want_lse[rows], rtol=1e-13, atol=1e-13), i
+    # a scattered subset of one block's rows
+    rows = np.array([16 * 9 + 1, 16 * 9 + 7, 16 * 9 + 15])
+    o, _ = oracle.prefill_block_rows(q[rows], k, v, kind, B, 1, 4, 0.3, rows)
+    assert np.allclose(o, want[rows], rtol=1e-12, atol=1e-12)
+
+
+def test_prefill_block_rows_closed_forms():
+    rng = _rng(28)
+    T, D, B = 64, 8, 16
+    q, k, v = (_bf16_values(rng, (T, D)) for _ in range(3))
+    # row 0 sees only key 0: o = v[0], lse = scale * q0 . k0
+    o, lse = oracle.prefill_block_rows(q[:1], k, v, 0, B, 1, 4, 0.5, [0])
+    assert np.array_equal(o[0], v[0]) and lse[0] == pytest.approx(0.5 * q[0] @ k[0], rel=1e-15)
+    # identical keys: the row is the mean of the values it may see
+    kk = np.repeat(k[:1], T, axis=0)
+    rows = np.arange(48, 64)
+    o, _ = oracle.prefill_block_rows(q[rows], kk, v, 0, B, 1, 4, 0.5, rows)
+    for r, t in enumerate(rows):
+        assert np.allclose(o[r], v[:t + 1].mean(axis=0), rtol=1e-12, atol=1e-12)
+    # rows of two different blocks are refused
+    with pytest.raises(AssertionError):
+        oracle.prefill_block_rows(q[[15, 16]], k, v, 0, B, 1, 4, 0.5, [15, 16])
+
+
 def test_method_constants_in_workloads():
     c = _golden("method_constants.json")
     for make in synth.DECODE_CONFIGS.values():
