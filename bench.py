@@ -44,7 +44,8 @@ sys.path.insert(0, ROOT)
 
 LAYERS = 32
 REUSE = 4
-DEFAULT_STEPS = 6000
+DEFAULT_STEPS = 6000          # GPU arm: 32-layer steps
+DEFAULT_REF_STEPS = 200      # reference arm: layer-steps of the oracle (~20 s on one core)
 DEFAULT_WARMUP = 8
 METRIC = "sparse decode attn µs/step & HBM GB/s; block-sparse prefill TFLOP/s"
 
@@ -137,25 +138,20 @@ def stats_build_bytes(w):
     return rd + wr
 
 
-def decode_traffic():
-    """DRAM bytes (read + write) per decode-attention launch from the committed
-    ncu summary, provided the kernel source is still the one it measured."""
+def kernel_traffic(kernel):
+    """DRAM bytes (read + write) per launch of `kernel` from the committed ncu
+    record (profiles/traffic.json), provided the kernel's source file still
+    hashes to the one the counters were taken on; otherwise None."""
     import hashlib
-    summ = os.path.join(ROOT, "profiles", "decode_attn_llama3_8b_decode.md")
-    src = os.path.join(ROOT, "block_sparse_attention_page_b200", "csrc", "decode_attn.cu")
     try:
-        fields = {}
-        with open(summ) as f:
-            for line in f:
-                if line.startswith("- ") and ":" in line:
-                    k, v = line[2:].split(":", 1)
-                    fields[k.strip()] = v.strip().strip("`")
-        with open(src, "rb") as f:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            rec = json.load(f)[kernel]
+        with open(os.path.join(ROOT, rec["source"]), "rb") as f:
             digest = hashlib.sha256(f.read()).hexdigest()
-        if fields.get("decode_attn.cu sha256") != digest:
+        if rec["source_sha256"] != digest:
             return None
-        return float(fields["traffic bytes per launch"])
-    except (OSError, KeyError, ValueError):
+        return float(rec["traffic_bytes_per_launch"])
+    except (OSError, KeyError, ValueError, TypeError):
         return None
 
 
@@ -250,123 +246,286 @@ def whole_job_value(bytes_per_rank_step, steps, ws, elapsed_max_s):
 
 # --- the CPU oracle baseline ----------------------------------------------------
 
-def oracle_step_sample(w, budget_s=12.0, max_pairs=None):
-    """Time the oracle's decode step (stats of the retrieval heads already
-    built, as on the GPU; then S^j -> P^m -> top-K -> attention per pair) on a
-    bounded sample of (sequence, KV head) pairs; returns seconds per layer-step
-    extrapolated from the pairs timed, and what was sampled."""
-    import oracle
+def host_cpu():
+    """The host's CPU model and core counts."""
+    model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    try:
+        usable = len(os.sched_getaffinity(0))
+    except (AttributeError, OSError):
+        usable = os.cpu_count()
+    return {"model": model, "nproc": os.cpu_count(), "usable_cores": usable}
+
+
+class OraclePair:
+    """One (sequence, KV head) of the decode workload in the oracle's hands:
+    q, K and V widened to float64, and for a retrieval head its page statistics
+    (built once beforehand, as the GPU builds them once after the prefill).
+    visit() is what one decode step costs this pair: the page selection
+    (S^j -> P^m -> top-K) when `select` is set, and the attention over the
+    attended pages -- the gather of their tokens included."""
+
+    def __init__(self, w, b, h):
+        import oracle
+        G = w.G
+        self.w, self.kind = w, int(w.head_kind[h])
+        self.n = int(w.ctx_lens[b])
+        self.q = oracle.widen_bf16(w.q[b, h * G:(h + 1) * G])
+        self.k = oracle.widen_bf16(w.k_seq(b, h))
+        self.v = oracle.widen_bf16(w.v_seq(b, h))
+        self.stats = oracle.page_stats(self.k, w.N_L) if self.kind == 0 else None
+        self.pages = None
+        self.scale = 1.0 / math.sqrt(w.D)
+
+    def visit(self, select):
+        import oracle
+        w = self.w
+        if self.kind == 0:
+            if select or self.pages is None:
+                P = oracle.physical_scores(oracle.logical_scores(self.q, *self.stats), w.g)
+                self.pages = oracle.select_top_k(P, w.top_k)
+            pages = self.pages
+        else:
+            pages = oracle.streaming_pages(self.n, w.N_P, w.sink, w.local)
+        oracle.decode_attention(self.q, self.k, self.v, oracle.page_tokens(pages, self.n, w.N_P),
+                                self.scale)
+
+
+def _one_thread():
+    """Limit BLAS / OpenMP pools of this process to one thread."""
     try:
         from threadpoolctl import threadpool_limits
-        lim = threadpool_limits(1)
+        return threadpool_limits(1)
     except Exception:
-        lim = None
-    G = w.G
-    scale = 1.0 / math.sqrt(w.D)
-    pairs = [(b, h) for b in range(w.B) for h in range(w.H_kv)]
-    t_sel = t_attn = 0.0
-    done = 0
-    t_start = time.perf_counter()
-    for (b, h) in pairs:
-        n = int(w.ctx_lens[b])
-        q = oracle.widen_bf16(w.q[b, h * G:(h + 1) * G])
-        k = oracle.widen_bf16(w.k_seq(b, h))
-        v = oracle.widen_bf16(w.v_seq(b, h))
-        if w.head_kind[h] == 0:
-            kmin, kmax = oracle.page_stats(k, w.N_L)      # built once, not timed (GPU: not per step)
-            t0 = time.perf_counter()
-            P = oracle.physical_scores(oracle.logical_scores(q, kmin, kmax), w.g)
-            pages = oracle.select_top_k(P, w.top_k)
-            t1 = time.perf_counter()
-            t_sel += t1 - t0
+        return None
+
+
+def oracle_layer_steps(pairs, t0, steps):
+    """Run layer-steps t0 .. t0 + steps - 1 over the given pairs (selection on
+    every REUSE-th step, as the GPU step reuses it); returns seconds."""
+    start = time.perf_counter()
+    for t in range(t0, t0 + steps):
+        for pr in pairs:
+            pr.visit(t % REUSE == 0)
+    return time.perf_counter() - start
+
+
+def oracle_single_thread(w, budget_s=8.0):
+    """The oracle's decode step on one thread: whole layer-steps (all pairs),
+    as many complete reuse windows as fit the budget.  Returns (s / layer-step,
+    layer-steps timed)."""
+    lim = _one_thread()
+    pairs = [OraclePair(w, b, h) for b in range(w.B) for h in range(w.H_kv)]
+    oracle_layer_steps(pairs, 0, 1)           # warm-up (selection made)
+    steps, elapsed = 0, 0.0
+    while elapsed < budget_s or steps < REUSE:
+        elapsed += oracle_layer_steps(pairs, REUSE + steps, REUSE)
+        steps += REUSE
+    del lim
+    return elapsed / steps, steps
+
+
+def _bundles(w):
+    """The workload's (sequence, KV head) pairs grouped into bundles of equal
+    cost: a retrieval pair with a streaming pair (their visits cost ~10:1)."""
+    P = w.B * w.H_kv
+    retr = [p for p in range(P) if w.head_kind[p % w.H_kv] == 0]
+    strm = [p for p in range(P) if w.head_kind[p % w.H_kv] != 0]
+    out = [list(x) for x in zip(retr, strm)]
+    rest = retr[len(out):] + strm[len(out):]
+    return out + [[p] for p in rest]
+
+
+def _oracle_worker(args):
+    """One process of the all-core run (spawned): builds its bundles of pairs,
+    waits for the others, then runs layer-steps [s0, s1) over them."""
+    bundle_ids, s0, s1, barrier = args
+    lim = _one_thread()
+    import synth
+    w = synth.llama3_8b_decode()
+    bundles = _bundles(w)
+    pairs = [OraclePair(w, p // w.H_kv, p % w.H_kv) for i in bundle_ids for p in bundles[i]]
+    oracle_layer_steps(pairs, 0, 1)
+    barrier.wait()
+    elapsed = oracle_layer_steps(pairs, s0, s1 - s0)
+    del lim
+    return elapsed
+
+
+def oracle_all_cores(w, t_single, budget_s=6.0):
+    """The oracle's decode step on the host's cores: one spawned process per
+    core, each holding whole bundles (a retrieval + a streaming pair).  With W
+    processes and nb bundles: W <= nb -> a process takes the bundles i with
+    i mod W = its index, for every layer-step; W = R * nb -> a process takes
+    one bundle and a contiguous 1/R of the layer-steps.  Every process starts
+    at a barrier; the S layer-steps take the slowest process's time.
+    t_single (s per layer-step on one thread) sizes S to about budget_s.
+    Returns (s / layer-step, processes, layer-steps)."""
+    import multiprocessing as mp
+    nb = len(_bundles(w))
+    cores = host_cpu()["usable_cores"] or 1
+    if cores >= nb:
+        R = cores // nb
+        nw = nb * R
+    else:
+        R, nw = 1, 1
+        while nw * 2 <= cores and nb % (nw * 2) == 0:
+            nw *= 2
+    per = max(REUSE, int(budget_s * nw / t_single / R) // REUSE * REUSE)  # steps per process
+    S = per * R
+    tasks = []
+    for i in range(nw):
+        if R == 1:
+            tasks.append(([b for b in range(nb) if b % nw == i], REUSE, REUSE + S))
         else:
-            t1 = time.perf_counter()
-            pages = oracle.streaming_pages(n, w.N_P, w.sink, w.local)
-        oracle.decode_attention(q, k, v, oracle.page_tokens(pages, n, w.N_P), scale)
-        t_attn += time.perf_counter() - t1
-        done += 1
-        if time.perf_counter() - t_start > budget_s or (max_pairs and done >= max_pairs):
-            break
-    if lim is not None:
-        lim.unregister() if hasattr(lim, "unregister") else None
-    frac = done / len(pairs)
-    per_step = (t_sel / REUSE + t_attn) / frac
-    return per_step, f"{done} of {len(pairs)} (sequence, KV head) pairs of one layer-step, " \
-                     f"selection amortised over {REUSE} steps, 1 thread"
+            rep = i // nb
+            tasks.append(([i % nb], REUSE + rep * per, REUSE + (rep + 1) * per))
+    env_keys = ("OMP_NUM_THREADS", "OPENBLAS_NUM_THREADS", "MKL_NUM_THREADS")
+    saved = {k: os.environ.get(k) for k in env_keys}
+    for k in env_keys:
+        os.environ[k] = "1"
+    try:
+        ctx = mp.get_context("spawn")
+        mgr = ctx.Manager()
+        barrier = mgr.Barrier(nw)
+        with ctx.Pool(nw) as pool:
+            res = pool.map(_oracle_worker, [t + (barrier,) for t in tasks], chunksize=1)
+        mgr.shutdown()
+    finally:
+        for k, v in saved.items():
+            if v is None:
+                os.environ.pop(k, None)
+            else:
+                os.environ[k] = v
+    return max(res) / S, nw, S
+
+
+def oracle_prefill_sample(threads_one=True, budget_rows=64):
+    """The oracle's block-sparse prefill on a bounded sample of the 128K
+    workload: two dense and two Lambda query heads, per head two full query
+    blocks (one early, one late) and `budget_rows` random rows.  The time of the
+    whole workload is extrapolated from it by the number of (row, key) pairs
+    each head kind computes.  Returns (extrapolated s, sample description)."""
+    import oracle
+    import synth
+    lim = _one_thread() if threads_one else None
+    w = synth.prefill_128k()
+    K, V = oracle.widen_bf16(w.k()), oracle.widen_bf16(w.v())
+    nb = -(-w.T // w.block)
+    scale = 1.0 / math.sqrt(w.D)
+    rng = np.random.default_rng(7)
+
+    def keys_of(kind, rows):
+        """(row, key) pairs the rows compute: keys s <= t of the blocks row t sees."""
+        t = np.asarray(rows, dtype=np.float64)
+        if kind == 0:
+            return float(np.sum(t + 1))
+        i = np.floor(t / w.block)
+        sink_end = np.minimum(w.sink_blocks, i + 1) * w.block
+        local_start = np.maximum(np.maximum(0, i - w.local_blocks + 1) * w.block, sink_end)
+        return float(np.sum(np.minimum(sink_end, t + 1) + np.maximum(0, t + 1 - local_start)))
+
+    t_kind, keys_kind = {0: 0.0, 1: 0.0}, {0: 0.0, 1: 0.0}
+    heads = [hq for hq in range(w.H_q) if w.head_kind[hq // w.G] == 0][:2] + \
+            [hq for hq in range(w.H_q) if w.head_kind[hq // w.G] == 1][:2]
+    for hq in heads:
+        hk, kind = hq // w.G, int(w.head_kind[hq // w.G])
+        kh, vh = np.ascontiguousarray(K[:, hk]), np.ascontiguousarray(V[:, hk])
+        groups = {}
+        for i in (int(rng.integers(2, nb // 4)), int(rng.integers(3 * nb // 4, nb))):
+            groups[i] = list(range(i * w.block, min((i + 1) * w.block, w.T)))
+        for t in rng.choice(w.T, budget_rows, replace=False):
+            groups.setdefault(int(t) // w.block, []).append(int(t))
+        for i, rows in groups.items():
+            rows = np.asarray(sorted(set(rows)))
+            qb = oracle.widen_bf16(w.q_rows(int(rows[0]), int(rows[-1]) + 1))[rows - rows[0], hq]
+            t0 = time.perf_counter()
+            oracle.prefill_block_rows(qb, kh, vh, kind, w.block, w.sink_blocks, w.local_blocks,
+                                      scale, rows)
+            t_kind[kind] += time.perf_counter() - t0
+            keys_kind[kind] += keys_of(kind, rows)
+    del lim
+    all_rows = np.arange(w.T)
+    n_heads = {kind: sum(1 for hq in range(w.H_q) if w.head_kind[hq // w.G] == kind)
+               for kind in (0, 1)}
+    total = sum(t_kind[k] / keys_kind[k] * keys_of(k, all_rows) * n_heads[k] for k in (0, 1))
+    sampled = sum(t_kind.values())
+    return total, (f"extrapolated: 2 dense + 2 Lambda query heads x (2 full query blocks + "
+                   f"{budget_rows} random rows) timed ({sampled:.1f} s), scaled to all "
+                   f"{w.H_q} heads x {w.T} rows by the (row, key) pairs of each head kind")
+
+
+def cpu_baseline(w, acct, tc_flops=None):
+    """The fp64 oracle timed on this host: the decode step on one thread and on
+    every core, and the prefill (extrapolated from a sample)."""
+    host = host_cpu()
+    t1, steps1 = oracle_single_thread(w)
+    tn, nw, S = oracle_all_cores(w, t1)
+    res = {"value": acct["step"] / tn / 1e9, "unit": "GB/s", "cores": nw, "kind": "oracle",
+           "sample": f"{S} layer-steps of the bench workload (all {w.B * w.H_kv} pairs, selection "
+                     f"every {REUSE}th step) over {nw} processes of one thread each, started "
+                     f"together; the slowest process's time",
+           "host": host,
+           "single_thread": {"value": acct["step"] / t1 / 1e9, "unit": "GB/s", "cores": 1,
+                             "us_per_layer_step": t1 * 1e6,
+                             "sample": f"{steps1} whole layer-steps on one thread"},
+           "us_per_layer_step": tn * 1e6}
+    if tc_flops is not None:
+        tp1, s1 = oracle_prefill_sample(True)
+        tpn, _ = oracle_prefill_sample(False)
+        res["prefill"] = {"single_thread": {"TFLOP/s": tc_flops / tp1 / 1e12, "s": tp1, "cores": 1},
+                          "all_cores_blas": {"TFLOP/s": tc_flops / tpn / 1e12, "s": tpn,
+                                             "cores": host["usable_cores"]},
+                          "sample": s1}
+    return res
 
 
 def reference_steps(w, steps, warmup):
-    """The oracle as timed steps of the reference arm: step t takes the
-    (sequence, KV head) pair t mod P of one layer -- its page selection
-    (S^j -> P^m -> top-K) on every REUSE-th visit, as the GPU step reuses it,
-    and its attention every visit -- so a step is a bounded sample of the
-    workload and K steps amount to K / P layer-steps.  The bf16 inputs are
-    widened once and the page statistics built once (as on the GPU), untimed;
-    one thread.  Returns (seconds of the K timed steps, layer-steps, sample)."""
-    import oracle
-    try:
-        from threadpoolctl import threadpool_limits
-        lim = threadpool_limits(1)
-    except Exception:
-        lim = None
-    G = w.G
-    scale = 1.0 / math.sqrt(w.D)
-    cache = []
-    for b in range(w.B):
-        n = int(w.ctx_lens[b])
-        for h in range(w.H_kv):
-            q = oracle.widen_bf16(w.q[b, h * G:(h + 1) * G])
-            k = oracle.widen_bf16(w.k_seq(b, h))
-            v = oracle.widen_bf16(w.v_seq(b, h))
-            stats = None
-            if w.head_kind[h] == 0:
-                stats = oracle.page_stats(k, w.N_L)
-                pages = oracle.select_top_k(
-                    oracle.physical_scores(oracle.logical_scores(q, *stats), w.g), w.top_k)
-            else:
-                pages = oracle.streaming_pages(n, w.N_P, w.sink, w.local)
-            toks = oracle.page_tokens(pages, n, w.N_P)
-            # the attended keys and values (the selection is the same at every visit)
-            cache.append((q, stats, np.ascontiguousarray(k[toks]), np.ascontiguousarray(v[toks])))
-    P = len(cache)
-
-    def step(t):
-        q, stats, ks, vs = cache[t % P]
-        if stats is not None and (t // P) % REUSE == 0:
-            oracle.select_top_k(oracle.physical_scores(oracle.logical_scores(q, *stats), w.g), w.top_k)
-        oracle.decode_attention(q, ks, vs, np.arange(len(ks)), scale)
-
-    for t in range(warmup):
-        step(t)
-    t0 = time.perf_counter()
-    for t in range(warmup, warmup + steps):
-        step(t)
-    elapsed = time.perf_counter() - t0
-    if lim is not None and hasattr(lim, "unregister"):
-        lim.unregister()
-    return elapsed, steps / P, (f"each step one (sequence, KV head) pair of one layer ({P} pairs, "
-                                f"selection on every {REUSE}th visit of a pair), 1 thread")
+    """The oracle as timed steps of the reference arm: a step is one whole
+    layer-step of the workload -- every (sequence, KV head) pair: its page
+    selection on every REUSE-th step (as the GPU step reuses it) and its
+    attention over the attended pages, their tokens gathered inside the step.
+    The bf16 inputs are widened and the page statistics built once (as on the
+    GPU), untimed; one thread.  Returns (seconds of the K timed steps, sample)."""
+    lim = _one_thread()
+    pairs = [OraclePair(w, b, h) for b in range(w.B) for h in range(w.H_kv)]
+    oracle_layer_steps(pairs, 0, warmup)
+    elapsed = oracle_layer_steps(pairs, warmup, steps)
+    del lim
+    nsel = sum(1 for t in range(warmup, warmup + steps) if t % REUSE == 0)
+    return elapsed, (f"each step one whole layer-step ({len(pairs)} pairs; selection on {nsel} of "
+                     f"the {steps} timed steps, every {REUSE}th), 1 thread")
 
 
 def reference_arm(args):
-    """The oracle as the reference arm: same metric / unit / config."""
+    """The oracle as the reference arm: same metric / unit / config; a step is
+    one layer of the GPU arm's 32-layer step."""
     ws, rank, _ = dist_env()
     if rank != 0:
         return 0
     import synth
     w = synth.llama3_8b_decode()
     acct = decode_bytes(w)
-    elapsed, layer_steps, sample = reference_steps(w, args.steps, args.warmup)
-    per_layer_step = elapsed / layer_steps
+    elapsed, sample = reference_steps(w, args.steps, args.warmup)
+    per_layer_step = elapsed / args.steps
     value = acct["step"] / per_layer_step / 1e9
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": per_layer_step * LAYERS * 1e3,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": per_layer_step * 1e3,
+        "step": "one layer-step of the workload (the GPU arm's step is 32 of them)",
         "us_per_layer_step": per_layer_step * 1e6, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": workload_config(w),
         "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle",
-                         "sample": sample + f"; {elapsed:.1f} s for {args.steps} steps"},
+                         "sample": sample + f"; {elapsed:.2f} s for {args.steps} steps",
+                         "host": host_cpu()},
         "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line))
@@ -388,7 +547,7 @@ def main():
     global LAYERS
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=DEFAULT_STEPS)
+    ap.add_argument("--steps", type=int, default=None)
     ap.add_argument("--warmup", type=int, default=DEFAULT_WARMUP)
     ap.add_argument("--impl", default="lserve", choices=["lserve", "reference"])
     ap.add_argument("--no-prefill", action="store_true", help="skip the prefill stage")
@@ -406,6 +565,8 @@ def main():
                     help="prefill sequence length (default: the 128K workload)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
+    if args.steps is None:
+        args.steps = DEFAULT_REF_STEPS if args.impl == "reference" else DEFAULT_STEPS
     LAYERS = max(1, args.layers)
     if args.impl == "reference":
         return reference_arm(args)
@@ -610,7 +771,7 @@ def main():
         "config": workload_config(w),
         "roofline": {"bound": "hbm", "kernel": "decode_attn_kernel (lserve_sparse_decode_attn)",
                      "achieved": attn_gbs, "peak": hbm_peak, "unit": "GB/s",
-                     "frac": attn_gbs / hbm_peak, "traffic": decode_traffic(),
+                     "frac": attn_gbs / hbm_peak, "traffic": kernel_traffic("decode_attn"),
                      "algorithmic_bytes": acct["attn"],
                      "peak_source": f"{peak_src} hbm_gbs (copy, burst); of {peak_src}",
                      "timing": "mean attention launch inside the timed region (CUDA events "
@@ -644,10 +805,8 @@ def main():
                                                     args.prefill_seq)
 
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:  # the oracle baseline: one GPU runs only
-        per_step, sample = oracle_step_sample(w, budget_s=15.0)
-        cpu_val = acct["step"] / per_step / 1e9
-        result["cpu_baseline"] = {"value": cpu_val, "unit": "GB/s", "cores": 1, "kind": "oracle",
-                                  "sample": sample}
+        pf = result["stages"].get("prefill", {}).get("flops")
+        result["cpu_baseline"] = cpu_baseline(w, acct, pf)
     if rank == 0:
         print(json.dumps(result))
     if ws > 1:

@@ -147,6 +147,11 @@ int lserve_prefill_to_pages(const lserve_paged_desc* desc, int32_t seq_len, cons
  * The block table must already hold the page of pos.  A position outside
  * [0, max_pages_per_seq * N_P) or a bad pool id skips that sequence and sets
  * LSERVE_ERR_BOUNDS (lserve_read_device_status).  No workspace.
+ * The page being appended to must belong to one sequence only: two sequences
+ * whose block tables name the same pool page at their append positions (a
+ * shared prefix page) would update that page's K / V row and statistics from
+ * two warps at once, and the result is undefined.  Pages shared read-only
+ * (before the append position) are fine.
  */
 int lserve_decode_append(const lserve_paged_desc* desc, const void* k_new, const void* v_new,
                          const int32_t* block_table, const int32_t* ctx_lens,
@@ -331,7 +336,10 @@ int lserve_blocksparse_prefill(const lserve_prefill_desc* desc, const void* q, c
  *   - every call on a device shares the array (the previous call's scores stay
  *     there and are overwritten): calls that overlap on the GPU race;
  *   - the first call on each device looks up the array's device address with
- *     that device current; make that first call before any stream capture.
+ *     that device current; make that first call before any stream capture;
+ *   - the current device must be the one `stream` belongs to (the array used
+ *     is the current device's), and its index must be below 64 (the library
+ *     caches one address per device index; higher indices get LSERVE_ERR_CUDA).
  */
 int lserve_page_select_noalloc(const lserve_paged_desc* desc, const void* q, const void* stats_pool,
                                const int32_t* block_table, const int32_t* ctx_lens,

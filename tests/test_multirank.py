@@ -82,7 +82,7 @@ def test_reference_arm_prints_one_json_line_on_rank0(monkeypatch):
     monkeypatch.setenv("RANK", "0")
     monkeypatch.setenv("WORLD_SIZE", "1")
     monkeypatch.setattr(bench, "reference_steps",
-                        lambda w, steps, warmup: (1e-3 * steps, steps / 32, "stub sample"))
+                        lambda w, steps, warmup: (1e-3 * steps, "stub sample"))
 
     class A:
         gpus, warmup, steps = 1, 3, 1
@@ -95,3 +95,18 @@ def test_reference_arm_prints_one_json_line_on_rank0(monkeypatch):
     assert rec["impl"] == "reference" and rec["unit"] == "GB/s" and rec["higher_is_better"]
     assert rec["cpu_baseline"]["kind"] == "oracle"
     assert rec["e2e"]["h2d_bytes_per_step"] == 0
+    # a reported step is a measured one: ms_per_step x steps = the timed seconds
+    assert rec["ms_per_step"] * rec["steps"] == pytest.approx(1e-3 * A.steps * 1e3)
+    assert rec["cpu_baseline"]["host"]["nproc"] >= 1
+
+
+def test_oracle_bundles_pair_every_retrieval_with_a_streaming_pair():
+    """The all-core oracle run splits the pairs into bundles of equal cost."""
+    import bench
+    import synth
+    w = synth.llama3_8b_decode()
+    bundles = bench._bundles(w)
+    flat = sorted(p for b in bundles for p in b)
+    assert flat == list(range(w.B * w.H_kv))
+    for b in bundles:
+        assert sorted(int(w.head_kind[p % w.H_kv]) for p in b) == [0, 1]

@@ -54,6 +54,47 @@ def test_noalloc_select_matches_workspace_select_twice():
         buf.q.copy_(-buf.q)
 
 
+def _noalloc(d, q, stats, bt, ctx, hk, top_k, sel, cnt):
+    return lserve.lib.lserve_page_select_noalloc(
+        ctypes.byref(d), ctypes.c_void_p(q.data_ptr()), ctypes.c_void_p(stats.data_ptr()),
+        ctypes.c_void_p(bt.data_ptr()), ctypes.c_void_p(ctx.data_ptr()), ctypes.c_void_p(hk.data_ptr()),
+        top_k, ctypes.c_void_p(sel.data_ptr()), ctypes.c_void_p(cnt.data_ptr()),
+        ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+
+
+def test_noalloc_select_allocates_nothing_and_accepts_the_limit():
+    """A shape of exactly 1,048,576 scores (the array's size: 8 sequences x 2
+    KV heads x a block table 65,536 pages wide) is accepted and selects what
+    the workspace path selects; torch's allocator sees no change across the
+    call (the call itself allocates no device memory)."""
+    w = synth.decode_workload(8, 4, 2, 64, 16, 64, 16, 64, 256,
+                              [3000, 64, 5000, 777, 4096, 1, 2500, 6000], seed=32)
+    buf = DecodeBuffers(w)
+    wide = 65536
+    assert w.B * w.H_kv * wide == 1 << 20
+    bt = torch.full((w.B, wide), -1, dtype=torch.int32, device=buf.block_table.device)
+    bt[:, :w.max_pages] = buf.block_table
+    d = lserve.paged_desc(w.B, w.H_q, w.H_kv, w.D, w.N_L, w.N_P, wide, w.num_pool_pages)
+    lserve.page_stats(d, buf.k_pool, bt, buf.ctx_lens, buf.head_kind, buf.stats[0])
+    ws = lserve.alloc_workspace(lserve.workspace_size(lserve.OP_SELECT, d, w.top_k))
+    sel_a = torch.full_like(buf.sel[0], -9)
+    cnt_a = torch.full_like(buf.sel_count[0], -9)
+    lserve.page_select(d, buf.q, buf.stats[0], bt, buf.ctx_lens, buf.head_kind, w.top_k, sel_a,
+                       cnt_a, workspace=ws)
+    sel_b = torch.full_like(sel_a, -9)
+    cnt_b = torch.full_like(cnt_a, -9)
+    torch.cuda.synchronize()
+    before = torch.cuda.memory_allocated()
+    for _ in range(2):
+        st = _noalloc(d, buf.q, buf.stats[0], bt, buf.ctx_lens, buf.head_kind, w.top_k, sel_b, cnt_b)
+        assert st == lserve.OK, lserve.status_string(st)
+    torch.cuda.synchronize()
+    assert torch.cuda.memory_allocated() == before
+    assert lserve.read_device_status() == lserve.OK
+    assert torch.equal(sel_a, sel_b) and torch.equal(cnt_a, cnt_b)
+    assert int(cnt_b.min()) >= 0
+
+
 def test_noalloc_select_rejects_too_large_shapes():
     d = lserve.paged_desc(64, 32, 8, 128, 16, 64, 4096, 64 * 4096)   # 2M scores > 1M
     st = lserve.lib.lserve_page_select_noalloc(ctypes.byref(d), None, None, None, None, None, 8, None,
