@@ -63,14 +63,14 @@ def _noalloc(d, q, stats, bt, ctx, hk, top_k, sel, cnt):
 
 
 def test_noalloc_select_allocates_nothing_and_accepts_the_limit():
-    """A shape of exactly 1,048,576 scores (the array's size: 8 sequences x 2
-    KV heads x a block table 65,536 pages wide) is accepted and selects what
+    """A shape of exactly 1,048,576 scores (the array's size: 16 sequences x 2
+    KV heads x a block table 32,768 pages wide) is accepted and selects what
     the workspace path selects; torch's allocator sees no change across the
     call (the call itself allocates no device memory)."""
-    w = synth.decode_workload(8, 4, 2, 64, 16, 64, 16, 64, 256,
-                              [3000, 64, 5000, 777, 4096, 1, 2500, 6000], seed=32)
+    w = synth.decode_workload(16, 4, 2, 64, 16, 64, 16, 64, 256,
+                              [3000, 64, 5000, 777, 4096, 1, 2500, 6000] * 2, seed=32)
     buf = DecodeBuffers(w)
-    wide = 65536
+    wide = 32768
     assert w.B * w.H_kv * wide == 1 << 20
     bt = torch.full((w.B, wide), -1, dtype=torch.int32, device=buf.block_table.device)
     bt[:, :w.max_pages] = buf.block_table
