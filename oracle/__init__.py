@@ -35,6 +35,8 @@ Readings where the pages are silent (each is listed in the design notes):
      (pool page, KV head, channel) over the page's valid tokens, codes decided
      in float32 (quantize_kv8); attention attends code * scale.
      (parity unpinned by the pages: they name KV quantization, not a scheme)
+  R18 4-bit KV cache (row f3): the R15 scheme with codes -7..7 (quantize_kv4),
+     two codes per byte in the device layout.       (parity unpinned, as R15)
   R17 sequence-sharded decode (row f4): shard r of N holds the contiguous
      physical pages [floor(M*r/N), floor(M*(r+1)/N)); each shard proposes its
      own top-K, the global top-K is re-made from the proposals, and the
@@ -64,7 +66,9 @@ from .lserve import (  # noqa: F401
     prefill_rows,
     prefill_block_rows,
     prefill_flops,
+    quantize_kv,
     quantize_kv8,
+    quantize_kv4,
     dequantize_kv8,
     dequantized_seq,
 )

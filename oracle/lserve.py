@@ -298,47 +298,62 @@ def prefill_block_rows(q: np.ndarray, k: np.ndarray, v: np.ndarray, kind: int, b
     return o, lse
 
 
-# --- quantized KV cache [R15] ------------------------------------------------
+# --- quantized KV cache [R15, R18] -------------------------------------------
 # The pages name KV-cache quantization (QServe KV4, combined with LServe's
 # sparsity in the abstract page) but give no scheme.  R15 reading: symmetric
 # int8 with one scale per (pool page, KV head, channel) over the page's valid
-# tokens; the integer codes are decided in float32 exactly as written below so
-# that both sides take the same decision; the attention attends the value
-# code * scale (a real number, exact in float64 here; each side rounds it as
-# its own arithmetic does).
+# tokens; R18: the same with 4-bit codes (-7..7).  The integer codes are
+# decided in float32 exactly as written below so that both sides take the
+# same decision; the attention attends the value code * scale (a real number,
+# exact in float64 here; each side rounds it as its own arithmetic does).
 
-def quantize_kv8(x_bits: np.ndarray):
-    """Codes and scales of one page of one KV head.
+def quantize_kv(x_bits: np.ndarray, qmax: int):
+    """Codes and scales of one page of one KV head, symmetric with codes in
+    [-qmax, qmax] (qmax = 127: 8-bit codes, R15; qmax = 7: 4-bit codes, R18).
 
     x_bits: bf16 bits [t][D] of the page's valid tokens (t >= 1).
-    amax_c = max_t |x[t][c]| (exact in float32); inv_c = float32(127) /
+    amax_c = max_t |x[t][c]| (exact in float32); inv_c = float32(qmax) /
     float32(amax_c); code = rint(float32(x) * inv_c) (float32 product, round
-    half to even), clamped to [-127, 127]; scale_c = float32(amax_c) /
-    float32(127).  A channel with amax 0 gets codes 0 and scale 0.
+    half to even), clamped to [-qmax, qmax]; scale_c = float32(amax_c) /
+    float32(qmax).  A channel with amax 0 gets codes 0 and scale 0.
     Returns (codes int8 [t][D], scale float32 [D]).
     """
     x = widen_bf16(x_bits).astype(np.float32)
+    q = np.float32(qmax)
     amax = np.max(np.abs(x), axis=0).astype(np.float32)
     with np.errstate(divide="ignore", invalid="ignore"):
-        inv = np.where(amax > 0, np.float32(127.0) / amax, np.float32(0.0)).astype(np.float32)
+        inv = np.where(amax > 0, q / amax, np.float32(0.0)).astype(np.float32)
     prod = (x * inv[None, :]).astype(np.float32)
-    codes = np.clip(np.rint(prod), -127, 127).astype(np.int8)
-    scale = (amax / np.float32(127.0)).astype(np.float32)
+    codes = np.clip(np.rint(prod), -qmax, qmax).astype(np.int8)
+    scale = (amax / q).astype(np.float32)
     return codes, scale
 
 
+def quantize_kv8(x_bits: np.ndarray):
+    """8-bit codes (R15): quantize_kv with qmax = 127."""
+    return quantize_kv(x_bits, 127)
+
+
+def quantize_kv4(x_bits: np.ndarray):
+    """4-bit codes (R18): quantize_kv with qmax = 7 (codes -7..7, so a code
+    and its negation are both representable in a signed nibble)."""
+    return quantize_kv(x_bits, 7)
+
+
 def dequantize_kv8(codes: np.ndarray, scale: np.ndarray) -> np.ndarray:
-    """code * scale per element, float64 (exact: 8-bit times 24-bit)."""
+    """code * scale per element, float64 (exact: an 8-bit integer times a
+    24-bit significand).  The same for 4-bit codes."""
     return codes.astype(np.float64) * scale.astype(np.float64)[None, :]
 
 
-def dequantized_seq(x_bits: np.ndarray, N_P: int) -> np.ndarray:
+def dequantized_seq(x_bits: np.ndarray, N_P: int, bits: int = 8) -> np.ndarray:
     """A sequence's K or V ([n][D] bf16 bits) as the quantized cache holds it:
-    each physical page of N_P tokens quantized on its own valid tokens, then
-    dequantized (float64 [n][D])."""
+    each physical page of N_P tokens quantized on its own valid tokens with
+    `bits`-bit codes, then dequantized (float64 [n][D])."""
+    qmax = {8: 127, 4: 7}[bits]
     n = x_bits.shape[0]
     out = np.empty(x_bits.shape, dtype=np.float64)
     for t0 in range(0, n, N_P):
-        c, s = quantize_kv8(x_bits[t0:t0 + N_P])
+        c, s = quantize_kv(x_bits[t0:t0 + N_P], qmax)
         out[t0:t0 + N_P] = dequantize_kv8(c, s)
     return out

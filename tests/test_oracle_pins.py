@@ -471,3 +471,49 @@ def test_kv8_lossless_on_grid_values():
     assert np.array_equal(np.abs(codes.astype(np.int64)), np.abs(ints))
     assert np.array_equal(codes.astype(np.int64), ints)
     assert np.array_equal(oracle.dequantize_kv8(codes, scale), oracle.widen_bf16(x))
+
+
+def test_kv4_hand_example():
+    # channel 0: amax 2 -> inv 3.5; 1 -> 3.5 -> 4 (half to even), -2 -> -7, 0.5 -> 1.75 -> 2
+    # channel 1: amax 7 -> inv 1; 2.5 -> 2 and 3.5 -> 4 (half to even), -7 -> -7
+    x = _bits([[1.0, 2.5], [-2.0, 3.5], [0.5, -7.0]])
+    codes, scale = oracle.quantize_kv4(x)
+    assert codes[:, 0].tolist() == [4, -7, 2]
+    assert codes[:, 1].tolist() == [2, 4, -7]
+    assert scale[0] == np.float32(2.0) / np.float32(7.0) and scale[1] == np.float32(1.0)
+
+
+def test_kv4_round_trip_error_and_range():
+    rng = np.random.default_rng(15)
+    x = _bits(rng.normal(size=(64, 128)) * rng.uniform(0.5, 8, size=128))
+    codes, scale = oracle.quantize_kv4(x)
+    assert codes.min() >= -7 and codes.max() <= 7
+    xf = oracle.widen_bf16(x)
+    amax = np.abs(xf).max(axis=0)
+    j = np.abs(xf).argmax(axis=0)
+    assert np.all(np.abs(codes[j, np.arange(128)]) == 7)
+    back = oracle.dequantize_kv8(codes, scale)
+    bound = amax / 7 / 2 * (1 + 1e-5)
+    assert np.all(np.abs(back - xf) <= bound[None, :])
+    # 4-bit codes are the 8-bit scheme with a coarser grid: same scales up to 127/7
+    _, s8 = oracle.quantize_kv8(x)
+    assert np.allclose(scale * 7, s8 * 127, rtol=1e-6)
+
+
+def test_kv4_is_odd_and_lossless_on_its_grid():
+    rng = np.random.default_rng(16)
+    x = _bits(rng.normal(size=(16, 64)))
+    c1, s1 = oracle.quantize_kv4(x)
+    c2, s2 = oracle.quantize_kv4(x ^ np.uint16(0x8000))
+    assert np.array_equal(c2, -c1) and np.array_equal(s1, s2)
+    ints = rng.integers(-7, 8, size=(40, 16))
+    ints[5] = 7
+    step = 2.0 ** rng.integers(-6, 3, size=16)
+    xg = _bits(ints * step)
+    codes, scale = oracle.quantize_kv4(xg)
+    assert np.array_equal(codes.astype(np.int64), ints)
+    assert np.array_equal(oracle.dequantize_kv8(codes, scale), oracle.widen_bf16(xg))
+    # a 4-bit dequantized sequence quantizes each page on its own
+    whole = oracle.dequantized_seq(x, 8, bits=4)
+    c, s = oracle.quantize_kv4(x[8:16])
+    assert np.array_equal(whole[8:16], oracle.dequantize_kv8(c, s))
