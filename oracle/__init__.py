@@ -27,6 +27,9 @@ Readings where the pages are silent (each is listed in the design notes):
   R4 ties go to the lowest page index; selections are reported ascending.
   R5 streaming decode is page-granular: sink pages [0, ceil(S/N_P)) plus every
      page holding one of the last L tokens.
+  R10 tokens appended during a reuse window: by default a retrieval head sees
+     them only if their page is selected; as an option it also attends every
+     token appended since its selection (attended_tokens with recent_from).
   R6 Lambda prefill: block row i sees blocks {0..sink-1} and
      [i - local + 1, i] (the diagonal counts as local).   (parity unpinned)
   R7 retrieval heads in prefill are dense causal.
@@ -53,6 +56,7 @@ from .lserve import (  # noqa: F401
     retrieval_pages,
     streaming_pages,
     page_tokens,
+    attended_tokens,
     decode_attention,
     decode_pair,
     shard_bounds,

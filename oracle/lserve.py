@@ -127,6 +127,19 @@ def decode_attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, tokens, scale:
     return o, zmax[:, 0] + np.log(lsum)
 
 
+def attended_tokens(pages, n: int, N_P: int, recent_from=None) -> np.ndarray:
+    """Token positions a decode step attends: the valid tokens of the given
+    physical pages (R2) and, when recent_from is given (reading R10's option:
+    retrieval heads also see every token appended since their selection was
+    made, whose pages the reused selection may not hold), every position in
+    [recent_from, n) -- a set, ascending, each token once."""
+    toks = page_tokens(pages, n, N_P)
+    if recent_from is None:
+        return toks
+    lo = max(0, min(int(recent_from), n))
+    return np.union1d(toks, np.arange(lo, n)).astype(np.int64)
+
+
 def decode_pair(q, k, v, n, kind, N_L, N_P, K, sink, local, scale):
     """One (sequence, KV head) of a decode step: retrieval heads pick top-K
     pages by S^j, streaming heads take sink + local pages; then attention.

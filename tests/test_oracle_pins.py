@@ -517,3 +517,36 @@ def test_kv4_is_odd_and_lossless_on_its_grid():
     whole = oracle.dequantized_seq(x, 8, bits=4)
     c, s = oracle.quantize_kv4(x[8:16])
     assert np.array_equal(whole[8:16], oracle.dequantize_kv8(c, s))
+
+
+# --- tokens appended since the last selection (R10 option) -----------------------
+
+def test_attended_tokens_recent_option_closed_forms():
+    n, N_P = 300, 64                       # pages 0..4, the last holding tokens 256..299
+    pages = [1, 3]
+    base = oracle.page_tokens(pages, n, N_P)
+    # no recent tokens, or none past n: the selected pages' tokens only
+    assert np.array_equal(oracle.attended_tokens(pages, n, N_P), base)
+    assert np.array_equal(oracle.attended_tokens(pages, n, N_P, recent_from=n), base)
+    # every token recent: all n tokens, each once
+    assert np.array_equal(oracle.attended_tokens(pages, n, N_P, recent_from=0), np.arange(n))
+    # recent tokens inside a selected page add nothing
+    assert np.array_equal(oracle.attended_tokens([1, 4], n, N_P, recent_from=290),
+                          oracle.page_tokens([1, 4], n, N_P))
+    # recent tokens outside the selection are added, in order
+    got = oracle.attended_tokens(pages, n, N_P, recent_from=296)
+    assert np.array_equal(got, np.concatenate([base, np.arange(296, 300)]))
+
+
+def test_decode_with_every_token_recent_is_dense_attention():
+    """recent_from = 0 turns any selection into dense attention over all n
+    tokens (torch SDPA, fp64)."""
+    rng = _rng(31)
+    n, D, G = 150, 16, 3
+    q, k, v = (_bf16_values(rng, s) for s in ((G, D), (n, D), (n, D)))
+    toks = oracle.attended_tokens([0], n, 64, recent_from=0)
+    o, _ = oracle.decode_attention(q, k, v, toks, 0.25)
+    want = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(q)[:, None], torch.from_numpy(k)[None].expand(G, n, D),
+        torch.from_numpy(v)[None].expand(G, n, D), scale=0.25)[:, 0].numpy()
+    assert np.allclose(o, want, rtol=1e-12, atol=1e-12)
