@@ -62,11 +62,13 @@ def peaks():
 
 # --- algorithmic byte / flop accounting (what the chosen sparsity touches) ----
 
-def decode_bytes(w):
+def decode_bytes(w, fused_append=False):
     """Bytes one decode step of one layer must move, amortising selection over
     the reuse interval.  KV: valid tokens of the attended pages, K and V, D*2
     bytes each.  Selection: the stats of every valid logical page of the
-    retrieval heads (2*D*2 bytes), the q vectors, scores and selection."""
+    retrieval heads (2*D*2 bytes), the q vectors, scores and selection.  With
+    fused_append the attention launch also appends the step's token (its K / V
+    rows and the statistics it updates, append_bytes)."""
     import oracle
     D, NP, NL = w.D, w.N_P, w.N_L
     kv = 0
@@ -88,15 +90,16 @@ def decode_bytes(w):
     q = w.B * w.H_q * D * 2
     out = w.B * w.H_q * D * 2
     sel_io = q + w.B * w.H_kv * (w.max_pages * 4 + w.top_k * 4 + 4)
-    attn = kv + q + out
+    attn = kv + q + out + (append_bytes(w) if fused_append else 0)
     select = stats + sel_io
     return dict(attn=attn, select=select, step=attn + select / REUSE, kv=kv, stats=stats)
 
 
-def decode_bytes_kv8(w):
-    """Bytes one decode-attention call over the int8 cache moves: the codes of
-    the attended pages (K and V, D bytes per token each), the two float32
-    channel-scale rows of every attended (page, head), q and the output."""
+def decode_bytes_kv8(w, bits=8):
+    """Bytes one decode-attention call over the quantized cache moves: the
+    codes of the attended pages (K and V, D * bits / 8 bytes per token each),
+    the two float32 channel-scale rows of every attended (page, head), q and
+    the output."""
     import oracle
     D, NP = w.D, w.N_P
     kv = 0
@@ -106,23 +109,23 @@ def decode_bytes_kv8(w):
         for h in range(w.H_kv):
             if w.head_kind[h] == 0:
                 k = min(w.top_k, npages)
-                kv += k * NP * D * 2 + k * 2 * D * 4
+                kv += k * NP * D * bits // 8 * 2 + k * 2 * D * 4
             else:
                 pages = oracle.streaming_pages(n, NP, w.sink, w.local)
                 toks = len(oracle.page_tokens(pages, n, NP))
-                kv += toks * D * 2 + len(pages) * 2 * D * 4
+                kv += toks * D * bits // 8 * 2 + len(pages) * 2 * D * 4
     return kv + 2 * w.B * w.H_q * D * 2
 
 
-def quantize_bytes(w):
-    """lserve_quantize_pages_kv8: read the valid bf16 K/V rows of every page,
-    write the int8 codes (whole pages) and the float32 scales."""
+def quantize_bytes(w, bits=8):
+    """lserve_quantize_pages_kv8 / _kv4: read the valid bf16 K/V rows of every
+    page, write the codes (whole pages) and the float32 scales."""
     rd = wr = 0
     for b in range(w.B):
         n = int(w.ctx_lens[b])
         npages = -(-n // w.N_P)
         rd += 2 * n * w.H_kv * w.D * 2
-        wr += 2 * npages * w.H_kv * (w.N_P * w.D + w.D * 4)
+        wr += 2 * npages * w.H_kv * (w.N_P * w.D * bits // 8 + w.D * 4)
     return rd + wr
 
 
@@ -556,7 +559,7 @@ def main():
     ap.add_argument("--layers", type=int, default=LAYERS,
                     help="layer replicas (fewer = a small case for profiling; < 32 may fit in L2)")
     ap.add_argument("--no-mha", action="store_true", help="skip the MHA decode stage")
-    ap.add_argument("--no-kv8", action="store_true", help="skip the int8-cache decode stages")
+    ap.add_argument("--no-kv8", action="store_true", help="skip the quantized-cache (8- and 4-bit) decode stages")
     ap.add_argument("--no-configs", action="store_true",
                     help="skip the long-decode and mixed-batch decode stages")
     ap.add_argument("--prefill-only", action="store_true",
@@ -605,7 +608,7 @@ def main():
     qs = [q_all[l] for l in range(LAYERS)]
     outs = [out_all[l] for l in range(LAYERS)]
     stream = torch.cuda.Stream(device=dev)
-    acct = decode_bytes(w)
+    acct = decode_bytes(w, fused_append=True)
 
     def stats_all():
         for l in range(LAYERS):
@@ -616,14 +619,25 @@ def main():
         lserve.page_select(d, qs[l], buf.stats[l], buf.block_table, buf.ctx_lens, buf.head_kind,
                            w.top_k, buf.sel[l], buf.sel_count[l], workspace=ws_sel)
 
+    # The step's new token of every sequence is appended in the attention launch
+    # (lserve_decode_step).  So that every step sees the same cache, the token
+    # appended is each sequence's last one again, with its own K / V (position
+    # n - 1, ctx_lens unchanged): the pools and statistics keep their contents.
+    last = [(int(w.block_table[b, (int(w.ctx_lens[b]) - 1) // w.N_P]),
+             (int(w.ctx_lens[b]) - 1) % w.N_P) for b in range(w.B)]
+    k_last = [torch.stack([buf.k_pools[l][pid, :, r] for pid, r in last]).contiguous()
+              for l in range(LAYERS)]
+    v_last = [torch.stack([buf.v_pools[l][pid, :, r] for pid, r in last]).contiguous()
+              for l in range(LAYERS)]
+
     def attn(l, overlap=False):
         # overlap: the kernel before this call is the previous layer's attention,
         # which writes none of the selection / block-table inputs, so the split
         # plan and first page lookups may run while it finishes (PDL)
-        lserve.sparse_decode_attn(d, qs[l], buf.k_pools[l], buf.v_pools[l], buf.block_table,
-                                  buf.ctx_lens, buf.head_kind, buf.sel[l], buf.sel_count[l], w.top_k,
-                                  w.sink, w.local, scale, outs[l], None, workspace=ws_dec,
-                                  overlap_prologue=overlap)
+        lserve.decode_step(d, qs[l], k_last[l], v_last[l], buf.k_pools[l], buf.v_pools[l],
+                           buf.stats[l], buf.block_table, buf.ctx_lens, buf.head_kind, buf.sel[l],
+                           buf.sel_count[l], w.top_k, w.sink, w.local, scale, outs[l], None,
+                           workspace=ws_dec, overlap_prologue=overlap)
 
     with torch.cuda.stream(stream):
         stats_all()
@@ -644,16 +658,9 @@ def main():
     g_select_only = capture(lambda: [select(l) for l in range(LAYERS)])
     g_stats = capture(stats_all)
 
-    # decode-time cache maintenance (lserve_decode_append), timed alone: each
-    # sequence's last token is written again with its own K/V (position n - 1,
-    # inside the block table), which leaves the cache and statistics unchanged
+    # the same cache maintenance as a launch of its own (lserve_decode_append),
+    # timed alone for comparison
     lens_last = (buf.ctx_lens - 1).to(torch.int32)
-    last = [(int(w.block_table[b, (int(w.ctx_lens[b]) - 1) // w.N_P]),
-             (int(w.ctx_lens[b]) - 1) % w.N_P) for b in range(w.B)]
-    k_last = [torch.stack([buf.k_pools[l][pid, :, r] for pid, r in last]).contiguous()
-              for l in range(LAYERS)]
-    v_last = [torch.stack([buf.v_pools[l][pid, :, r] for pid, r in last]).contiguous()
-              for l in range(LAYERS)]
 
     def append_all():
         for l in range(LAYERS):
@@ -731,7 +738,9 @@ def main():
         "stats_build": {"us": t_stats * 1e6, "GB/s": sb / t_stats / 1e9,
                         "frac": sb / t_stats / 1e9 / hbm_peak, "bytes": sb},
         "append": {"us": t_app * 1e6, "GB/s": app_bytes / t_app / 1e9, "bytes": app_bytes,
-                   "note": "lserve_decode_append per layer; launch-latency bound (16 KB of K/V)"},
+                   "note": "lserve_decode_append as a launch of its own, per layer (the bench's "
+                           "step appends inside the attention launch, lserve_decode_step); "
+                           "launch-latency bound (48 KB)"},
     }
     del g_stats, g_append
 
@@ -793,20 +802,22 @@ def main():
         result["stages"]["mixed_batch_decode"] = decode_config_stage(
             lserve, synth, dev, stream, hbm_peak, timed, synth.mixed_batch_decode, 3)
     if not args.no_kv8:
-        result["stages"]["attention_kv8"] = kv8_stage(lserve, synth, dev, stream, hbm_peak, timed,
-                                                      synth.llama3_8b_decode, 16,
-                                                      stages["attention"]["us"])
-        if not args.no_mha:
-            result["stages"]["attention_mha_kv8"] = kv8_stage(
-                lserve, synth, dev, stream, hbm_peak, timed, synth.llama2_7b_mha_decode, 8,
-                result["stages"]["attention_mha"]["us"])
+        for bits in (8, 4):
+            result["stages"][f"attention_kv{bits}"] = kv8_stage(
+                lserve, synth, dev, stream, hbm_peak, timed, synth.llama3_8b_decode, 16,
+                stages["attention"]["us"], bits)
+            if not args.no_mha:
+                result["stages"][f"attention_mha_kv{bits}"] = kv8_stage(
+                    lserve, synth, dev, stream, hbm_peak, timed, synth.llama2_7b_mha_decode, 8,
+                    result["stages"]["attention_mha"]["us"], bits)
     if not args.no_prefill:
         result["stages"]["prefill"] = prefill_stage(lserve, synth, dev, stream, tc_peak, timed,
                                                     args.prefill_seq)
 
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:  # the oracle baseline: one GPU runs only
         pf = result["stages"].get("prefill", {}).get("flops")
-        result["cpu_baseline"] = cpu_baseline(w, acct, pf)
+        # the oracle's step attends without appending: its bytes leave the append out
+        result["cpu_baseline"] = cpu_baseline(w, decode_bytes(w), pf)
     if rank == 0:
         print(json.dumps(result))
     if ws > 1:
@@ -1016,11 +1027,12 @@ def seqshard_timing(lserve, w, buf, d, dev, stream, timed, layers, N, scale):
                          f"partials {4 * B * H_q * (D + 1)} B per shard"}
 
 
-def kv8_stage(lserve, synth, dev, stream, hbm_peak, timed, make, layers, bf16_us):
-    """Decode attention over the int8 cache (lserve_sparse_decode_attn_kv8),
-    alone: the workload's pools quantized once (lserve_quantize_pages_kv8,
-    timed too), then `layers` replicas of the int8 pools attended back to back
-    (more bytes than L2 holds), the selection being the bf16 statistics'."""
+def kv8_stage(lserve, synth, dev, stream, hbm_peak, timed, make, layers, bf16_us, bits=8):
+    """Decode attention over the quantized cache (lserve_sparse_decode_attn_kv8
+    or _kv4 for bits = 8 / 4), alone: the workload's pools quantized once
+    (lserve_quantize_pages_kv8 / _kv4, timed too), then `layers` replicas of
+    the quantized pools attended back to back (more bytes than L2 holds), the
+    selection being the bf16 statistics'."""
     import torch
     from synth.device import DecodeBuffers
     w = make()
@@ -1028,14 +1040,15 @@ def kv8_stage(lserve, synth, dev, stream, hbm_peak, timed, make, layers, bf16_us
     d = lserve.paged_desc(w.B, w.H_q, w.H_kv, w.D, w.N_L, w.N_P, w.max_pages, w.num_pool_pages)
     wss = lserve.alloc_workspace(lserve.workspace_size(lserve.OP_SELECT, d, w.top_k), device=dev)
     wsd = lserve.alloc_workspace(lserve.workspace_size(lserve.OP_DECODE, d, w.top_k), device=dev)
-    k8 = torch.empty(w.pool_shape(), dtype=torch.int8, device=dev)
+    shape = w.pool_shape() if bits == 8 else w.pool_shape()[:-1] + (w.D // 2,)
+    k8 = torch.empty(shape, dtype=torch.int8, device=dev)
     v8 = torch.empty_like(k8)
     ks = torch.empty((w.num_pool_pages, w.H_kv, w.D), dtype=torch.float32, device=dev)
     vs = torch.empty_like(ks)
 
     def quantize():
         lserve.quantize_pages_kv8(d, buf.k_pool, buf.v_pool, buf.block_table, buf.ctx_lens, k8, v8,
-                                  ks, vs, stream=stream)
+                                  ks, vs, stream=stream, bits=bits)
     with torch.cuda.stream(stream):
         lserve.page_stats(d, buf.k_pool, buf.block_table, buf.ctx_lens, buf.head_kind, buf.stats[0])
         lserve.page_select(d, buf.q, buf.stats[0], buf.block_table, buf.ctx_lens, buf.head_kind,
@@ -1044,7 +1057,7 @@ def kv8_stage(lserve, synth, dev, stream, hbm_peak, timed, make, layers, bf16_us
     torch.cuda.synchronize()
     assert lserve.read_device_status(stream) == lserve.OK
     t_q = timed(quantize, 3) / 3
-    qb = quantize_bytes(w)
+    qb = quantize_bytes(w, bits)
     buf.k_pools = buf.v_pools = None  # the bf16 pools are not read below
     torch.cuda.empty_cache()
     pools = [(k8, v8, ks, vs)] + [(k8.clone(), v8.clone(), ks.clone(), vs.clone())
@@ -1057,7 +1070,7 @@ def kv8_stage(lserve, synth, dev, stream, hbm_peak, timed, make, layers, bf16_us
             lserve.sparse_decode_attn_kv8(d, buf.q, a, b, c, e, buf.block_table, buf.ctx_lens,
                                           buf.head_kind, buf.sel[0], buf.sel_count[0], w.top_k,
                                           w.sink, w.local, scale, outs[l], None, workspace=wsd,
-                                          overlap_prologue=l > 0)
+                                          overlap_prologue=l > 0, bits=bits)
     with torch.cuda.stream(stream):
         attn_all()
     torch.cuda.synchronize()
@@ -1070,14 +1083,14 @@ def kv8_stage(lserve, synth, dev, stream, hbm_peak, timed, make, layers, bf16_us
             g.replay()
     reps = 20
     t = timed(lambda: g.replay(), reps) / (reps * layers)
-    bts = decode_bytes_kv8(w)
+    bts = decode_bytes_kv8(w, bits)
     del g, pools
     torch.cuda.empty_cache()
     return {"us": t * 1e6, "GB/s": bts / t / 1e9, "frac": bts / t / 1e9 / hbm_peak, "bytes": bts,
             "speedup_vs_bf16_cache": bf16_us / (t * 1e6),
             "quantize": {"us": t_q * 1e6, "GB/s": qb / t_q / 1e9, "frac": qb / t_q / 1e9 / hbm_peak,
-                         "bytes": qb, "what": "lserve_quantize_pages_kv8 of the whole cache"},
-            "workload": f"{w.name} (int8 cache): B={w.B} n={int(w.ctx_lens[0])} H_q={w.H_q} "
+                         "bytes": qb, "what": f"lserve_quantize_pages_kv{bits} of the whole cache"},
+            "workload": f"{w.name} ({bits}-bit cache): B={w.B} n={int(w.ctx_lens[0])} H_q={w.H_q} "
                         f"H_kv={w.H_kv} D={w.D} N_P={w.N_P} top_k={w.top_k}"}
 
 

@@ -34,6 +34,7 @@ EXPORTED = [
     "lserve_decode_append", "lserve_prefill_to_pages", "lserve_quantize_pages_kv8",
     "lserve_sparse_decode_attn_kv8", "lserve_seqshard_bounds", "lserve_seqshard_sel_stride",
     "lserve_seqshard_candidates", "lserve_seqshard_merge", "lserve_seqshard_combine",
+    "lserve_quantize_pages_kv4", "lserve_sparse_decode_attn_kv4", "lserve_decode_step",
 ]
 DECODE_OVERLAP_PROLOGUE = 1
 DECODE_OUT_F32 = 2
@@ -82,6 +83,11 @@ def _load(path):
     lib.lserve_sparse_decode_attn_kv8.argtypes = [P(PagedDesc), vp, vp, vp, vp, vp, vp, vp, vp, vp,
                                                   vp, i32, i32, i32, ctypes.c_float, vp, vp,
                                                   ctypes.c_uint32, vp, sz, vp]
+    lib.lserve_quantize_pages_kv4.argtypes = lib.lserve_quantize_pages_kv8.argtypes
+    lib.lserve_decode_step.argtypes = [P(PagedDesc), vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i32,
+                                       i32, i32, vp, ctypes.c_float, vp, vp, ctypes.c_uint32, vp,
+                                       sz, vp]
+    lib.lserve_sparse_decode_attn_kv4.argtypes = lib.lserve_sparse_decode_attn_kv8.argtypes
     lib.lserve_page_select_noalloc.argtypes = [P(PagedDesc), vp, vp, vp, vp, vp, i32, vp, vp, vp]
     pi32 = P(i32)
     lib.lserve_seqshard_bounds.argtypes = [i32, i32, i32, i32, pi32, pi32, pi32]
@@ -106,7 +112,9 @@ def _load(path):
                  "lserve_bounds_checked", "lserve_quantize_pages_kv8",
                  "lserve_sparse_decode_attn_kv8", "lserve_sparse_decode_attn_ex",
                  "lserve_decode_append", "lserve_prefill_to_pages", "lserve_seqshard_bounds",
-                 "lserve_seqshard_candidates", "lserve_seqshard_merge", "lserve_seqshard_combine"):
+                 "lserve_seqshard_candidates", "lserve_seqshard_merge", "lserve_seqshard_combine",
+                 "lserve_quantize_pages_kv4", "lserve_sparse_decode_attn_kv4",
+                 "lserve_decode_step"):
         getattr(lib, name).restype = ctypes.c_int
     return lib
 
@@ -211,11 +219,13 @@ def prefill_to_pages(desc, seq_len, k, v, block_table, head_kind, k_pool, v_pool
 
 
 def quantize_pages_kv8(desc, k_pool, v_pool, block_table, ctx_lens, k_pool8, v_pool8, k_scale,
-                       v_scale, stream=None):
-    """lserve_quantize_pages_kv8: int8 codes (int8 tensors shaped like the
-    pools) and float32 per-(page, head, channel) scales ([pool pages][H_kv][D])
-    of every page the block table references."""
-    _check("lserve_quantize_pages_kv8", lib.lserve_quantize_pages_kv8(
+                       v_scale, stream=None, bits=8):
+    """lserve_quantize_pages_kv8 (bits=8: int8 tensors shaped like the pools)
+    or lserve_quantize_pages_kv4 (bits=4: uint8 [pool pages][H_kv][N_P][D/2],
+    two codes per byte), with float32 per-(page, head, channel) scales
+    ([pool pages][H_kv][D]) of every page the block table references."""
+    name = {8: "lserve_quantize_pages_kv8", 4: "lserve_quantize_pages_kv4"}[bits]
+    _check(name, getattr(lib, name)(
         ctypes.byref(desc), _ptr(k_pool), _ptr(v_pool), _ptr(block_table), _ptr(ctx_lens),
         _ptr(k_pool8), _ptr(v_pool8), _ptr(k_scale), _ptr(v_scale), _stream(stream)))
 
@@ -223,15 +233,32 @@ def quantize_pages_kv8(desc, k_pool, v_pool, block_table, ctx_lens, k_pool8, v_p
 def sparse_decode_attn_kv8(desc, q, k_pool8, v_pool8, k_scale, v_scale, block_table, ctx_lens,
                            head_kind, sel, sel_count, top_k, sink_tokens, local_tokens,
                            softmax_scale, out, lse=None, workspace=None, stream=None,
-                           overlap_prologue=False):
-    """lserve_sparse_decode_attn_kv8: sparse decode attention over the int8 cache."""
+                           overlap_prologue=False, bits=8):
+    """lserve_sparse_decode_attn_kv8 / _kv4: sparse decode attention over the
+    8-bit or 4-bit cache."""
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     flags = DECODE_OVERLAP_PROLOGUE if overlap_prologue else 0
-    _check("lserve_sparse_decode_attn_kv8", lib.lserve_sparse_decode_attn_kv8(
+    name = {8: "lserve_sparse_decode_attn_kv8", 4: "lserve_sparse_decode_attn_kv4"}[bits]
+    _check(name, getattr(lib, name)(
         ctypes.byref(desc), _ptr(q), _ptr(k_pool8), _ptr(v_pool8), _ptr(k_scale), _ptr(v_scale),
         _ptr(block_table), _ptr(ctx_lens), _ptr(head_kind), _ptr(sel), _ptr(sel_count), top_k,
         sink_tokens, local_tokens, float(softmax_scale), _ptr(out), _ptr(lse), flags,
         _ptr(workspace), ws_bytes, _stream(stream)))
+
+
+def decode_step(desc, q, k_new, v_new, k_pool, v_pool, stats_pool, block_table, ctx_lens,
+                head_kind, sel, sel_count, top_k, sink_tokens, local_tokens, softmax_scale, out,
+                lse=None, recent_from=None, workspace=None, stream=None, overlap_prologue=False):
+    """lserve_decode_step: append the new tokens (k_new / v_new, or None) and
+    attend, in one launch; ctx_lens counts the new token."""
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    flags = DECODE_OVERLAP_PROLOGUE if overlap_prologue else 0
+    _check("lserve_decode_step", lib.lserve_decode_step(
+        ctypes.byref(desc), _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_pool), _ptr(v_pool),
+        _ptr(stats_pool), _ptr(block_table), _ptr(ctx_lens), _ptr(head_kind), _ptr(sel),
+        _ptr(sel_count), top_k, sink_tokens, local_tokens, _ptr(recent_from),
+        float(softmax_scale), _ptr(out), _ptr(lse), flags, _ptr(workspace), ws_bytes,
+        _stream(stream)))
 
 
 def blocksparse_prefill(desc, q, k, v, head_kind_host, softmax_scale, out, lse=None, workspace=None,

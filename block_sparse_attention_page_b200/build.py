@@ -20,7 +20,7 @@ CSRC = os.path.join(HERE, "csrc")
 ROOT = os.path.dirname(HERE)
 SOURCES = ["api.cu", "page_stats.cu", "page_select.cu", "decode_attn.cu", "decode_append.cu",
            "prefill.cu", "prefill_to_pages.cu", "select_noalloc.cu",
-           "quantize_kv8.cu", "seq_shard.cu"]
+           "quantize_kv.cu", "seq_shard.cu"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
          "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr", "-I", os.path.join(ROOT, "include")]

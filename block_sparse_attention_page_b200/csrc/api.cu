@@ -419,7 +419,7 @@ int decode_params(const lserve_paged_desc* desc, const void* q, const int32_t* b
   const int D = desc->head_dim, G = desc->num_q_heads / desc->num_kv_heads;
   const int P = desc->batch * desc->num_kv_heads;
   if (P > kDecodeMaxPairs) return LSERVE_ERR_UNSUPPORTED;
-  const int tile_rows = desc->physical_page < kDecodeTileMax ? desc->physical_page : kDecodeTileMax;
+  const int tile_rows = decode_tile_rows(desc->physical_page);
   grid = decode_grid(current_sm_count());
   {
     // Small calls use fewer CTAs: from the host-side shapes, a pair attends at
@@ -445,13 +445,11 @@ int decode_params(const lserve_paged_desc* desc, const void* q, const int32_t* b
   if (flags & LSERVE_DECODE_OUT_F32) p.out_f32 = static_cast<float*>(out);
   else p.out = static_cast<__nv_bfloat16*>(out);
   p.lse = lse;
+  // workspace: the pairs' merge epochs, then one tagged partial slot per CTA
+  // (decode_workspace_bytes sizes it for the device's largest grid)
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  const size_t cnt_bytes = ((size_t)(P + 1) * 4 + 255) / 256 * 256;
-  const size_t slots = (size_t)grid + P;
-  const size_t o_bytes = (slots * G * D * 4 + 255) / 256 * 256;
-  p.counters = reinterpret_cast<uint32_t*>(ws);
-  p.part_o = reinterpret_cast<float*>(ws + cnt_bytes);
-  p.part_ml = reinterpret_cast<float*>(ws + cnt_bytes + o_bytes);
+  p.epochs = reinterpret_cast<uint32_t*>(ws);
+  p.parts = reinterpret_cast<unsigned long long*>(ws + ((size_t)P * 4 + 255) / 256 * 256);
   p.batch = desc->batch;
   p.num_q_heads = desc->num_q_heads;
   p.num_kv_heads = desc->num_kv_heads;
@@ -463,6 +461,7 @@ int decode_params(const lserve_paged_desc* desc, const void* q, const int32_t* b
   p.local = local_tokens;
   p.tile_rows = tile_rows;
   p.tiles_per_page = desc->physical_page / tile_rows;
+  p.consumer_warps = decode_consumer_warps();
   p.scale_log2 = softmax_scale * 1.4426950408889634f;
   p.wait_limit = wait_limit();
   p.overlap_prologue = (flags & LSERVE_DECODE_OVERLAP_PROLOGUE) ? 1 : 0;
@@ -499,14 +498,17 @@ int lserve_sparse_decode_attn_ex(const lserve_paged_desc* desc, const void* q, c
   return cuda_status(launch_decode(p, kmap, vmap, D, G, grid, static_cast<cudaStream_t>(stream)));
 }
 
-int lserve_sparse_decode_attn_kv8(const lserve_paged_desc* desc, const void* q, const void* k_pool8,
-                                  const void* v_pool8, const float* k_scale, const float* v_scale,
-                                  const int32_t* block_table, const int32_t* ctx_lens,
-                                  const uint8_t* head_kind, const int32_t* sel,
-                                  const int32_t* sel_count, int32_t top_k, int32_t sink_tokens,
-                                  int32_t local_tokens, float softmax_scale, void* out, float* lse,
-                                  uint32_t flags, void* workspace, size_t workspace_bytes,
-                                  void* stream) {
+}  // extern "C"
+
+namespace {
+// decode over a quantized cache (bits = 8 or 4)
+int decode_quant_entry(const lserve_paged_desc* desc, const void* q, const void* k_pool8,
+                       const void* v_pool8, const float* k_scale, const float* v_scale,
+                       const int32_t* block_table, const int32_t* ctx_lens,
+                       const uint8_t* head_kind, const int32_t* sel, const int32_t* sel_count,
+                       int32_t top_k, int32_t sink_tokens, int32_t local_tokens,
+                       float softmax_scale, void* out, float* lse, uint32_t flags, void* workspace,
+                       size_t workspace_bytes, void* stream, int bits) {
   if (!k_pool8 || !v_pool8 || !k_scale || !v_scale) return LSERVE_ERR_INVALID_ARG;
   if (!aligned(k_pool8, 16) || !aligned(v_pool8, 16) || !aligned(k_scale, 16) || !aligned(v_scale, 16))
     return LSERVE_ERR_INVALID_ARG;
@@ -521,12 +523,75 @@ int lserve_sparse_decode_attn_kv8(const lserve_paged_desc* desc, const void* q, 
   p.k_scale = k_scale;
   p.v_scale = v_scale;
   const int D = desc->head_dim, G = desc->num_q_heads / desc->num_kv_heads;
-  return cuda_status(launch_decode_kv8(p, D, G, grid, static_cast<cudaStream_t>(stream)));
+  return cuda_status(launch_decode_quant(p, D, G, bits, grid, static_cast<cudaStream_t>(stream)));
+}
+}  // namespace
+
+extern "C" {
+
+int lserve_decode_step(const lserve_paged_desc* desc, const void* q, const void* k_new,
+                       const void* v_new, void* k_pool, void* v_pool, void* stats_pool,
+                       const int32_t* block_table, const int32_t* ctx_lens,
+                       const uint8_t* head_kind, const int32_t* sel, const int32_t* sel_count,
+                       int32_t top_k, int32_t sink_tokens, int32_t local_tokens,
+                       const int32_t* recent_from, float softmax_scale, void* out, float* lse,
+                       uint32_t flags, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!k_pool || !v_pool || !aligned(k_pool, 16) || !aligned(v_pool, 16)) return LSERVE_ERR_INVALID_ARG;
+  if ((k_new == nullptr) != (v_new == nullptr)) return LSERVE_ERR_INVALID_ARG;
+  if (k_new && (!stats_pool || !aligned(k_new, 16) || !aligned(v_new, 16) || !aligned(stats_pool, 16)))
+    return LSERVE_ERR_INVALID_ARG;
+  if (recent_from && !aligned(recent_from, 4)) return LSERVE_ERR_INVALID_ARG;
+  DecodeParams p;
+  int grid = 0;
+  const int st = decode_params(desc, q, block_table, ctx_lens, head_kind, sel, sel_count, top_k,
+                               sink_tokens, local_tokens, softmax_scale, out, lse, flags, workspace,
+                               workspace_bytes, p, grid);
+  if (st != LSERVE_OK) return st;
+  p.k_new = static_cast<const __nv_bfloat16*>(k_new);
+  p.v_new = static_cast<const __nv_bfloat16*>(v_new);
+  p.k_pool_w = static_cast<__nv_bfloat16*>(k_pool);
+  p.v_pool_w = static_cast<__nv_bfloat16*>(v_pool);
+  p.stats_w = static_cast<__nv_bfloat16*>(stats_pool);
+  p.logical_page = desc->logical_page;
+  p.recent_from = recent_from;
+  const int D = desc->head_dim, G = desc->num_q_heads / desc->num_kv_heads;
+  const uint64_t rows = (uint64_t)desc->num_pool_pages * desc->num_kv_heads * desc->physical_page;
+  CUtensorMap kmap, vmap;
+  if (!make_map_tiled(&kmap, k_pool, 3, 64, D / 64, rows, 64, D / 64, p.tile_rows) ||
+      !make_map_tiled(&vmap, v_pool, 3, 64, D / 64, rows, 64, D / 64, p.tile_rows))
+    return LSERVE_ERR_CUDA;
+  return cuda_status(launch_decode(p, kmap, vmap, D, G, grid, static_cast<cudaStream_t>(stream)));
 }
 
-int lserve_quantize_pages_kv8(const lserve_paged_desc* desc, const void* k_pool, const void* v_pool,
+int lserve_sparse_decode_attn_kv8(const lserve_paged_desc* desc, const void* q, const void* k_pool8,
+                                  const void* v_pool8, const float* k_scale, const float* v_scale,
+                                  const int32_t* block_table, const int32_t* ctx_lens,
+                                  const uint8_t* head_kind, const int32_t* sel,
+                                  const int32_t* sel_count, int32_t top_k, int32_t sink_tokens,
+                                  int32_t local_tokens, float softmax_scale, void* out, float* lse,
+                                  uint32_t flags, void* workspace, size_t workspace_bytes,
+                                  void* stream) {
+  return decode_quant_entry(desc, q, k_pool8, v_pool8, k_scale, v_scale, block_table, ctx_lens,
+                            head_kind, sel, sel_count, top_k, sink_tokens, local_tokens,
+                            softmax_scale, out, lse, flags, workspace, workspace_bytes, stream, 8);
+}
+
+int lserve_sparse_decode_attn_kv4(const lserve_paged_desc* desc, const void* q, const void* k_pool4,
+                                  const void* v_pool4, const float* k_scale, const float* v_scale,
+                                  const int32_t* block_table, const int32_t* ctx_lens,
+                                  const uint8_t* head_kind, const int32_t* sel,
+                                  const int32_t* sel_count, int32_t top_k, int32_t sink_tokens,
+                                  int32_t local_tokens, float softmax_scale, void* out, float* lse,
+                                  uint32_t flags, void* workspace, size_t workspace_bytes,
+                                  void* stream) {
+  return decode_quant_entry(desc, q, k_pool4, v_pool4, k_scale, v_scale, block_table, ctx_lens,
+                            head_kind, sel, sel_count, top_k, sink_tokens, local_tokens,
+                            softmax_scale, out, lse, flags, workspace, workspace_bytes, stream, 4);
+}
+
+static int quantize_entry(const lserve_paged_desc* desc, const void* k_pool, const void* v_pool,
                               const int32_t* block_table, const int32_t* ctx_lens, void* k_pool8,
-                              void* v_pool8, float* k_scale, float* v_scale, void* stream) {
+                              void* v_pool8, float* k_scale, float* v_scale, void* stream, int bits) {
   if (!valid_paged(desc)) return LSERVE_ERR_INVALID_ARG;
   if (!k_pool || !v_pool || !block_table || !ctx_lens || !k_pool8 || !v_pool8 || !k_scale || !v_scale)
     return LSERVE_ERR_INVALID_ARG;
@@ -554,7 +619,21 @@ int lserve_quantize_pages_kv8(const lserve_paged_desc* desc, const void* k_pool,
   p.num_pool_pages = desc->num_pool_pages;
   p.status = device_status_word();
   if (!p.status) return LSERVE_ERR_CUDA;
-  return cuda_status(launch_quantize_kv8(p, desc->head_dim, static_cast<cudaStream_t>(stream)));
+  return cuda_status(launch_quantize_kv(p, desc->head_dim, bits, static_cast<cudaStream_t>(stream)));
+}
+
+int lserve_quantize_pages_kv8(const lserve_paged_desc* desc, const void* k_pool, const void* v_pool,
+                              const int32_t* block_table, const int32_t* ctx_lens, void* k_pool8,
+                              void* v_pool8, float* k_scale, float* v_scale, void* stream) {
+  return quantize_entry(desc, k_pool, v_pool, block_table, ctx_lens, k_pool8, v_pool8, k_scale,
+                        v_scale, stream, 8);
+}
+
+int lserve_quantize_pages_kv4(const lserve_paged_desc* desc, const void* k_pool, const void* v_pool,
+                              const int32_t* block_table, const int32_t* ctx_lens, void* k_pool4,
+                              void* v_pool4, float* k_scale, float* v_scale, void* stream) {
+  return quantize_entry(desc, k_pool, v_pool, block_table, ctx_lens, k_pool4, v_pool4, k_scale,
+                        v_scale, stream, 4);
 }
 
 int lserve_seqshard_bounds(int32_t ctx_len, int32_t physical_page, int32_t rank,

@@ -9,13 +9,16 @@
 // SM).  Every SM therefore streams the same number of KV bytes, however unequal
 // the pairs are (64 selected pages next to ~10 sink + local pages).
 //
-// Per CTA: one producer warp and kConsumerWarps consumer warps.
+// Per CTA: one producer warp and W = 8 consumer warps, one CTA per SM.  (A
+// two-CTAs-per-SM shape -- W = 4, 32-token tiles, at most 112 KB of shared
+// memory each, so that the next call's CTAs are resident while this call
+// runs -- measured 1.5x slower on the 8B layer and is not instantiated.)
 //   producer : its lanes resolve 32 tiles at a time (pair, page ordinal,
 //              block-table lookup); then, stage by stage of an S-deep ring, it
 //              waits until every consumer warp has released the stage and
 //              refills it -- K and V by TMA (128-byte swizzle), the pair's q by
 //              a 1-D bulk copy.
-//   consumers: every warp owns 1/kConsumerWarps of each tile's tokens and keeps
+//   consumers: every warp owns 1/W of each tile's tokens and keeps
 //              its own online-softmax state, so a tile needs no CTA-wide
 //              barrier.  An iteration takes one tile, or two consecutive tiles
 //              of the same pair.
@@ -29,10 +32,17 @@
 //              registers across tiles, rescaled only when a running max grew.
 // Pair boundaries come from the tile plan in shared memory, so all consumer
 // warps agree on them whatever the data.  At a boundary the warps' states are
-// merged in shared memory.  A pair covered by one CTA is finalised there;
-// otherwise each CTA writes an unnormalised (o, m, l) partial and the last CTA
-// to finish the pair (per-pair counter in the workspace) merges the partials
-// with log-sum-exp weights and resets the counter to zero.
+// merged in shared memory.  A pair covered by one CTA is finalised there.  A
+// pair split over CTAs c_f .. c_l is merged by c_f, the CTA holding its first
+// tile (the pair closes c_f's range, so c_f reaches it last): every other CTA
+// c of the pair holds it as its FIRST pair and writes its unnormalised
+// (o, m, l) partial into its own workspace slot as tagged 8-byte words
+// {value, tag}, and c_f polls those words until their tags match, then merges
+// them with log-sum-exp weights.  No fence, counter or atomic is involved: a
+// word is one single-copy atomic store, and the tag carries the pair and the
+// pair's merge epoch (a per-pair counter that c_f advances at the end of
+// every call, whatever happened), so words left by an earlier call -- even
+// one that ended in a timeout -- never match.
 #include <cstring>
 
 #include "common.cuh"
@@ -42,9 +52,6 @@ namespace lserve {
 
 namespace {
 
-constexpr int kConsumerWarps = 8;
-constexpr int kThreads = (kConsumerWarps + 1) * 32;  // + the producer warp
-constexpr int kConsumerThreads = kConsumerWarps * 32;
 constexpr int kBarConsumers = 1;       // named barrier of the consumer warps
 constexpr int kMaxGrid = 512;          // CTAs whose range starts the range table holds
 constexpr unsigned kFull = 0xffffffffu;
@@ -55,38 +62,125 @@ __device__ __forceinline__ void store_out(const DecodeParams& p, size_t i, float
   else p.out[i] = __float2bfloat16_rn(v);
 }
 
-// Pages the pair attends (retrieval: the selection; streaming: sink + local).
+// Recent pages of a retrieval pair (the option of attending every token since
+// the selection): the pages [ra, rz] holding positions [recent_from[b], n);
+// those the selection holds are attended as selected pages.  The selection is
+// ascending, so its entries in [ra, rz] are among its last rz - ra + 1.
+__device__ __forceinline__ bool recent_range(const DecodeParams& p, int b, int n, int& ra, int& rz,
+                                             int& rf) {
+  if (!p.recent_from || n <= 0) return false;
+  rf = max(0, min(p.recent_from[b], n));
+  if (rf >= n) return false;
+  ra = rf / p.physical_page;
+  rz = (n - 1) / p.physical_page;
+  return true;
+}
+__device__ __forceinline__ bool in_sel_tail(const int32_t* s, int nsel, int R, int m) {
+  for (int i = max(0, nsel - R); i < nsel; ++i)
+    if (s[i] == m) return true;
+  return false;
+}
+
+// Selected pages of a retrieval pair the attention takes (the clamped count).
+__device__ __forceinline__ int sel_pages(const DecodeParams& p, int pair, int npages) {
+  return min(max(p.sel_count[pair], 0), min(p.top_k, npages));
+}
+
+// Pages the pair attends (retrieval: the selection, plus the recent pages it
+// does not hold; streaming: sink + local).
 __device__ __forceinline__ int pair_pages(const DecodeParams& p, int pair) {
   const int b = pair / p.num_kv_heads, h = pair - b * p.num_kv_heads;
   const int n = p.ctx_lens[b];
   const int kind = p.head_kind[h];
-  const int nsel = p.sel_count[pair];  // loaded whatever the kind: one round trip
   const int NP = p.physical_page;
   const int npages = (n + NP - 1) / NP;
-  if (kind == 0) return min(max(nsel, 0), min(p.top_k, npages));
+  if (kind == 0) {
+    const int nsel = sel_pages(p, pair, npages);
+    int ra, rz, rf;
+    if (!recent_range(p, b, n, ra, rz, rf)) return nsel;
+    const int32_t* s = p.sel + (size_t)pair * p.top_k;
+    int extra = 0;
+    for (int m = ra; m <= rz; ++m) extra += in_sel_tail(s, nsel, rz - ra + 1, m) ? 0 : 1;
+    return nsel + extra;
+  }
   const int ns = min((p.sink + NP - 1) / NP, npages);
   const int ls = max(max(0, n - p.local) / NP, ns);
   return ns + max(0, npages - ls);
 }
 
-// Q8: the int8 cache -- K / V tiles of 1-byte codes followed by the page's
-// K and V channel scales (float32 [D] each); otherwise bf16 tiles.
-template <int D, int G, bool Q8 = false>
+// The appended token's rows: K and V into the pools, and for a retrieval
+// head its logical page's k_min / k_max (a page's first token starts them),
+// exact in bf16.  One warp per (sequence, KV head); lanes take 16-byte
+// chunks (D / 8 of them per row).
+template <int D>
+__device__ __forceinline__ void append_rows(const DecodeParams& p, int pair, int lane) {
+  const int b = pair / p.num_kv_heads, h = pair - b * p.num_kv_heads;
+  const int n = p.ctx_lens[b];
+  if (n <= 0) return;
+  const int t = n - 1, NP = p.physical_page, m = t / NP;
+  int pid = -1;
+  if (m < p.max_pages) pid = p.block_table[(size_t)b * p.max_pages + m];
+  if (pid < 0 || pid >= p.num_pool_pages) {
+    if (lane == 0) raise_status(p.status, LSERVE_ERR_BOUNDS);
+    return;
+  }
+  constexpr int C16 = D / 8;  // 16-byte chunks per row
+  const size_t row = ((size_t)pid * p.num_kv_heads + h) * NP + (t - m * NP);
+  const size_t src = ((size_t)b * p.num_kv_heads + h) * D;
+  if (lane < C16) {
+    const uint4 k = *reinterpret_cast<const uint4*>(p.k_new + src + lane * 8);
+    *reinterpret_cast<uint4*>(p.k_pool_w + row * D + lane * 8) = k;
+    if (p.head_kind[h] == 0) {
+      const int g = NP / p.logical_page, sub = (t - m * NP) / p.logical_page;
+      __nv_bfloat16* st = p.stats_w + (((size_t)pid * p.num_kv_heads + h) * g + sub) * 2 * D + lane * 8;
+      uint4 lo = k, hi = k;
+      if (t % p.logical_page != 0) {
+        const uint4 a = *reinterpret_cast<const uint4*>(st), z = *reinterpret_cast<const uint4*>(st + D);
+        const __nv_bfloat162* kk = reinterpret_cast<const __nv_bfloat162*>(&k);
+        const __nv_bfloat162* aa = reinterpret_cast<const __nv_bfloat162*>(&a);
+        const __nv_bfloat162* zz = reinterpret_cast<const __nv_bfloat162*>(&z);
+        __nv_bfloat162* ll = reinterpret_cast<__nv_bfloat162*>(&lo);
+        __nv_bfloat162* hh = reinterpret_cast<__nv_bfloat162*>(&hi);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          ll[i] = __hmin2(aa[i], kk[i]);
+          hh[i] = __hmax2(zz[i], kk[i]);
+        }
+      }
+      *reinterpret_cast<uint4*>(st) = lo;
+      *reinterpret_cast<uint4*>(st + D) = hi;
+    }
+  } else if (lane < 2 * C16) {
+    const int c = lane - C16;
+    *reinterpret_cast<uint4*>(p.v_pool_w + row * D + c * 8) =
+        *reinterpret_cast<const uint4*>(p.v_new + src + c * 8);
+  }
+}
+
+// QB = 8 / 4: the quantized cache -- K / V tiles of 8- or 4-bit codes
+// followed by the page's K and V channel scales (float32 [D] each); QB = 0:
+// bf16 tiles.  TR tokens per tile, W consumer warps; W = 4 is the
+// two-CTAs-per-SM shape (at most 112 KB of shared memory each), W = 8 takes a
+// whole SM.
+template <int D, int G, int QB, int TR, int W>
 struct DecLayout {
-  static constexpr int kTileK = kDecodeTileMax * D * (Q8 ? 1 : 2);       // K (or V) tile bytes
-  static constexpr int kScales = Q8 ? 2 * D * 4 : 0;                     // K, V channel scales
+  static constexpr int kRow = D * (QB == 0 ? 16 : QB) / 8;               // bytes per K (or V) row
+  static constexpr int kTileK = TR * kRow;                               // K (or V) tile bytes
+  static constexpr int kScales = QB ? 2 * D * 4 : 0;                     // K, V channel scales
   static constexpr int oScale = 2 * kTileK;                              // stage offsets
   static constexpr int oQ = oScale + kScales;
   static constexpr int kStageQ = G * D * 2;
-  static constexpr int kStage = (oQ + kStageQ + 1023) / 1024 * 1024;
-  static constexpr int kPs = 2 * kDecodeTileMax * G * 8;                 // p of two tiles
-  static constexpr int kOw = kConsumerWarps * G * D * 4;                 // o per warp
-  static constexpr int kMl = kConsumerWarps * G * 2 * 4;                 // (m, l) per warp
-  static constexpr int kSc = (kConsumerWarps + 1) * G * 4;               // merge weights + max
+  static constexpr int oNew = oQ + kStageQ;                              // appended K, V rows (bf16)
+  static constexpr int kNew = QB ? 0 : 2 * D * 2;
+  static constexpr int kStage = (oNew + kNew + 1023) / 1024 * 1024;
+  static constexpr int kPs = 2 * TR * G * 8;                            // p of two tiles
+  static constexpr int kOw = W * G * D * 4;                              // o per warp
+  static constexpr int kMl = W * G * 2 * 4;                              // (m, l) per warp
+  static constexpr int kSc = (W + 1) * G * 4;                            // merge weights + max
   static constexpr int kOff = ((kDecodeMaxPairs + 1) * 4 + 15) / 16 * 16;
   static constexpr int kCst = ((kMaxGrid + 1) * 4 + 15) / 16 * 16;
   static constexpr int kFixed = kPs + kOw + kMl + kSc + kOff + kCst + 1024;
-  static constexpr int kBudget = 227 * 1024 - 1024;
+  static constexpr int kBudget = W <= 4 ? 112 * 1024 : 227 * 1024 - 1024;
   static constexpr int kStagesFit = (kBudget - kFixed) / kStage;
   static constexpr int kStages = kStagesFit > 8 ? 8 : kStagesFit;
   // offsets (stages first: 1024-aligned for the swizzled TMA tiles)
@@ -133,6 +227,28 @@ __device__ __forceinline__ int pair_of(const int* off, int u, int P) {
     if (off[mid] <= u) lo = mid; else hi = mid - 1;
   }
   return lo;
+}
+
+// Tagged partial words: {float value, tag} as one 64-bit store / load.  The
+// tag is the pair's merge epoch for this call (11 low bits: the pair; pairs
+// are < 2048) -- a word from any earlier call or another pair differs.
+__device__ __forceinline__ uint32_t part_tag(uint32_t epoch, int pair) {
+  return (epoch << 11) | (uint32_t)pair;
+}
+__device__ __forceinline__ void st_word(unsigned long long* a, float v, uint32_t tag) {
+  const unsigned long long w = ((unsigned long long)tag << 32) | __float_as_uint(v);
+  asm volatile("st.relaxed.gpu.global.b64 [%0], %1;" ::"l"(a), "l"(w) : "memory");
+}
+__device__ __forceinline__ unsigned long long ld_word(const unsigned long long* a) {
+  unsigned long long w;
+  asm volatile("ld.relaxed.gpu.global.b64 %0, [%1];" : "=l"(w) : "l"(a) : "memory");
+  return w;
+}
+__device__ __forceinline__ bool word_ok(unsigned long long w, uint32_t tag) {
+  return (uint32_t)(w >> 32) == tag;
+}
+__device__ __forceinline__ float word_val(unsigned long long w) {
+  return __uint_as_float((uint32_t)w);
 }
 
 // Bounded wait that gives up at once when another warp already timed out.
@@ -192,19 +308,62 @@ __device__ __forceinline__ void join_step(const float (&in)[N], float (&out)[N >
 template <int V>
 constexpr int join_out() { return V >= 8 ? V / 8 : 1; }
 
-// Four int8 codes (one 32-bit word, lowest byte first) times their channel
-// scales.  A code c becomes the float 2^23 + (c + 128) by placing the byte
-// c ^ 0x80 in the mantissa of 2^23; subtracting 2^23 + 128 leaves c exactly.
-__device__ __forceinline__ void dequant4_s8(uint32_t w, float2 s01, float2 s23, float2& x01,
-                                            float2& x23) {
+// Quantized codes -> fp16 pairs, exactly (|code| <= 127 fits fp16's 11-bit
+// significand).  8-bit: a byte c placed as the low byte of the fp16 1024 + x
+// (0x64xx: 1024 .. 1279, step 1) after flipping its sign bit gives
+// 1024 + (c + 128); subtracting 1152 leaves c.  Word w (codes of channels
+// 4m .. 4m+3, lowest byte first) gives the pairs (4m, 4m+1) and (4m+2, 4m+3).
+__device__ __forceinline__ void codes8_to_f16(uint32_t w, uint32_t& p01, uint32_t& p23) {
   const uint32_t u = w ^ 0x80808080u;
-  const float2 bias = make_float2(-8388736.f, -8388736.f);
-  const float2 f01 = make_float2(__uint_as_float(__byte_perm(u, 0x4B000000u, 0x7440)),
-                                 __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7441)));
-  const float2 f23 = make_float2(__uint_as_float(__byte_perm(u, 0x4B000000u, 0x7442)),
-                                 __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7443)));
-  x01 = __fmul2_rn(__fadd2_rn(f01, bias), s01);
-  x23 = __fmul2_rn(__fadd2_rn(f23, bias), s23);
+  const uint32_t x = __byte_perm(u, 0x64646464u, 0x4140);
+  const uint32_t y = __byte_perm(u, 0x64646464u, 0x4342);
+  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(p01) : "r"(x), "r"(0x64806480u));
+  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(p23) : "r"(y), "r"(0x64806480u));
+}
+// 4-bit: nibble c of channel 8m + j (lowest nibble first) flipped by 8 is
+// c + 8 in 1..15; ORed into the fp16 1024 and less 1032 it is c.  Word w
+// (channels 8m .. 8m+7) gives the pairs (8m + j, 8m + j + 4), j = 0..3.
+__device__ __forceinline__ uint32_t codes4_pair(uint32_t u, int j) {
+  const uint32_t x = ((u >> (4 * j)) & 0x000F000Fu) | 0x64006400u;
+  uint32_t r;
+  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(x), "r"(0x64086408u));
+  return r;
+}
+// channel offset (inside a lane's run) of element e of pair p of QB-bit codes
+__host__ __device__ constexpr int pair_channel(int QB, int p, int e) {
+  return QB == 4 ? 8 * (p / 4) + (p % 4) + 4 * e : 2 * p + e;
+}
+__device__ __forceinline__ uint32_t f32x2_to_f16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+__device__ __forceinline__ uint32_t hmul2(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+__device__ __forceinline__ float f16_lo(uint32_t w) { return __half2float(__ushort_as_half((unsigned short)(w & 0xFFFFu))); }
+__device__ __forceinline__ float f16_hi(uint32_t w) { return __half2float(__ushort_as_half((unsigned short)(w >> 16))); }
+// 8x8 b16 matrix transposed across the warp (lane L holds row L/4, columns
+// 2*(L%4) + {0,1} before and after)
+__device__ __forceinline__ uint32_t movmatrix_t(uint32_t x) {
+  uint32_t r;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(r) : "r"(x));
+  return r;
+}
+__device__ __forceinline__ void mma_16816_f16(float (&d)[4], uint32_t a0, uint32_t a2, uint32_t b0,
+                                              uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9},"
+      " {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ void mma_1688_f16(float (&d)[4], uint32_t a0, uint32_t b0) {
+  asm("mma.sync.aligned.m16n8k8.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5}, {%6},"
+      " {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(0u), "r"(b0));
 }
 
 // Warp-level tensor-core tiles (mma.sync, bf16 in, fp32 accumulate).  The
@@ -244,12 +403,14 @@ __device__ __forceinline__ void join_dots(const float (&d)[V], float (&out)[join
 
 }  // namespace
 
-template <int D, int G, int TR, bool Q8>
-__global__ void __launch_bounds__(kThreads, 1)
+template <int D, int G, int TR, int QB, int W>
+__global__ void __launch_bounds__((W + 1) * 32, W <= 4 ? 2 : 1)
 decode_attn_kernel(const __grid_constant__ DecodeParams p, const __grid_constant__ CUtensorMap kmap,
                    const __grid_constant__ CUtensorMap vmap) {
-  using L = DecLayout<D, G, Q8>;
-  constexpr int W = kConsumerWarps;
+  using L = DecLayout<D, G, QB, TR, W>;
+  constexpr bool Q8 = QB != 0;             // a quantized cache (8- or 4-bit codes)
+  constexpr int kThreads = (W + 1) * 32;   // consumer warps + the producer warp
+  constexpr int kConsumerThreads = W * 32;
   constexpr int S = L::kStages;
   constexpr int HB = G < 4 ? G : 4;      // heads whose q a QK lane holds at a time
   constexpr int NHB = G / HB;            // head blocks (2 for G = 8)
@@ -280,7 +441,7 @@ decode_attn_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
   int* info = reinterpret_cast<int*>(smem + L::oInfo);     // valid tokens of the stage's tile
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::oFull);
   uint64_t* empty = reinterpret_cast<uint64_t*>(smem + L::oEmpty);
-  // [0..15] scan, [18] abort, [20..21] pairs to merge, [24..27] zeros
+  // [0..15] scan, [18] abort, [24..27] zeros
   int* misc = reinterpret_cast<int*>(smem + L::oMisc);
   volatile int* abort_flag = misc + 18;
   const uint8_t* zero16 = reinterpret_cast<const uint8_t*>(misc + 24);  // 16 zero bytes
@@ -302,7 +463,6 @@ decode_attn_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
       mbar_init(&empty[s], W);
     }
     misc[18] = 0;
-    misc[20] = misc[21] = -1;  // pairs to merge at the end (first, last of the range)
     misc[24] = misc[25] = misc[26] = misc[27] = 0;
     fence_mbar_init();
   }
@@ -352,6 +512,8 @@ decode_attn_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
   // =========================== producer warp ===============================
   if (warp == W) {
     // descriptor of tile u: (pair, first row in the [pool rows][D] view, valid tokens)
+    // valid is packed with the first token the tile attends (lo, recent pages)
+    // and 1 + the row of the appended token (0: none): valid | lo << 8 | (row + 1) << 16
     auto lookup = [&](int u, int& pair, int& row, int& valid) {
       pair = pair_of(off, u, P);
       const int local = u - off[pair];
@@ -360,9 +522,22 @@ decode_attn_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
       const int n = p.ctx_lens[b];
       const int NP = p.physical_page;
       const int npages = (n + NP - 1) / NP;
-      int m;
+      int m, lo = 0;
       if (p.head_kind[h] == 0) {
-        m = p.sel[(size_t)pair * p.top_k + li];
+        const int nsel = sel_pages(p, pair, npages);
+        if (li < nsel) {
+          m = p.sel[(size_t)pair * p.top_k + li];
+        } else {  // the (li - nsel)-th recent page the selection does not hold
+          m = -1;
+          int ra, rz, rf;
+          if (recent_range(p, b, n, ra, rz, rf)) {
+            const int32_t* s = p.sel + (size_t)pair * p.top_k;
+            int r = li - nsel;
+            for (int j = ra; j <= rz && m < 0; ++j)
+              if (!in_sel_tail(s, nsel, rz - ra + 1, j) && r-- == 0) m = j;
+            if (m >= 0) lo = max(0, rf - m * NP);
+          }
+        }
       } else {
         const int ns = min((p.sink + NP - 1) / NP, npages);
         const int ls = max(max(0, n - p.local) / NP, ns);
@@ -378,6 +553,10 @@ decode_attn_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
       }
       row = (int)(((long long)pid * p.num_kv_heads + h) * NP + sub * TR);
       valid = max(0, min(TR, n - m * NP - sub * TR));
+      const int lo_t = min(valid, max(0, lo - sub * TR));
+      const int ta = p.k_new ? n - 1 - (m * NP + sub * TR) : -1;  // the appended token's row
+      const int fix = (ta >= lo_t && ta < valid) ? ta : -1;
+      valid |= (lo_t << 8) | ((fix + 1) << 16);
     };
     int issued = 0;
     bool alive = true;
@@ -401,18 +580,24 @@ decode_attn_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
             const int b = pr / p.num_kv_heads, h = pr - b * p.num_kv_heads;
             uint8_t* st = smem + s * L::kStage;
             if constexpr (Q8) {
-              // codes: one contiguous TR x D byte tile each; then the page's scales
+              // codes: one contiguous TR-row tile each; then the page's scales
               const size_t ph = (size_t)row / p.physical_page;  // pool page * H_kv + head
-              mbar_arrive_expect_tx(&full[s], 2 * TR * D + L::kScales + L::kStageQ);
-              bulk_load_1d_hint(st, p.k8 + (size_t)row * D, TR * D, &full[s], pol);
-              bulk_load_1d_hint(st + L::kTileK, p.v8 + (size_t)row * D, TR * D, &full[s], pol);
+              mbar_arrive_expect_tx(&full[s], 2 * L::kTileK + L::kScales + L::kStageQ);
+              bulk_load_1d_hint(st, p.k8 + (size_t)row * L::kRow, L::kTileK, &full[s], pol);
+              bulk_load_1d_hint(st + L::kTileK, p.v8 + (size_t)row * L::kRow, L::kTileK, &full[s], pol);
               bulk_load_1d(st + L::oScale, p.k_scale + ph * D, D * 4, &full[s]);
               bulk_load_1d(st + L::oScale + D * 4, p.v_scale + ph * D, D * 4, &full[s]);
             } else {
-              mbar_arrive_expect_tx(&full[s], 2 * TR * D * 2 + L::kStageQ);
+              const bool has_new = (val >> 16) != 0;  // the tile holds the appended token
+              mbar_arrive_expect_tx(&full[s], 2 * TR * D * 2 + L::kStageQ + (has_new ? L::kNew : 0));
               // one contiguous TR x D tile each: 3-D view (64 channels, D/64 halves, rows)
               tma_load_3d_hint(st, &kmap, 0, 0, row, &full[s], pol);
               tma_load_3d_hint(st + L::kTileK, &vmap, 0, 0, row, &full[s], pol);
+              if (has_new) {  // its K / V rows from k_new / v_new, next to the tile
+                const size_t src = ((size_t)b * p.num_kv_heads + h) * D;
+                bulk_load_1d(st + L::oNew, p.k_new + src, D * 2, &full[s]);
+                bulk_load_1d(st + L::oNew + D * 2, p.v_new + src, D * 2, &full[s]);
+              }
             }
             bulk_load_1d(st + L::oQ, p.q + ((size_t)b * p.num_q_heads + (size_t)h * G) * D,
                          L::kStageQ, &full[s]);
@@ -430,11 +615,27 @@ decode_attn_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
     // after a timeout: let the copies still in flight land before the CTA exits
     if (!alive && lane == 0)
       for (int k = max(0, issued - S); k < issued; ++k) mbar_wait(&full[k % S], (k / S) & 1, lim, p.status);
+    // The appended tokens' rows go to the pools and statistics (pairs dealt
+    // round-robin over the CTAs).  This launch reads those rows from k_new /
+    // v_new instead, so its own TMA copies of them may see either content.
+    if (p.k_new) {
+      if (ntiles == 0) pdl_wait_prior_grid();  // the pools may be in use by the kernel before
+      for (int pr = cta; pr < P; pr += NC) append_rows<D>(p, pr, lane);
+    }
     return;
   }
 
   // =========================== consumer warps ==============================
   pdl_wait_prior_grid();  // no global write before the previous kernel completes
+  // Split pairs at the ends of this CTA's range: the first pair, if it began
+  // in an earlier CTA, gets a partial written to this CTA's slot; the last
+  // pair, if it begins here and goes on into later CTAs, is merged here.
+  const int first_pair = ntiles > 0 ? pair_of(off, u0, P) : -1;
+  const int last_pair = ntiles > 0 ? pair_of(off, u1 - 1, P) : -1;
+  const int merge_pair =
+      (last_pair >= 0 && off[last_pair] >= u0 && off[last_pair + 1] > u1) ? last_pair : -1;
+  const uint32_t e_first = (first_pair >= 0 && off[first_pair] < u0) ? __ldcg(p.epochs + first_pair) : 0u;
+  const uint32_t e_merge = merge_pair >= 0 ? __ldcg(p.epochs + merge_pair) : 0u;
   // pairs with nothing to attend (n = 0): zero output, lse = -inf
   if (cta == 0) {
     for (int pr = tid; pr < P; pr += kConsumerThreads) {
@@ -457,12 +658,7 @@ decode_attn_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
   // consecutive 128-byte swizzle rows)
   uint32_t koff[R][KCH];
   uint32_t voff[PVN];
-  if constexpr (Q8) {  // unswizzled byte rows of D codes
-#pragma unroll
-    for (int r = 0; r < R; ++r) koff[r][0] = (wt0 + 4 * r + tok_l) * D + qtr * CPT;
-#pragma unroll
-    for (int j = 0; j < PVN; ++j) voff[j] = L::kTileK + (pv_t0 + j) * D + 4 * quad;
-  } else {
+  if constexpr (!Q8) {
 #pragma unroll
     for (int r = 0; r < R; ++r)
 #pragma unroll
@@ -494,6 +690,7 @@ decode_attn_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
   // ldmatrix.trans; O (rows = heads, 8 channels per n-tile) stays in
   // registers across the pair's tiles.
   constexpr bool kMma = !Q8 && G >= 4;  // G < 4: most MMA rows would be padding
+  constexpr bool kQmma = Q8;             // the quantized cache: tensor cores for every G
   constexpr int KS = D / 16;   // QK k-steps
   constexpr int CPL = D / 4;   // channels per lane in the QK operands
   constexpr int NTl = D / 8;   // PV n-tiles (8 channels each)
@@ -596,6 +793,128 @@ decode_attn_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
     }
   };
 
+  // ---- tensor-core consumer of the quantized cache (QB = 8 or 4, every G).
+  // The fragments are those above, in fp16: a lane's QK operand is its
+  // token's run of CPL channels, whose codes convert to fp16 exactly; the
+  // page's K channel scales go into q instead (q' = q * k_scale, rounded once
+  // to fp16, per tile), so S = q' . code.  For PV the lane forms its token's
+  // V' = code * v_scale (fp16) and movmatrix transposes each 8 x 8 block into
+  // the B fragment.  Pair p of a lane's run holds channels pair_channel(QB, p,
+  // 0 / 1); n-tile p of O therefore holds, in fragment columns 2*qq + e,
+  // channel CPL*qq + pair_channel(QB, p, e).
+  constexpr int QBB = QB ? QB : 8;
+  constexpr int CB = CPL * QBB / 8;          // code bytes of a lane's run
+  constexpr int NP2 = CPL / 2;               // pairs of a lane's run
+  uint32_t qbf[CPL / 2];                     // q of head hr (bf16 pairs, natural order); 0 on padding rows
+  // this lane's run of codes of token row t of the tile at `tile`, as fp16 pairs
+  auto run_codes = [&](const uint8_t* tile, int t, uint32_t (&pr)[NP2]) {
+    const uint8_t* cp = tile + t * L::kRow + CB * qq;
+    uint32_t w[CB / 4];
+#pragma unroll
+    for (int i = 0; i < CB / 16; ++i) {
+      const uint4 v = reinterpret_cast<const uint4*>(cp)[i];
+      w[4 * i] = v.x;
+      w[4 * i + 1] = v.y;
+      w[4 * i + 2] = v.z;
+      w[4 * i + 3] = v.w;
+    }
+    if constexpr (CB % 16 == 8) {
+      const uint2 v = reinterpret_cast<const uint2*>(cp)[CB / 8 - 1];
+      w[CB / 4 - 2] = v.x;
+      w[CB / 4 - 1] = v.y;
+    }
+#pragma unroll
+    for (int m = 0; m < CB / 4; ++m) {
+      if constexpr (QB == 8) {
+        codes8_to_f16(w[m], pr[2 * m], pr[2 * m + 1]);
+      } else {
+        const uint32_t u = w[m] ^ 0x88888888u;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) pr[4 * m + j] = codes4_pair(u, j);
+      }
+    }
+  };
+  // f(pair, scale of its channel 0, scale of its channel 1) for every pair of
+  // this lane's run, the page's K (which = 0) or V (1) channel scales read 8
+  // channels at a time
+  auto for_scale_pairs = [&](const uint8_t* st, int which, auto&& f) {
+    const float4* sp = reinterpret_cast<const float4*>(st + L::oScale + which * D * 4) + qq * (CPL / 4);
+#pragma unroll
+    for (int m = 0; m < CPL / 8; ++m) {
+      const float4 a = sp[2 * m], b = sp[2 * m + 1];
+      const float c[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int pp = 4 * m + j;
+        f(pp, c[pair_channel(QBB, pp, 0) - 8 * m], c[pair_channel(QBB, pp, 1) - 8 * m]);
+      }
+    }
+  };
+  auto q_chan = [&](int c) -> float {  // q of head hr, channel CPL*qq + c
+    return (c & 1) ? bf16_hi(qbf[c / 2]) : bf16_lo(qbf[c / 2]);
+  };
+  auto load_q_qmma = [&](const uint8_t* st) {
+#pragma unroll
+    for (int i = 0; i < CPL / 8; ++i) {
+      uint4 w = make_uint4(0u, 0u, 0u, 0u);
+      if (real_row) w = reinterpret_cast<const uint4*>(st + L::oQ + (hr * D + CPL * qq) * 2)[i];
+      qbf[4 * i] = w.x;
+      qbf[4 * i + 1] = w.y;
+      qbf[4 * i + 2] = w.z;
+      qbf[4 * i + 3] = w.w;
+    }
+  };
+  // S of the warp's 8 tokens of tile st over the quantized keys
+  auto qk_qmma = [&](const uint8_t* st, float (&sa)[4], float (&sb)[4]) {
+    uint32_t qf[NP2];
+    for_scale_pairs(st, 0, [&](int pp, float s0, float s1) {
+      qf[pp] = f32x2_to_f16x2(q_chan(pair_channel(QBB, pp, 0)) * s0, q_chan(pair_channel(QBB, pp, 1)) * s1);
+    });
+    uint32_t kc[NP2];
+    run_codes(st, mt0 + hr, kc);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) sa[i] = sb[i] = 0.f;
+#pragma unroll
+    for (int k2 = 0; k2 < KS; ++k2) {
+      if (k2 & 1) mma_16816_f16(sb, qf[2 * k2], qf[2 * k2 + 1], kc[2 * k2], kc[2 * k2 + 1]);
+      else mma_16816_f16(sa, qf[2 * k2], qf[2 * k2 + 1], kc[2 * k2], kc[2 * k2 + 1]);
+    }
+  };
+  // V' = code * v_scale of the warp's token mt0 + hr of tile st, transposed into
+  // the B fragments of the NP2 n-tiles
+  auto v_frags = [&](const uint8_t* st, uint32_t (&vb)[NP2]) {
+    uint32_t vc[NP2];
+    run_codes(st + L::kTileK, mt0 + hr, vc);
+    for_scale_pairs(st, 1, [&](int pp, float s0, float s1) {
+      vb[pp] = movmatrix_t(hmul2(vc[pp], f32x2_to_f16x2(s0, s1)));
+    });
+  };
+  auto pv_qmma = [&](const uint8_t* st0, const uint8_t* st1, int nt, const float (&pr)[2][2]) {
+    uint32_t ah[2], al[2];
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      ah[i] = f32x2_to_f16x2(pr[i][0], pr[i][1]);
+      al[i] = f32x2_to_f16x2(pr[i][0] - f16_lo(ah[i]), pr[i][1] - f16_hi(ah[i]));
+    }
+    uint32_t v0[NP2];
+    v_frags(st0, v0);
+    if (nt == 2) {
+      uint32_t v1[NP2];
+      v_frags(st1, v1);
+#pragma unroll
+      for (int n = 0; n < NP2; ++n) {
+        mma_16816_f16(om[n], ah[0], ah[1], v0[n], v1[n]);
+        mma_16816_f16(om[n], al[0], al[1], v0[n], v1[n]);
+      }
+    } else {
+#pragma unroll
+      for (int n = 0; n < NP2; ++n) {
+        mma_1688_f16(om[n], ah[0], v0[n]);
+        mma_1688_f16(om[n], al[0], v0[n]);
+      }
+    }
+  };
+
   auto load_q = [&](const uint8_t* st, int hb) {  // bf16 q of the stage -> this lane's eighth
 #pragma unroll
     for (int h = 0; h < HB; ++h) {
@@ -611,45 +930,9 @@ decode_attn_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
     }
   };
 
-  // partial dots of tile st for the rows of this lane: d[g * R + r]
+  // partial dots of tile st for the rows of this lane: d[g * R + r] (bf16 cache)
   auto qk_tile = [&](const uint8_t* st, float (&d)[V], int hb) {
-    if constexpr (Q8) {
-      // this lane's CPT channel scales of the tile's page
-      float2 sk[CPT / 2];
-      const float4* skp = reinterpret_cast<const float4*>(st + L::oScale) + qtr * (CPT / 4);
-#pragma unroll
-      for (int i = 0; i < CPT / 4; ++i) {
-        const float4 s4 = skp[i];
-        sk[2 * i] = make_float2(s4.x, s4.y);
-        sk[2 * i + 1] = make_float2(s4.z, s4.w);
-      }
-#pragma unroll
-      for (int r = 0; r < R; ++r) {
-        uint32_t cw[CPT / 4];
-        if constexpr (CPT == 16) {
-          const uint4 w = *reinterpret_cast<const uint4*>(st + koff[r][0]);
-          cw[0] = w.x; cw[1] = w.y; cw[2] = w.z; cw[3] = w.w;
-        } else {
-          const uint2 w = *reinterpret_cast<const uint2*>(st + koff[r][0]);
-          cw[0] = w.x; cw[1] = w.y;
-        }
-        float2 acc[HB];
-#pragma unroll
-        for (int h = 0; h < HB; ++h) acc[h] = make_float2(0.f, 0.f);
-#pragma unroll
-        for (int i = 0; i < CPT / 4; ++i) {
-          float2 k01, k23;
-          dequant4_s8(cw[i], sk[2 * i], sk[2 * i + 1], k01, k23);
-#pragma unroll
-          for (int h = 0; h < HB; ++h) {
-            acc[h] = __ffma2_rn(qreg[h][2 * i + 0], k01, acc[h]);
-            acc[h] = __ffma2_rn(qreg[h][2 * i + 1], k23, acc[h]);
-          }
-        }
-#pragma unroll
-        for (int h = 0; h < HB; ++h) d[(hb * HB + h) * R + r] = acc[h].x + acc[h].y;
-      }
-    } else {
+    {
 #pragma unroll
       for (int r = 0; r < R; ++r) {
         float2 acc[HB];
@@ -676,25 +959,13 @@ decode_attn_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
 
   // o += p v over this lane's tokens of tile st (tokens past `valid` read zeros)
   auto pv_tile = [&](const uint8_t* st, int i, int valid) {
-    float2 sv01, sv23;  // Q8: this lane's four channel scales of V
-    if constexpr (Q8) {
-      const float4 s4 = reinterpret_cast<const float4*>(st + L::oScale + D * 4)[quad];
-      sv01 = make_float2(s4.x, s4.y);
-      sv23 = make_float2(s4.z, s4.w);
-    }
 #pragma unroll
     for (int j = 0; j < PVN; ++j) {
       const int t = pv_t0 + j;
       const uint8_t* vp = t < valid ? st + voff[j] : zero16;
-      float2 v01, v23;
-      if constexpr (Q8) {
-        dequant4_s8(*reinterpret_cast<const uint32_t*>(vp), sv01, sv23, v01, v23);
-      } else {
-        const uint2 vw = *reinterpret_cast<const uint2*>(vp);
-        v01 = bf16x2_to_float2(vw.x);
-        v23 = bf16x2_to_float2(vw.y);
-      }
-      const float2* pt = ps + (i * kDecodeTileMax + t) * G;
+      const uint2 vw = *reinterpret_cast<const uint2*>(vp);
+      const float2 v01 = bf16x2_to_float2(vw.x), v23 = bf16x2_to_float2(vw.y);
+      const float2* pt = ps + (i * TR + t) * G;
       if constexpr (G >= 2) {
 #pragma unroll
         for (int g2 = 0; g2 < G / 2; ++g2) {
@@ -713,28 +984,26 @@ decode_attn_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
     }
   };
 
-  // CTAs holding tiles of the pair (CTAs whose range is empty write nothing)
-  auto seg_count = [&](int pair) {
-    const int c_first = cta_of(cst, off[pair], NC), c_last = cta_of(cst, off[pair + 1] - 1, NC);
-    int nseg = 0;
-    for (int cc = c_first; cc <= c_last; ++cc) nseg += cta_busy(cst, cc) ? 1 : 0;
-    return nseg;
-  };
-
   // End of a pair segment (every consumer warp arrives here at the same tile):
-  // merge the warps, then finalise, or publish a partial and maybe merge the
-  // pair's partials across CTAs.
+  // merge the warps, then finalise the pair, or publish this CTA's partial, or
+  // (the pair's merging CTA) fold in the other CTAs' partials and finalise.
   auto flush = [&](int pair) {
-    if constexpr (kMma) {
+    if constexpr (kMma || kQmma) {
       float lw = l_run;  // row sum of head hr over the warp's tokens: the row's 4 lanes
       lw += __shfl_xor_sync(kFull, lw, 1);
       lw += __shfl_xor_sync(kFull, lw, 2);
       if (real_row) {
         if (qq == 0) mlw[warp * G + hr] = make_float2(m_run, lw);
+        float* orow = ow + (warp * G + hr) * D;
 #pragma unroll
-        for (int n = 0; n < NTl; ++n)
-          *reinterpret_cast<float2*>(ow + (warp * G + hr) * D + 8 * n + 2 * qq) =
-              make_float2(om[n][0], om[n][1]);
+        for (int n = 0; n < NTl; ++n) {
+          if constexpr (kQmma) {  // n-tile n = pair n of the lanes' runs
+            orow[CPL * qq + pair_channel(QBB, n, 0)] = om[n][0];
+            orow[CPL * qq + pair_channel(QBB, n, 1)] = om[n][1];
+          } else {
+            *reinterpret_cast<float2*>(orow + 8 * n + 2 * qq) = make_float2(om[n][0], om[n][1]);
+          }
+        }
       }
     } else {
     float lw = l_run;  // row sum of this lane's head over the warp's tokens
@@ -776,11 +1045,14 @@ decode_attn_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
     const int b = pair / p.num_kv_heads, h = pair - b * p.num_kv_heads;
     // only the first and the last pair of a CTA's range can reach into other CTAs
     const bool whole = off[pair] >= u0 && off[pair + 1] <= u1;
-    const size_t slot = (size_t)cta + pair;
+    const bool merger = !whole && pair == merge_pair;
+    const uint32_t tag = part_tag((merger ? e_merge : e_first) + 1u, pair);
+    constexpr int kSlot = G * D + 2 * G;  // words per partial
+    // this CTA's own (o, l, M) of each of the thread's outputs
+    float o_[NOUT], l_[NOUT], M_[NOUT];
 #pragma unroll
     for (int i = 0; i < NOUT; ++i) {
-      const int j = tid + i * kConsumerThreads;
-      if (j >= G * D || !live) continue;
+      const int j = min(tid + i * kConsumerThreads, G * D - 1);
       const int g = j / D, c = j - g * D;
       float o = 0.f, l = 0.f;
 #pragma unroll
@@ -789,138 +1061,164 @@ decode_attn_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
         o += wt * ow[(w * G + g) * D + c];
         l += wt * mlw[w * G + g].y;
       }
-      const float M = msc[W * G + g];
-      const size_t qh = (size_t)b * p.num_q_heads + (size_t)h * G + g;
-      if (whole) {
-        const bool empty_row = !(l > 0.f);
-        store_out(p, qh * D + c, empty_row ? 0.f : o / l);
-        if (c == 0 && p.lse)
-          p.lse[qh] = empty_row ? -INFINITY : (M + __log2f(l)) * 0.69314718055994530942f;
-      } else {
-        p.part_o[(slot * G + g) * D + c] = o;
-        if (c == 0) *reinterpret_cast<float2*>(p.part_ml + (slot * G + g) * 2) = make_float2(M, l);
-      }
+      o_[i] = o;
+      l_[i] = l;
+      M_[i] = msc[W * G + g];
     }
-    named_sync(kBarConsumers, kConsumerThreads);  // ow / mlw / msc free again, partial written
-    // A partial: one thread publishes it (the barrier above ordered every
-    // thread's stores before its fence) and counts the pair's finished
-    // segments; the CTA that completes the count merges the pair at its end.
-    // Only warp 0 waits for the fence (counting at the kernel's end instead
-    // measured slower: the merges then start later).
-    if (!whole && live && tid == 0) {
-      __threadfence();
-      if (atomicAdd(&p.counters[pair], 1u) == (unsigned)(seg_count(pair) - 1))
-        misc[20 + (off[pair] < u0 ? 0 : 1)] = pair;
-    }
-  };
-
-  // Merge every partial (o, m, l) of a pair with log-sum-exp weights; the
-  // counter goes back to zero for the next call.  The (m, l) of all segments
-  // are loaded at once into the (now free) merge buffer, the weights
-  // 2^(m_s - M) computed once per (segment, head), and each output sums its
-  // segments with independent loads -- a couple of L2 round trips, however
-  // many CTAs the pair spans.
-  auto merge_partials = [&](int pair) {
-    const int b = pair / p.num_kv_heads, h = pair - b * p.num_kv_heads;
-    const int c_first = cta_of(cst, off[pair], NC), c_last = cta_of(cst, off[pair + 1] - 1, NC);
-    const int nc = c_last - c_first + 1;
-    constexpr int kCap = L::kOw / 8;  // float2 slots of the merge buffer
-    float2* wml = reinterpret_cast<float2*>(ow);  // [segment][head]: (m, l)
-    constexpr int kPre = 12;  // o partials of the first segments, loaded with the (m, l)
-    if (nc * G <= kCap) {
-      // one round of loads: every (m, l) into shared memory and the first
-      // kPre segments' o of this thread's outputs into registers
-      float opre[NOUT][kPre];
-#pragma unroll
-      for (int i = 0; i < NOUT; ++i) {
-        const int j = min(tid + i * kConsumerThreads, G * D - 1);
-        const int g = j / D, c = j - g * D;
-#pragma unroll
-        for (int u = 0; u < kPre; ++u)
-          opre[i][u] = (u < nc && cta_busy(cst, c_first + u))
-                           ? __ldcg(p.part_o + (((size_t)(c_first + u) + pair) * G + g) * D + c)
-                           : 0.f;
-      }
-      for (int i = tid; i < nc * G; i += kConsumerThreads) {
-        const int cc = c_first + i / G, g = i - (i / G) * G;
-        wml[i] = cta_busy(cst, cc)
-                     ? __ldcg(reinterpret_cast<const float2*>(p.part_ml + (((size_t)cc + pair) * G + g) * 2))
-                     : make_float2(-INFINITY, 0.f);
-      }
-      named_sync(kBarConsumers, kConsumerThreads);
-      // each output: M over the segments, weights 2^(m_s - M), weighted sums
+    if (!whole && !merger) {  // a later segment of a split pair: publish the partial
+      unsigned long long* sl = p.parts + (size_t)cta * kSlot;
 #pragma unroll
       for (int i = 0; i < NOUT; ++i) {
         const int j = tid + i * kConsumerThreads;
-        if (j >= G * D) continue;
+        if (j >= G * D || !live) continue;
         const int g = j / D, c = j - g * D;
-        float M = -INFINITY;
-        for (int sgi = 0; sgi < nc; ++sgi) M = fmaxf(M, wml[sgi * G + g].x);
-        float o = 0.f, lsum = 0.f;
-#pragma unroll
-        for (int u = 0; u < kPre; ++u) {
-          if (u < nc) {
-            const float2 ml = wml[u * G + g];
-            const float wt = ml.x == -INFINITY ? 0.f : exp2f(ml.x - M);
-            o += wt * opre[i][u];
-            lsum += wt * ml.y;
-          }
+        st_word(sl + g * D + c, o_[i], tag);
+        if (c == 0) {
+          st_word(sl + G * D + g, M_[i], tag);
+          st_word(sl + G * D + G + g, l_[i], tag);
         }
-        constexpr int kBatch = 8;  // independent loads in flight per thread
-        for (int s0 = kPre; s0 < nc; s0 += kBatch) {
-          float os[kBatch];
-#pragma unroll
-          for (int u = 0; u < kBatch; ++u) {
-            const int sgi = s0 + u;
-            os[u] = (sgi < nc && cta_busy(cst, c_first + sgi))
-                        ? __ldcg(p.part_o + (((size_t)(c_first + sgi) + pair) * G + g) * D + c)
-                        : 0.f;
+      }
+    }
+    bool got = true;
+    if (merger && live) {
+      // Fold in the partials of CTAs cta+1 .. c_last (those with tiles), every
+      // word polled until its tag matches.  Up to kBatch1 segments, each output
+      // loads its o, m and l words of all of them in one round and folds them
+      // in with running log-sum-exp weights.  Beyond that, every (m, l) word is
+      // first staged in shared memory (the p buffer is idle here), one word per
+      // thread, then each output loads its o words kBatch segments at a time
+      // with weights 2^(m_s - M) of the common maximum.
+      const int c_last = cta_of(cst, off[pair + 1] - 1, NC);
+      const int nseg = c_last - cta;
+      const long long t_poll = clock64();
+      float2* mls = reinterpret_cast<float2*>(ps);  // [segment][head]: (m, l)
+      // up to kBatch1 segments: one round of loads per output (its o, m, l words
+      // of every segment at once); more: the (m, l) words staged first
+      constexpr int kBatch1 = 8;
+      const bool staged = nseg > kBatch1 && nseg * G <= L::kPs / 8;
+      if (staged) {
+        for (int i = tid; i < nseg * G; i += kConsumerThreads) {
+          const int sg = i / G, g = i - sg * G, cc = cta + 1 + sg;
+          float2 ml = make_float2(-INFINITY, 0.f);
+          if (cta_busy(cst, cc)) {
+            const unsigned long long* sl = p.parts + (size_t)cc * kSlot;
+            unsigned long long wm = ld_word(sl + G * D + g), wl = ld_word(sl + G * D + G + g);
+            while (!(word_ok(wm, tag) && word_ok(wl, tag))) {
+              if ((uint64_t)(clock64() - t_poll) > lim) {
+                got = false;
+                break;
+              }
+              if (!word_ok(wm, tag)) wm = ld_word(sl + G * D + g);
+              if (!word_ok(wl, tag)) wl = ld_word(sl + G * D + G + g);
+            }
+            ml = make_float2(word_val(wm), word_val(wl));
           }
+          mls[i] = ml;
+        }
+        got = named_sync_and(kBarConsumers, kConsumerThreads, got);
+      }
+      constexpr int kBatch = G >= 8 ? 8 : 16;  // segments whose o words are loaded at once
 #pragma unroll
-          for (int u = 0; u < kBatch; ++u) {
-            if (s0 + u < nc) {
-              const float2 ml = wml[(s0 + u) * G + g];
-              const float wt = ml.x == -INFINITY ? 0.f : exp2f(ml.x - M);
-              o += wt * os[u];
-              lsum += wt * ml.y;
+      for (int i = 0; i < NOUT; ++i) {
+        const int j = tid + i * kConsumerThreads;
+        if (j >= G * D || !got) continue;
+        const int g = j / D, c = j - g * D;
+        float M = M_[i], o = o_[i], l = l_[i];
+        if (staged) {  // the common maximum first, then one weighted sum
+          float Mt = M;
+          for (int sg = 0; sg < nseg; ++sg) Mt = fmaxf(Mt, mls[sg * G + g].x);
+          if (Mt != -INFINITY) {
+            const float a = exp2f(M - Mt);
+            o *= a;
+            l *= a;
+          }
+          for (int s0 = 0; s0 < nseg && got; s0 += kBatch) {
+            unsigned long long wo[kBatch];
+#pragma unroll
+            for (int u = 0; u < kBatch; ++u) {
+              const int cc = cta + 1 + s0 + u;
+              wo[u] = 0ull;
+              if (s0 + u < nseg && cta_busy(cst, cc))
+                wo[u] = ld_word(p.parts + (size_t)cc * kSlot + g * D + c);
+            }
+#pragma unroll
+            for (int u = 0; u < kBatch; ++u) {
+              const int cc = cta + 1 + s0 + u;
+              if (s0 + u >= nseg || !cta_busy(cst, cc) || !got) continue;
+              while (!word_ok(wo[u], tag)) {
+                if ((uint64_t)(clock64() - t_poll) > lim) {
+                  got = false;
+                  break;
+                }
+                wo[u] = ld_word(p.parts + (size_t)cc * kSlot + g * D + c);
+              }
+              const float2 ml = mls[(s0 + u) * G + g];
+              if (!got || ml.x == -INFINITY) continue;
+              const float wt = exp2f(ml.x - Mt);
+              o += word_val(wo[u]) * wt;
+              l += ml.y * wt;
+            }
+          }
+          M = Mt;
+        } else {  // few segments (or too many to stage): o, m, l words per output
+          for (int c0 = cta + 1; c0 <= c_last && got; c0 += kBatch1) {
+            unsigned long long wo[kBatch1], wm[kBatch1], wl[kBatch1];
+#pragma unroll
+            for (int u = 0; u < kBatch1; ++u) {
+              const int cc = c0 + u;
+              wo[u] = wm[u] = wl[u] = 0ull;
+              if (cc <= c_last && cta_busy(cst, cc)) {
+                const unsigned long long* sl = p.parts + (size_t)cc * kSlot;
+                wo[u] = ld_word(sl + g * D + c);
+                wm[u] = ld_word(sl + G * D + g);
+                wl[u] = ld_word(sl + G * D + G + g);
+              }
+            }
+#pragma unroll
+            for (int u = 0; u < kBatch1; ++u) {
+              const int cc = c0 + u;
+              if (cc > c_last || !cta_busy(cst, cc) || !got) continue;
+              const unsigned long long* sl = p.parts + (size_t)cc * kSlot;
+              while (!(word_ok(wo[u], tag) && word_ok(wm[u], tag) && word_ok(wl[u], tag))) {
+                if ((uint64_t)(clock64() - t_poll) > lim) {
+                  got = false;
+                  break;
+                }
+                if (!word_ok(wo[u], tag)) wo[u] = ld_word(sl + g * D + c);
+                if (!word_ok(wm[u], tag)) wm[u] = ld_word(sl + G * D + g);
+                if (!word_ok(wl[u], tag)) wl[u] = ld_word(sl + G * D + G + g);
+              }
+              if (!got) continue;
+              const float ms = word_val(wm[u]);
+              const float Mn = fmaxf(M, ms);
+              if (Mn == -INFINITY) continue;  // both parts empty so far
+              const float a = exp2f(M - Mn), bw = exp2f(ms - Mn);
+              o = o * a + word_val(wo[u]) * bw;
+              l = l * a + word_val(wl[u]) * bw;
+              M = Mn;
             }
           }
         }
-        const size_t qh = (size_t)b * p.num_q_heads + (size_t)h * G + g;
-        const bool empty_row = !(lsum > 0.f);
-        store_out(p, qh * D + c, empty_row ? 0.f : o / lsum);
-        if (c == 0 && p.lse)
-          p.lse[qh] = empty_row ? -INFINITY : (M + __log2f(lsum)) * 0.69314718055994530942f;
+        o_[i] = o;
+        l_[i] = l;
+        M_[i] = M;
       }
-      named_sync(kBarConsumers, kConsumerThreads);  // the buffer is free for the next merge
-    } else {  // more segments than the buffer holds: one segment at a time
+      if (!got && tid == 0) raise_status(p.status, LSERVE_ERR_TIMEOUT);
+    }
+    if ((whole || merger) && live && got) {
 #pragma unroll
       for (int i = 0; i < NOUT; ++i) {
         const int j = tid + i * kConsumerThreads;
         if (j >= G * D) continue;
         const int g = j / D, c = j - g * D;
-        float M = -INFINITY, o = 0.f, lsum = 0.f;
-        for (int cc = c_first; cc <= c_last; ++cc) {
-          const bool busy = cta_busy(cst, cc);
-          const size_t sl = (size_t)cc + pair;
-          const float2 ml = busy ? __ldcg(reinterpret_cast<const float2*>(p.part_ml + (sl * G + g) * 2))
-                                 : make_float2(-INFINITY, 0.f);
-          const float os = busy ? __ldcg(p.part_o + (sl * G + g) * D + c) : 0.f;
-          const float Mn = fmaxf(M, ml.x);
-          if (Mn == -INFINITY) continue;
-          const float sc = exp2f(M - Mn), wt = exp2f(ml.x - Mn);
-          o = o * sc + wt * os;
-          lsum = lsum * sc + wt * ml.y;
-          M = Mn;
-        }
         const size_t qh = (size_t)b * p.num_q_heads + (size_t)h * G + g;
-        const bool empty_row = !(lsum > 0.f);
-        store_out(p, qh * D + c, empty_row ? 0.f : o / lsum);
+        const bool empty_row = !(l_[i] > 0.f);
+        store_out(p, qh * D + c, empty_row ? 0.f : o_[i] / l_[i]);
         if (c == 0 && p.lse)
-          p.lse[qh] = empty_row ? -INFINITY : (M + __log2f(lsum)) * 0.69314718055994530942f;
+          p.lse[qh] = empty_row ? -INFINITY : (M_[i] + __log2f(l_[i])) * 0.69314718055994530942f;
       }
     }
-    if (tid == 0) p.counters[pair] = 0u;
+    named_sync(kBarConsumers, kConsumerThreads);  // ow / mlw / msc / ps free again
   };
 
   // Each iteration takes one tile, or two consecutive tiles of the same pair:
@@ -934,7 +1232,7 @@ decode_attn_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
       pend = off[cur + 1] - u0;
       m_run = -INFINITY;
       l_run = 0.f;
-      if constexpr (kMma) {
+      if constexpr (kMma || kQmma) {
 #pragma unroll
         for (int n = 0; n < NTl; ++n) om[n][0] = om[n][1] = 0.f;
       } else {
@@ -948,24 +1246,57 @@ decode_attn_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
     const bool ok0 = __all_sync(kFull, stage_wait(&full[s0], (k / S) & 1, lim, p.status, abort_flag));
     const bool ok1 =
         nt == 2 && __all_sync(kFull, stage_wait(&full[s1], ((k + 1) / S) & 1, lim, p.status, abort_flag));
-    const int valid0 = ok0 ? info[s0] : 0;
-    const int valid1 = ok1 ? info[s1] : 0;
+    const int inf0 = ok0 ? info[s0] : 0, inf1 = ok1 ? info[s1] : 0;
+    const int valid0 = inf0 & 0xFF, valid1 = inf1 & 0xFF;        // tokens [lo, valid) attended
+    const int lo0 = (inf0 >> 8) & 0xFF, lo1 = (inf1 >> 8) & 0xFF;
     const uint8_t* st0 = smem + s0 * L::kStage;
     const uint8_t* st1 = smem + s1 * L::kStage;
-    if constexpr (kMma) {
-      if (need_q) load_q_mma(st0);
+    if constexpr (!Q8) {
+      if (p.k_new) {
+        // the appended token's K / V row of a tile comes from k_new / v_new (the
+        // producer copied them next to the tile): the warp that owns the row
+        // overwrites it in the stage (no other warp reads it)
+        constexpr int TPO = (kMma ? 8 : TPW);  // tokens of a tile per owning warp
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+          const int fx = ((i == 0 ? inf0 : inf1) >> 16) - 1;
+          if (fx >= 0 && fx / TPO == warp && (i == 0 || nt == 2)) {
+            uint8_t* st = smem + (i == 0 ? s0 : s1) * L::kStage;
+            constexpr int C16 = D / 8;
+            if (lane < 2 * C16) {
+              const int c = lane % C16;
+              const uint4 v = reinterpret_cast<const uint4*>(st + L::oNew)[lane];  // K chunks, then V
+              *reinterpret_cast<uint4*>(st + (lane < C16 ? 0 : L::kTileK) +
+                                        sw128_offset(NBOX * fx + c / 8, c % 8)) = v;
+            }
+            __syncwarp();
+          }
+        }
+      }
+    }
+    if constexpr (kMma || kQmma) {
+      if (need_q) {
+        if constexpr (kQmma) load_q_qmma(st0);
+        else load_q_mma(st0);
+      }
       need_q = false;
       if (has_tok) {
         float sa[2][4], sb[2][4];
-        qk_mma(st0, sa[0], sb[0]);
-        if (nt == 2) qk_mma(st1, sa[1], sb[1]);
+        if constexpr (kQmma) {
+          qk_qmma(st0, sa[0], sb[0]);
+          if (nt == 2) qk_qmma(st1, sa[1], sb[1]);
+        } else {
+          qk_mma(st0, sa[0], sb[0]);
+          if (nt == 2) qk_mma(st1, sa[1], sb[1]);
+        }
         float x[2][2];
 #pragma unroll
         for (int i = 0; i < 2; ++i)
 #pragma unroll
           for (int j = 0; j < 2; ++j) {
             const int tok = mt0 + 2 * qq + j;
-            const bool ok = i == 0 ? tok < valid0 : (nt == 2 && tok < valid1);
+            const bool ok = i == 0 ? (tok >= lo0 && tok < valid0)
+                                   : (nt == 2 && tok >= lo1 && tok < valid1);
             x[i][j] = ok ? (sa[i][j] + sb[i][j]) * p.scale_log2 : -INFINITY;
           }
         float mx = fmaxf(fmaxf(x[0][0], x[0][1]), fmaxf(x[1][0], x[1][1]));
@@ -992,7 +1323,8 @@ decode_attn_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
             om[n][1] *= alpha;
           }
         }
-        pv_mma(s0, s1, nt, pr, valid0, valid1);
+        if constexpr (kQmma) pv_qmma(st0, st1, nt, pr);
+        else pv_mma(s0, s1, nt, pr, valid0, valid1);
       }
     } else {
     if constexpr (NHB == 1) {
@@ -1014,8 +1346,8 @@ decode_attn_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
 #pragma unroll
     for (int j = 0; j < C; ++j) {
       const int tok = wt0 + 4 * (my_r0 + j) + tok_l;
-      x[0][j] = tok < valid0 ? x[0][j] * p.scale_log2 : -INFINITY;
-      x[1][j] = tok < valid1 ? x[1][j] * p.scale_log2 : -INFINITY;
+      x[0][j] = (tok >= lo0 && tok < valid0) ? x[0][j] * p.scale_log2 : -INFINITY;
+      x[1][j] = (tok >= lo1 && tok < valid1) ? x[1][j] * p.scale_log2 : -INFINITY;
     }
 
     // ---- online softmax of this lane's head: warp max over its rows and tokens
@@ -1041,7 +1373,7 @@ decode_attn_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
         const float pr = fast_ex2(x[i][j] - m_use);  // x = -inf gives 0
         lsum += pr;
         const int tok = wt0 + 4 * (my_r0 + j) + tok_l;
-        if (i == 0 || nt == 2) ps[(i * kDecodeTileMax + tok) * G + my_g] = make_float2(pr, pr);
+        if (i == 0 || nt == 2) ps[(i * TR + tok) * G + my_g] = make_float2(pr, pr);
       }
     l_run = lsum;
     __syncwarp();
@@ -1073,49 +1405,63 @@ decode_attn_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
     k += nt;
   }
   if (cur >= 0) flush(cur);
-  // the pairs this CTA completed: merge their partials
-  named_sync(kBarConsumers, kConsumerThreads);
-  if (misc[20] >= 0) merge_partials(misc[20]);
-  if (misc[21] >= 0) merge_partials(misc[21]);
+  // The merged pair's epoch advances whatever happened above (a timeout
+  // included), so no word of this call matches a later call's tags.
+  if (tid == 0 && merge_pair >= 0) {
+    asm volatile("st.relaxed.gpu.global.b32 [%0], %1;" ::"l"(p.epochs + merge_pair), "r"(e_merge + 1u)
+                 : "memory");
+  }
 }
 
 size_t decode_workspace_bytes(int pairs, int grid, int G, int D) {
-  const size_t cnt = ((size_t)pairs * 4 + 255) / 256 * 256;
-  const size_t slots = (size_t)grid + pairs;
-  const size_t o = (slots * G * D * 4 + 255) / 256 * 256;
-  return cnt + o + slots * G * 2 * 4;
+  const size_t ep = ((size_t)pairs * 4 + 255) / 256 * 256;  // epochs
+  return ep + (size_t)grid * (G * D + 2 * G) * 8;             // one tagged partial per CTA
 }
 
 int decode_grid(int sm_count) { return sm_count; }
 
+int decode_consumer_warps() { return 8; }
+
+int decode_tile_rows(int physical_page) {
+  return physical_page < kDecodeTileMax ? physical_page : kDecodeTileMax;
+}
+
 namespace {
 // launched as a programmatic dependent of the previous work on the stream
-template <int D, int G, bool Q8>
-cudaError_t launch_decode_t(const DecodeParams& p, const CUtensorMap& kmap, const CUtensorMap& vmap,
+template <int D, int G, int QB, int TR, int W>
+cudaError_t launch_decode_w(const DecodeParams& p, const CUtensorMap& kmap, const CUtensorMap& vmap,
                             int grid, cudaStream_t stream) {
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(kThreads);
+  cfg.blockDim = dim3((W + 1) * 32);
   cfg.stream = stream;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  cfg.dynamicSmemBytes = DecLayout<D, G, Q8>::kBytes + 1024;
-  auto kern = p.tile_rows == 64 ? decode_attn_kernel<D, G, 64, Q8> : decode_attn_kernel<D, G, 32, Q8>;
+  cfg.dynamicSmemBytes = DecLayout<D, G, QB, TR, W>::kBytes + 1024;
+  auto kern = decode_attn_kernel<D, G, TR, QB, W>;
   const cudaError_t e = set_smem_once((const void*)kern, (int)cfg.dynamicSmemBytes);
   if (e != cudaSuccess) return e;
   return cudaLaunchKernelEx(&cfg, kern, p, kmap, vmap);
 }
 
-template <bool Q8>
+template <int D, int G, int QB>
+cudaError_t launch_decode_t(const DecodeParams& p, const CUtensorMap& kmap, const CUtensorMap& vmap,
+                            int grid, cudaStream_t stream) {
+  if (p.consumer_warps != 8) return cudaErrorInvalidValue;
+  if (p.tile_rows == 64) return launch_decode_w<D, G, QB, 64, 8>(p, kmap, vmap, grid, stream);
+  return launch_decode_w<D, G, QB, 32, 8>(p, kmap, vmap, grid, stream);
+}
+
+template <int QB>
 cudaError_t launch_decode_any(const DecodeParams& p, const CUtensorMap& kmap, const CUtensorMap& vmap,
                               int D, int G, int grid, cudaStream_t stream) {
   if (grid < 1 || grid > kMaxGrid) return cudaErrorInvalidValue;
   if (p.tile_rows != 64 && p.tile_rows != 32) return cudaErrorInvalidValue;
 #define LSERVE_DECODE_CASE(DD, GG) \
-  if (D == DD && G == GG) return launch_decode_t<DD, GG, Q8>(p, kmap, vmap, grid, stream);
+  if (D == DD && G == GG) return launch_decode_t<DD, GG, QB>(p, kmap, vmap, grid, stream);
   LSERVE_DECODE_CASE(64, 1)
   LSERVE_DECODE_CASE(64, 2)
   LSERVE_DECODE_CASE(64, 4)
@@ -1131,13 +1477,16 @@ cudaError_t launch_decode_any(const DecodeParams& p, const CUtensorMap& kmap, co
 
 cudaError_t launch_decode(const DecodeParams& p, const CUtensorMap& kmap, const CUtensorMap& vmap,
                           int D, int G, int grid, cudaStream_t stream) {
-  return launch_decode_any<false>(p, kmap, vmap, D, G, grid, stream);
+  return launch_decode_any<0>(p, kmap, vmap, D, G, grid, stream);
 }
 
-cudaError_t launch_decode_kv8(const DecodeParams& p, int D, int G, int grid, cudaStream_t stream) {
-  CUtensorMap unused;  // the int8 tiles are plain bulk copies: no tensor map
+cudaError_t launch_decode_quant(const DecodeParams& p, int D, int G, int bits, int grid,
+                                cudaStream_t stream) {
+  CUtensorMap unused;  // the quantized tiles are plain bulk copies: no tensor map
   memset(&unused, 0, sizeof(unused));
-  return launch_decode_any<true>(p, unused, unused, D, G, grid, stream);
+  if (bits == 8) return launch_decode_any<8>(p, unused, unused, D, G, grid, stream);
+  if (bits == 4) return launch_decode_any<4>(p, unused, unused, D, G, grid, stream);
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace lserve

@@ -61,23 +61,40 @@ struct DecodeParams {
   __nv_bfloat16* out;     // bf16 [B][H_q][D], or null when out_f32 is set
   float* out_f32;         // float [B][H_q][D] instead (LSERVE_DECODE_OUT_F32)
   float* lse;
-  uint32_t* counters;     // workspace [P]: segments finished per pair; zero between calls
-  float* part_o;          // workspace [(grid + P)][G][D]: unnormalised partial outputs
-  float* part_ml;         // workspace [(grid + P)][G][2]: (running max, row sum) per partial
+  // Split pairs (workspace).  A CTA writes at most one partial: the part of
+  // its first pair that began in an earlier CTA.  Each word is 8 bytes, a
+  // float value in the low half and a tag in the high half (one single-copy
+  // atomic store), so the merging CTA can poll the words themselves.
+  uint32_t* epochs;              // [P]: epoch of the pair's last split merge
+  unsigned long long* parts;     // [grid][G*D + 2*G]: o[G][D], m[G], l[G] words
   unsigned int* status;
   int batch, num_q_heads, num_kv_heads, physical_page, max_pages, num_pool_pages;
   int top_k, sink, local;
-  int tile_rows;          // tokens per tile: min(N_P, 64)
+  int tile_rows;          // tokens per tile (decode_tile_rows)
   int tiles_per_page;
+  int consumer_warps;     // 8: one CTA per SM; 4: two co-resident CTAs per SM
   float scale_log2;       // softmax_scale * log2(e)
   uint64_t wait_limit;
   int overlap_prologue;   // plan + first lookups may run before the preceding kernel ends
-  // int8 cache (lserve_sparse_decode_attn_kv8): codes [pool rows][D] and
-  // float scales [num_pool_pages][H_kv][D]; null for the bf16 cache
+  // quantized cache (lserve_sparse_decode_attn_kv8 / _kv4): codes [pool rows]
+  // [D] bytes (8-bit) or [D/2] bytes (4-bit, two per byte) and float scales
+  // [num_pool_pages][H_kv][D]; null for the bf16 cache
   const int8_t* k8;
   const int8_t* v8;
   const float* k_scale;
   const float* v_scale;
+  // lserve_decode_step: the new token of sequence b sits at position
+  // ctx_lens[b] - 1; its K / V rows (k_new / v_new, bf16 [B][H_kv][D]) are
+  // written to the pools and the retrieval heads' page statistics in this
+  // launch and attended from k_new / v_new (null: no append)
+  const __nv_bfloat16* k_new;
+  const __nv_bfloat16* v_new;
+  __nv_bfloat16* k_pool_w;
+  __nv_bfloat16* v_pool_w;
+  __nv_bfloat16* stats_w;
+  int logical_page;
+  // retrieval heads also attend positions [recent_from[b], ctx_lens[b]) (null: off)
+  const int32_t* recent_from;
 };
 
 // lserve_decode_append: one warp per (sequence, KV head)
@@ -124,7 +141,7 @@ struct QuantParams {
   unsigned int* status;
   int batch, num_kv_heads, physical_page, max_pages, num_pool_pages;
 };
-cudaError_t launch_quantize_kv8(const QuantParams& p, int D, cudaStream_t stream);
+cudaError_t launch_quantize_kv(const QuantParams& p, int D, int bits, cudaStream_t stream);
 
 // Sequence-sharded decode (seq_shard.cu): shard `rank` of `num_shards` holds
 // pages [floor(M*rank/N), floor(M*(rank+1)/N)) of each sequence.
@@ -162,10 +179,14 @@ cudaError_t launch_page_stats(const StatsParams& p, int D, int max_logical_pages
 cudaError_t launch_page_select(const SelectParams& p, int D, cudaStream_t stream);
 cudaError_t launch_decode(const DecodeParams& p, const CUtensorMap& kmap, const CUtensorMap& vmap,
                           int D, int G, int grid, cudaStream_t stream);
-// the int8-cache variant (p.k8 / p.v8 / p.k_scale / p.v_scale set; no tensor maps)
-cudaError_t launch_decode_kv8(const DecodeParams& p, int D, int G, int grid, cudaStream_t stream);
+// the quantized-cache variants, bits = 8 or 4 (p.k8 / p.v8 / p.k_scale / p.v_scale
+// set; no tensor maps)
+cudaError_t launch_decode_quant(const DecodeParams& p, int D, int G, int bits, int grid,
+                                cudaStream_t stream);
 size_t decode_workspace_bytes(int pairs, int grid, int G, int D);
 int decode_grid(int sm_count);
+int decode_consumer_warps();
+int decode_tile_rows(int physical_page);
 
 cudaError_t launch_wait_timeout_probe(uint64_t cycles, unsigned int* status, cudaStream_t stream);
 

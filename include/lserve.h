@@ -200,9 +200,12 @@ int lserve_page_select(const lserve_paged_desc* desc, const void* q, const void*
  *   lse  float [B][H_q] natural-log sum of exp(scale * q.k), or NULL.
  * A head with no token to attend (n_b = 0) gets out = 0, lse = -inf.
  * workspace: lserve_workspace_size(LSERVE_OP_DECODE, desc, top_k) bytes,
- * 256-byte aligned and ZERO-FILLED before its first use: besides the split
- * partials it holds per-pair completion counters, which every successful call
- * leaves at zero again (after an error, zero it again).  Calls that may run
+ * 256-byte aligned and ZERO-FILLED once before its first use.  It holds the
+ * partial results of pairs split over several thread blocks, each word tagged
+ * with the pair and a per-pair merge epoch kept in the workspace too; every
+ * call advances the epochs it uses, also when it ends in an error (a
+ * timeout), so leftovers of any earlier call are never mistaken for this
+ * call's: the workspace never needs re-zeroing.  Calls that may run
  * concurrently need separate workspaces.
  * Limits: B * H_kv <= 2048; N_P = 32 or a multiple of 64.
  */
@@ -249,6 +252,40 @@ int lserve_sparse_decode_attn_ex(const lserve_paged_desc* desc, const void* q, c
                                  size_t workspace_bytes, void* stream);
 
 /*
+ * lserve_decode_step -- one decode step in one launch: append each sequence's
+ * new token to the paged cache and attend.
+ * [技術的詳細 › 動的スパーシティ (the k_min / k_max statistics a new token
+ *  updates) and › Reusable Page Selection (a selection is reused for k steps;
+ *  the pages do not say whether tokens appended meanwhile are seen -- this
+ *  call offers both readings); the attention as lserve_sparse_decode_attn.]
+ *
+ * ctx_lens[b] counts the new token: it sits at position t = ctx_lens[b] - 1.
+ *   k_new, v_new  bf16 [B][H_kv][D] (16-byte aligned), or both NULL (no append):
+ *                 written to row t of the pools, and for retrieval heads into
+ *                 the k_min / k_max of logical page t / N_L (exactly as
+ *                 lserve_decode_append), in the same launch; the attention
+ *                 reads the new token from k_new / v_new, never from the pool.
+ *   recent_from   int32 [B] or NULL.  NULL: a retrieval head attends the valid
+ *                 tokens of its selected pages (the new token only if its page
+ *                 is selected).  Given: it also attends every position in
+ *                 [recent_from[b], ctx_lens[b]) -- e.g. the length when its
+ *                 selection was made -- each token once.
+ * Streaming heads attend the sink + local pages of ctx_lens[b] tokens (the new
+ * token always).  Everything else -- sel, outputs, workspace, flags -- as
+ * lserve_sparse_decode_attn_ex; LSERVE_DECODE_OVERLAP_PROLOGUE also requires
+ * that the kernel before writes no recent_from.  The block table must already
+ * hold the page of position t; a sequence with ctx_lens[b] = 0 appends nothing.
+ * The appended page must belong to one sequence (see lserve_decode_append).
+ */
+int lserve_decode_step(const lserve_paged_desc* desc, const void* q, const void* k_new,
+                       const void* v_new, void* k_pool, void* v_pool, void* stats_pool,
+                       const int32_t* block_table, const int32_t* ctx_lens,
+                       const uint8_t* head_kind, const int32_t* sel, const int32_t* sel_count,
+                       int32_t top_k, int32_t sink_tokens, int32_t local_tokens,
+                       const int32_t* recent_from, float softmax_scale, void* out, float* lse,
+                       uint32_t flags, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * lserve_quantize_pages_kv8 -- an int8 copy of the paged K / V cache.
  * [LServe abstract page: the unified sparse attention is combined with a
  *  quantized KV cache (QServe's KV4 in the end-to-end results); the pages give
@@ -277,20 +314,61 @@ int lserve_quantize_pages_kv8(const lserve_paged_desc* desc, const void* k_pool,
                               void* v_pool8, float* k_scale, float* v_scale, void* stream);
 
 /*
+ * lserve_quantize_pages_kv4 -- a 4-bit copy of the paged K / V cache.
+ * [LServe abstract page: the sparse attention combined with QServe's KV4 in
+ *  the end-to-end results; the pages give no scheme.  This library's scheme:
+ *  the int8 scheme above with codes -7..7.]
+ *
+ * As lserve_quantize_pages_kv8 with 7 in place of 127:
+ *   code    = rint(x * (7 / amax_c)) clamped to [-7, 7]  (float32, ties to even)
+ *   scale_c = amax_c / 7
+ *   k_pool4 / v_pool4  uint8 [num_pool_pages][H_kv][N_P][D/2]: two codes per
+ *                      byte as 4-bit two's complement, channel 2i in the low
+ *                      nibble and 2i+1 in the high nibble; rows past `valid`
+ *                      are 0;
+ *   k_scale / v_scale  float [num_pool_pages][H_kv][D].
+ * A quarter of the bf16 cache's bytes (plus the scales).  No workspace; all
+ * pointers 16-byte aligned.
+ */
+int lserve_quantize_pages_kv4(const lserve_paged_desc* desc, const void* k_pool, const void* v_pool,
+                              const int32_t* block_table, const int32_t* ctx_lens, void* k_pool4,
+                              void* v_pool4, float* k_scale, float* v_scale, void* stream);
+
+/*
  * lserve_sparse_decode_attn_kv8 -- lserve_sparse_decode_attn_ex over the int8
  * cache that lserve_quantize_pages_kv8 writes.
  * [Same pages as lserve_sparse_decode_attn; the quantized cache as above.]
  *
  * Every attended token contributes k = code_k * k_scale and v = code_v *
- * v_scale of its page (fp32 arithmetic); pages, softmax, outputs, lse,
- * flags and workspace are exactly those of lserve_sparse_decode_attn_ex with
- * the same arguments.  k_pool8 / v_pool8 int8 [num_pool_pages][H_kv][N_P][D],
+ * v_scale of its page; pages, softmax, outputs, lse, flags and workspace are
+ * exactly those of lserve_sparse_decode_attn_ex with the same arguments.
+ * Arithmetic: tensor cores in fp16 -- the codes are exact in fp16, q * k_scale
+ * and code_v * v_scale are rounded to fp16 (11-bit significand; q * k_scale
+ * must lie within fp16's range), products accumulate in fp32, the softmax is
+ * fp32.  k_pool8 / v_pool8 int8 [num_pool_pages][H_kv][N_P][D],
  * k_scale / v_scale float [num_pool_pages][H_kv][D], all 16-byte aligned.
  * Each attended page moves N_P*D bytes of K codes and of V codes plus 2*D*4
  * bytes of scales: about half the bf16 call's traffic.
  */
 int lserve_sparse_decode_attn_kv8(const lserve_paged_desc* desc, const void* q, const void* k_pool8,
                                   const void* v_pool8, const float* k_scale, const float* v_scale,
+                                  const int32_t* block_table, const int32_t* ctx_lens,
+                                  const uint8_t* head_kind, const int32_t* sel,
+                                  const int32_t* sel_count, int32_t top_k, int32_t sink_tokens,
+                                  int32_t local_tokens, float softmax_scale, void* out, float* lse,
+                                  uint32_t flags, void* workspace, size_t workspace_bytes,
+                                  void* stream);
+
+/*
+ * lserve_sparse_decode_attn_kv4 -- lserve_sparse_decode_attn_kv8 over the
+ * 4-bit cache that lserve_quantize_pages_kv4 writes (k_pool4 / v_pool4 uint8
+ * [num_pool_pages][H_kv][N_P][D/2], two codes per byte; scales as kv8).  Each
+ * attended page moves N_P*D/2 bytes of K codes and of V codes plus 2*D*4
+ * bytes of scales: about a quarter of the bf16 call's traffic.
+ * [Same pages as lserve_sparse_decode_attn; the 4-bit cache as above.]
+ */
+int lserve_sparse_decode_attn_kv4(const lserve_paged_desc* desc, const void* q, const void* k_pool4,
+                                  const void* v_pool4, const float* k_scale, const float* v_scale,
                                   const int32_t* block_table, const int32_t* ctx_lens,
                                   const uint8_t* head_kind, const int32_t* sel,
                                   const int32_t* sel_count, int32_t top_k, int32_t sink_tokens,

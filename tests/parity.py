@@ -57,9 +57,11 @@ def run_decode_path(buf: DecodeBuffers, layer: int = 0, scale=None):
     )
 
 
-def run_decode_path_kv8(buf: DecodeBuffers, layer: int = 0, scale=None, overlap=False):
-    """stats -> select on the bf16 cache, then quantize the pools to int8 and
-    decode over the int8 cache; returns host copies (plus codes and scales)."""
+def run_decode_path_kv8(buf: DecodeBuffers, layer: int = 0, scale=None, overlap=False, bits=8):
+    """stats -> select on the bf16 cache, then quantize the pools to `bits`-bit
+    codes (8: int8 [pool][H_kv][N_P][D]; 4: uint8 [pool][H_kv][N_P][D/2], two
+    codes per byte) and decode over the quantized cache; returns host copies
+    (plus codes and scales)."""
     w = buf.w
     d = desc_of(w)
     scale = 1.0 / math.sqrt(w.D) if scale is None else scale
@@ -67,18 +69,19 @@ def run_decode_path_kv8(buf: DecodeBuffers, layer: int = 0, scale=None, overlap=
                       buf.stats[layer])
     lserve.page_select(d, buf.q, buf.stats[layer], buf.block_table, buf.ctx_lens, buf.head_kind,
                        w.top_k, buf.sel[layer], buf.sel_count[layer], phys_scores=buf.scores)
-    k8 = torch.full(w.pool_shape(), 99, dtype=torch.int8, device=buf.device)
-    v8 = torch.full(w.pool_shape(), -99, dtype=torch.int8, device=buf.device)
+    shape = w.pool_shape() if bits == 8 else w.pool_shape()[:-1] + (w.D // 2,)
+    k8 = torch.full(shape, 99, dtype=torch.int8, device=buf.device)
+    v8 = torch.full(shape, -99, dtype=torch.int8, device=buf.device)
     ks = torch.full((w.num_pool_pages, w.H_kv, w.D), float("nan"), dtype=torch.float32,
                     device=buf.device)
     vs = torch.full_like(ks, float("nan"))
     lserve.quantize_pages_kv8(d, buf.k_pools[layer], buf.v_pools[layer], buf.block_table,
-                              buf.ctx_lens, k8, v8, ks, vs)
+                              buf.ctx_lens, k8, v8, ks, vs, bits=bits)
     ws = lserve.alloc_workspace(lserve.workspace_size(lserve.OP_DECODE, d, w.top_k))
     lserve.sparse_decode_attn_kv8(d, buf.q, k8, v8, ks, vs, buf.block_table, buf.ctx_lens,
                                   buf.head_kind, buf.sel[layer], buf.sel_count[layer], w.top_k,
                                   w.sink, w.local, scale, buf.out, buf.lse, workspace=ws,
-                                  overlap_prologue=overlap)
+                                  overlap_prologue=overlap, bits=bits)
     torch.cuda.synchronize()
     st = lserve.read_device_status()
     assert st == lserve.OK, lserve.status_string(st)
@@ -90,23 +93,42 @@ def run_decode_path_kv8(buf: DecodeBuffers, layer: int = 0, scale=None, overlap=
         out=oracle.widen_bf16(bf16_bits(buf.out)),
         lse=buf.lse.cpu().numpy().astype(np.float64),
         scale=scale,
-        k8=k8, v8=v8, k_scale=ks, v_scale=vs,
+        k8=k8, v8=v8, k_scale=ks, v_scale=vs, bits=bits,
     )
+
+
+def unpack_codes4(packed: np.ndarray) -> np.ndarray:
+    """uint8 [..][D/2] -> int8 [..][D]: channel 2i is the low nibble of byte i,
+    2i+1 the high nibble, each a 4-bit two's complement code."""
+    u = packed.astype(np.uint8)
+    lo = (u & 0xF).astype(np.int8)
+    hi = (u >> 4).astype(np.int8)
+    lo = np.where(lo >= 8, lo - 16, lo).astype(np.int8)
+    hi = np.where(hi >= 8, hi - 16, hi).astype(np.int8)
+    out = np.empty(packed.shape[:-1] + (packed.shape[-1] * 2,), dtype=np.int8)
+    out[..., 0::2] = lo
+    out[..., 1::2] = hi
+    return out
 
 
 def check_quantized_pages(w, res, b, h):
     """Codes and scales of every page of (b, h), K and V, bit for bit against
-    the oracle's quantize_kv8; rows past the valid tokens hold code 0."""
+    the oracle's quantize_kv8 / quantize_kv4; rows past the valid tokens hold
+    code 0."""
     n = int(w.ctx_lens[b])
+    bits = res.get("bits", 8)
+    quant = oracle.quantize_kv8 if bits == 8 else oracle.quantize_kv4
     for key in ("k8", "v8", "k_scale", "v_scale"):   # one device -> host copy per call
         if key + "_np" not in res:
             res[key + "_np"] = res[key].cpu().numpy()
+            if bits == 4 and key in ("k8", "v8"):
+                res[key + "_np"] = unpack_codes4(res[key + "_np"].view(np.uint8))
     for name, bits, codes_all, scale_all in (("K", w.k_seq(b, h), res["k8_np"], res["k_scale_np"]),
                                              ("V", w.v_seq(b, h), res["v8_np"], res["v_scale_np"])):
         for m in range(-(-n // w.N_P)):
             pid = int(w.block_table[b, m])
             t0, t1 = m * w.N_P, min((m + 1) * w.N_P, n)
-            codes, sc = oracle.quantize_kv8(bits[t0:t1])
+            codes, sc = quant(bits[t0:t1])
             got_c = codes_all[pid, h]
             got_s = scale_all[pid, h]
             assert np.array_equal(got_c[:t1 - t0], codes), (name, b, h, m)
@@ -180,8 +202,9 @@ def check_outputs(w, res, b, h, q, k, v, pages, stats_out=None):
 
 def check_pair(w, res, b, h, errs=None, check_stats_bits=True, kv8=False):
     """Full parity of one (sequence, KV head): stats, scores, selection, output.
-    kv8: the attention read the int8 cache, so the oracle attends the
-    dequantized keys and values (pages and statistics stay those of bf16 K)."""
+    kv8: the attention read the quantized cache (res["bits"]: 8 or 4), so the
+    oracle attends the dequantized keys and values (pages and statistics stay
+    those of bf16 K)."""
     G = w.G
     n = int(w.ctx_lens[b])
     q = oracle.widen_bf16(w.q[b, h * G:(h + 1) * G])
@@ -191,8 +214,8 @@ def check_pair(w, res, b, h, errs=None, check_stats_bits=True, kv8=False):
     v = oracle.widen_bf16(v_bits)
     k_att, v_att = k, v
     if kv8:
-        k_att = oracle.dequantized_seq(k_bits, w.N_P)
-        v_att = oracle.dequantized_seq(v_bits, w.N_P)
+        k_att = oracle.dequantized_seq(k_bits, w.N_P, res.get("bits", 8))
+        v_att = oracle.dequantized_seq(v_bits, w.N_P, res.get("bits", 8))
     if w.head_kind[h] == 0:
         if n > 0:
             if check_stats_bits:

@@ -1,7 +1,8 @@
-"""GPU parity of the quantized-KV decode (the int8 cache): the page quantizer
-bit for bit against the oracle's quantize_kv8, and sparse decode attention
-over the int8 cache against the fp64 oracle attending the dequantized keys
-and values (code * scale), on the same seeded inputs and selections."""
+"""GPU parity of the quantized-KV decode (the 8-bit and the 4-bit cache): the
+page quantizer bit for bit against the oracle's quantize_kv8 / quantize_kv4,
+and sparse decode attention over the quantized cache against the fp64 oracle
+attending the dequantized keys and values (code * scale), on the same seeded
+inputs and selections."""
 import numpy as np
 import pytest
 import torch
@@ -25,30 +26,36 @@ CASES = [
 ]
 
 
+BITS = [8, 4]
+
+
+@pytest.mark.parametrize("bits", BITS)
 @pytest.mark.parametrize("case", CASES)
-def test_kv8_quantizer_and_decode_shapes(case):
+def test_kv8_quantizer_and_decode_shapes(case, bits):
     B, H_q, H_kv, D, N_L, N_P, K, S, L, lens, shuffle = case
     w = synth.decode_workload(B, H_q, H_kv, D, N_L, N_P, K, S, L, lens, seed=5151 + D + N_P,
                               shuffle=shuffle)
-    res = run_decode_path_kv8(DecodeBuffers(w, pad=synth.BF16_NAN))
+    res = run_decode_path_kv8(DecodeBuffers(w, pad=synth.BF16_NAN), bits=bits)
     for b in range(w.B):
         for h in range(w.H_kv):
             check_quantized_pages(w, res, b, h)
             check_pair(w, res, b, h, kv8=True)
 
 
-def test_kv8_tiny_workload():
+@pytest.mark.parametrize("bits", BITS)
+def test_kv8_tiny_workload(bits):
     w = synth.tiny_decode()
-    res = run_decode_path_kv8(DecodeBuffers(w, pad=synth.BF16_NAN))
+    res = run_decode_path_kv8(DecodeBuffers(w, pad=synth.BF16_NAN), bits=bits)
     for h in range(w.H_kv):
         check_quantized_pages(w, res, 0, h)
         check_pair(w, res, 0, h, kv8=True)
     assert list(res["sel"][0, 0]) == w.planted_pages[(0, 0)]
 
 
-def test_kv8_llama3_8b_decode_full():
+@pytest.mark.parametrize("bits", BITS)
+def test_kv8_llama3_8b_decode_full(bits):
     w = synth.llama3_8b_decode()
-    res = run_decode_path_kv8(DecodeBuffers(w))
+    res = run_decode_path_kv8(DecodeBuffers(w), bits=bits)
     errs = []
     for b in range(w.B):
         for h in range(w.H_kv):
@@ -59,10 +66,11 @@ def test_kv8_llama3_8b_decode_full():
           max(e[2] for e in errs))
 
 
-def test_kv8_mixed_batch_and_mha_sampled_pairs():
+@pytest.mark.parametrize("bits", BITS)
+def test_kv8_mixed_batch_and_mha_sampled_pairs(bits):
     for make, seed in ((synth.mixed_batch_decode, 21), (synth.llama2_7b_mha_decode, 22)):
         w = make()
-        res = run_decode_path_kv8(DecodeBuffers(w))
+        res = run_decode_path_kv8(DecodeBuffers(w), bits=bits)
         rng = np.random.default_rng(seed)
         pairs = [(int(b), int(h)) for b, h in zip(rng.integers(0, w.B, 8), rng.integers(0, w.H_kv, 8))]
         pairs += [(0, 0), (w.B - 1, w.H_kv - 1)]
@@ -72,22 +80,25 @@ def test_kv8_mixed_batch_and_mha_sampled_pairs():
         assert np.all(np.isfinite(res["out"]))
 
 
-def test_kv8_overlap_flag_is_bitwise_identical_and_close_to_bf16():
+@pytest.mark.parametrize("bits", BITS)
+def test_kv8_overlap_flag_is_bitwise_identical_and_close_to_bf16(bits):
     w = synth.decode_workload(2, 32, 8, 128, 16, 64, 16, 128, 512, [20000, 33333], seed=3)
     buf = DecodeBuffers(w)
-    r1 = run_decode_path_kv8(buf)
-    r2 = run_decode_path_kv8(buf, overlap=True)
+    r1 = run_decode_path_kv8(buf, bits=bits)
+    r2 = run_decode_path_kv8(buf, overlap=True, bits=bits)
     assert np.array_equal(r1["out"], r2["out"]) and np.array_equal(r1["lse"], r2["lse"])
-    # int8 per-page scales keep the output near the bf16 cache's (same pages)
+    # per-page scales keep the output near the bf16 cache's (same pages): int8
+    # within 0.05, 4-bit codes (a step of amax / 7) within 0.5
     rb = run_decode_path(buf)
     assert np.array_equal(rb["sel"], r1["sel"])
-    assert np.max(np.abs(rb["out"] - r1["out"])) < 0.05
+    assert np.max(np.abs(rb["out"] - r1["out"])) < (0.05 if bits == 8 else 0.5)
 
 
-def test_kv8_empty_sequence_and_bad_pool_id():
+@pytest.mark.parametrize("bits", BITS)
+def test_kv8_empty_sequence_and_bad_pool_id(bits):
     w = synth.decode_workload(2, 8, 2, 128, 16, 64, 4, 64, 256, [0, 3000], seed=8)
     buf = DecodeBuffers(w)
-    res = run_decode_path_kv8(buf)
+    res = run_decode_path_kv8(buf, bits=bits)
     assert np.all(res["out"][0] == 0) and np.all(np.isneginf(res["lse"][0]))
     for h in range(2):
         check_pair(w, res, 1, h, kv8=True)
@@ -96,6 +107,6 @@ def test_kv8_empty_sequence_and_bad_pool_id():
     bt = buf.block_table.clone()
     bt[1, 3] = w.num_pool_pages + 5
     lserve.quantize_pages_kv8(d, buf.k_pool, buf.v_pool, bt, buf.ctx_lens, res["k8"], res["v8"],
-                              res["k_scale"], res["v_scale"])
+                              res["k_scale"], res["v_scale"], bits=bits)
     assert lserve.read_device_status() == lserve.ERR_BOUNDS
     assert lserve.read_device_status() == lserve.OK

@@ -117,3 +117,55 @@ def test_output_does_not_depend_on_the_split():
         pages = ([int(x) for x in res["sel"][0, h, :int(res["sel_count"][0, h])]] if w.head_kind[h] == 0
                  else oracle.streaming_pages(n, w.N_P, w.sink, w.local))
         check_outputs(w, res2, 0, h, q, k, v, pages)
+
+
+def _decode(w, buf, d, ws, out, lse, scale):
+    lserve.sparse_decode_attn(d, buf.q, buf.k_pool, buf.v_pool, buf.block_table, buf.ctx_lens,
+                              buf.head_kind, buf.sel[0], buf.sel_count[0], w.top_k, w.sink, w.local,
+                              scale, out, lse, workspace=ws)
+    torch.cuda.synchronize()
+    assert lserve.read_device_status() == lserve.OK
+
+
+def test_workspace_leftovers_are_never_merged():
+    """The decode workspace heals itself: split partials are tagged with their
+    pair and a per-pair merge epoch, so words that an earlier call left behind
+    (here: every partial word of the previous call kept with its tag, its value
+    replaced by NaN, as a call that stopped before merging would leave them)
+    are ignored, and a workspace last used by a call of another shape needs no
+    re-zeroing.  Each later call gives bit for bit the first call's output."""
+    w = synth.llama3_8b_decode()
+    buf = DecodeBuffers(w)
+    res = run_decode_path(buf)
+    d = desc_of(w)
+    w2 = synth.decode_workload(3, 16, 2, 128, 16, 64, 16, 64, 256, [20000, 3000, 40000], seed=74)
+    d2 = desc_of(w2)
+    nbytes = max(lserve.workspace_size(lserve.OP_DECODE, d, w.top_k),
+                 lserve.workspace_size(lserve.OP_DECODE, d2, w2.top_k))
+    ws = lserve.alloc_workspace(nbytes)
+    out = torch.empty_like(buf.out)
+    lse = torch.empty_like(buf.lse)
+    _decode(w, buf, d, ws, out, lse, res["scale"])
+    ref_o, ref_l = out.clone(), lse.clone()
+    assert torch.equal(ref_o, buf.out)                       # same split as run_decode_path's call
+    P = w.B * w.H_kv
+    head = (P * 4 + 255) // 256 * 256                        # the epochs, then the partial words
+    assert int(ws[:P * 4].view(torch.int32).max()) >= 1      # the call did merge split pairs
+    words = ws[head:].view(torch.int64)
+    nan_low = torch.tensor(0x7FC00000, dtype=torch.int64, device=ws.device)
+    for _ in range(2):
+        # keep every word's tag (high half), poison its value (low half)
+        words.copy_((words & ~0xFFFFFFFF) | nan_low)
+        out.fill_(0)
+        _decode(w, buf, d, ws, out, lse, res["scale"])
+        assert torch.equal(out, ref_o) and torch.equal(lse, ref_l)
+    # the same workspace after a call of another shape (G = 8, two KV heads)
+    buf2 = DecodeBuffers(w2)
+    run_decode_path(buf2)
+    lserve.sparse_decode_attn(d2, buf2.q, buf2.k_pool, buf2.v_pool, buf2.block_table,
+                              buf2.ctx_lens, buf2.head_kind, buf2.sel[0], buf2.sel_count[0],
+                              w2.top_k, w2.sink, w2.local, res["scale"], buf2.out, buf2.lse,
+                              workspace=ws)
+    out.fill_(0)
+    _decode(w, buf, d, ws, out, lse, res["scale"])
+    assert torch.equal(out, ref_o) and torch.equal(lse, ref_l)
