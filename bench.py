@@ -632,12 +632,13 @@ def main():
 
     def attn(l, overlap=False):
         # overlap: the kernel before this call is the previous layer's attention,
-        # which writes none of the selection / block-table inputs, so the split
-        # plan and first page lookups may run while it finishes (PDL)
+        # which writes none of the selection / block-table inputs nor this
+        # layer's pools, so the split plan, the first page lookups and the first
+        # tiles' copies may start while it finishes (PDL)
         lserve.decode_step(d, qs[l], k_last[l], v_last[l], buf.k_pools[l], buf.v_pools[l],
                            buf.stats[l], buf.block_table, buf.ctx_lens, buf.head_kind, buf.sel[l],
                            buf.sel_count[l], w.top_k, w.sink, w.local, scale, outs[l], None,
-                           workspace=ws_dec, overlap_prologue=overlap)
+                           workspace=ws_dec, overlap_prologue=overlap, prefetch_kv=overlap)
 
     with torch.cuda.stream(stream):
         stats_all()
@@ -798,7 +799,11 @@ def main():
         result["stages"]["attention_mha"] = mha_stage(lserve, synth, dev, stream, hbm_peak, timed)
     if not args.no_configs:
         result["stages"]["long_decode_256k"] = decode_config_stage(
-            lserve, synth, dev, stream, hbm_peak, timed, synth.long_decode_256k, 16, shards=4)
+            lserve, synth, dev, stream, hbm_peak, timed, synth.long_decode_256k, 16,
+            shards=4 if ws == 1 else 1)
+        if ws > 1:  # the 256K sequence split over the ranks, NCCL exchanges timed
+            result["stages"]["long_decode_256k_seq_sharded"] = seqshard_stage(
+                lserve, synth, dev, stream, hbm_peak, timed, rank, ws, args.warmup)
         result["stages"]["mixed_batch_decode"] = decode_config_stage(
             lserve, synth, dev, stream, hbm_peak, timed, synth.mixed_batch_decode, 3)
     if not args.no_kv8:
@@ -851,7 +856,7 @@ def mha_stage(lserve, synth, dev, stream, hbm_peak, timed, layers=8):
             lserve.sparse_decode_attn(d, buf.q, buf.k_pools[l], buf.v_pools[l], buf.block_table,
                                       buf.ctx_lens, buf.head_kind, buf.sel[l], buf.sel_count[l],
                                       w.top_k, w.sink, w.local, scale, outs[l], None, workspace=wsd,
-                                      overlap_prologue=l > 0)
+                                      overlap_prologue=l > 0, prefetch_kv=l > 0)
     with torch.cuda.stream(stream):
         attn_all()
     torch.cuda.synchronize()
@@ -896,7 +901,7 @@ def decode_config_stage(lserve, synth, dev, stream, hbm_peak, timed, make, layer
             lserve.sparse_decode_attn(d, buf.q, buf.k_pools[l], buf.v_pools[l], buf.block_table,
                                       buf.ctx_lens, buf.head_kind, buf.sel[l], buf.sel_count[l],
                                       w.top_k, w.sink, w.local, scale, outs[l], None, workspace=wsd,
-                                      overlap_prologue=l > 0)
+                                      overlap_prologue=l > 0, prefetch_kv=l > 0)
     with torch.cuda.stream(stream):
         for l in range(layers):
             lserve.page_stats(d, buf.k_pools[l], buf.block_table, buf.ctx_lens, buf.head_kind,
@@ -1027,6 +1032,62 @@ def seqshard_timing(lserve, w, buf, d, dev, stream, timed, layers, N, scale):
                          f"partials {4 * B * H_q * (D + 1)} B per shard"}
 
 
+def seqshard_stage(lserve, synth, dev, stream, hbm_peak, timed, rank, ws, warmup, layers=8,
+                   steps=64):
+    """The 256K long decode as one sequence split over the ws ranks (rank r
+    holds the physical pages [floor(M r / ws), floor(M (r + 1) / ws)) of every
+    layer, reading R17): per layer-step each rank attends its share of the
+    chosen pages, all-gathers the float partials over NCCL and combines them;
+    every REUSE-th step it first scores its own pages, all-gathers its top-K
+    proposals and merges them (SeqShardStep, the exchanges on the stream).
+    `layers` replicas, `steps` layer-steps timed (after `warmup`), eager
+    launches, max over ranks.  Bytes: those of the whole unsharded step."""
+    import torch
+    from synth.device import DecodeBuffers
+    w = synth.long_decode_256k()
+    buf = DecodeBuffers(w, device=dev, layers=layers)
+    B, H_q, H_kv, D, K = w.B, w.H_q, w.H_kv, w.D, w.top_k
+    d = lserve.paged_desc(B, H_q, H_kv, D, w.N_L, w.N_P, w.max_pages, w.num_pool_pages)
+    bounds = [lserve.seqshard_bounds(int(w.ctx_lens[b]), w.N_P, rank, ws) for b in range(B)]
+    stride = lserve.seqshard_sel_stride(d, K, w.sink, w.local)
+    ml = max([stride, 1] + [hi - lo for lo, hi, _ in bounds])
+    bt = np.full((B, ml), -1, dtype=np.int32)
+    for b, (lo, hi, _) in enumerate(bounds):
+        bt[b, :hi - lo] = w.block_table[b, lo:hi]
+    dr = lserve.paged_desc(B, H_q, H_kv, D, w.N_L, w.N_P, ml, w.num_pool_pages)
+    bt_r = torch.from_numpy(bt).to(dev)
+    ctx_r = torch.tensor([n for _, _, n in bounds], dtype=torch.int32, device=dev)
+    shards = [lserve.SeqShardStep(dr, rank, ws, K, w.sink, w.local, device=dev)
+              for _ in range(layers)]
+    outs = [torch.empty((B, H_q, D), dtype=torch.bfloat16, device=dev) for _ in range(layers)]
+    scale = 1.0 / math.sqrt(D)
+    with torch.cuda.stream(stream):
+        for l in range(layers):  # the statistics of this rank's pages
+            lserve.page_stats(dr, buf.k_pools[l], bt_r, ctx_r, buf.head_kind, buf.stats[l])
+
+    def step(t):
+        for l in range(layers):
+            if t % REUSE == 0:
+                shards[l].select(buf.q, buf.stats[l], bt_r, ctx_r, buf.ctx_lens, buf.head_kind)
+            shards[l].attend(buf.q, buf.k_pools[l], buf.v_pools[l], bt_r, ctx_r, scale, outs[l])
+
+    with torch.cuda.stream(stream):
+        for t in range(max(warmup, REUSE)):
+            step(t)
+    torch.cuda.synchronize()
+    assert lserve.read_device_status(stream) == lserve.OK
+    el = timed(lambda: [step(t) for t in range(steps)])
+    el = max_over_ranks(el, ws, dev)
+    per = el / (steps * layers)
+    acct = decode_bytes(w)
+    return {"ranks": ws, "us_per_layer_step": per * 1e6, "GB/s_per_step": acct["step"] / per / 1e9,
+            "layers": layers, "steps": steps,
+            "what": "SeqShardStep per layer: attention over the rank's chosen pages, NCCL "
+                    "all-gather of (o, lse), combine; every 4th step also scores, all-gathers "
+                    "proposals and merges; eager launches; the bytes of the unsharded step",
+            "workload": f"{w.name}: B={B} n={int(w.ctx_lens[0])} split over {ws} ranks"}
+
+
 def kv8_stage(lserve, synth, dev, stream, hbm_peak, timed, make, layers, bf16_us, bits=8):
     """Decode attention over the quantized cache (lserve_sparse_decode_attn_kv8
     or _kv4 for bits = 8 / 4), alone: the workload's pools quantized once
@@ -1070,7 +1131,7 @@ def kv8_stage(lserve, synth, dev, stream, hbm_peak, timed, make, layers, bf16_us
             lserve.sparse_decode_attn_kv8(d, buf.q, a, b, c, e, buf.block_table, buf.ctx_lens,
                                           buf.head_kind, buf.sel[0], buf.sel_count[0], w.top_k,
                                           w.sink, w.local, scale, outs[l], None, workspace=wsd,
-                                          overlap_prologue=l > 0, bits=bits)
+                                          overlap_prologue=l > 0, prefetch_kv=l > 0, bits=bits)
     with torch.cuda.stream(stream):
         attn_all()
     torch.cuda.synchronize()

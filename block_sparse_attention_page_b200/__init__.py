@@ -38,6 +38,7 @@ EXPORTED = [
 ]
 DECODE_OVERLAP_PROLOGUE = 1
 DECODE_OUT_F32 = 2
+DECODE_PREFETCH_KV = 4
 
 
 class LServeError(RuntimeError):
@@ -122,6 +123,11 @@ def _load(path):
 lib = _load(library_path())
 
 
+def _decode_flags(overlap_prologue, prefetch_kv):
+    return ((DECODE_OVERLAP_PROLOGUE if overlap_prologue else 0) |
+            (DECODE_PREFETCH_KV if prefetch_kv else 0))
+
+
 def _ptr(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
@@ -179,14 +185,15 @@ def page_select_noalloc(desc, q, stats_pool, block_table, ctx_lens, head_kind, t
 
 def sparse_decode_attn(desc, q, k_pool, v_pool, block_table, ctx_lens, head_kind, sel, sel_count,
                        top_k, sink_tokens, local_tokens, softmax_scale, out, lse=None,
-                       workspace=None, stream=None, overlap_prologue=False, out_f32=False):
+                       workspace=None, stream=None, overlap_prologue=False, out_f32=False,
+                       prefetch_kv=False):
     """lserve_sparse_decode_attn; overlap_prologue=True or out_f32=True call
     lserve_sparse_decode_attn_ex with LSERVE_DECODE_OVERLAP_PROLOGUE (the caller
     guarantees the previous kernel on the stream writes none of block_table,
-    ctx_lens, head_kind, sel, sel_count) or LSERVE_DECODE_OUT_F32 (`out` is a
-    float32 tensor)."""
+    ctx_lens, head_kind, sel, sel_count; with prefetch_kv also no KV page this
+    call reads) or LSERVE_DECODE_OUT_F32 (`out` is a float32 tensor)."""
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    flags = (DECODE_OVERLAP_PROLOGUE if overlap_prologue else 0) | (DECODE_OUT_F32 if out_f32 else 0)
+    flags = _decode_flags(overlap_prologue, prefetch_kv) | (DECODE_OUT_F32 if out_f32 else 0)
     if flags:
         _check("lserve_sparse_decode_attn_ex", lib.lserve_sparse_decode_attn_ex(
             ctypes.byref(desc), _ptr(q), _ptr(k_pool), _ptr(v_pool), _ptr(block_table),
@@ -233,11 +240,11 @@ def quantize_pages_kv8(desc, k_pool, v_pool, block_table, ctx_lens, k_pool8, v_p
 def sparse_decode_attn_kv8(desc, q, k_pool8, v_pool8, k_scale, v_scale, block_table, ctx_lens,
                            head_kind, sel, sel_count, top_k, sink_tokens, local_tokens,
                            softmax_scale, out, lse=None, workspace=None, stream=None,
-                           overlap_prologue=False, bits=8):
+                           overlap_prologue=False, bits=8, prefetch_kv=False):
     """lserve_sparse_decode_attn_kv8 / _kv4: sparse decode attention over the
     8-bit or 4-bit cache."""
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    flags = DECODE_OVERLAP_PROLOGUE if overlap_prologue else 0
+    flags = _decode_flags(overlap_prologue, prefetch_kv)
     name = {8: "lserve_sparse_decode_attn_kv8", 4: "lserve_sparse_decode_attn_kv4"}[bits]
     _check(name, getattr(lib, name)(
         ctypes.byref(desc), _ptr(q), _ptr(k_pool8), _ptr(v_pool8), _ptr(k_scale), _ptr(v_scale),
@@ -248,11 +255,12 @@ def sparse_decode_attn_kv8(desc, q, k_pool8, v_pool8, k_scale, v_scale, block_ta
 
 def decode_step(desc, q, k_new, v_new, k_pool, v_pool, stats_pool, block_table, ctx_lens,
                 head_kind, sel, sel_count, top_k, sink_tokens, local_tokens, softmax_scale, out,
-                lse=None, recent_from=None, workspace=None, stream=None, overlap_prologue=False):
+                lse=None, recent_from=None, workspace=None, stream=None, overlap_prologue=False,
+                prefetch_kv=False):
     """lserve_decode_step: append the new tokens (k_new / v_new, or None) and
     attend, in one launch; ctx_lens counts the new token."""
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    flags = DECODE_OVERLAP_PROLOGUE if overlap_prologue else 0
+    flags = _decode_flags(overlap_prologue, prefetch_kv)
     _check("lserve_decode_step", lib.lserve_decode_step(
         ctypes.byref(desc), _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_pool), _ptr(v_pool),
         _ptr(stats_pool), _ptr(block_table), _ptr(ctx_lens), _ptr(head_kind), _ptr(sel),

@@ -99,6 +99,27 @@ bool make_map_tiled(CUtensorMap* m, const void* base, int rank, uint64_t d0, uin
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Rows of quantized codes (row_bytes = D or D / 2 bytes): a 2-D byte view,
+// box_rows whole rows a copy, swizzled by the row width (128, 64 or 32 bytes)
+// so that the rows a warp reads at once fall in different shared-memory banks.
+bool make_map_codes(CUtensorMap* m, const void* base, uint64_t rows, uint32_t row_bytes,
+                    uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  CUtensorMapSwizzle sw;
+  if (row_bytes == 128) sw = CU_TENSOR_MAP_SWIZZLE_128B;
+  else if (row_bytes == 64) sw = CU_TENSOR_MAP_SWIZZLE_64B;
+  else if (row_bytes == 32) sw = CU_TENSOR_MAP_SWIZZLE_32B;
+  else return false;
+  cuuint64_t dims[2] = {row_bytes, rows};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {row_bytes, box_rows};
+  cuuint32_t es[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 uint64_t wait_limit() { return g_wait_limit; }
 int current_sm_count() { return sm_count_current(); }
 
@@ -402,7 +423,8 @@ int decode_params(const lserve_paged_desc* desc, const void* q, const int32_t* b
                   float softmax_scale, void* out, float* lse, uint32_t flags, void* workspace,
                   size_t workspace_bytes, DecodeParams& p, int& grid) {
   if (!valid_paged(desc)) return LSERVE_ERR_INVALID_ARG;
-  if (flags & ~(uint32_t)(LSERVE_DECODE_OVERLAP_PROLOGUE | LSERVE_DECODE_OUT_F32))
+  if (flags & ~(uint32_t)(LSERVE_DECODE_OVERLAP_PROLOGUE | LSERVE_DECODE_OUT_F32 |
+                          LSERVE_DECODE_PREFETCH_KV))
     return LSERVE_ERR_INVALID_ARG;
   if (!q || !block_table || !ctx_lens || !head_kind || !sel || !sel_count || !out)
     return LSERVE_ERR_INVALID_ARG;
@@ -465,6 +487,7 @@ int decode_params(const lserve_paged_desc* desc, const void* q, const int32_t* b
   p.scale_log2 = softmax_scale * 1.4426950408889634f;
   p.wait_limit = wait_limit();
   p.overlap_prologue = (flags & LSERVE_DECODE_OVERLAP_PROLOGUE) ? 1 : 0;
+  p.prefetch_kv = (p.overlap_prologue && (flags & LSERVE_DECODE_PREFETCH_KV)) ? 1 : 0;
   p.status = device_status_word();
   if (!p.status) return LSERVE_ERR_CUDA;
   return LSERVE_OK;
@@ -523,7 +546,13 @@ int decode_quant_entry(const lserve_paged_desc* desc, const void* q, const void*
   p.k_scale = k_scale;
   p.v_scale = v_scale;
   const int D = desc->head_dim, G = desc->num_q_heads / desc->num_kv_heads;
-  return cuda_status(launch_decode_quant(p, D, G, bits, grid, static_cast<cudaStream_t>(stream)));
+  const uint64_t rows = (uint64_t)desc->num_pool_pages * desc->num_kv_heads * desc->physical_page;
+  CUtensorMap kmap, vmap;
+  if (!make_map_codes(&kmap, k_pool8, rows, (uint32_t)(D * bits / 8), p.tile_rows) ||
+      !make_map_codes(&vmap, v_pool8, rows, (uint32_t)(D * bits / 8), p.tile_rows))
+    return LSERVE_ERR_CUDA;
+  return cuda_status(launch_decode_quant(p, kmap, vmap, D, G, bits, grid,
+                                         static_cast<cudaStream_t>(stream)));
 }
 }  // namespace
 

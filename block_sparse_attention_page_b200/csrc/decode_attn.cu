@@ -166,7 +166,12 @@ template <int D, int G, int QB, int TR, int W>
 struct DecLayout {
   static constexpr int kRow = D * (QB == 0 ? 16 : QB) / 8;               // bytes per K (or V) row
   static constexpr int kTileK = TR * kRow;                               // K (or V) tile bytes
-  static constexpr int kScales = QB ? 2 * D * 4 : 0;                     // K, V channel scales
+  // K, V channel scales: four segments of D/4 channels (one per lane quad
+  // position of the MMA fragments) at a padded stride, so that the four
+  // segments a warp reads at once fall in different shared-memory banks
+  static constexpr int kScaleSeg = D;                                    // bytes: D/4 floats
+  static constexpr int kScaleSegP = kScaleSeg + 32;
+  static constexpr int kScales = QB ? 2 * 4 * kScaleSegP : 0;
   static constexpr int oScale = 2 * kTileK;                              // stage offsets
   static constexpr int oQ = oScale + kScales;
   static constexpr int kStageQ = G * D * 2;
@@ -466,11 +471,9 @@ decode_attn_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
     misc[24] = misc[25] = misc[26] = misc[27] = 0;
     fence_mbar_init();
   }
-  if constexpr (!Q8) {
-    if (tid == 32) {
-      tma_prefetch_desc(&kmap);
-      tma_prefetch_desc(&vmap);
-    }
+  if (tid == 32) {
+    tma_prefetch_desc(&kmap);
+    tma_prefetch_desc(&vmap);
   }
 
   // ---- plan: tiles per pair -> exclusive prefix off[0..P] in shared memory
@@ -561,12 +564,73 @@ decode_attn_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
     int issued = 0;
     bool alive = true;
     const uint64_t pol = l2_policy_evict_first();  // KV tiles: read once
+    // the stage's tile (and for the quantized cache its page's scales): expect
+    // every byte of the stage, then the copies that read no output of the
+    // previous kernel
+    auto issue_kv = [&](int s, int pr, int row, int val) {
+      uint8_t* st = smem + s * L::kStage;
+      if constexpr (Q8) {
+        const size_t ph = (size_t)row / p.physical_page;  // pool page * H_kv + head
+        mbar_arrive_expect_tx(&full[s], 2 * L::kTileK + 2 * 4 * L::kScaleSeg + L::kStageQ);
+        // rows swizzled by their width (tensor maps of the code pools)
+        tma_load_2d_hint(st, &kmap, 0, row, &full[s], pol);
+        tma_load_2d_hint(st + L::kTileK, &vmap, 0, row, &full[s], pol);
+#pragma unroll
+        for (int sg = 0; sg < 4; ++sg) {
+          bulk_load_1d(st + L::oScale + sg * L::kScaleSegP, p.k_scale + ph * D + sg * (D / 4),
+                       L::kScaleSeg, &full[s]);
+          bulk_load_1d(st + L::oScale + (4 + sg) * L::kScaleSegP, p.v_scale + ph * D + sg * (D / 4),
+                       L::kScaleSeg, &full[s]);
+        }
+      } else {
+        const bool has_new = (val >> 16) != 0;  // the tile holds the appended token
+        mbar_arrive_expect_tx(&full[s], 2 * TR * D * 2 + L::kStageQ + (has_new ? L::kNew : 0));
+        // one contiguous TR x D tile each: 3-D view (64 channels, D/64 halves, rows)
+        tma_load_3d_hint(st, &kmap, 0, 0, row, &full[s], pol);
+        tma_load_3d_hint(st + L::kTileK, &vmap, 0, 0, row, &full[s], pol);
+      }
+    };
+    // the copies of what the previous kernel may write: q, the appended rows
+    auto issue_rest = [&](int s, int pr, int val) {
+      uint8_t* st = smem + s * L::kStage;
+      const int b = pr / p.num_kv_heads, h = pr - b * p.num_kv_heads;
+      if constexpr (!Q8) {
+        if ((val >> 16) != 0) {  // its K / V rows from k_new / v_new, next to the tile
+          const size_t src = ((size_t)b * p.num_kv_heads + h) * D;
+          bulk_load_1d(st + L::oNew, p.k_new + src, D * 2, &full[s]);
+          bulk_load_1d(st + L::oNew + D * 2, p.v_new + src, D * 2, &full[s]);
+        }
+      }
+      bulk_load_1d(st + L::oQ, p.q + ((size_t)b * p.num_q_heads + (size_t)h * G) * D, L::kStageQ,
+                   &full[s]);
+    };
     for (int kb = 0; kb < ntiles && alive; kb += 32) {
       int tp = 0, trow = 0, tval = 0;
       if (kb + lane < ntiles) lookup(u0 + kb + lane, tp, trow, tval);
-      if (kb == 0) pdl_wait_prior_grid();  // q and the KV pools may come from the previous kernel
       const int nb = min(32, ntiles - kb);
-      for (int j = 0; j < nb; ++j) {
+      int j0 = 0;
+      if (kb == 0) {
+        // With LSERVE_DECODE_PREFETCH_KV the first stages' KV copies go out
+        // before the previous kernel completes (it writes no page this call
+        // reads); q and the appended rows may be its outputs and wait for it.
+        const int kpre = p.prefetch_kv ? min(S, nb) : 0;
+        for (int j = 0; j < kpre; ++j) {
+          const int pr = __shfl_sync(kFull, tp, j), row = __shfl_sync(kFull, trow, j);
+          const int val = __shfl_sync(kFull, tval, j);
+          if (lane == 0) {
+            info[j] = val;
+            issue_kv(j, pr, row, val);
+          }
+        }
+        pdl_wait_prior_grid();
+        for (int j = 0; j < kpre; ++j) {
+          const int pr = __shfl_sync(kFull, tp, j), val = __shfl_sync(kFull, tval, j);
+          if (lane == 0) issue_rest(j, pr, val);
+        }
+        j0 = kpre;
+        issued = kpre;
+      }
+      for (int j = j0; j < nb; ++j) {
         const int k = kb + j, s = k % S;
         const int pr = __shfl_sync(kFull, tp, j);
         const int row = __shfl_sync(kFull, trow, j);
@@ -577,30 +641,8 @@ decode_attn_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
           if (ok && !*abort_flag) {
             fence_proxy_async_smem();  // the consumers' reads of the stage come first
             info[s] = val;
-            const int b = pr / p.num_kv_heads, h = pr - b * p.num_kv_heads;
-            uint8_t* st = smem + s * L::kStage;
-            if constexpr (Q8) {
-              // codes: one contiguous TR-row tile each; then the page's scales
-              const size_t ph = (size_t)row / p.physical_page;  // pool page * H_kv + head
-              mbar_arrive_expect_tx(&full[s], 2 * L::kTileK + L::kScales + L::kStageQ);
-              bulk_load_1d_hint(st, p.k8 + (size_t)row * L::kRow, L::kTileK, &full[s], pol);
-              bulk_load_1d_hint(st + L::kTileK, p.v8 + (size_t)row * L::kRow, L::kTileK, &full[s], pol);
-              bulk_load_1d(st + L::oScale, p.k_scale + ph * D, D * 4, &full[s]);
-              bulk_load_1d(st + L::oScale + D * 4, p.v_scale + ph * D, D * 4, &full[s]);
-            } else {
-              const bool has_new = (val >> 16) != 0;  // the tile holds the appended token
-              mbar_arrive_expect_tx(&full[s], 2 * TR * D * 2 + L::kStageQ + (has_new ? L::kNew : 0));
-              // one contiguous TR x D tile each: 3-D view (64 channels, D/64 halves, rows)
-              tma_load_3d_hint(st, &kmap, 0, 0, row, &full[s], pol);
-              tma_load_3d_hint(st + L::kTileK, &vmap, 0, 0, row, &full[s], pol);
-              if (has_new) {  // its K / V rows from k_new / v_new, next to the tile
-                const size_t src = ((size_t)b * p.num_kv_heads + h) * D;
-                bulk_load_1d(st + L::oNew, p.k_new + src, D * 2, &full[s]);
-                bulk_load_1d(st + L::oNew + D * 2, p.v_new + src, D * 2, &full[s]);
-              }
-            }
-            bulk_load_1d(st + L::oQ, p.q + ((size_t)b * p.num_q_heads + (size_t)h * G) * D,
-                         L::kStageQ, &full[s]);
+            issue_kv(s, pr, row, val);
+            issue_rest(s, pr, val);
           } else {
             ok = 0;
           }
@@ -806,20 +848,26 @@ decode_attn_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
   constexpr int CB = CPL * QBB / 8;          // code bytes of a lane's run
   constexpr int NP2 = CPL / 2;               // pairs of a lane's run
   uint32_t qbf[CPL / 2];                     // q of head hr (bf16 pairs, natural order); 0 on padding rows
+  // Byte `o` of code row t of a tile: the tensor map swizzles 16-byte chunks by
+  // the row width (128-, 64- or 32-byte mode): chunk ^= (t * kRow / 128) & M.
+  auto code_at = [&](const uint8_t* tile, int t, int o) -> const uint8_t* {
+    constexpr int M = L::kRow == 128 ? 7 : (L::kRow == 64 ? 3 : 1);
+    const int sw = ((t * L::kRow) >> 7) & M;
+    return tile + t * L::kRow + ((((o >> 4) ^ sw)) << 4) + (o & 15);
+  };
   // this lane's run of codes of token row t of the tile at `tile`, as fp16 pairs
   auto run_codes = [&](const uint8_t* tile, int t, uint32_t (&pr)[NP2]) {
-    const uint8_t* cp = tile + t * L::kRow + CB * qq;
     uint32_t w[CB / 4];
 #pragma unroll
     for (int i = 0; i < CB / 16; ++i) {
-      const uint4 v = reinterpret_cast<const uint4*>(cp)[i];
+      const uint4 v = *reinterpret_cast<const uint4*>(code_at(tile, t, CB * qq + 16 * i));
       w[4 * i] = v.x;
       w[4 * i + 1] = v.y;
       w[4 * i + 2] = v.z;
       w[4 * i + 3] = v.w;
     }
     if constexpr (CB % 16 == 8) {
-      const uint2 v = reinterpret_cast<const uint2*>(cp)[CB / 8 - 1];
+      const uint2 v = *reinterpret_cast<const uint2*>(code_at(tile, t, CB * qq + CB - 8));
       w[CB / 4 - 2] = v.x;
       w[CB / 4 - 1] = v.y;
     }
@@ -838,7 +886,7 @@ decode_attn_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
   // this lane's run, the page's K (which = 0) or V (1) channel scales read 8
   // channels at a time
   auto for_scale_pairs = [&](const uint8_t* st, int which, auto&& f) {
-    const float4* sp = reinterpret_cast<const float4*>(st + L::oScale + which * D * 4) + qq * (CPL / 4);
+    const float4* sp = reinterpret_cast<const float4*>(st + L::oScale + (4 * which + qq) * L::kScaleSegP);
 #pragma unroll
     for (int m = 0; m < CPL / 8; ++m) {
       const float4 a = sp[2 * m], b = sp[2 * m + 1];
@@ -1480,12 +1528,11 @@ cudaError_t launch_decode(const DecodeParams& p, const CUtensorMap& kmap, const 
   return launch_decode_any<0>(p, kmap, vmap, D, G, grid, stream);
 }
 
-cudaError_t launch_decode_quant(const DecodeParams& p, int D, int G, int bits, int grid,
+cudaError_t launch_decode_quant(const DecodeParams& p, const CUtensorMap& kmap,
+                                const CUtensorMap& vmap, int D, int G, int bits, int grid,
                                 cudaStream_t stream) {
-  CUtensorMap unused;  // the quantized tiles are plain bulk copies: no tensor map
-  memset(&unused, 0, sizeof(unused));
-  if (bits == 8) return launch_decode_any<8>(p, unused, unused, D, G, grid, stream);
-  if (bits == 4) return launch_decode_any<4>(p, unused, unused, D, G, grid, stream);
+  if (bits == 8) return launch_decode_any<8>(p, kmap, vmap, D, G, grid, stream);
+  if (bits == 4) return launch_decode_any<4>(p, kmap, vmap, D, G, grid, stream);
   return cudaErrorInvalidValue;
 }
 

@@ -76,6 +76,7 @@ struct DecodeParams {
   float scale_log2;       // softmax_scale * log2(e)
   uint64_t wait_limit;
   int overlap_prologue;   // plan + first lookups may run before the preceding kernel ends
+  int prefetch_kv;        // the first stages' KV copies too (the preceding kernel writes no page)
   // quantized cache (lserve_sparse_decode_attn_kv8 / _kv4): codes [pool rows]
   // [D] bytes (8-bit) or [D/2] bytes (4-bit, two per byte) and float scales
   // [num_pool_pages][H_kv][D]; null for the bf16 cache
@@ -181,7 +182,8 @@ cudaError_t launch_decode(const DecodeParams& p, const CUtensorMap& kmap, const 
                           int D, int G, int grid, cudaStream_t stream);
 // the quantized-cache variants, bits = 8 or 4 (p.k8 / p.v8 / p.k_scale / p.v_scale
 // set; no tensor maps)
-cudaError_t launch_decode_quant(const DecodeParams& p, int D, int G, int bits, int grid,
+cudaError_t launch_decode_quant(const DecodeParams& p, const CUtensorMap& kmap,
+                                const CUtensorMap& vmap, int D, int G, int bits, int grid,
                                 cudaStream_t stream);
 size_t decode_workspace_bytes(int pairs, int grid, int G, int D);
 int decode_grid(int sm_count);
@@ -199,6 +201,8 @@ bool make_map_2d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
                  uint32_t box_rows);
 bool make_map_tiled(CUtensorMap* m, const void* base, int rank, uint64_t d0, uint64_t d1, uint64_t d2,
                     uint32_t b0, uint32_t b1, uint32_t b2);
+bool make_map_codes(CUtensorMap* m, const void* base, uint64_t rows, uint32_t row_bytes,
+                    uint32_t box_rows);
 uint64_t wait_limit();
 int current_sm_count();
 unsigned int* device_status_word();

@@ -238,11 +238,22 @@ int lserve_sparse_decode_attn(const lserve_paged_desc* desc, const void* q, cons
  *                                      normalised output before bf16
  *                                      rounding), e.g. a shard's partial
  *                                      for lserve_seqshard_combine.
+ *   LSERVE_DECODE_PREFETCH_KV          with LSERVE_DECODE_OVERLAP_PROLOGUE
+ *                                      (ignored without it): the caller also
+ *                                      guarantees that the kernel just before
+ *                                      writes no KV-pool page (nor quantized
+ *                                      code or scale) this call reads, so the
+ *                                      first tiles' copies start before that
+ *                                      kernel completes (consecutive layers'
+ *                                      calls; a QKV projection that writes q
+ *                                      and the new token only).  q and the
+ *                                      appended rows still wait for it.
  * Any other bit: LSERVE_ERR_INVALID_ARG.  Everything else as
  * lserve_sparse_decode_attn.
  */
 #define LSERVE_DECODE_OVERLAP_PROLOGUE 1u
 #define LSERVE_DECODE_OUT_F32 2u
+#define LSERVE_DECODE_PREFETCH_KV 4u
 int lserve_sparse_decode_attn_ex(const lserve_paged_desc* desc, const void* q, const void* k_pool,
                                  const void* v_pool, const int32_t* block_table,
                                  const int32_t* ctx_lens, const uint8_t* head_kind,

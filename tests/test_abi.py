@@ -126,7 +126,7 @@ def test_workspace_size_of_select():
 
 def test_decode_ex_rejects_unknown_flags():
     d = _desc()
-    for flags in (4, 8, 0x80000000):
+    for flags in (8, 16, 0x80000000):
         st = lserve.lib.lserve_sparse_decode_attn_ex(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, FAKE,
                                                      FAKE, FAKE, FAKE, 8, 64, 256, 0.125, FAKE, None,
                                                      flags, None, 0, None)
@@ -176,4 +176,4 @@ def test_kv8_calls_reject_null_misaligned_and_bad_scalars():
     assert _decode8(d, out=None) == lserve.ERR_INVALID_ARG
     assert _decode8(d, top_k=0) == lserve.ERR_INVALID_ARG
     assert _decode8(d, top_k=33) == lserve.ERR_INVALID_ARG
-    assert _decode8(d, flags=4) == lserve.ERR_INVALID_ARG
+    assert _decode8(d, flags=8) == lserve.ERR_INVALID_ARG

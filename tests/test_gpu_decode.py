@@ -182,7 +182,7 @@ def test_overlapped_prologue_across_layers_is_bitwise_identical():
     ws = lserve.alloc_workspace(lserve.workspace_size(lserve.OP_DECODE, d, w.top_k))
     scale = 1.0 / math.sqrt(w.D)
 
-    def run(overlap):
+    def run(overlap, prefetch=False):
         outs = [torch.zeros_like(buf.out) for _ in range(layers)]
         lses = [torch.zeros_like(buf.lse) for _ in range(layers)]
         for rep in range(2):
@@ -190,12 +190,14 @@ def test_overlapped_prologue_across_layers_is_bitwise_identical():
                 lserve.sparse_decode_attn(d, buf.q, buf.k_pools[l], buf.v_pools[l], buf.block_table,
                                           buf.ctx_lens, buf.head_kind, buf.sel[l], buf.sel_count[l],
                                           w.top_k, w.sink, w.local, scale, outs[l], lses[l],
-                                          workspace=ws, overlap_prologue=overlap)
+                                          workspace=ws, overlap_prologue=overlap, prefetch_kv=prefetch)
         torch.cuda.synchronize()
         assert lserve.read_device_status() == lserve.OK
         return outs, lses
 
     plain_o, plain_l = run(False)
     ov_o, ov_l = run(True)
+    pf_o, pf_l = run(True, prefetch=True)   # the first tiles' copies before the previous layer ends
     for l in range(layers):
         assert torch.equal(plain_o[l], ov_o[l]) and torch.equal(plain_l[l], ov_l[l])
+        assert torch.equal(plain_o[l], pf_o[l]) and torch.equal(plain_l[l], pf_l[l])
