@@ -566,6 +566,10 @@ def main():
                     help="run only the prefill stage (profiling)")
     ap.add_argument("--prefill-seq", type=int, default=None,
                     help="prefill sequence length (default: the 128K workload)")
+    ap.add_argument("--profile", default=None,
+                    help="set up one workload and launch one decode call --steps times, then exit "
+                         "(a small case for ncu): WORKLOAD:CACHE with WORKLOAD in "
+                         "8b|mha|256k|mixed and CACHE in bf16|kv8|kv4")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
     if args.steps is None:
@@ -589,6 +593,8 @@ def main():
     from synth.device import DecodeBuffers
 
     hbm_peak, tc_peak, tc_sustained, peak_src = peaks()
+    if args.profile:
+        return profile_case(lserve, synth, dev, args.profile, args.steps)
     if args.prefill_only:
         res = prefill_stage(lserve, synth, dev, torch.cuda.Stream(device=dev), tc_peak, None,
                             args.prefill_seq)
@@ -1030,6 +1036,49 @@ def seqshard_timing(lserve, w, buf, d, dev, stream, timed, layers, N, scale):
             "us_per_layer_step": (t_att + t_sel / REUSE) * 1e6,
             "not_timed": f"two all-gathers per step across GPUs: proposals {8 * B * H_kv * K} B and "
                          f"partials {4 * B * H_q * (D + 1)} B per shard"}
+
+
+def profile_case(lserve, synth, dev, spec, launches):
+    """One decode call of one workload, launched `launches` times after its
+    set-up (statistics, selection, quantization): the small case the ncu
+    captures in profiles/ run."""
+    import torch
+    from synth.device import DecodeBuffers
+    wname, cache = spec.split(":")
+    make = {"8b": synth.llama3_8b_decode, "mha": synth.llama2_7b_mha_decode,
+            "256k": synth.long_decode_256k, "mixed": synth.mixed_batch_decode}[wname]
+    w = make()
+    buf = DecodeBuffers(w, device=dev)
+    d = lserve.paged_desc(w.B, w.H_q, w.H_kv, w.D, w.N_L, w.N_P, w.max_pages, w.num_pool_pages)
+    wss = lserve.alloc_workspace(lserve.workspace_size(lserve.OP_SELECT, d, w.top_k), device=dev)
+    wsd = lserve.alloc_workspace(lserve.workspace_size(lserve.OP_DECODE, d, w.top_k), device=dev)
+    lserve.page_stats(d, buf.k_pool, buf.block_table, buf.ctx_lens, buf.head_kind, buf.stats[0])
+    lserve.page_select(d, buf.q, buf.stats[0], buf.block_table, buf.ctx_lens, buf.head_kind,
+                       w.top_k, buf.sel[0], buf.sel_count[0], workspace=wss)
+    scale = 1.0 / math.sqrt(w.D)
+    bits = {"bf16": 0, "kv8": 8, "kv4": 4}[cache]
+    if bits:
+        shape = w.pool_shape() if bits == 8 else w.pool_shape()[:-1] + (w.D // 2,)
+        k8 = torch.empty(shape, dtype=torch.int8, device=dev)
+        v8 = torch.empty_like(k8)
+        ks = torch.empty((w.num_pool_pages, w.H_kv, w.D), dtype=torch.float32, device=dev)
+        vs = torch.empty_like(ks)
+        lserve.quantize_pages_kv8(d, buf.k_pool, buf.v_pool, buf.block_table, buf.ctx_lens, k8, v8,
+                                  ks, vs, bits=bits)
+    for _ in range(max(1, launches)):
+        if bits:
+            lserve.sparse_decode_attn_kv8(d, buf.q, k8, v8, ks, vs, buf.block_table, buf.ctx_lens,
+                                          buf.head_kind, buf.sel[0], buf.sel_count[0], w.top_k,
+                                          w.sink, w.local, scale, buf.out, None, workspace=wsd,
+                                          bits=bits)
+        else:
+            lserve.sparse_decode_attn(d, buf.q, buf.k_pool, buf.v_pool, buf.block_table,
+                                      buf.ctx_lens, buf.head_kind, buf.sel[0], buf.sel_count[0],
+                                      w.top_k, w.sink, w.local, scale, buf.out, None, workspace=wsd)
+    torch.cuda.synchronize()
+    assert lserve.read_device_status() == lserve.OK
+    print(json.dumps({"profile": spec, "launches": launches}))
+    return 0
 
 
 def seqshard_stage(lserve, synth, dev, stream, hbm_peak, timed, rank, ws, warmup, layers=8,
