@@ -75,10 +75,19 @@ __device__ __forceinline__ bool recent_range(const DecodeParams& p, int b, int n
   rz = (n - 1) / p.physical_page;
   return true;
 }
-__device__ __forceinline__ bool in_sel_tail(const int32_t* s, int nsel, int R, int m) {
-  for (int i = max(0, nsel - R); i < nsel; ++i)
-    if (s[i] == m) return true;
-  return false;
+// First index of the ascending selection s[0..nsel) whose page is >= ra: the
+// selected pages among the recent ones are s[i0 .. nsel) (all are <= rz).
+__device__ __forceinline__ int sel_tail_start(const int32_t* s, int nsel, int ra) {
+  int i = nsel;
+  while (i > 0 && s[i - 1] >= ra) --i;
+  return i;
+}
+// The r-th recent page (0-based, ascending) that the selection does not hold:
+// ra + r, pushed up by one for every selected page at or below it.
+__device__ __forceinline__ int recent_page(const int32_t* s, int i0, int nsel, int ra, int r) {
+  int j = ra + r;
+  for (int i = i0; i < nsel && s[i] <= j; ++i) ++j;
+  return j;
 }
 
 // Selected pages of a retrieval pair the attention takes (the clamped count).
@@ -99,9 +108,7 @@ __device__ __forceinline__ int pair_pages(const DecodeParams& p, int pair) {
     int ra, rz, rf;
     if (!recent_range(p, b, n, ra, rz, rf)) return nsel;
     const int32_t* s = p.sel + (size_t)pair * p.top_k;
-    int extra = 0;
-    for (int m = ra; m <= rz; ++m) extra += in_sel_tail(s, nsel, rz - ra + 1, m) ? 0 : 1;
-    return nsel + extra;
+    return nsel + max(0, (rz - ra + 1) - (nsel - sel_tail_start(s, nsel, ra)));
   }
   const int ns = min((p.sink + NP - 1) / NP, npages);
   const int ls = max(max(0, n - p.local) / NP, ns);
@@ -535,10 +542,11 @@ decode_attn_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
           int ra, rz, rf;
           if (recent_range(p, b, n, ra, rz, rf)) {
             const int32_t* s = p.sel + (size_t)pair * p.top_k;
-            int r = li - nsel;
-            for (int j = ra; j <= rz && m < 0; ++j)
-              if (!in_sel_tail(s, nsel, rz - ra + 1, j) && r-- == 0) m = j;
-            if (m >= 0) lo = max(0, rf - m * NP);
+            const int j = recent_page(s, sel_tail_start(s, nsel, ra), nsel, ra, li - nsel);
+            if (j <= rz) {
+              m = j;
+              lo = max(0, rf - m * NP);
+            }
           }
         }
       } else {

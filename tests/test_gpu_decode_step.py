@@ -144,3 +144,44 @@ def test_decode_step_without_append_equals_sparse_decode_attn():
     torch.cuda.synchronize()
     assert lserve.read_device_status() == lserve.OK
     assert torch.equal(buf.out, o2) and torch.equal(buf.lse, l2)
+
+
+def test_decode_step_every_token_recent_is_dense_attention():
+    """recent_from = 0: every retrieval head attends all n tokens (one step,
+    appending), which the oracle computes as dense attention; long windows
+    cost the plan no more than the selection's length."""
+    w = synth.decode_workload(2, 8, 2, 128, 16, 64, 4, 64, 256, [3001, 9000], seed=9400)
+    buf = DecodeBuffers(w)
+    d = desc_of(w)
+    lens0 = np.array(w.ctx_lens, dtype=np.int32) - 1        # the last token is the appended one
+    lserve.page_stats(d, buf.k_pool, buf.block_table, torch.from_numpy(lens0).cuda(), buf.head_kind,
+                      buf.stats[0])
+    lserve.page_select(d, buf.q, buf.stats[0], buf.block_table, torch.from_numpy(lens0).cuda(),
+                       buf.head_kind, w.top_k, buf.sel[0], buf.sel_count[0], phys_scores=buf.scores)
+    K = [[w.k_seq(b, h) for h in range(w.H_kv)] for b in range(w.B)]
+    V = [[w.v_seq(b, h) for h in range(w.H_kv)] for b in range(w.B)]
+    kn = np.stack([np.stack([K[b][h][lens0[b]] for h in range(w.H_kv)]) for b in range(w.B)])
+    vn = np.stack([np.stack([V[b][h][lens0[b]] for h in range(w.H_kv)]) for b in range(w.B)])
+    zero = torch.zeros(w.B, dtype=torch.int32, device="cuda")
+    ws = lserve.alloc_workspace(lserve.workspace_size(lserve.OP_DECODE, d, w.top_k))
+    scale = 1.0 / math.sqrt(w.D)
+    lserve.decode_step(d, buf.q, bf16_tensor(kn), bf16_tensor(vn), buf.k_pool, buf.v_pool,
+                       buf.stats[0], buf.block_table, buf.ctx_lens, buf.head_kind, buf.sel[0],
+                       buf.sel_count[0], w.top_k, w.sink, w.local, scale, buf.out, buf.lse,
+                       recent_from=zero, workspace=ws)
+    torch.cuda.synchronize()
+    assert lserve.read_device_status() == lserve.OK
+    out = oracle.widen_bf16(bf16_bits(buf.out))
+    G = w.G
+    for b in range(w.B):
+        n = int(w.ctx_lens[b])
+        for h in range(w.H_kv):
+            q = oracle.widen_bf16(w.q[b, h * G:(h + 1) * G])
+            if w.head_kind[h] == 0:
+                toks = np.arange(n)
+            else:
+                toks = oracle.page_tokens(oracle.streaming_pages(n, w.N_P, w.sink, w.local), n, w.N_P)
+            o, _ = oracle.decode_attention(q, oracle.widen_bf16(K[b][h]), oracle.widen_bf16(V[b][h]),
+                                           toks, scale)
+            err = np.abs(out[b, h * G:(h + 1) * G] - o)
+            assert err.max() <= OUT_MAX_ABS and err.mean() <= OUT_MEAN_ABS, (b, h, err.max())
