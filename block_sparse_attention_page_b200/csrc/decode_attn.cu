@@ -37,13 +37,17 @@
 // tile (the pair closes c_f's range, so c_f reaches it last): every other CTA
 // c of the pair holds it as its FIRST pair and writes its unnormalised
 // (o, m, l) partial into its own workspace slot as tagged 8-byte words
-// {value, tag}, and c_f polls those words until their tags match, then merges
-// them with log-sum-exp weights.  No fence, counter or atomic is involved: a
-// word is one single-copy atomic store, and the tag carries the pair and the
-// pair's merge epoch (a per-pair counter that c_f advances at the end of
-// every call, whatever happened), so words left by an earlier call -- even
-// one that ended in a timeout -- never match.
+// {value, tag}.  c_f polls only the small (m, l) words (one warp's worth of
+// loads per poll: polling every o word as well put ~60 KB per poll on the
+// SM's load path and slowed the merge), stages them in shared memory, then
+// reads each o word once (checking its tag too) and merges with log-sum-exp
+// weights.  No fence, counter or atomic is involved: a word is one
+// single-copy atomic store, and the tag carries the pair and the pair's merge
+// epoch (a per-pair counter that c_f advances at the end of every call,
+// whatever happened), so words left by an earlier call -- even one that ended
+// in a timeout -- never match.
 #include <cstring>
+#include <type_traits>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -101,10 +105,11 @@ __device__ __forceinline__ int pair_pages(const DecodeParams& p, int pair) {
   const int b = pair / p.num_kv_heads, h = pair - b * p.num_kv_heads;
   const int n = p.ctx_lens[b];
   const int kind = p.head_kind[h];
+  const int sc = p.sel_count[pair];  // loaded with the other two (one round trip)
   const int NP = p.physical_page;
   const int npages = (n + NP - 1) / NP;
   if (kind == 0) {
-    const int nsel = sel_pages(p, pair, npages);
+    const int nsel = min(max(sc, 0), min(p.top_k, npages));
     int ra, rz, rf;
     if (!recent_range(p, b, n, ra, rz, rf)) return nsel;
     const int32_t* s = p.sel + (size_t)pair * p.top_k;
@@ -188,10 +193,9 @@ struct DecLayout {
   static constexpr int kPs = 2 * TR * G * 8;                            // p of two tiles
   static constexpr int kOw = W * G * D * 4;                              // o per warp
   static constexpr int kMl = W * G * 2 * 4;                              // (m, l) per warp
-  static constexpr int kSc = (W + 1) * G * 4;                            // merge weights + max
   static constexpr int kOff = ((kDecodeMaxPairs + 1) * 4 + 15) / 16 * 16;
   static constexpr int kCst = ((kMaxGrid + 1) * 4 + 15) / 16 * 16;
-  static constexpr int kFixed = kPs + kOw + kMl + kSc + kOff + kCst + 1024;
+  static constexpr int kFixed = kPs + kOw + kMl + kOff + kCst + 1024;
   static constexpr int kBudget = W <= 4 ? 112 * 1024 : 227 * 1024 - 1024;
   static constexpr int kStagesFit = (kBudget - kFixed) / kStage;
   static constexpr int kStages = kStagesFit > 8 ? 8 : kStagesFit;
@@ -199,8 +203,7 @@ struct DecLayout {
   static constexpr int oPs = kStages * kStage;
   static constexpr int oOw = oPs + kPs;
   static constexpr int oMl = oOw + kOw;
-  static constexpr int oSc = oMl + kMl;
-  static constexpr int oOff = (oSc + kSc + 15) / 16 * 16;
+  static constexpr int oOff = (oMl + kMl + 15) / 16 * 16;
   static constexpr int oCst = oOff + kOff;
   static constexpr int oInfo = oCst + kCst;
   static constexpr int oFull = (oInfo + kStages * 4 + 7) / 8 * 8;
@@ -208,16 +211,24 @@ struct DecLayout {
   static constexpr int oMisc = (oEmpty + kStages * 8 + 15) / 16 * 16;
   static constexpr int kBytes = oMisc + 128;
   static_assert(kStages >= 2, "decode ring needs two stages");
-  static_assert(oPs % 16 == 0 && oOw % 16 == 0 && oMl % 16 == 0 && oSc % 16 == 0 &&
+  static_assert(kStages * kStage >= kMaxGrid * G * 8, "the idle ring stages the merge's (m, l) words");
+  static_assert(oPs % 16 == 0 && oOw % 16 == 0 && oMl % 16 == 0 &&
                     oOff % 16 == 0 && oCst % 16 == 0 && oInfo % 4 == 0 && oFull % 8 == 0 &&
                     oEmpty % 8 == 0 && oMisc % 16 == 0,
                 "decode shared-memory arrays must keep their alignment");
   static_assert(kBytes <= kBudget, "decode shared memory over budget");
 };
 
-// cst[c] = floor(U * c / NC) is the first tile of CTA c's range (cst[NC] = U).
-// CTA whose range holds tile u: the largest c < NC with cst[c] <= u (ranges
-// can be empty when U < NC; the largest such c is the one that owns u).
+// First tile of CTA c's range, floor(U * c / NC) (c = NC gives U), in 32-bit
+// arithmetic: U = q * NC + r, so U * c / NC = q * c + r * c / NC with
+// r * c < NC^2.
+__device__ __forceinline__ int range_start(int U, int c, int NC) {
+  const int q = U / NC, r = U - q * NC;
+  return q * c + (r * c) / NC;
+}
+// cst[c] = range_start(U, c, NC).  CTA whose range holds tile u: the largest
+// c < NC with cst[c] <= u (ranges can be empty when U < NC; the largest such c
+// is the one that owns u).
 __device__ __forceinline__ int cta_of(const int* cst, int u, int NC) {
   int lo = 0, hi = NC - 1;
   while (lo < hi) {
@@ -242,10 +253,12 @@ __device__ __forceinline__ int pair_of(const int* off, int u, int P) {
 }
 
 // Tagged partial words: {float value, tag} as one 64-bit store / load.  The
-// tag is the pair's merge epoch for this call (11 low bits: the pair; pairs
-// are < 2048) -- a word from any earlier call or another pair differs.
+// tag is the pair's merge epoch for this call (20 bits) over the pair (11 low
+// bits; pairs are < 2048), with the top bit set so that a zeroed word never
+// matches -- a word from another pair, or from any of the pair's previous
+// 2^20 - 1 calls, differs.
 __device__ __forceinline__ uint32_t part_tag(uint32_t epoch, int pair) {
-  return (epoch << 11) | (uint32_t)pair;
+  return 0x80000000u | ((epoch & 0xFFFFFu) << 11) | (uint32_t)pair;
 }
 __device__ __forceinline__ void st_word(unsigned long long* a, float v, uint32_t tag) {
   const unsigned long long w = ((unsigned long long)tag << 32) | __float_as_uint(v);
@@ -255,6 +268,17 @@ __device__ __forceinline__ unsigned long long ld_word(const unsigned long long* 
   unsigned long long w;
   asm volatile("ld.relaxed.gpu.global.b64 %0, [%1];" : "=l"(w) : "l"(a) : "memory");
   return w;
+}
+// Two adjacent words (16-byte aligned) in one access; each word is still a
+// single-copy atomic 8-byte element.
+__device__ __forceinline__ void st_word2(unsigned long long* a, float v0, float v1, uint32_t tag) {
+  const unsigned long long w0 = ((unsigned long long)tag << 32) | __float_as_uint(v0);
+  const unsigned long long w1 = ((unsigned long long)tag << 32) | __float_as_uint(v1);
+  asm volatile("st.relaxed.gpu.global.v2.b64 [%0], {%1, %2};" ::"l"(a), "l"(w0), "l"(w1) : "memory");
+}
+__device__ __forceinline__ void ld_word2(const unsigned long long* a, unsigned long long& w0,
+                                         unsigned long long& w1) {
+  asm volatile("ld.relaxed.gpu.global.v2.b64 {%0, %1}, [%2];" : "=l"(w0), "=l"(w1) : "l"(a) : "memory");
 }
 __device__ __forceinline__ bool word_ok(unsigned long long w, uint32_t tag) {
   return (uint32_t)(w >> 32) == tag;
@@ -447,7 +471,6 @@ decode_attn_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
   float2* ps = reinterpret_cast<float2*>(smem + L::oPs);   // [tile 0/1][token][head] (p, p)
   float* ow = reinterpret_cast<float*>(smem + L::oOw);     // [warp][head][D]
   float2* mlw = reinterpret_cast<float2*>(smem + L::oMl);  // [warp][head] (m, l)
-  float* msc = reinterpret_cast<float*>(smem + L::oSc);    // [warp][head] weights, [head] max
   int* off = reinterpret_cast<int*>(smem + L::oOff);
   int* cst = reinterpret_cast<int*>(smem + L::oCst);
   int* info = reinterpret_cast<int*>(smem + L::oInfo);     // valid tokens of the stage's tile
@@ -512,9 +535,9 @@ decode_attn_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
     if (tid == kThreads - 1) off[P] = base + incl;
     __syncthreads();
   }
-  const long long U = off[P];
-  for (int c = tid; c <= NC; c += kThreads) cst[c] = (int)(U * c / NC);
-  const int u0 = (int)(U * cta / NC), u1 = (int)(U * (cta + 1) / NC);
+  const int U = off[P];
+  for (int c = tid; c <= NC; c += kThreads) cst[c] = range_start(U, c, NC);
+  const int u0 = range_start(U, cta, NC), u1 = range_start(U, cta + 1, NC);
   const int ntiles = u1 - u0;
 
   __syncthreads();  // range table, barrier init and plan visible to every warp
@@ -1043,7 +1066,9 @@ decode_attn_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
   // End of a pair segment (every consumer warp arrives here at the same tile):
   // merge the warps, then finalise the pair, or publish this CTA's partial, or
   // (the pair's merging CTA) fold in the other CTAs' partials and finalise.
-  auto flush = [&](int pair) {
+  // fin: the flush after the loop (the only one that can merge other CTAs' partials)
+  auto flush = [&](int pair, auto fin) {
+  constexpr bool kFinal = decltype(fin)::value;
     if constexpr (kMma || kQmma) {
       float lw = l_run;  // row sum of head hr over the warp's tokens: the row's 4 lanes
       lw += __shfl_xor_sync(kFull, lw, 1);
@@ -1087,194 +1112,149 @@ decode_attn_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
             make_float4(o_acc[g][0].x, o_acc[g][0].y, o_acc[g][1].x, o_acc[g][1].y);
     }
     }
-    const bool live = named_sync_and(kBarConsumers, kConsumerThreads, !*abort_flag);
-    if (tid < W * G) {  // weight of warp w's state for head g: 2^(m_w - max over warps)
-      const int g = tid % G;
-      float M = -INFINITY;
-#pragma unroll
-      for (int w = 0; w < W; ++w) M = fmaxf(M, mlw[w * G + g].x);
-      const float mw = mlw[tid].x;
-      msc[tid] = mw == -INFINITY ? 0.f : fast_ex2(mw - M);
-      if (tid < G) msc[W * G + g] = M;
-    }
-    named_sync(kBarConsumers, kConsumerThreads);
     const int b = pair / p.num_kv_heads, h = pair - b * p.num_kv_heads;
     // only the first and the last pair of a CTA's range can reach into other CTAs
     const bool whole = off[pair] >= u0 && off[pair + 1] <= u1;
-    const bool merger = !whole && pair == merge_pair;
+    // the merged pair is the last of the range: only the flush after the loop merges
+    const bool merger = kFinal && !whole && pair == merge_pair;
     const uint32_t tag = part_tag((merger ? e_merge : e_first) + 1u, pair);
-    constexpr int kSlot = G * D + 2 * G;  // words per partial
-    // this CTA's own (o, l, M) of each of the thread's outputs
-    float o_[NOUT], l_[NOUT], M_[NOUT];
+    // Partial of a CTA (its workspace slot): o words [G][D], then (m, l) word
+    // pairs [G][2].  A thread's NOUT outputs are the consecutive channels
+    // c0 .. c0 + NOUT - 1 of one head g (NOUT <= 2: one 16-byte access).
+    constexpr int kSlot = G * D + 2 * G;
+    const int j0 = tid * NOUT;
+    const bool has_out = j0 < G * D;
+    const int g = (has_out ? j0 : 0) / D, c0 = (has_out ? j0 : 0) - g * D;
+    const bool live = named_sync_and(kBarConsumers, kConsumerThreads, !*abort_flag);
+    // this CTA's own (o, m, l) of the thread's outputs: the warps' states
+    // weighted by 2^(m_w - max over warps)
+    float o_[NOUT], M = -INFINITY, l = 0.f;
 #pragma unroll
-    for (int i = 0; i < NOUT; ++i) {
-      const int j = min(tid + i * kConsumerThreads, G * D - 1);
-      const int g = j / D, c = j - g * D;
-      float o = 0.f, l = 0.f;
+    for (int w = 0; w < W; ++w) M = fmaxf(M, mlw[w * G + g].x);
 #pragma unroll
-      for (int w = 0; w < W; ++w) {
-        const float wt = msc[w * G + g];
-        o += wt * ow[(w * G + g) * D + c];
-        l += wt * mlw[w * G + g].y;
-      }
-      o_[i] = o;
-      l_[i] = l;
-      M_[i] = msc[W * G + g];
+    for (int i = 0; i < NOUT; ++i) o_[i] = 0.f;
+#pragma unroll
+    for (int w = 0; w < W; ++w) {
+      const float2 ml = mlw[w * G + g];
+      const float wt = ml.x == -INFINITY ? 0.f : fast_ex2(ml.x - M);
+      l += wt * ml.y;
+#pragma unroll
+      for (int i = 0; i < NOUT; ++i) o_[i] += wt * ow[(w * G + g) * D + c0 + i];
     }
-    if (!whole && !merger) {  // a later segment of a split pair: publish the partial
+    if (!whole && !merger && live && has_out) {  // a later segment of a split pair: publish
       unsigned long long* sl = p.parts + (size_t)cta * kSlot;
+      if constexpr (NOUT == 1) {
+        st_word(sl + g * D + c0, o_[0], tag);
+      } else {
 #pragma unroll
-      for (int i = 0; i < NOUT; ++i) {
-        const int j = tid + i * kConsumerThreads;
-        if (j >= G * D || !live) continue;
-        const int g = j / D, c = j - g * D;
-        st_word(sl + g * D + c, o_[i], tag);
-        if (c == 0) {
-          st_word(sl + G * D + g, M_[i], tag);
-          st_word(sl + G * D + G + g, l_[i], tag);
-        }
+        for (int i = 0; i < NOUT; i += 2) st_word2(sl + g * D + c0 + i, o_[i], o_[i + 1], tag);
       }
+      if (c0 == 0) st_word2(sl + G * D + 2 * g, M, l, tag);
     }
     bool got = true;
-    if (merger && live) {
-      // Fold in the partials of CTAs cta+1 .. c_last (those with tiles), every
-      // word polled until its tag matches.  Up to kBatch1 segments, each output
-      // loads its o, m and l words of all of them in one round and folds them
-      // in with running log-sum-exp weights.  Beyond that, every (m, l) word is
-      // first staged in shared memory (the p buffer is idle here), one word per
-      // thread, then each output loads its o words kBatch segments at a time
-      // with weights 2^(m_s - M) of the common maximum.
-      const int c_last = cta_of(cst, off[pair + 1] - 1, NC);
-      const int nseg = c_last - cta;
-      const long long t_poll = clock64();
-      float2* mls = reinterpret_cast<float2*>(ps);  // [segment][head]: (m, l)
-      // up to kBatch1 segments: one round of loads per output (its o, m, l words
-      // of every segment at once); more: the (m, l) words staged first
-      constexpr int kBatch1 = 8;
-      const bool staged = nseg > kBatch1 && nseg * G <= L::kPs / 8;
-      if (staged) {
-        for (int i = tid; i < nseg * G; i += kConsumerThreads) {
-          const int sg = i / G, g = i - sg * G, cc = cta + 1 + sg;
+    if constexpr (kFinal) {
+      if (merger && live) {
+        // Fold in the partials of CTAs cta+1 .. c_last (those with tiles).
+        // First the (m, l) word pairs, one (segment, head) entry per thread
+        // (a warp's worth of small loads per poll), each polled until its tag
+        // matches and staged in shared memory -- the stage ring, idle now.
+        // Then every thread loads its o words, kBatch segments at a time
+        // (stale words are loaded again together), and adds them with weights
+        // 2^(m_s - M) of the common maximum M.
+        const int c_last = cta_of(cst, off[pair + 1] - 1, NC);
+        const int nseg = c_last - cta, nml = nseg * G;
+        float2* mls = reinterpret_cast<float2*>(smem);  // [segment][head]: (m, l)
+        const long long t_poll = clock64();
+        for (int i = tid; i < nml; i += kConsumerThreads) {
+          const int cc = cta + 1 + i / G, gg = i % G;
           float2 ml = make_float2(-INFINITY, 0.f);
           if (cta_busy(cst, cc)) {
-            const unsigned long long* sl = p.parts + (size_t)cc * kSlot;
-            unsigned long long wm = ld_word(sl + G * D + g), wl = ld_word(sl + G * D + G + g);
-            while (!(word_ok(wm, tag) && word_ok(wl, tag))) {
+            const unsigned long long* a = p.parts + (size_t)cc * kSlot + G * D + 2 * gg;
+            unsigned long long wm, wl;
+            while (true) {
+              ld_word2(a, wm, wl);
+              if (word_ok(wm, tag) && word_ok(wl, tag)) break;
               if ((uint64_t)(clock64() - t_poll) > lim) {
                 got = false;
                 break;
               }
-              if (!word_ok(wm, tag)) wm = ld_word(sl + G * D + g);
-              if (!word_ok(wl, tag)) wl = ld_word(sl + G * D + G + g);
             }
             ml = make_float2(word_val(wm), word_val(wl));
           }
           mls[i] = ml;
         }
         got = named_sync_and(kBarConsumers, kConsumerThreads, got);
-      }
-      constexpr int kBatch = G >= 8 ? 8 : 16;  // segments whose o words are loaded at once
-#pragma unroll
-      for (int i = 0; i < NOUT; ++i) {
-        const int j = tid + i * kConsumerThreads;
-        if (j >= G * D || !got) continue;
-        const int g = j / D, c = j - g * D;
-        float M = M_[i], o = o_[i], l = l_[i];
-        if (staged) {  // the common maximum first, then one weighted sum
+        if (has_out && got) {
           float Mt = M;
           for (int sg = 0; sg < nseg; ++sg) Mt = fmaxf(Mt, mls[sg * G + g].x);
           if (Mt != -INFINITY) {
             const float a = exp2f(M - Mt);
-            o *= a;
+#pragma unroll
+            for (int i = 0; i < NOUT; ++i) o_[i] *= a;
             l *= a;
           }
+          constexpr int kBatch = 16 / NOUT;  // segments whose o words are in flight at once
           for (int s0 = 0; s0 < nseg && got; s0 += kBatch) {
-            unsigned long long wo[kBatch];
+            unsigned long long wo[kBatch][NOUT];
+            bool us[kBatch];
+            auto load_o = [&](int u) {
+              const unsigned long long* sl = p.parts + (size_t)(cta + 1 + s0 + u) * kSlot + g * D + c0;
+              if constexpr (NOUT == 1) {
+                wo[u][0] = ld_word(sl);
+              } else {
+#pragma unroll
+                for (int i = 0; i < NOUT; i += 2) ld_word2(sl + i, wo[u][i], wo[u][i + 1]);
+              }
+            };
+            auto seg_ok = [&](int u) {
+              bool ok = true;
+#pragma unroll
+              for (int i = 0; i < NOUT; ++i) ok = ok && word_ok(wo[u][i], tag);
+              return ok;
+            };
 #pragma unroll
             for (int u = 0; u < kBatch; ++u) {
-              const int cc = cta + 1 + s0 + u;
-              wo[u] = 0ull;
-              if (s0 + u < nseg && cta_busy(cst, cc))
-                wo[u] = ld_word(p.parts + (size_t)cc * kSlot + g * D + c);
+              us[u] = s0 + u < nseg && cta_busy(cst, cta + 1 + s0 + u);
+              if (us[u]) load_o(u);
+            }
+            while (true) {
+              bool pending = false;
+#pragma unroll
+              for (int u = 0; u < kBatch; ++u) pending |= us[u] && !seg_ok(u);
+              if (!pending) break;
+              if ((uint64_t)(clock64() - t_poll) > lim) {
+                got = false;
+                break;
+              }
+#pragma unroll
+              for (int u = 0; u < kBatch; ++u)
+                if (us[u] && !seg_ok(u)) load_o(u);
             }
 #pragma unroll
             for (int u = 0; u < kBatch; ++u) {
-              const int cc = cta + 1 + s0 + u;
-              if (s0 + u >= nseg || !cta_busy(cst, cc) || !got) continue;
-              while (!word_ok(wo[u], tag)) {
-                if ((uint64_t)(clock64() - t_poll) > lim) {
-                  got = false;
-                  break;
-                }
-                wo[u] = ld_word(p.parts + (size_t)cc * kSlot + g * D + c);
-              }
+              if (!us[u] || !got) continue;
               const float2 ml = mls[(s0 + u) * G + g];
-              if (!got || ml.x == -INFINITY) continue;
+              if (ml.x == -INFINITY) continue;
               const float wt = exp2f(ml.x - Mt);
-              o += word_val(wo[u]) * wt;
+#pragma unroll
+              for (int i = 0; i < NOUT; ++i) o_[i] += word_val(wo[u][i]) * wt;
               l += ml.y * wt;
             }
           }
           M = Mt;
-        } else {  // few segments (or too many to stage): o, m, l words per output
-          for (int c0 = cta + 1; c0 <= c_last && got; c0 += kBatch1) {
-            unsigned long long wo[kBatch1], wm[kBatch1], wl[kBatch1];
-#pragma unroll
-            for (int u = 0; u < kBatch1; ++u) {
-              const int cc = c0 + u;
-              wo[u] = wm[u] = wl[u] = 0ull;
-              if (cc <= c_last && cta_busy(cst, cc)) {
-                const unsigned long long* sl = p.parts + (size_t)cc * kSlot;
-                wo[u] = ld_word(sl + g * D + c);
-                wm[u] = ld_word(sl + G * D + g);
-                wl[u] = ld_word(sl + G * D + G + g);
-              }
-            }
-#pragma unroll
-            for (int u = 0; u < kBatch1; ++u) {
-              const int cc = c0 + u;
-              if (cc > c_last || !cta_busy(cst, cc) || !got) continue;
-              const unsigned long long* sl = p.parts + (size_t)cc * kSlot;
-              while (!(word_ok(wo[u], tag) && word_ok(wm[u], tag) && word_ok(wl[u], tag))) {
-                if ((uint64_t)(clock64() - t_poll) > lim) {
-                  got = false;
-                  break;
-                }
-                if (!word_ok(wo[u], tag)) wo[u] = ld_word(sl + g * D + c);
-                if (!word_ok(wm[u], tag)) wm[u] = ld_word(sl + G * D + g);
-                if (!word_ok(wl[u], tag)) wl[u] = ld_word(sl + G * D + G + g);
-              }
-              if (!got) continue;
-              const float ms = word_val(wm[u]);
-              const float Mn = fmaxf(M, ms);
-              if (Mn == -INFINITY) continue;  // both parts empty so far
-              const float a = exp2f(M - Mn), bw = exp2f(ms - Mn);
-              o = o * a + word_val(wo[u]) * bw;
-              l = l * a + word_val(wl[u]) * bw;
-              M = Mn;
-            }
-          }
         }
-        o_[i] = o;
-        l_[i] = l;
-        M_[i] = M;
+        if (!got && tid == 0) raise_status(p.status, LSERVE_ERR_TIMEOUT);
       }
-      if (!got && tid == 0) raise_status(p.status, LSERVE_ERR_TIMEOUT);
     }
-    if ((whole || merger) && live && got) {
+    if ((whole || merger) && live && got && has_out) {
+      const size_t qh = (size_t)b * p.num_q_heads + (size_t)h * G + g;
+      const bool empty_row = !(l > 0.f);
 #pragma unroll
-      for (int i = 0; i < NOUT; ++i) {
-        const int j = tid + i * kConsumerThreads;
-        if (j >= G * D) continue;
-        const int g = j / D, c = j - g * D;
-        const size_t qh = (size_t)b * p.num_q_heads + (size_t)h * G + g;
-        const bool empty_row = !(l_[i] > 0.f);
-        store_out(p, qh * D + c, empty_row ? 0.f : o_[i] / l_[i]);
-        if (c == 0 && p.lse)
-          p.lse[qh] = empty_row ? -INFINITY : (M_[i] + __log2f(l_[i])) * 0.69314718055994530942f;
-      }
+      for (int i = 0; i < NOUT; ++i) store_out(p, qh * D + c0 + i, empty_row ? 0.f : o_[i] / l);
+      if (c0 == 0 && p.lse)
+        p.lse[qh] = empty_row ? -INFINITY : (M + __log2f(l)) * 0.69314718055994530942f;
     }
-    named_sync(kBarConsumers, kConsumerThreads);  // ow / mlw / msc / ps free again
+    named_sync(kBarConsumers, kConsumerThreads);  // ow / mlw / ps free again
   };
 
   // Each iteration takes one tile, or two consecutive tiles of the same pair:
@@ -1283,7 +1263,7 @@ decode_attn_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
   bool need_q = false;
   for (int k = 0; k < ntiles;) {
     if (k >= pend) {  // first tile of a new pair (same decision in every consumer warp)
-      if (cur >= 0) flush(cur);
+      if (cur >= 0) flush(cur, std::false_type{});
       cur = pair_of(off, u0 + k, P);
       pend = off[cur + 1] - u0;
       m_run = -INFINITY;
@@ -1460,7 +1440,7 @@ decode_attn_kernel(const __grid_constant__ DecodeParams p, const __grid_constant
     }
     k += nt;
   }
-  if (cur >= 0) flush(cur);
+  if (cur >= 0) flush(cur, std::true_type{});
   // The merged pair's epoch advances whatever happened above (a timeout
   // included), so no word of this call matches a later call's tags.
   if (tid == 0 && merge_pair >= 0) {
