@@ -61,6 +61,46 @@ def peaks():
 
 
 # --- algorithmic byte / flop accounting (what the chosen sparsity touches) ----
+# Plain counting of the pages and blocks the method touches (the reading the
+# kernels implement), kept here so that the measurement legs run nothing of
+# the oracle; tests/test_bench_accounting.py checks these counts against it.
+
+def stream_pages(n, NP, sink, local):
+    """Pages a streaming head attends at length n: the sink pages
+    [0, ceil(sink / N_P)) and every page holding one of the last `local` tokens."""
+    if n <= 0:
+        return []
+    npages = -(-n // NP)
+    ns = min(-(-sink // NP), npages)
+    ls = max(max(0, n - local) // NP, ns)
+    return list(range(ns)) + list(range(ls, npages))
+
+
+def valid_tokens(pages, n, NP):
+    """Tokens of the given pages that lie below length n."""
+    return sum(max(0, min(NP, n - m * NP)) for m in pages)
+
+
+def prefill_flops(T, H_q, H_kv, D, block, head_kind, sink_blocks, local_blocks):
+    """Work counted as the pages count it: full block tiles (two matmuls of
+    2*block*block*D flops each) per query head; a retrieval KV head's rows
+    visit blocks 0..i, a streaming head's the sink blocks and the local
+    window [i - local + 1, i]."""
+    nb = -(-T // block)
+    G = H_q // H_kv
+    tiles = 0
+    for h in range(H_kv):
+        if int(head_kind[h]) == 0:
+            cnt = nb * (nb + 1) // 2
+        else:
+            cnt = 0
+            for i in range(nb):
+                s_hi = min(sink_blocks, i + 1)   # sink blocks [0, s_hi)
+                l_lo = max(0, i - local_blocks + 1)  # local blocks [l_lo, i]
+                cnt += s_hi + (i - l_lo + 1) - max(0, s_hi - l_lo)
+        tiles += G * cnt
+    return tiles * 4.0 * block * block * D
+
 
 def decode_bytes(w, fused_append=False):
     """Bytes one decode step of one layer must move, amortising selection over
@@ -69,7 +109,6 @@ def decode_bytes(w, fused_append=False):
     retrieval heads (2*D*2 bytes), the q vectors, scores and selection.  With
     fused_append the attention launch also appends the step's token (its K / V
     rows and the statistics it updates, append_bytes)."""
-    import oracle
     D, NP, NL = w.D, w.N_P, w.N_L
     kv = 0
     stats = 0
@@ -84,8 +123,7 @@ def decode_bytes(w, fused_append=False):
                 kv += k * NP * D * 2 * 2
                 stats += (-(-n // NL)) * 2 * D * 2
             else:
-                pages = oracle.streaming_pages(n, NP, w.sink, w.local)
-                toks = len(oracle.page_tokens(pages, n, NP))
+                toks = valid_tokens(stream_pages(n, NP, w.sink, w.local), n, NP)
                 kv += toks * D * 2 * 2
     q = w.B * w.H_q * D * 2
     out = w.B * w.H_q * D * 2
@@ -100,7 +138,6 @@ def decode_bytes_kv8(w, bits=8):
     codes of the attended pages (K and V, D * bits / 8 bytes per token each),
     the two float32 channel-scale rows of every attended (page, head), q and
     the output."""
-    import oracle
     D, NP = w.D, w.N_P
     kv = 0
     for b in range(w.B):
@@ -111,8 +148,8 @@ def decode_bytes_kv8(w, bits=8):
                 k = min(w.top_k, npages)
                 kv += k * NP * D * bits // 8 * 2 + k * 2 * D * 4
             else:
-                pages = oracle.streaming_pages(n, NP, w.sink, w.local)
-                toks = len(oracle.page_tokens(pages, n, NP))
+                pages = stream_pages(n, NP, w.sink, w.local)
+                toks = valid_tokens(pages, n, NP)
                 kv += toks * D * bits // 8 * 2 + len(pages) * 2 * D * 4
     return kv + 2 * w.B * w.H_q * D * 2
 
@@ -1208,7 +1245,6 @@ def prefill_stage(lserve, synth, dev, stream, tc_peak, timed, seq=None):
     """Block-sparse prefill on the 128K workload (or `seq` tokens of the same
     shape): TFLOP/s over computed blocks."""
     import torch
-    import oracle
     w = synth.prefill_128k() if seq is None else synth.prefill_workload(
         seq, 32, 8, 128, 128, 1004, name=f"prefill_{seq}")
     if timed is None:
@@ -1255,18 +1291,32 @@ def prefill_stage(lserve, synth, dev, stream, tc_peak, timed, seq=None):
             to_pages()
         torch.cuda.synchronize()
         t_tp = timed(to_pages, 3) / 3
+
+        # the same hand-over fused into the prefill kernel (its epilogue)
+        def paged():
+            lserve.blocksparse_prefill_paged(d, pd, pb.q, pb.k, pb.v, list(w.head_kind), scale,
+                                             pb.out, bt, kp, vp, sp, workspace=wsb, stream=stream)
+        with torch.cuda.stream(stream):
+            paged()
+        torch.cuda.synchronize()
+        t_pg = timed(paged, 3) / 3
+        assert lserve.read_device_status(stream) == lserve.OK
         retr = int(sum(1 for h in range(w.H_kv) if w.head_kind[h] == 0))
         tp_bytes = 2 * 2 * w.T * w.H_kv * w.D * 2 + retr * (-(-w.T // N_L)) * 2 * w.D * 2
         del kp, vp, sp
     except lserve.LServeError as e:
         return {"unavailable": str(e)}
-    flops = oracle.prefill_flops(w.T, w.H_q, w.H_kv, w.D, w.block, w.head_kind, w.sink_blocks,
-                                 w.local_blocks)
+    flops = prefill_flops(w.T, w.H_q, w.H_kv, w.D, w.block, w.head_kind, w.sink_blocks,
+                          w.local_blocks)
     tf = flops / t / 1e12
     return {"ms": t * 1e3, "TFLOP/s": tf, "frac": tf / tc_peak, "flops": flops,
             "to_pages": {"us": t_tp * 1e6, "GB/s": tp_bytes / t_tp / 1e9, "bytes": tp_bytes,
                          "what": "lserve_prefill_to_pages: K/V into the paged pools (N_P=64) "
                                  "+ page statistics (N_L=16), one pass"},
+            "paged": {"ms": t_pg * 1e3, "TFLOP/s": flops / t_pg / 1e12,
+                      "frac": flops / t_pg / 1e12 / tc_peak,
+                      "what": "lserve_blocksparse_prefill_paged: the prefill with the same hand-over "
+                              "(N_P=64, N_L=16) in its kernel's epilogue"},
             "workload": f"{w.name}: T={w.T} H_q={w.H_q} H_kv={w.H_kv} D={w.D} block={w.block} "
                         f"Lambda({w.sink_blocks},{w.local_blocks}) on KV heads 4-7"}
 

@@ -35,6 +35,7 @@ EXPORTED = [
     "lserve_sparse_decode_attn_kv8", "lserve_seqshard_bounds", "lserve_seqshard_sel_stride",
     "lserve_seqshard_candidates", "lserve_seqshard_merge", "lserve_seqshard_combine",
     "lserve_quantize_pages_kv4", "lserve_sparse_decode_attn_kv4", "lserve_decode_step",
+    "lserve_blocksparse_prefill_paged",
 ]
 DECODE_OVERLAP_PROLOGUE = 1
 DECODE_OUT_F32 = 2
@@ -80,6 +81,9 @@ def _load(path):
     lib.lserve_prefill_to_pages.argtypes = [P(PagedDesc), i32, vp, vp, vp, vp, vp, vp, vp, vp]
     lib.lserve_blocksparse_prefill.argtypes = [P(PrefillDesc), vp, vp, vp, vp, ctypes.c_float, vp, vp,
                                                vp, sz, vp]
+    lib.lserve_blocksparse_prefill_paged.argtypes = [P(PrefillDesc), P(PagedDesc), vp, vp, vp, vp,
+                                                     ctypes.c_float, vp, vp, vp, vp, vp, vp, vp, sz,
+                                                     vp]
     lib.lserve_quantize_pages_kv8.argtypes = [P(PagedDesc), vp, vp, vp, vp, vp, vp, vp, vp, vp]
     lib.lserve_sparse_decode_attn_kv8.argtypes = [P(PagedDesc), vp, vp, vp, vp, vp, vp, vp, vp, vp,
                                                   vp, i32, i32, i32, ctypes.c_float, vp, vp,
@@ -276,6 +280,21 @@ def blocksparse_prefill(desc, q, k, v, head_kind_host, softmax_scale, out, lse=N
     _check("lserve_blocksparse_prefill", lib.lserve_blocksparse_prefill(
         ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), ctypes.cast(hk, ctypes.c_void_p),
         float(softmax_scale), _ptr(out), _ptr(lse), _ptr(workspace), ws_bytes, _stream(stream)))
+
+
+def blocksparse_prefill_paged(desc, paged_desc, q, k, v, head_kind_host, softmax_scale, out,
+                              block_table, k_pool, v_pool, stats_pool, lse=None, workspace=None,
+                              stream=None):
+    """lserve_blocksparse_prefill_paged: the prefill, and from the same kernel
+    this sequence's K/V into the paged pools (through block_table) with the
+    retrieval heads' page statistics."""
+    hk = (ctypes.c_uint8 * len(head_kind_host))(*[int(x) for x in head_kind_host])
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check("lserve_blocksparse_prefill_paged", lib.lserve_blocksparse_prefill_paged(
+        ctypes.byref(desc), ctypes.byref(paged_desc), _ptr(q), _ptr(k), _ptr(v),
+        ctypes.cast(hk, ctypes.c_void_p), float(softmax_scale), _ptr(out), _ptr(lse),
+        _ptr(block_table), _ptr(k_pool), _ptr(v_pool), _ptr(stats_pool), _ptr(workspace), ws_bytes,
+        _stream(stream)))
 
 
 # --- sequence-sharded decode (one long sequence over several GPUs) -------------

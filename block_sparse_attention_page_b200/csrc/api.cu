@@ -788,4 +788,26 @@ int lserve_blocksparse_prefill(const lserve_prefill_desc* desc, const void* q, c
                        workspace_bytes, static_cast<cudaStream_t>(stream));
 }
 
+int lserve_blocksparse_prefill_paged(const lserve_prefill_desc* desc, const lserve_paged_desc* paged,
+                                     const void* q, const void* k, const void* v,
+                                     const uint8_t* head_kind_host, float softmax_scale, void* out,
+                                     float* lse, const int32_t* block_table, void* k_pool,
+                                     void* v_pool, void* stats_pool, void* workspace,
+                                     size_t workspace_bytes, void* stream) {
+  if (!desc || !valid_paged(paged)) return LSERVE_ERR_INVALID_ARG;
+  if (!block_table || !k_pool || !v_pool || !stats_pool) return LSERVE_ERR_INVALID_ARG;
+  if (!aligned(k_pool, 16) || !aligned(v_pool, 16) || !aligned(stats_pool, 16) ||
+      !aligned(block_table, 4))
+    return LSERVE_ERR_INVALID_ARG;
+  if (paged->head_dim != desc->head_dim || paged->num_kv_heads != desc->num_kv_heads)
+    return LSERVE_ERR_INVALID_ARG;
+  const int st = supported_paged(paged);
+  if (st != LSERVE_OK) return st;
+  if ((long long)desc->seq_len > (long long)paged->max_pages_per_seq * paged->physical_page)
+    return LSERVE_ERR_INVALID_ARG;
+  return prefill_paged_entry(desc, paged, q, k, v, head_kind_host, softmax_scale, out, lse,
+                             block_table, k_pool, v_pool, stats_pool, workspace, workspace_bytes,
+                             static_cast<cudaStream_t>(stream));
+}
+
 }  // extern "C"

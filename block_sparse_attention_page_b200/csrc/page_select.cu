@@ -11,7 +11,8 @@
 //    pages gives the physical score.
 // 2. page_topk_kernel: one CTA per (sequence, retrieval head) finds the K-th
 //    largest score by an 8-bit radix select over order-preserving integer
-//    keys, stopping once the bucket holding it has at most kTopkCand keys,
+//    keys (from the highest bit on which the keys differ), stopping once the
+//    bucket holding it has at most kTopkCand keys,
 //    which are ranked exactly by (score, page index); then it compacts the
 //    winners in ascending page order with one block scan.  Ties go to the
 //    lowest page indices.
@@ -151,6 +152,7 @@ __global__ void __launch_bounds__(kTopkThreads) page_topk_kernel(SelectParams p)
   __shared__ int sh_digit, sh_above, sh_bucket, sh_ncand;
   __shared__ int cand[kTopkCand];
   __shared__ uint32_t warp_tot[kTopkThreads / 32];
+  __shared__ uint32_t warp_max[kTopkThreads / 32], warp_min[kTopkThreads / 32];
   const int b = blockIdx.y, h = blockIdx.x, tid = threadIdx.x;
   const int lane = tid & 31, warp = tid >> 5;
   const size_t pair = (size_t)b * p.num_kv_heads + h;
@@ -175,15 +177,42 @@ __global__ void __launch_bounds__(kTopkThreads) page_topk_kernel(SelectParams p)
     return;
   }
   const float* sc = p.scores + pair * p.max_pages;
-  for (int m = tid; m < M; m += blockDim.x) keys[m] = order_key(sc[m]);
+  uint32_t kmx = 0u, kmn = 0xFFFFFFFFu;
+  for (int m = tid; m < M; m += blockDim.x) {
+    const uint32_t k = order_key(sc[m]);
+    keys[m] = k;
+    kmx = max(kmx, k);
+    kmn = min(kmn, k);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    kmx = max(kmx, __shfl_xor_sync(0xffffffffu, kmx, o));
+    kmn = min(kmn, __shfl_xor_sync(0xffffffffu, kmn, o));
+  }
+  if (lane == 0) {
+    warp_max[warp] = kmx;
+    warp_min[warp] = kmn;
+  }
   __syncthreads();
+  for (int w = 0; w < (int)(blockDim.x / 32); ++w) {
+    kmx = max(kmx, warp_max[w]);
+    kmn = min(kmn, warp_min[w]);
+  }
 
-  // Radix select of the K-th largest key, 8 bits at a time from the top, until
-  // the bucket that holds it has at most kTopkCand keys; those few are then
-  // ranked exactly by (key, page index).  `need` keys of the bucket are kept.
-  uint32_t prefix = 0, mask = 0;
+  // Radix select of the K-th largest key, at most 8 bits at a time from the
+  // top, until the bucket that holds it has at most kTopkCand keys; those few
+  // are then ranked exactly by (key, page index).  `need` keys of the bucket
+  // are kept.  The high bits on which the largest and the smallest key agree
+  // are common to every key and decide nothing, so the first digit is the
+  // (up to) 8 bits just below them (scores of similar magnitude share their
+  // top byte: starting at bit 31 would spend a pass on it).
+  const int hb = kmx == kmn ? -1 : 31 - __clz(kmx ^ kmn);  // highest bit where keys differ
+  uint32_t mask = hb >= 31 ? 0u : (0xFFFFFFFFu << (hb + 1));
+  uint32_t prefix = kmx & mask;
   int need = K, bucket = M;
-  for (int shift = 24; shift >= 0 && bucket > kTopkCand; shift -= 8) {
+  for (int hi = hb; hi >= 0 && bucket > kTopkCand;) {
+    const int shift = max(0, hi - 7);
+    const uint32_t dmask = (2u << (hi - shift)) - 1u;  // this pass's digit: bits [shift, hi]
     for (int i = tid; i < 256; i += blockDim.x) hist[i] = 0;
     __syncthreads();
     // warp-aggregated: the lanes holding the same digit add their count once
@@ -192,7 +221,7 @@ __global__ void __launch_bounds__(kTopkThreads) page_topk_kernel(SelectParams p)
       const int m = base + tid;
       const uint32_t k = m < M ? keys[m] : 0u;
       const bool act = m < M && (k & mask) == prefix;
-      const uint32_t digit = act ? (k >> shift) & 255u : 256u;
+      const uint32_t digit = act ? (k >> shift) & dmask : 256u;
       const unsigned peers = __match_any_sync(0xffffffffu, digit);
       if (act && lane == __ffs(peers) - 1) atomicAdd(&hist[digit], __popc(peers));
     }
@@ -227,8 +256,9 @@ __global__ void __launch_bounds__(kTopkThreads) page_topk_kernel(SelectParams p)
     __syncthreads();
     need -= sh_above;
     prefix |= (uint32_t)sh_digit << shift;
-    mask |= 255u << shift;
+    mask |= dmask << shift;
     bucket = sh_bucket;
+    hi = shift - 1;
   }
   uint8_t* chosen = reinterpret_cast<uint8_t*>(keys + M);  // [M], valid for bucket members
   const bool ranked = bucket <= kTopkCand;
@@ -251,8 +281,8 @@ __global__ void __launch_bounds__(kTopkThreads) page_topk_kernel(SelectParams p)
     }
     __syncthreads();
   }
-  // Otherwise all four digits were used and the bucket's keys are all equal:
-  // the `need` lowest page indices among them are kept.
+  // Otherwise every bit was used and the bucket's keys are all equal: the
+  // `need` lowest page indices among them are kept.
 
   // Compaction in ascending page order: one block scan of (above, kept) counts
   // over contiguous per-thread chunks.

@@ -11,7 +11,7 @@
 // of the row (all j <= i for dense heads; sink tiles and the local window for
 // streaming heads) -- the block skipping of the method.
 //
-// Warp roles (192 threads):
+// Warp roles (224 threads):
 //   warp 0     TMA producer: Q tile, then K and V tiles into two-stage rings
 //              (3-D tensor maps over [T][H][D], 128-byte swizzle, no multicast)
 //   warp 1     tensor-memory owner and single-thread MMA issuer:
@@ -22,6 +22,9 @@
 //              bf16 into shared memory (swizzled like a TMA tile), rescales O
 //              in TMEM only when the row max grows by more than 2^8, and runs
 //              the epilogue O / l -> bf16 and the log-sum-exp.
+//   warp 6     page writer (lserve_blocksparse_prefill_paged only): the
+//              diagonal key tile of each KV head into the paged pools and the
+//              page statistics, while the tile is in its ring stage.
 // MMA order S_0, S_1, PV_0, S_2, PV_1, ... keeps the tensor core on S_{j+1}
 // while the softmax warps work on S_j.
 #include <algorithm>
@@ -39,7 +42,7 @@ namespace {
 
 constexpr int kBM = 128;            // query rows per tile (MMA M)
 constexpr int kBN = 128;            // keys per key tile (MMA N of S, K of PV)
-constexpr int kThreads = 192;
+constexpr int kThreads = 224;          // 7 warps; warp 6 writes the paged cache
 constexpr float kRescaleLog2 = 8.0f;  // rescale O only when the max grows by > 2^8
 constexpr int kMaxHeads = 256;
 
@@ -60,6 +63,12 @@ struct PrefillParams {
   int n_dense_pairs, n_stream_pairs;
   uint8_t dense_pairs[kMaxHeads / 2];
   uint8_t stream_pairs[kMaxHeads / 2];
+  // paged epilogue (lserve_blocksparse_prefill_paged; pg_k_pool == nullptr: none)
+  __nv_bfloat16* pg_k_pool;
+  __nv_bfloat16* pg_v_pool;
+  __nv_bfloat16* pg_stats;
+  const int32_t* pg_block_table;  // this sequence's page ordinal -> pool id
+  int pg_np, pg_nl, pg_box_rows, pg_max_pages, pg_num_pool_pages;
 };
 
 template <int D>
@@ -71,7 +80,7 @@ struct Layout {
   static constexpr int kV = kK + 2 * kTile;       // 2 stages
   static constexpr int kP = kV + 2 * kTile;       // P: 128 x 128 bf16, 2 boxes
   static constexpr int kBar = kP + 2 * kBox;
-  static constexpr int kNumBars = 17;
+  static constexpr int kNumBars = 19;
   static constexpr int kBytes = kBar + kNumBars * 8 + 16;
 };
 
@@ -113,12 +122,154 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, uint64
   return __all_sync(0xffffffffu, ok);
 }
 
+// Paged epilogue of one key tile (row kt of KV head h), run by the whole
+// producer warp while the tile is still in its ring stage: K and V rows
+// [kt*kBN, min(kt*kBN + kBN, T)) go to the pools through the block table --
+// whole boxes of pg_box_rows rows by TMA stores, the rows of a page that the
+// sequence fills only partly by plain stores of its valid rows -- and, for a
+// retrieval head, every logical page of the tile gets the bf16 min / max of
+// its valid keys per channel (the same values lserve_page_stats and
+// lserve_prefill_to_pages write).  Returns after the TMA stores have read the
+// stage.  ks / vs: the stage's K and V tiles (NBOX swizzled 128-row boxes).
+template <int D>
+__device__ void page_out(const PrefillParams& p, const CUtensorMap* kpm, const CUtensorMap* vpm,
+                         const uint8_t* ks, const uint8_t* vs, int kt, int h, int lane) {
+  constexpr int NBOX = D / 64;
+  constexpr int kBoxBytes = kBM * 128;
+  constexpr int CPL = D / 32;  // channels of a lane in the statistics (4 or 2)
+  const int t0 = kt * kBN, tend = min(t0 + kBN, p.T);
+  const int NP = p.pg_np, NL = p.pg_nl, BR = p.pg_box_rows, g = NP / NL;
+  // byte offset of channel c of tile row r in a stage (128-byte swizzle per box)
+  auto off = [&](int r, int c) {
+    const int chunk = (c % 64) / 8;
+    return (uint32_t)((c / 64) * kBoxBytes + r * 128 + ((chunk ^ (r & 7)) << 4) + (c % 8) * 2);
+  };
+  bool issued = false;
+  // the tile's block-table entries (at most kBN / 32 pages), one lane each, in one round trip
+  const int m0 = t0 / NP;
+  int pid_l = -1;
+  if (m0 + lane < p.pg_max_pages && (m0 + lane) * NP < tend) pid_l = p.pg_block_table[m0 + lane];
+  for (int m = m0; m * NP < tend; ++m) {
+    const int a = max(t0, m * NP) - t0, e = min(tend, (m + 1) * NP) - t0;  // tile rows [a, e)
+    const int pid = __shfl_sync(0xffffffffu, pid_l, m - m0);
+    if (pid < 0 || pid >= p.pg_num_pool_pages) {
+      if (lane == 0) raise_status(p.status, LSERVE_ERR_BOUNDS);
+      continue;
+    }
+    const size_t prow = ((size_t)pid * p.H_kv + h) * NP + (size_t)(t0 + a - m * NP);  // pool row of a
+    if ((e - a) % BR == 0) {
+      if (lane == 0) {
+        fence_proxy_async_smem();  // the copies below read what the tile loads wrote
+        for (int r = a; r < e; r += BR)
+          for (int bx = 0; bx < NBOX; ++bx) {
+            tma_store_3d(kpm, 0, bx, (int32_t)(prow + (r - a)), ks + bx * kBoxBytes + r * 128);
+            tma_store_3d(vpm, 0, bx, (int32_t)(prow + (r - a)), vs + bx * kBoxBytes + r * 128);
+          }
+      }
+      issued = true;
+    } else {  // the sequence's last, partly filled page: its valid rows
+      for (int i = lane; i < (e - a) * (D / 8); i += 32) {
+        const int r = a + i / (D / 8), c = (i % (D / 8)) * 8;
+        const size_t dst = (prow + (size_t)(r - a)) * D + c;
+        *reinterpret_cast<uint4*>(p.pg_k_pool + dst) = *reinterpret_cast<const uint4*>(ks + off(r, c));
+        *reinterpret_cast<uint4*>(p.pg_v_pool + dst) = *reinterpret_cast<const uint4*>(vs + off(r, c));
+      }
+    }
+    if (p.kv_kind[h] != 0) continue;  // streaming heads need no statistics
+    for (int lp = (t0 + a) / NL; lp * NL < t0 + e; ++lp) {
+      const int ra = lp * NL - t0, rb = min((lp + 1) * NL, tend) - t0;
+      const uint32_t kPosInf2 = 0x7F807F80u, kNegInf2 = 0xFF80FF80u;
+      __nv_bfloat162 mn[CPL / 2], mx[CPL / 2];
+#pragma unroll
+      for (int k = 0; k < CPL / 2; ++k) {
+        mn[k] = *reinterpret_cast<const __nv_bfloat162*>(&kPosInf2);
+        mx[k] = *reinterpret_cast<const __nv_bfloat162*>(&kNegInf2);
+      }
+      for (int r = ra; r < rb; ++r) {
+#pragma unroll
+        for (int k = 0; k < CPL / 2; ++k) {
+          const __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162*>(ks + off(r, lane * CPL + 2 * k));
+          mn[k] = __hmin2(mn[k], v);
+          mx[k] = __hmax2(mx[k], v);
+        }
+      }
+      __nv_bfloat16* st = p.pg_stats + ((((size_t)pid * p.H_kv + h) * g) + (lp - m * g)) * 2 * D + lane * CPL;
+#pragma unroll
+      for (int k = 0; k < CPL / 2; ++k) {
+        reinterpret_cast<__nv_bfloat162*>(st)[k] = mn[k];
+        reinterpret_cast<__nv_bfloat162*>(st + D)[k] = mx[k];
+      }
+    }
+  }
+  if (issued && lane == 0) {
+    bulk_commit();
+    bulk_wait_read();  // the stage may be refilled
+  }
+  __syncwarp();
+}
+
+// The page writer warp: follows the CTA's work tiles as the producer deals
+// them (the same tile order and key-tile counts), and for every tile of a KV
+// head's first query head writes the pages of its diagonal key tile -- the
+// row's last key tile -- as soon as that tile's K and V have landed, then
+// arrives on pg_done[stage].  The producer waits on pg_done before it refills
+// that stage, so the tile stays in shared memory until it is written.  The
+// MMA and softmax warps never wait on it.
+// kv_issued[s]: fills of stage s the producer has issued.  A parity wait only
+// tells phases apart within one phase of the barrier's current one, so the
+// writer (which may run ahead of the producer) first waits until its tile's
+// fill has been issued; the producer cannot refill the stage after it until
+// the writer releases it, so that fill's phase is then the barrier's current
+// or just-completed one.
+template <int D, typename L, typename TileAt>
+__device__ void page_writer(const PrefillParams& p, const CUtensorMap* kpm, const CUtensorMap* vpm,
+                            uint8_t* smem, uint64_t* k_full, uint64_t* v_full, uint64_t* pg_done,
+                            const volatile uint32_t* kv_issued, int total, TileAt tile_of, int lane) {
+  const uint64_t lim = p.wait_limit;
+  // waits by lane 0 alone (the other lanes idle at the broadcast)
+  auto wait_issued = [&](int s, uint32_t want) -> bool {
+    bool ok = true;
+    if (lane == 0) {
+      const long long t0 = clock64();
+      while (kv_issued[s] < want) {
+        if ((uint64_t)(clock64() - t0) > lim) {
+          raise_status(p.status, LSERVE_ERR_TIMEOUT);
+          ok = false;
+          break;
+        }
+      }
+    }
+    return __shfl_sync(0xffffffffu, ok, 0);
+  };
+  auto wait1 = [&](uint64_t* bar, uint32_t parity) -> bool {
+    bool ok = true;
+    if (lane == 0) ok = mbar_wait(bar, parity, lim, p.status);
+    return __shfl_sync(0xffffffffu, ok, 0);
+  };
+  int kv_use = 0;
+  for (int r = 0;; ++r) {
+    const int idx = cta_tile(r, blockIdx.x, gridDim.x);
+    if (idx >= total) break;
+    const TileRef t = tile_of(idx);
+    const int hkv = t.hq / p.G;
+    kv_use += kv_range(p, p.kv_kind[hkv], t.qt).count();
+    if (t.hq % p.G != 0) continue;
+    const int kvi = kv_use - 1, s = kvi & 1, n = kvi >> 1;
+    if (!wait_issued(s, (uint32_t)n + 1) || !wait1(&k_full[s], n & 1) || !wait1(&v_full[s], n & 1))
+      break;
+    page_out<D>(p, kpm, vpm, smem + L::kK + s * L::kTile, smem + L::kV + s * L::kTile, t.qt, hkv, lane);
+    if (lane == 0) mbar_arrive(&pg_done[s]);
+  }
+  if (lane == 0) bulk_wait_all();  // the pools' TMA writes are complete
+}
+
 }  // namespace
 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
 prefill_kernel(const __grid_constant__ PrefillParams p, const __grid_constant__ CUtensorMap qmap,
-               const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap) {
+               const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
+               const __grid_constant__ CUtensorMap kpm, const __grid_constant__ CUtensorMap vpm) {
   using L = Layout<D>;
   constexpr int NBOX = D / 64;
   extern __shared__ uint8_t smem_raw[];
@@ -135,10 +286,13 @@ prefill_kernel(const __grid_constant__ PrefillParams p, const __grid_constant__ 
   uint64_t* p_full = bars + 14;
   uint64_t* p_free = bars + 15;
   uint64_t* o_free = bars + 16;
+  uint64_t* pg_done = bars + 17;  // [2]: the page writer is done with the stage's tile
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::kBar + L::kNumBars * 8);
+  volatile uint32_t* kv_issued = tmem_holder + 1;  // [2]: fills of each stage issued
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
+    kv_issued[0] = kv_issued[1] = 0u;
     mbar_init(q_full, 1);
     mbar_init(q_empty, 1);
     for (int s = 0; s < 2; ++s) {
@@ -148,6 +302,7 @@ prefill_kernel(const __grid_constant__ PrefillParams p, const __grid_constant__ 
       mbar_init(&v_empty[s], 1);
       mbar_init(&s_full[s], 1);
       mbar_init(&s_free[s], 128);
+      mbar_init(&pg_done[s], 1);
     }
     mbar_init(p_full, 128);
     mbar_init(p_free, 1);
@@ -168,14 +323,40 @@ prefill_kernel(const __grid_constant__ PrefillParams p, const __grid_constant__ 
   const int grid = gridDim.x;
   const uint64_t lim = p.wait_limit;
 
-  if (warp == 0) {
+  if (warp == 6) {
+    // ------------------------------------------------------------ page writer
+    if (p.pg_k_pool)
+      page_writer<D, L>(p, &kpm, &vpm, smem, k_full, v_full, pg_done, kv_issued, total,
+                        [&](int idx) { return tile_at(p, idx); }, lane);
+  } else if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
+    // Lane 0 alone; lanes 1-31 of warp 0 do nothing (they must not fall into
+    // the softmax branch below).  With the paged epilogue, a stage that holds
+    // a KV head's diagonal key tile (visited once, by the group's first query
+    // head) is refilled only after the page writer has released it.
     if (lane == 0) {
       tma_prefetch_desc(&qmap);
       tma_prefetch_desc(&kmap);
       tma_prefetch_desc(&vmap);
+      const bool paged = p.pg_k_pool != nullptr;
       int q_use = 0, kv_use = 0;
-      for (int r = 0;; ++r) {
+      // stage 0 / 1 holds a diagonal tile the page writer has not released yet;
+      // ep0 / ep1 count the writer's releases (the pg_done phases) per stage
+      bool owe0 = false, owe1 = false;
+      int ep0 = 0, ep1 = 0;
+      auto wait_writer = [&](int s) -> bool {
+        if (!mbar_wait(&pg_done[s], (s ? ep1 : ep0) & 1, lim, p.status)) return false;
+        if (s) {
+          ++ep1;
+          owe1 = false;
+        } else {
+          ++ep0;
+          owe0 = false;
+        }
+        return true;
+      };
+      bool ok = true;
+      for (int r = 0; ok; ++r) {
         const int idx = cta_tile(r, blockIdx.x, grid);
         if (idx >= total) break;
         const TileRef t = tile_at(p, idx);
@@ -186,12 +367,12 @@ prefill_kernel(const __grid_constant__ PrefillParams p, const __grid_constant__ 
         for (int bx = 0; bx < NBOX; ++bx)
           tma_load_3d(smem + L::kQ + bx * L::kBox, &qmap, bx * 64, t.hq, t.qt * kBM, q_full);
         ++q_use;
-        bool ok = true;
         const int nkv = kr.count();
         for (int j = 0; j < nkv && ok; ++j) {
           const int kt = kr.at(j);
           const int s = kv_use & 1, n = kv_use >> 1;
           if (n > 0 && !mbar_wait(&k_empty[s], (n - 1) & 1, lim, p.status)) { ok = false; break; }
+          if ((s ? owe1 : owe0) && !wait_writer(s)) { ok = false; break; }
           mbar_arrive_expect_tx(&k_full[s], L::kTile);
           for (int bx = 0; bx < NBOX; ++bx)
             tma_load_3d(smem + L::kK + s * L::kTile + bx * L::kBox, &kmap, bx * 64, hkv, kt * kBN,
@@ -201,9 +382,13 @@ prefill_kernel(const __grid_constant__ PrefillParams p, const __grid_constant__ 
           for (int bx = 0; bx < NBOX; ++bx)
             tma_load_3d(smem + L::kV + s * L::kTile + bx * L::kBox, &vmap, bx * 64, hkv, kt * kBN,
                         &v_full[s]);
+          kv_issued[s] = (uint32_t)n + 1;  // for the page writer
+          if (paged && t.hq % p.G == 0 && kt == t.qt) {  // the writer's tile
+            if (s) owe1 = true;
+            else owe0 = true;
+          }
           ++kv_use;
         }
-        if (!ok) break;
       }
     }
   } else if (warp == 1) {
@@ -424,7 +609,9 @@ prefill_kernel(const __grid_constant__ PrefillParams p, const __grid_constant__ 
 // leaves the tensor core waiting for its one softmax warpgroup.
 //   warp 0        TMA producer: Q of both heads, K and V into two-stage rings
 //   warp 1        tensor-memory owner (all 512 columns) and MMA issuer
-//   warps 2, 3    idle (they only lend their registers)
+//   warp 2        page writer (lserve_blocksparse_prefill_paged only), as in
+//                 prefill_kernel
+//   warp 3        idle (it only lends its registers)
 //   warps 4-7     softmax of head A (thread r: query row r = TMEM lane r)
 //   warps 8-11    softmax of head B
 // An S commit also covers the PV issued before it: when a softmax warpgroup
@@ -443,7 +630,7 @@ struct PairLayout {
   static constexpr int kK = kQ + 2 * kTile;     // 2 stages
   static constexpr int kV = kK + 2 * kTile;     // 2 stages
   static constexpr int kBar = kV + 2 * kTile;
-  static constexpr int kNumBars = 19;
+  static constexpr int kNumBars = 21;
   static constexpr int kBytes = kBar + kNumBars * 8 + 16;
 };
 
@@ -458,7 +645,8 @@ __device__ __forceinline__ TileRef pair_tile_at(const PrefillParams& p, int idx)
 template <int D>
 __global__ void __launch_bounds__(kPairThreads, 1)
 prefill_pair_kernel(const __grid_constant__ PrefillParams p, const __grid_constant__ CUtensorMap qmap,
-                    const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap) {
+                    const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
+                    const __grid_constant__ CUtensorMap kpm, const __grid_constant__ CUtensorMap vpm) {
   using L = PairLayout<D>;
   constexpr int NBOX = D / 64;
   extern __shared__ uint8_t smem_raw[];
@@ -474,10 +662,13 @@ prefill_pair_kernel(const __grid_constant__ PrefillParams p, const __grid_consta
   uint64_t* p_full = bars + 12;   // [head]
   uint64_t* pv_done = bars + 14;  // [head]: the tile's last PV has completed
   uint64_t* o_free = bars + 16;   // [head]: the epilogue has read O
+  uint64_t* pg_done = bars + 19;  // [2]: the page writer is done with the stage's tile
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::kBar + L::kNumBars * 8);
+  volatile uint32_t* kv_issued = tmem_holder + 1;  // [2]: fills of each stage issued
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
+    kv_issued[0] = kv_issued[1] = 0u;
     mbar_init(q_full, 1);
     mbar_init(q_empty, 1);
     for (int s = 0; s < 2; ++s) {
@@ -489,6 +680,7 @@ prefill_pair_kernel(const __grid_constant__ PrefillParams p, const __grid_consta
       mbar_init(&p_full[s], 128);
       mbar_init(&pv_done[s], 1);
       mbar_init(&o_free[s], 128);
+      mbar_init(&pg_done[s], 1);
     }
     fence_mbar_init();
   }
@@ -513,11 +705,28 @@ prefill_pair_kernel(const __grid_constant__ PrefillParams p, const __grid_consta
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kPairRegsCtl));
     if (warp == 0 && lane == 0) {
       // ------------------------------------------------------------ TMA producer
+      // A stage holding a diagonal key tile of the paged epilogue is refilled
+      // after the page writer (warp 2) releases it, as in prefill_kernel.
       tma_prefetch_desc(&qmap);
       tma_prefetch_desc(&kmap);
       tma_prefetch_desc(&vmap);
+      const bool paged = p.pg_k_pool != nullptr;
       int q_use = 0, kv_use = 0;
-      for (int r = 0;; ++r) {
+      bool owe0 = false, owe1 = false;  // as in prefill_kernel
+      int ep0 = 0, ep1 = 0;
+      auto wait_writer = [&](int s) -> bool {
+        if (!mbar_wait(&pg_done[s], (s ? ep1 : ep0) & 1, lim, p.status)) return false;
+        if (s) {
+          ++ep1;
+          owe1 = false;
+        } else {
+          ++ep0;
+          owe0 = false;
+        }
+        return true;
+      };
+      bool ok = true;
+      for (int r = 0; ok; ++r) {
         const int idx = cta_tile(r, blockIdx.x, grid);
         if (idx >= total) break;
         const TileRef t = pair_tile_at(p, idx);  // t.hq: head A, head B = t.hq + 1
@@ -530,12 +739,12 @@ prefill_pair_kernel(const __grid_constant__ PrefillParams p, const __grid_consta
             tma_load_3d(smem + L::kQ + x * L::kTile + bx * L::kBox, &qmap, bx * 64, t.hq + x,
                         t.qt * kBM, q_full);
         ++q_use;
-        bool ok = true;
         const int nkv = kr.count();
         for (int j = 0; j < nkv && ok; ++j) {
           const int kt = kr.at(j);
           const int s = kv_use & 1, n = kv_use >> 1;
           if (n > 0 && !mbar_wait(&k_empty[s], (n - 1) & 1, lim, p.status)) { ok = false; break; }
+          if ((s ? owe1 : owe0) && !wait_writer(s)) { ok = false; break; }
           mbar_arrive_expect_tx(&k_full[s], L::kTile);
           for (int bx = 0; bx < NBOX; ++bx)
             tma_load_3d(smem + L::kK + s * L::kTile + bx * L::kBox, &kmap, bx * 64, hkv, kt * kBN,
@@ -545,10 +754,19 @@ prefill_pair_kernel(const __grid_constant__ PrefillParams p, const __grid_consta
           for (int bx = 0; bx < NBOX; ++bx)
             tma_load_3d(smem + L::kV + s * L::kTile + bx * L::kBox, &vmap, bx * 64, hkv, kt * kBN,
                         &v_full[s]);
+          kv_issued[s] = (uint32_t)n + 1;  // for the page writer
+          if (paged && t.hq % p.G == 0 && kt == t.qt) {  // the writer's tile
+            if (s) owe1 = true;
+            else owe0 = true;
+          }
           ++kv_use;
         }
-        if (!ok) break;
       }
+    } else if (warp == 2) {
+      // ------------------------------------------------------------ page writer
+      if (p.pg_k_pool)
+        page_writer<D, L>(p, &kpm, &vpm, smem, k_full, v_full, pg_done, kv_issued, total,
+                          [&](int idx) { return pair_tile_at(p, idx); }, lane);
     } else if (warp == 1 && lane == 0) {
       // ------------------------------------------------------------ MMA issuer
       constexpr uint32_t idesc_s = tc::idesc_bf16_f32(kBM, kBN, false, false);
@@ -766,6 +984,24 @@ size_t prefill_workspace_bytes(const lserve_prefill_desc* d) {
 int prefill_entry(const lserve_prefill_desc* d, const void* q, const void* k, const void* v,
                   const uint8_t* head_kind_host, float softmax_scale, void* out, float* lse,
                   void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  return prefill_paged_entry(d, nullptr, q, k, v, head_kind_host, softmax_scale, out, lse, nullptr,
+                             nullptr, nullptr, nullptr, workspace, workspace_bytes, stream);
+}
+
+static int gcd_int(int a, int b) {
+  while (b) {
+    const int t = a % b;
+    a = b;
+    b = t;
+  }
+  return a;
+}
+
+int prefill_paged_entry(const lserve_prefill_desc* d, const lserve_paged_desc* pd, const void* q,
+                        const void* k, const void* v, const uint8_t* head_kind_host,
+                        float softmax_scale, void* out, float* lse, const int32_t* block_table,
+                        void* k_pool, void* v_pool, void* stats_pool, void* workspace,
+                        size_t workspace_bytes, cudaStream_t stream) {
   (void)workspace;
   (void)workspace_bytes;
   if (!d || !q || !k || !v || !head_kind_host || !out) return LSERVE_ERR_INVALID_ARG;
@@ -821,6 +1057,26 @@ int prefill_entry(const lserve_prefill_desc* d, const void* q, const void* k, co
       !make_map_3d(&km, k, d->seq_len, d->num_kv_heads, d->head_dim) ||
       !make_map_3d(&vm, v, d->seq_len, d->num_kv_heads, d->head_dim))
     return LSERVE_ERR_CUDA;
+  // paged epilogue: the pools as [rows][D] (3-D: 64 channels, D/64 halves,
+  // rows), box = 64 channels x 1 half x gcd(N_P, 128) rows, 128-byte swizzle
+  // (a box is a row range of one swizzled 128-row box of the stage)
+  CUtensorMap kpm = km, vpm = vm;
+  if (pd) {
+    const uint64_t rows = (uint64_t)pd->num_pool_pages * pd->num_kv_heads * pd->physical_page;
+    const int br = gcd_int(pd->physical_page, kBN);
+    if (!make_map_tiled(&kpm, k_pool, 3, 64, d->head_dim / 64, rows, 64, 1, (uint32_t)br) ||
+        !make_map_tiled(&vpm, v_pool, 3, 64, d->head_dim / 64, rows, 64, 1, (uint32_t)br))
+      return LSERVE_ERR_CUDA;
+    p.pg_k_pool = static_cast<__nv_bfloat16*>(k_pool);
+    p.pg_v_pool = static_cast<__nv_bfloat16*>(v_pool);
+    p.pg_stats = static_cast<__nv_bfloat16*>(stats_pool);
+    p.pg_block_table = block_table;
+    p.pg_np = pd->physical_page;
+    p.pg_nl = pd->logical_page;
+    p.pg_box_rows = br;
+    p.pg_max_pages = pd->max_pages_per_seq;
+    p.pg_num_pool_pages = pd->num_pool_pages;
+  }
   const int sms = current_sm_count();
   if (sms <= 0) return LSERVE_ERR_CUDA;
   const int tiles = (paired ? d->num_q_heads / 2 : d->num_q_heads) * p.n_qt;
@@ -835,23 +1091,23 @@ int prefill_entry(const lserve_prefill_desc* d, const void* q, const void* k, co
       const int smem = std::max(PairLayout<128>::kBytes + 1024, kOneCtaSmem);
       e = set_smem_once((const void*)prefill_pair_kernel<128>, smem);
       if (e != cudaSuccess) return LSERVE_ERR_CUDA;
-      prefill_pair_kernel<128><<<grid, kPairThreads, smem, stream>>>(p, qm, km, vm);
+      prefill_pair_kernel<128><<<grid, kPairThreads, smem, stream>>>(p, qm, km, vm, kpm, vpm);
     } else {
       const int smem = std::max(PairLayout<64>::kBytes + 1024, kOneCtaSmem);
       e = set_smem_once((const void*)prefill_pair_kernel<64>, smem);
       if (e != cudaSuccess) return LSERVE_ERR_CUDA;
-      prefill_pair_kernel<64><<<grid, kPairThreads, smem, stream>>>(p, qm, km, vm);
+      prefill_pair_kernel<64><<<grid, kPairThreads, smem, stream>>>(p, qm, km, vm, kpm, vpm);
     }
   } else if (d->head_dim == 128) {
     const int smem = std::max(Layout<128>::kBytes + 1024, kOneCtaSmem);
     e = set_smem_once((const void*)prefill_kernel<128>, smem);
     if (e != cudaSuccess) return LSERVE_ERR_CUDA;
-    prefill_kernel<128><<<grid, kThreads, smem, stream>>>(p, qm, km, vm);
+    prefill_kernel<128><<<grid, kThreads, smem, stream>>>(p, qm, km, vm, kpm, vpm);
   } else {
     const int smem = std::max(Layout<64>::kBytes + 1024, kOneCtaSmem);
     e = set_smem_once((const void*)prefill_kernel<64>, smem);
     if (e != cudaSuccess) return LSERVE_ERR_CUDA;
-    prefill_kernel<64><<<grid, kThreads, smem, stream>>>(p, qm, km, vm);
+    prefill_kernel<64><<<grid, kThreads, smem, stream>>>(p, qm, km, vm, kpm, vpm);
   }
   return cudaGetLastError() == cudaSuccess ? LSERVE_OK : LSERVE_ERR_CUDA;
 }

@@ -410,6 +410,36 @@ int lserve_blocksparse_prefill(const lserve_prefill_desc* desc, const void* q, c
                                void* stream);
 
 /*
+ * lserve_blocksparse_prefill_paged -- lserve_blocksparse_prefill that also
+ * hands the sequence to the paged decode cache from inside the same kernel:
+ * K / V through the block table into the pools and the retrieval heads' page
+ * statistics (what lserve_prefill_to_pages writes, without its second pass).
+ * [統一ブロックスパースアテンション as lserve_blocksparse_prefill; 階層的ページング:
+ *  logical pages of N_L tokens inside physical pages of N_P tokens; 技術的詳細 ›
+ *  動的スパーシティ: k_min^j / k_max^j of logical page j.]
+ *
+ * desc, q, k, v, head_kind_host, softmax_scale, out, lse, workspace: as
+ * lserve_blocksparse_prefill (out and lse are bit-identical to it).
+ * paged: the cache (batch unused; head_dim and num_kv_heads equal desc's;
+ * N_L, N_P as lserve_page_stats supports); block_table int32
+ * [max_pages_per_seq] of THIS sequence (page ordinal -> pool id), covering
+ * seq_len tokens; k_pool / v_pool bf16 [num_pool_pages][H_kv][N_P][D],
+ * stats_pool bf16 [num_pool_pages][H_kv][g][2][D] (16-byte aligned).  Token t
+ * of KV head h goes to pool id block_table[t / N_P], row t % N_P; rows past
+ * seq_len are not written; retrieval heads (head_kind_host[h] == 0) get the
+ * k_min / k_max of every logical page.  Each key block of 128 tokens is
+ * written by the work tile of its KV head's first query head that ends on it
+ * (the diagonal block), while the block is in shared memory.  A bad pool id
+ * skips that page and sets LSERVE_ERR_BOUNDS.
+ */
+int lserve_blocksparse_prefill_paged(const lserve_prefill_desc* desc, const lserve_paged_desc* paged,
+                                     const void* q, const void* k, const void* v,
+                                     const uint8_t* head_kind_host, float softmax_scale, void* out,
+                                     float* lse, const int32_t* block_table, void* k_pool,
+                                     void* v_pool, void* stats_pool, void* workspace,
+                                     size_t workspace_bytes, void* stream);
+
+/*
  * lserve_page_select_noalloc -- lserve_page_select for callers that cannot
  * allocate device memory.  (The LServe pages have no counterpart: this is a
  * deployment convenience of this library.)

@@ -118,6 +118,31 @@ def test_prefill_rejects_bad_descriptors():
         assert st in (lserve.ERR_INVALID_ARG, lserve.ERR_UNSUPPORTED)
 
 
+def test_prefill_paged_rejects_bad_arguments():
+    # every check precedes a launch: bad paged descriptors, mismatched heads /
+    # head_dim, a table too short for the sequence, null or misaligned pools
+    hk = (ctypes.c_uint8 * 2)(0, 1)
+    d = lserve.prefill_desc(1000, 4, 2, 64, 64, 1, 4)
+    good = lserve.paged_desc(1, 4, 2, 64, 16, 64, 16, 32)
+
+    def call(pd, bt=FAKE, kp=FAKE, vp=FAKE, sp=FAKE, desc=d):
+        return lserve.lib.lserve_blocksparse_prefill_paged(
+            ctypes.byref(desc), ctypes.byref(pd), FAKE, FAKE, FAKE, ctypes.cast(hk, ctypes.c_void_p),
+            0.125, FAKE, None, bt, kp, vp, sp, None, 0, None)
+
+    assert call(lserve.paged_desc(1, 4, 2, 64, 16, 40, 16, 32)) == lserve.ERR_INVALID_ARG  # N_P % N_L
+    assert call(lserve.paged_desc(1, 4, 2, 128, 16, 64, 16, 32)) == lserve.ERR_INVALID_ARG  # head_dim
+    assert call(lserve.paged_desc(1, 4, 4, 64, 16, 64, 16, 32)) == lserve.ERR_INVALID_ARG  # H_kv
+    assert call(lserve.paged_desc(1, 4, 2, 64, 16, 64, 15, 32)) == lserve.ERR_INVALID_ARG  # 15 pages < 1000
+    assert call(lserve.paged_desc(1, 4, 2, 64, 24, 96, 16, 32)) == lserve.ERR_UNSUPPORTED  # N_L = 24
+    assert call(good, bt=None) == lserve.ERR_INVALID_ARG
+    assert call(good, kp=None) == lserve.ERR_INVALID_ARG
+    assert call(good, sp=ctypes.c_void_p(FAKE.value + 8)) == lserve.ERR_INVALID_ARG
+    assert call(good, bt=ctypes.c_void_p(FAKE.value + 2)) == lserve.ERR_INVALID_ARG
+    bad = lserve.prefill_desc(0, 4, 2, 64, 64, 1, 4)
+    assert call(good, desc=bad) in (lserve.ERR_INVALID_ARG, lserve.ERR_UNSUPPORTED)
+
+
 def test_workspace_size_of_select():
     d = _desc()
     assert lserve.workspace_size(lserve.OP_SELECT, d) >= 1 * 2 * 32 * 4
