@@ -11,7 +11,7 @@
 // of the row (all j <= i for dense heads; sink tiles and the local window for
 // streaming heads) -- the block skipping of the method.
 //
-// Warp roles (224 threads):
+// Warp roles (192 threads; 224 in the paged-epilogue variant):
 //   warp 0     TMA producer: Q tile, then K and V tiles into two-stage rings
 //              (3-D tensor maps over [T][H][D], 128-byte swizzle, no multicast)
 //   warp 1     tensor-memory owner and single-thread MMA issuer:
@@ -42,7 +42,7 @@ namespace {
 
 constexpr int kBM = 128;            // query rows per tile (MMA M)
 constexpr int kBN = 128;            // keys per key tile (MMA N of S, K of PV)
-constexpr int kThreads = 224;          // 7 warps; warp 6 writes the paged cache
+constexpr int kThreads = 224;  // 7 warps; warp 6 writes the paged cache (kPaged only)
 constexpr float kRescaleLog2 = 8.0f;  // rescale O only when the max grows by > 2^8
 constexpr int kMaxHeads = 256;
 
@@ -160,10 +160,13 @@ __device__ void page_out(const PrefillParams& p, const CUtensorMap* kpm, const C
     if ((e - a) % BR == 0) {
       if (lane == 0) {
         fence_proxy_async_smem();  // the copies below read what the tile loads wrote
+        // evict-first: the pools are not read again by this kernel, the K / V
+        // tiles that later query tiles re-read should keep their L2 lines
+        const uint64_t pol = l2_policy_evict_first();
         for (int r = a; r < e; r += BR)
           for (int bx = 0; bx < NBOX; ++bx) {
-            tma_store_3d(kpm, 0, bx, (int32_t)(prow + (r - a)), ks + bx * kBoxBytes + r * 128);
-            tma_store_3d(vpm, 0, bx, (int32_t)(prow + (r - a)), vs + bx * kBoxBytes + r * 128);
+            tma_store_3d_hint(kpm, 0, bx, (int32_t)(prow + (r - a)), ks + bx * kBoxBytes + r * 128, pol);
+            tma_store_3d_hint(vpm, 0, bx, (int32_t)(prow + (r - a)), vs + bx * kBoxBytes + r * 128, pol);
           }
       }
       issued = true;
@@ -265,8 +268,8 @@ __device__ void page_writer(const PrefillParams& p, const CUtensorMap* kpm, cons
 
 }  // namespace
 
-template <int D>
-__global__ void __launch_bounds__(kThreads, 1)
+template <int D, bool kPaged>
+__global__ void __launch_bounds__(kPaged ? kThreads : kThreads - 32, 1)
 prefill_kernel(const __grid_constant__ PrefillParams p, const __grid_constant__ CUtensorMap qmap,
                const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
                const __grid_constant__ CUtensorMap kpm, const __grid_constant__ CUtensorMap vpm) {
@@ -292,7 +295,7 @@ prefill_kernel(const __grid_constant__ PrefillParams p, const __grid_constant__ 
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
-    kv_issued[0] = kv_issued[1] = 0u;
+    if (kPaged) kv_issued[0] = kv_issued[1] = 0u;
     mbar_init(q_full, 1);
     mbar_init(q_empty, 1);
     for (int s = 0; s < 2; ++s) {
@@ -302,7 +305,7 @@ prefill_kernel(const __grid_constant__ PrefillParams p, const __grid_constant__ 
       mbar_init(&v_empty[s], 1);
       mbar_init(&s_full[s], 1);
       mbar_init(&s_free[s], 128);
-      mbar_init(&pg_done[s], 1);
+      if (kPaged) mbar_init(&pg_done[s], 1);
     }
     mbar_init(p_full, 128);
     mbar_init(p_free, 1);
@@ -323,11 +326,10 @@ prefill_kernel(const __grid_constant__ PrefillParams p, const __grid_constant__ 
   const int grid = gridDim.x;
   const uint64_t lim = p.wait_limit;
 
-  if (warp == 6) {
+  if (kPaged && warp == 6) {
     // ------------------------------------------------------------ page writer
-    if (p.pg_k_pool)
-      page_writer<D, L>(p, &kpm, &vpm, smem, k_full, v_full, pg_done, kv_issued, total,
-                        [&](int idx) { return tile_at(p, idx); }, lane);
+    page_writer<D, L>(p, &kpm, &vpm, smem, k_full, v_full, pg_done, kv_issued, total,
+                      [&](int idx) { return tile_at(p, idx); }, lane);
   } else if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     // Lane 0 alone; lanes 1-31 of warp 0 do nothing (they must not fall into
@@ -338,7 +340,6 @@ prefill_kernel(const __grid_constant__ PrefillParams p, const __grid_constant__ 
       tma_prefetch_desc(&qmap);
       tma_prefetch_desc(&kmap);
       tma_prefetch_desc(&vmap);
-      const bool paged = p.pg_k_pool != nullptr;
       int q_use = 0, kv_use = 0;
       // stage 0 / 1 holds a diagonal tile the page writer has not released yet;
       // ep0 / ep1 count the writer's releases (the pg_done phases) per stage
@@ -372,7 +373,7 @@ prefill_kernel(const __grid_constant__ PrefillParams p, const __grid_constant__ 
           const int kt = kr.at(j);
           const int s = kv_use & 1, n = kv_use >> 1;
           if (n > 0 && !mbar_wait(&k_empty[s], (n - 1) & 1, lim, p.status)) { ok = false; break; }
-          if ((s ? owe1 : owe0) && !wait_writer(s)) { ok = false; break; }
+          if (kPaged && (s ? owe1 : owe0) && !wait_writer(s)) { ok = false; break; }
           mbar_arrive_expect_tx(&k_full[s], L::kTile);
           for (int bx = 0; bx < NBOX; ++bx)
             tma_load_3d(smem + L::kK + s * L::kTile + bx * L::kBox, &kmap, bx * 64, hkv, kt * kBN,
@@ -382,10 +383,12 @@ prefill_kernel(const __grid_constant__ PrefillParams p, const __grid_constant__ 
           for (int bx = 0; bx < NBOX; ++bx)
             tma_load_3d(smem + L::kV + s * L::kTile + bx * L::kBox, &vmap, bx * 64, hkv, kt * kBN,
                         &v_full[s]);
-          kv_issued[s] = (uint32_t)n + 1;  // for the page writer
-          if (paged && t.hq % p.G == 0 && kt == t.qt) {  // the writer's tile
-            if (s) owe1 = true;
-            else owe0 = true;
+          if (kPaged) {
+            kv_issued[s] = (uint32_t)n + 1;  // for the page writer
+            if (t.hq % p.G == 0 && kt == t.qt) {  // the writer's tile
+              if (s) owe1 = true;
+              else owe0 = true;
+            }
           }
           ++kv_use;
         }
@@ -642,7 +645,7 @@ __device__ __forceinline__ TileRef pair_tile_at(const PrefillParams& p, int idx)
 }
 }  // namespace
 
-template <int D>
+template <int D, bool kPaged>
 __global__ void __launch_bounds__(kPairThreads, 1)
 prefill_pair_kernel(const __grid_constant__ PrefillParams p, const __grid_constant__ CUtensorMap qmap,
                     const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
@@ -668,7 +671,7 @@ prefill_pair_kernel(const __grid_constant__ PrefillParams p, const __grid_consta
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
-    kv_issued[0] = kv_issued[1] = 0u;
+    if (kPaged) kv_issued[0] = kv_issued[1] = 0u;
     mbar_init(q_full, 1);
     mbar_init(q_empty, 1);
     for (int s = 0; s < 2; ++s) {
@@ -680,7 +683,7 @@ prefill_pair_kernel(const __grid_constant__ PrefillParams p, const __grid_consta
       mbar_init(&p_full[s], 128);
       mbar_init(&pv_done[s], 1);
       mbar_init(&o_free[s], 128);
-      mbar_init(&pg_done[s], 1);
+      if (kPaged) mbar_init(&pg_done[s], 1);
     }
     fence_mbar_init();
   }
@@ -703,14 +706,52 @@ prefill_pair_kernel(const __grid_constant__ PrefillParams p, const __grid_consta
 
   if (warp < 4) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kPairRegsCtl));
-    if (warp == 0 && lane == 0) {
+    if (!kPaged && warp == 0 && lane == 0) {
+      // (the kernel without the paged epilogue)
+      // ------------------------------------------------------------ TMA producer
+      tma_prefetch_desc(&qmap);
+      tma_prefetch_desc(&kmap);
+      tma_prefetch_desc(&vmap);
+      int q_use = 0, kv_use = 0;
+      for (int r = 0;; ++r) {
+        const int idx = cta_tile(r, blockIdx.x, grid);
+        if (idx >= total) break;
+        const TileRef t = pair_tile_at(p, idx);  // t.hq: head A, head B = t.hq + 1
+        const int hkv = t.hq / p.G;
+        const KvRange kr = kv_range(p, p.kv_kind[hkv], t.qt);
+        if (q_use > 0 && !mbar_wait(q_empty, (q_use - 1) & 1, lim, p.status)) break;
+        mbar_arrive_expect_tx(q_full, 2 * L::kTile);
+        for (int x = 0; x < 2; ++x)
+          for (int bx = 0; bx < NBOX; ++bx)
+            tma_load_3d(smem + L::kQ + x * L::kTile + bx * L::kBox, &qmap, bx * 64, t.hq + x,
+                        t.qt * kBM, q_full);
+        ++q_use;
+        bool ok = true;
+        const int nkv = kr.count();
+        for (int j = 0; j < nkv && ok; ++j) {
+          const int kt = kr.at(j);
+          const int s = kv_use & 1, n = kv_use >> 1;
+          if (n > 0 && !mbar_wait(&k_empty[s], (n - 1) & 1, lim, p.status)) { ok = false; break; }
+          mbar_arrive_expect_tx(&k_full[s], L::kTile);
+          for (int bx = 0; bx < NBOX; ++bx)
+            tma_load_3d(smem + L::kK + s * L::kTile + bx * L::kBox, &kmap, bx * 64, hkv, kt * kBN,
+                        &k_full[s]);
+          if (n > 0 && !mbar_wait(&v_empty[s], (n - 1) & 1, lim, p.status)) { ok = false; break; }
+          mbar_arrive_expect_tx(&v_full[s], L::kTile);
+          for (int bx = 0; bx < NBOX; ++bx)
+            tma_load_3d(smem + L::kV + s * L::kTile + bx * L::kBox, &vmap, bx * 64, hkv, kt * kBN,
+                        &v_full[s]);
+          ++kv_use;
+        }
+        if (!ok) break;
+      }
+    } else if (kPaged && warp == 0 && lane == 0) {
       // ------------------------------------------------------------ TMA producer
       // A stage holding a diagonal key tile of the paged epilogue is refilled
       // after the page writer (warp 2) releases it, as in prefill_kernel.
       tma_prefetch_desc(&qmap);
       tma_prefetch_desc(&kmap);
       tma_prefetch_desc(&vmap);
-      const bool paged = p.pg_k_pool != nullptr;
       int q_use = 0, kv_use = 0;
       bool owe0 = false, owe1 = false;  // as in prefill_kernel
       int ep0 = 0, ep1 = 0;
@@ -744,7 +785,7 @@ prefill_pair_kernel(const __grid_constant__ PrefillParams p, const __grid_consta
           const int kt = kr.at(j);
           const int s = kv_use & 1, n = kv_use >> 1;
           if (n > 0 && !mbar_wait(&k_empty[s], (n - 1) & 1, lim, p.status)) { ok = false; break; }
-          if ((s ? owe1 : owe0) && !wait_writer(s)) { ok = false; break; }
+          if (kPaged && (s ? owe1 : owe0) && !wait_writer(s)) { ok = false; break; }
           mbar_arrive_expect_tx(&k_full[s], L::kTile);
           for (int bx = 0; bx < NBOX; ++bx)
             tma_load_3d(smem + L::kK + s * L::kTile + bx * L::kBox, &kmap, bx * 64, hkv, kt * kBN,
@@ -754,19 +795,20 @@ prefill_pair_kernel(const __grid_constant__ PrefillParams p, const __grid_consta
           for (int bx = 0; bx < NBOX; ++bx)
             tma_load_3d(smem + L::kV + s * L::kTile + bx * L::kBox, &vmap, bx * 64, hkv, kt * kBN,
                         &v_full[s]);
-          kv_issued[s] = (uint32_t)n + 1;  // for the page writer
-          if (paged && t.hq % p.G == 0 && kt == t.qt) {  // the writer's tile
-            if (s) owe1 = true;
-            else owe0 = true;
+          if (kPaged) {
+            kv_issued[s] = (uint32_t)n + 1;  // for the page writer
+            if (t.hq % p.G == 0 && kt == t.qt) {  // the writer's tile
+              if (s) owe1 = true;
+              else owe0 = true;
+            }
           }
           ++kv_use;
         }
       }
-    } else if (warp == 2) {
+    } else if (kPaged && warp == 2) {
       // ------------------------------------------------------------ page writer
-      if (p.pg_k_pool)
-        page_writer<D, L>(p, &kpm, &vpm, smem, k_full, v_full, pg_done, kv_issued, total,
-                          [&](int idx) { return pair_tile_at(p, idx); }, lane);
+      page_writer<D, L>(p, &kpm, &vpm, smem, k_full, v_full, pg_done, kv_issued, total,
+                        [&](int idx) { return pair_tile_at(p, idx); }, lane);
     } else if (warp == 1 && lane == 0) {
       // ------------------------------------------------------------ MMA issuer
       constexpr uint32_t idesc_s = tc::idesc_bf16_f32(kBM, kBN, false, false);
@@ -1089,25 +1131,29 @@ int prefill_paged_entry(const lserve_prefill_desc* d, const lserve_paged_desc* p
     // 512 tensor-memory columns: one CTA per SM (its shared memory alone guarantees that)
     if (d->head_dim == 128) {
       const int smem = std::max(PairLayout<128>::kBytes + 1024, kOneCtaSmem);
-      e = set_smem_once((const void*)prefill_pair_kernel<128>, smem);
+      e = set_smem_once(pd ? (const void*)prefill_pair_kernel<128, true> : (const void*)prefill_pair_kernel<128, false>, smem);
       if (e != cudaSuccess) return LSERVE_ERR_CUDA;
-      prefill_pair_kernel<128><<<grid, kPairThreads, smem, stream>>>(p, qm, km, vm, kpm, vpm);
+      if (pd) prefill_pair_kernel<128, true><<<grid, kPairThreads, smem, stream>>>(p, qm, km, vm, kpm, vpm);
+      else prefill_pair_kernel<128, false><<<grid, kPairThreads, smem, stream>>>(p, qm, km, vm, kpm, vpm);
     } else {
       const int smem = std::max(PairLayout<64>::kBytes + 1024, kOneCtaSmem);
-      e = set_smem_once((const void*)prefill_pair_kernel<64>, smem);
+      e = set_smem_once(pd ? (const void*)prefill_pair_kernel<64, true> : (const void*)prefill_pair_kernel<64, false>, smem);
       if (e != cudaSuccess) return LSERVE_ERR_CUDA;
-      prefill_pair_kernel<64><<<grid, kPairThreads, smem, stream>>>(p, qm, km, vm, kpm, vpm);
+      if (pd) prefill_pair_kernel<64, true><<<grid, kPairThreads, smem, stream>>>(p, qm, km, vm, kpm, vpm);
+      else prefill_pair_kernel<64, false><<<grid, kPairThreads, smem, stream>>>(p, qm, km, vm, kpm, vpm);
     }
   } else if (d->head_dim == 128) {
     const int smem = std::max(Layout<128>::kBytes + 1024, kOneCtaSmem);
-    e = set_smem_once((const void*)prefill_kernel<128>, smem);
+    e = set_smem_once(pd ? (const void*)prefill_kernel<128, true> : (const void*)prefill_kernel<128, false>, smem);
     if (e != cudaSuccess) return LSERVE_ERR_CUDA;
-    prefill_kernel<128><<<grid, kThreads, smem, stream>>>(p, qm, km, vm, kpm, vpm);
+    if (pd) prefill_kernel<128, true><<<grid, kThreads, smem, stream>>>(p, qm, km, vm, kpm, vpm);
+    else prefill_kernel<128, false><<<grid, kThreads - 32, smem, stream>>>(p, qm, km, vm, kpm, vpm);
   } else {
     const int smem = std::max(Layout<64>::kBytes + 1024, kOneCtaSmem);
-    e = set_smem_once((const void*)prefill_kernel<64>, smem);
+    e = set_smem_once(pd ? (const void*)prefill_kernel<64, true> : (const void*)prefill_kernel<64, false>, smem);
     if (e != cudaSuccess) return LSERVE_ERR_CUDA;
-    prefill_kernel<64><<<grid, kThreads, smem, stream>>>(p, qm, km, vm, kpm, vpm);
+    if (pd) prefill_kernel<64, true><<<grid, kThreads, smem, stream>>>(p, qm, km, vm, kpm, vpm);
+    else prefill_kernel<64, false><<<grid, kThreads - 32, smem, stream>>>(p, qm, km, vm, kpm, vpm);
   }
   return cudaGetLastError() == cudaSuccess ? LSERVE_OK : LSERVE_ERR_CUDA;
 }
