@@ -29,14 +29,16 @@ namespace lserve {
 //   S^j = sum_i Qp[i] * k_max^j[i] + Qn[i] * k_min^j[i]
 // with Qp[i] = sum_h max(q_h[i], 0) and Qn[i] = sum_h min(q_h[i], 0).
 // The stats loads go to shared memory by cp.async (16 bytes per lane and
-// load, each lane to its own slots), not to registers: with 71 registers
-// three blocks fit per SM and ~192 KB of statistics are in flight per SM --
-// staged in registers (127 of them) the kernel held two blocks per SM and
-// reached half the HBM bandwidth.
+// load, each lane to its own slots), not to registers: with 70 registers
+// seven 4-warp blocks (32 KB of staging each) fit per SM and ~224 KB of
+// statistics are in flight per SM; the 8B layer's 1,024 working blocks then
+// run in one wave (eight 8-warp blocks a pair ran in ~1.15 waves and were 3%
+// slower on the 8B layer and the mixed batch).  Staged in registers (127 of
+// them) the kernel held two blocks per SM and reached half the HBM bandwidth.
 constexpr int kScoreSmem = kScoreWarps * kScorePagesPerWarp * kScoreSteps * 2 * 32 * 16;
 
 template <int D, int G>
-__global__ void __launch_bounds__(kScoreWarps * 32, 3)
+__global__ void __launch_bounds__(kScoreWarps * 32, 7)
 page_score_kernel(SelectParams p) {
   constexpr int LPR = D / 8;      // lanes per logical page (16 channels x 8 = 128)
   constexpr int LPI = 32 / LPR;   // logical pages per warp step
