@@ -9,7 +9,7 @@
 namespace lserve {
 
 constexpr int kStatsWarps = 8;   // warps per CTA of the stats kernel
-constexpr int kScoreWarps = 4;   // warps per CTA of the score kernel (7 CTAs per SM)
+constexpr int kScoreWarps = 4;   // warps per CTA of the score kernel (6 CTAs per SM)
 constexpr int kScorePagesPerWarp = 4;
 constexpr int kScoreSteps = 2;        // warp steps (of 32 / (D/8) logical pages) loaded at once
 constexpr int kTopkThreads = 512;

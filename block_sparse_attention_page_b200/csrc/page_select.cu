@@ -30,11 +30,11 @@ namespace lserve {
 // with Qp[i] = sum_h max(q_h[i], 0) and Qn[i] = sum_h min(q_h[i], 0).
 // The stats loads go to shared memory by cp.async (16 bytes per lane and
 // load, each lane to its own slots), not to registers: with 70 registers
-// seven 4-warp blocks (32 KB of staging each) fit per SM and ~224 KB of
-// statistics are in flight per SM; the 8B layer's 1,024 working blocks then
-// run in one wave (eight 8-warp blocks a pair ran in ~1.15 waves and were 3%
-// slower on the 8B layer and the mixed batch).  Staged in registers (127 of
-// them) the kernel held two blocks per SM and reached half the HBM bandwidth.
+// six 4-warp blocks (32 KB of staging each; shared memory is the limit) run
+// per SM with ~192 KB of statistics in flight -- finer blocks than three
+// 8-warp ones with the same bytes in flight: 3% faster on the 8B layer and on
+// the mixed batch.  Staged in registers (127 of them) the kernel held two
+// blocks per SM and reached half the HBM bandwidth.
 constexpr int kScoreSmem = kScoreWarps * kScorePagesPerWarp * kScoreSteps * 2 * 32 * 16;
 
 template <int D, int G>
