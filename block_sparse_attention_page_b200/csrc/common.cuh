@@ -126,28 +126,6 @@ __device__ __forceinline__ void tma_load_3d(void* smem_dst, const CUtensorMap* m
       "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
       : "memory");
 }
-// TMA tiled store from shared memory (bulk-group completion): the 3-D map's
-// box is written at coordinates (x, y, z); x is 0 here.  commit + wait_read
-// make the source shared memory reusable, wait_all the writes complete.
-__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, int32_t x, int32_t y, int32_t z,
-                                             const void* smem_src) {
-  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.tile.bulk_group [%0, {%1, %2, %3}], [%4];"
-               ::"l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(smem_src))
-               : "memory");
-}
-__device__ __forceinline__ void tma_store_3d_hint(const CUtensorMap* map, int32_t x, int32_t y,
-                                                  int32_t z, const void* smem_src, uint64_t policy) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.global.shared::cta.tile.bulk_group.L2::cache_hint"
-      " [%0, {%1, %2, %3}], [%4], %5;" ::"l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z),
-      "r"(smem_u32(smem_src)), "l"(policy)
-      : "memory");
-}
-__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void bulk_wait_read() {
-  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
-}
-__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 // L2 policy for data read exactly once (the KV tiles of a decode step): its
 // lines are the first to go, so the small metadata arrays, q and the split
 // partials that every launch re-reads stay in L2.

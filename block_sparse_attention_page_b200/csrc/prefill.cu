@@ -22,9 +22,9 @@
 //              bf16 into shared memory (swizzled like a TMA tile), rescales O
 //              in TMEM only when the row max grows by more than 2^8, and runs
 //              the epilogue O / l -> bf16 and the log-sum-exp.
-//   warp 6     page writer (lserve_blocksparse_prefill_paged only): the
-//              diagonal key tile of each KV head into the paged pools and the
-//              page statistics, while the tile is in its ring stage.
+//   warp 6     page writer (lserve_blocksparse_prefill_paged only): each key
+//              tile of a KV head into the paged pools and its page
+//              statistics, read from the kernel's own K / V inputs.
 // MMA order S_0, S_1, PV_0, S_2, PV_1, ... keeps the tensor core on S_{j+1}
 // while the softmax warps work on S_j.
 #include <algorithm>
@@ -63,12 +63,14 @@ struct PrefillParams {
   int n_dense_pairs, n_stream_pairs;
   uint8_t dense_pairs[kMaxHeads / 2];
   uint8_t stream_pairs[kMaxHeads / 2];
-  // paged epilogue (lserve_blocksparse_prefill_paged; pg_k_pool == nullptr: none)
+  // paged epilogue (lserve_blocksparse_prefill_paged only)
+  const __nv_bfloat16* pg_k_in;   // the prefill's K and V, [T][H_kv][D]
+  const __nv_bfloat16* pg_v_in;
   __nv_bfloat16* pg_k_pool;
   __nv_bfloat16* pg_v_pool;
   __nv_bfloat16* pg_stats;
   const int32_t* pg_block_table;  // this sequence's page ordinal -> pool id
-  int pg_np, pg_nl, pg_box_rows, pg_max_pages, pg_num_pool_pages;
+  int pg_np, pg_nl, pg_max_pages, pg_num_pool_pages;
 };
 
 template <int D>
@@ -80,7 +82,7 @@ struct Layout {
   static constexpr int kV = kK + 2 * kTile;       // 2 stages
   static constexpr int kP = kV + 2 * kTile;       // P: 128 x 128 bf16, 2 boxes
   static constexpr int kBar = kP + 2 * kBox;
-  static constexpr int kNumBars = 19;
+  static constexpr int kNumBars = 17;
   static constexpr int kBytes = kBar + kNumBars * 8 + 16;
 };
 
@@ -122,148 +124,91 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, uint64
   return __all_sync(0xffffffffu, ok);
 }
 
-// Paged epilogue of one key tile (row kt of KV head h), run by the whole
-// producer warp while the tile is still in its ring stage: K and V rows
-// [kt*kBN, min(kt*kBN + kBN, T)) go to the pools through the block table --
-// whole boxes of pg_box_rows rows by TMA stores, the rows of a page that the
-// sequence fills only partly by plain stores of its valid rows -- and, for a
-// retrieval head, every logical page of the tile gets the bf16 min / max of
-// its valid keys per channel (the same values lserve_page_stats and
-// lserve_prefill_to_pages write).  Returns after the TMA stores have read the
-// stage.  ks / vs: the stage's K and V tiles (NBOX swizzled 128-row boxes).
+// Paged epilogue of key tile kt of KV head h, run by one warp: the rows
+// [kt*kBN, min(kt*kBN + kBN, T)) of the prefill's K and V go to their pool
+// rows through the block table, and for a retrieval head every logical page
+// of the tile gets the bf16 min / max of its keys per channel (the values
+// lserve_page_stats and lserve_prefill_to_pages write).  The rows are read
+// from the kernel's own K / V inputs -- the tile loads of this kernel keep
+// them in L2 -- with plain 16-byte loads (D/8 lanes a row, 32 / (D/8) rows a
+// step) and stored the same way, so the writer never holds a ring stage and
+// waits on nothing.
 template <int D>
-__device__ void page_out(const PrefillParams& p, const CUtensorMap* kpm, const CUtensorMap* vpm,
-                         const uint8_t* ks, const uint8_t* vs, int kt, int h, int lane) {
-  constexpr int NBOX = D / 64;
-  constexpr int kBoxBytes = kBM * 128;
-  constexpr int CPL = D / 32;  // channels of a lane in the statistics (4 or 2)
+__device__ void page_out(const PrefillParams& p, int kt, int h, int lane) {
+  constexpr int LPR = D / 8;     // lanes per row
+  constexpr int RPI = 32 / LPR;  // rows of one warp-wide step
   const int t0 = kt * kBN, tend = min(t0 + kBN, p.T);
-  const int NP = p.pg_np, NL = p.pg_nl, BR = p.pg_box_rows, g = NP / NL;
-  // byte offset of channel c of tile row r in a stage (128-byte swizzle per box)
-  auto off = [&](int r, int c) {
-    const int chunk = (c % 64) / 8;
-    return (uint32_t)((c / 64) * kBoxBytes + r * 128 + ((chunk ^ (r & 7)) << 4) + (c % 8) * 2);
-  };
-  bool issued = false;
-  // the tile's block-table entries (at most kBN / 32 pages), one lane each, in one round trip
+  const int NP = p.pg_np, NL = p.pg_nl, g = NP / NL;
+  const int r0 = lane / LPR, c = (lane % LPR) * 8;
+  const size_t src_stride = (size_t)p.H_kv * D;  // between tokens of [T][H_kv][D]
+  // the tile's block-table entries (at most kBN / 32 pages), one lane each
   const int m0 = t0 / NP;
   int pid_l = -1;
   if (m0 + lane < p.pg_max_pages && (m0 + lane) * NP < tend) pid_l = p.pg_block_table[m0 + lane];
-  for (int m = m0; m * NP < tend; ++m) {
-    const int a = max(t0, m * NP) - t0, e = min(tend, (m + 1) * NP) - t0;  // tile rows [a, e)
+  const uint32_t kPosInf2 = 0x7F807F80u, kNegInf2 = 0xFF80FF80u;
+  for (int lp = t0 / NL; lp * NL < tend; ++lp) {  // logical pages of the tile (N_L divides kBN)
+    const int m = lp / g, sub = lp - m * g;
     const int pid = __shfl_sync(0xffffffffu, pid_l, m - m0);
-    if (pid < 0 || pid >= p.pg_num_pool_pages) {
+    if (pid < 0 || pid >= p.pg_num_pool_pages) {  // bad entry: the page is skipped and flagged
       if (lane == 0) raise_status(p.status, LSERVE_ERR_BOUNDS);
       continue;
     }
-    const size_t prow = ((size_t)pid * p.H_kv + h) * NP + (size_t)(t0 + a - m * NP);  // pool row of a
-    if ((e - a) % BR == 0) {
-      if (lane == 0) {
-        fence_proxy_async_smem();  // the copies below read what the tile loads wrote
-        // evict-first: the pools are not read again by this kernel, the K / V
-        // tiles that later query tiles re-read should keep their L2 lines
-        const uint64_t pol = l2_policy_evict_first();
-        for (int r = a; r < e; r += BR)
-          for (int bx = 0; bx < NBOX; ++bx) {
-            tma_store_3d_hint(kpm, 0, bx, (int32_t)(prow + (r - a)), ks + bx * kBoxBytes + r * 128, pol);
-            tma_store_3d_hint(vpm, 0, bx, (int32_t)(prow + (r - a)), vs + bx * kBoxBytes + r * 128, pol);
-          }
-      }
-      issued = true;
-    } else {  // the sequence's last, partly filled page: its valid rows
-      for (int i = lane; i < (e - a) * (D / 8); i += 32) {
-        const int r = a + i / (D / 8), c = (i % (D / 8)) * 8;
-        const size_t dst = (prow + (size_t)(r - a)) * D + c;
-        *reinterpret_cast<uint4*>(p.pg_k_pool + dst) = *reinterpret_cast<const uint4*>(ks + off(r, c));
-        *reinterpret_cast<uint4*>(p.pg_v_pool + dst) = *reinterpret_cast<const uint4*>(vs + off(r, c));
+    const int valid = min(NL, tend - lp * NL);
+    const size_t src0 = (size_t)lp * NL * src_stride + (size_t)h * D + c;
+    const size_t dst0 = (((size_t)pid * p.H_kv + h) * NP + (size_t)sub * NL) * D + c;
+    __nv_bfloat162 mn[4], mx[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      mn[k] = *reinterpret_cast<const __nv_bfloat162*>(&kPosInf2);
+      mx[k] = *reinterpret_cast<const __nv_bfloat162*>(&kNegInf2);
+    }
+    for (int r = r0; r < valid; r += RPI) {
+      const uint4 kr = ldg_nc_v4(p.pg_k_in + src0 + (size_t)r * src_stride);
+      const uint4 vr = ldg_nc_v4(p.pg_v_in + src0 + (size_t)r * src_stride);
+      *reinterpret_cast<uint4*>(p.pg_k_pool + dst0 + (size_t)r * D) = kr;
+      *reinterpret_cast<uint4*>(p.pg_v_pool + dst0 + (size_t)r * D) = vr;
+      const __nv_bfloat162* v = reinterpret_cast<const __nv_bfloat162*>(&kr);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        mn[k] = __hmin2(mn[k], v[k]);
+        mx[k] = __hmax2(mx[k], v[k]);
       }
     }
     if (p.kv_kind[h] != 0) continue;  // streaming heads need no statistics
-    for (int lp = (t0 + a) / NL; lp * NL < t0 + e; ++lp) {
-      const int ra = lp * NL - t0, rb = min((lp + 1) * NL, tend) - t0;
-      const uint32_t kPosInf2 = 0x7F807F80u, kNegInf2 = 0xFF80FF80u;
-      __nv_bfloat162 mn[CPL / 2], mx[CPL / 2];
+    // reduce over the row groups of the warp (lanes holding the same channels)
 #pragma unroll
-      for (int k = 0; k < CPL / 2; ++k) {
-        mn[k] = *reinterpret_cast<const __nv_bfloat162*>(&kPosInf2);
-        mx[k] = *reinterpret_cast<const __nv_bfloat162*>(&kNegInf2);
-      }
-      for (int r = ra; r < rb; ++r) {
+    for (int o = LPR; o < 32; o <<= 1) {
 #pragma unroll
-        for (int k = 0; k < CPL / 2; ++k) {
-          const __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162*>(ks + off(r, lane * CPL + 2 * k));
-          mn[k] = __hmin2(mn[k], v);
-          mx[k] = __hmax2(mx[k], v);
-        }
-      }
-      __nv_bfloat16* st = p.pg_stats + ((((size_t)pid * p.H_kv + h) * g) + (lp - m * g)) * 2 * D + lane * CPL;
-#pragma unroll
-      for (int k = 0; k < CPL / 2; ++k) {
-        reinterpret_cast<__nv_bfloat162*>(st)[k] = mn[k];
-        reinterpret_cast<__nv_bfloat162*>(st + D)[k] = mx[k];
+      for (int k = 0; k < 4; ++k) {
+        uint32_t a = *reinterpret_cast<uint32_t*>(&mn[k]);
+        uint32_t z = *reinterpret_cast<uint32_t*>(&mx[k]);
+        a = __shfl_xor_sync(0xffffffffu, a, o);
+        z = __shfl_xor_sync(0xffffffffu, z, o);
+        mn[k] = __hmin2(mn[k], *reinterpret_cast<__nv_bfloat162*>(&a));
+        mx[k] = __hmax2(mx[k], *reinterpret_cast<__nv_bfloat162*>(&z));
       }
     }
+    if (r0 == 0) {
+      __nv_bfloat16* st = p.pg_stats + ((((size_t)pid * p.H_kv + h) * g) + sub) * 2 * D + c;
+      *reinterpret_cast<uint4*>(st) = *reinterpret_cast<uint4*>(mn);
+      *reinterpret_cast<uint4*>(st + D) = *reinterpret_cast<uint4*>(mx);
+    }
   }
-  if (issued && lane == 0) {
-    bulk_commit();
-    bulk_wait_read();  // the stage may be refilled
-  }
-  __syncwarp();
 }
 
-// The page writer warp: follows the CTA's work tiles as the producer deals
-// them (the same tile order and key-tile counts), and for every tile of a KV
-// head's first query head writes the pages of its diagonal key tile -- the
-// row's last key tile -- as soon as that tile's K and V have landed, then
-// arrives on pg_done[stage].  The producer waits on pg_done before it refills
-// that stage, so the tile stays in shared memory until it is written.  The
-// MMA and softmax warps never wait on it.
-// kv_issued[s]: fills of stage s the producer has issued.  A parity wait only
-// tells phases apart within one phase of the barrier's current one, so the
-// writer (which may run ahead of the producer) first waits until its tile's
-// fill has been issued; the producer cannot refill the stage after it until
-// the writer releases it, so that fill's phase is then the barrier's current
-// or just-completed one.
-template <int D, typename L, typename TileAt>
-__device__ void page_writer(const PrefillParams& p, const CUtensorMap* kpm, const CUtensorMap* vpm,
-                            uint8_t* smem, uint64_t* k_full, uint64_t* v_full, uint64_t* pg_done,
-                            const volatile uint32_t* kv_issued, int total, TileAt tile_of, int lane) {
-  const uint64_t lim = p.wait_limit;
-  // waits by lane 0 alone (the other lanes idle at the broadcast)
-  auto wait_issued = [&](int s, uint32_t want) -> bool {
-    bool ok = true;
-    if (lane == 0) {
-      const long long t0 = clock64();
-      while (kv_issued[s] < want) {
-        if ((uint64_t)(clock64() - t0) > lim) {
-          raise_status(p.status, LSERVE_ERR_TIMEOUT);
-          ok = false;
-          break;
-        }
-      }
-    }
-    return __shfl_sync(0xffffffffu, ok, 0);
-  };
-  auto wait1 = [&](uint64_t* bar, uint32_t parity) -> bool {
-    bool ok = true;
-    if (lane == 0) ok = mbar_wait(bar, parity, lim, p.status);
-    return __shfl_sync(0xffffffffu, ok, 0);
-  };
-  int kv_use = 0;
+// The page writer warp: follows the CTA's work tiles (the producer's order)
+// and, for every tile of a KV head's first query head, writes the pages of
+// its diagonal key tile -- each key tile of a head is the diagonal tile of
+// exactly one such work tile.  It reads only the kernel's inputs and writes
+// only the paged cache, so nothing else in the kernel waits on it.
+template <int D, typename TileAt>
+__device__ void page_writer(const PrefillParams& p, int total, TileAt tile_of, int lane) {
   for (int r = 0;; ++r) {
     const int idx = cta_tile(r, blockIdx.x, gridDim.x);
     if (idx >= total) break;
     const TileRef t = tile_of(idx);
-    const int hkv = t.hq / p.G;
-    kv_use += kv_range(p, p.kv_kind[hkv], t.qt).count();
-    if (t.hq % p.G != 0) continue;
-    const int kvi = kv_use - 1, s = kvi & 1, n = kvi >> 1;
-    if (!wait_issued(s, (uint32_t)n + 1) || !wait1(&k_full[s], n & 1) || !wait1(&v_full[s], n & 1))
-      break;
-    page_out<D>(p, kpm, vpm, smem + L::kK + s * L::kTile, smem + L::kV + s * L::kTile, t.qt, hkv, lane);
-    if (lane == 0) mbar_arrive(&pg_done[s]);
+    if (t.hq % p.G == 0) page_out<D>(p, t.qt, t.hq / p.G, lane);
   }
-  if (lane == 0) bulk_wait_all();  // the pools' TMA writes are complete
 }
 
 }  // namespace
@@ -271,8 +216,7 @@ __device__ void page_writer(const PrefillParams& p, const CUtensorMap* kpm, cons
 template <int D, bool kPaged>
 __global__ void __launch_bounds__(kPaged ? kThreads : kThreads - 32, 1)
 prefill_kernel(const __grid_constant__ PrefillParams p, const __grid_constant__ CUtensorMap qmap,
-               const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
-               const __grid_constant__ CUtensorMap kpm, const __grid_constant__ CUtensorMap vpm) {
+               const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap) {
   using L = Layout<D>;
   constexpr int NBOX = D / 64;
   extern __shared__ uint8_t smem_raw[];
@@ -289,13 +233,10 @@ prefill_kernel(const __grid_constant__ PrefillParams p, const __grid_constant__ 
   uint64_t* p_full = bars + 14;
   uint64_t* p_free = bars + 15;
   uint64_t* o_free = bars + 16;
-  uint64_t* pg_done = bars + 17;  // [2]: the page writer is done with the stage's tile
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::kBar + L::kNumBars * 8);
-  volatile uint32_t* kv_issued = tmem_holder + 1;  // [2]: fills of each stage issued
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
-    if (kPaged) kv_issued[0] = kv_issued[1] = 0u;
     mbar_init(q_full, 1);
     mbar_init(q_empty, 1);
     for (int s = 0; s < 2; ++s) {
@@ -305,7 +246,6 @@ prefill_kernel(const __grid_constant__ PrefillParams p, const __grid_constant__ 
       mbar_init(&v_empty[s], 1);
       mbar_init(&s_full[s], 1);
       mbar_init(&s_free[s], 128);
-      if (kPaged) mbar_init(&pg_done[s], 1);
     }
     mbar_init(p_full, 128);
     mbar_init(p_free, 1);
@@ -328,36 +268,15 @@ prefill_kernel(const __grid_constant__ PrefillParams p, const __grid_constant__ 
 
   if (kPaged && warp == 6) {
     // ------------------------------------------------------------ page writer
-    page_writer<D, L>(p, &kpm, &vpm, smem, k_full, v_full, pg_done, kv_issued, total,
-                      [&](int idx) { return tile_at(p, idx); }, lane);
+    page_writer<D>(p, total, [&](int idx) { return tile_at(p, idx); }, lane);
   } else if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
-    // Lane 0 alone; lanes 1-31 of warp 0 do nothing (they must not fall into
-    // the softmax branch below).  With the paged epilogue, a stage that holds
-    // a KV head's diagonal key tile (visited once, by the group's first query
-    // head) is refilled only after the page writer has released it.
     if (lane == 0) {
       tma_prefetch_desc(&qmap);
       tma_prefetch_desc(&kmap);
       tma_prefetch_desc(&vmap);
       int q_use = 0, kv_use = 0;
-      // stage 0 / 1 holds a diagonal tile the page writer has not released yet;
-      // ep0 / ep1 count the writer's releases (the pg_done phases) per stage
-      bool owe0 = false, owe1 = false;
-      int ep0 = 0, ep1 = 0;
-      auto wait_writer = [&](int s) -> bool {
-        if (!mbar_wait(&pg_done[s], (s ? ep1 : ep0) & 1, lim, p.status)) return false;
-        if (s) {
-          ++ep1;
-          owe1 = false;
-        } else {
-          ++ep0;
-          owe0 = false;
-        }
-        return true;
-      };
-      bool ok = true;
-      for (int r = 0; ok; ++r) {
+      for (int r = 0;; ++r) {
         const int idx = cta_tile(r, blockIdx.x, grid);
         if (idx >= total) break;
         const TileRef t = tile_at(p, idx);
@@ -368,12 +287,12 @@ prefill_kernel(const __grid_constant__ PrefillParams p, const __grid_constant__ 
         for (int bx = 0; bx < NBOX; ++bx)
           tma_load_3d(smem + L::kQ + bx * L::kBox, &qmap, bx * 64, t.hq, t.qt * kBM, q_full);
         ++q_use;
+        bool ok = true;
         const int nkv = kr.count();
         for (int j = 0; j < nkv && ok; ++j) {
           const int kt = kr.at(j);
           const int s = kv_use & 1, n = kv_use >> 1;
           if (n > 0 && !mbar_wait(&k_empty[s], (n - 1) & 1, lim, p.status)) { ok = false; break; }
-          if (kPaged && (s ? owe1 : owe0) && !wait_writer(s)) { ok = false; break; }
           mbar_arrive_expect_tx(&k_full[s], L::kTile);
           for (int bx = 0; bx < NBOX; ++bx)
             tma_load_3d(smem + L::kK + s * L::kTile + bx * L::kBox, &kmap, bx * 64, hkv, kt * kBN,
@@ -383,15 +302,9 @@ prefill_kernel(const __grid_constant__ PrefillParams p, const __grid_constant__ 
           for (int bx = 0; bx < NBOX; ++bx)
             tma_load_3d(smem + L::kV + s * L::kTile + bx * L::kBox, &vmap, bx * 64, hkv, kt * kBN,
                         &v_full[s]);
-          if (kPaged) {
-            kv_issued[s] = (uint32_t)n + 1;  // for the page writer
-            if (t.hq % p.G == 0 && kt == t.qt) {  // the writer's tile
-              if (s) owe1 = true;
-              else owe0 = true;
-            }
-          }
           ++kv_use;
         }
+        if (!ok) break;
       }
     }
   } else if (warp == 1) {
@@ -633,7 +546,7 @@ struct PairLayout {
   static constexpr int kK = kQ + 2 * kTile;     // 2 stages
   static constexpr int kV = kK + 2 * kTile;     // 2 stages
   static constexpr int kBar = kV + 2 * kTile;
-  static constexpr int kNumBars = 21;
+  static constexpr int kNumBars = 19;
   static constexpr int kBytes = kBar + kNumBars * 8 + 16;
 };
 
@@ -648,8 +561,7 @@ __device__ __forceinline__ TileRef pair_tile_at(const PrefillParams& p, int idx)
 template <int D, bool kPaged>
 __global__ void __launch_bounds__(kPairThreads, 1)
 prefill_pair_kernel(const __grid_constant__ PrefillParams p, const __grid_constant__ CUtensorMap qmap,
-                    const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
-                    const __grid_constant__ CUtensorMap kpm, const __grid_constant__ CUtensorMap vpm) {
+                    const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap) {
   using L = PairLayout<D>;
   constexpr int NBOX = D / 64;
   extern __shared__ uint8_t smem_raw[];
@@ -665,13 +577,10 @@ prefill_pair_kernel(const __grid_constant__ PrefillParams p, const __grid_consta
   uint64_t* p_full = bars + 12;   // [head]
   uint64_t* pv_done = bars + 14;  // [head]: the tile's last PV has completed
   uint64_t* o_free = bars + 16;   // [head]: the epilogue has read O
-  uint64_t* pg_done = bars + 19;  // [2]: the page writer is done with the stage's tile
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::kBar + L::kNumBars * 8);
-  volatile uint32_t* kv_issued = tmem_holder + 1;  // [2]: fills of each stage issued
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
-    if (kPaged) kv_issued[0] = kv_issued[1] = 0u;
     mbar_init(q_full, 1);
     mbar_init(q_empty, 1);
     for (int s = 0; s < 2; ++s) {
@@ -683,7 +592,6 @@ prefill_pair_kernel(const __grid_constant__ PrefillParams p, const __grid_consta
       mbar_init(&p_full[s], 128);
       mbar_init(&pv_done[s], 1);
       mbar_init(&o_free[s], 128);
-      if (kPaged) mbar_init(&pg_done[s], 1);
     }
     fence_mbar_init();
   }
@@ -706,8 +614,7 @@ prefill_pair_kernel(const __grid_constant__ PrefillParams p, const __grid_consta
 
   if (warp < 4) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kPairRegsCtl));
-    if (!kPaged && warp == 0 && lane == 0) {
-      // (the kernel without the paged epilogue)
+    if (warp == 0 && lane == 0) {
       // ------------------------------------------------------------ TMA producer
       tma_prefetch_desc(&qmap);
       tma_prefetch_desc(&kmap);
@@ -745,70 +652,9 @@ prefill_pair_kernel(const __grid_constant__ PrefillParams p, const __grid_consta
         }
         if (!ok) break;
       }
-    } else if (kPaged && warp == 0 && lane == 0) {
-      // ------------------------------------------------------------ TMA producer
-      // A stage holding a diagonal key tile of the paged epilogue is refilled
-      // after the page writer (warp 2) releases it, as in prefill_kernel.
-      tma_prefetch_desc(&qmap);
-      tma_prefetch_desc(&kmap);
-      tma_prefetch_desc(&vmap);
-      int q_use = 0, kv_use = 0;
-      bool owe0 = false, owe1 = false;  // as in prefill_kernel
-      int ep0 = 0, ep1 = 0;
-      auto wait_writer = [&](int s) -> bool {
-        if (!mbar_wait(&pg_done[s], (s ? ep1 : ep0) & 1, lim, p.status)) return false;
-        if (s) {
-          ++ep1;
-          owe1 = false;
-        } else {
-          ++ep0;
-          owe0 = false;
-        }
-        return true;
-      };
-      bool ok = true;
-      for (int r = 0; ok; ++r) {
-        const int idx = cta_tile(r, blockIdx.x, grid);
-        if (idx >= total) break;
-        const TileRef t = pair_tile_at(p, idx);  // t.hq: head A, head B = t.hq + 1
-        const int hkv = t.hq / p.G;
-        const KvRange kr = kv_range(p, p.kv_kind[hkv], t.qt);
-        if (q_use > 0 && !mbar_wait(q_empty, (q_use - 1) & 1, lim, p.status)) break;
-        mbar_arrive_expect_tx(q_full, 2 * L::kTile);
-        for (int x = 0; x < 2; ++x)
-          for (int bx = 0; bx < NBOX; ++bx)
-            tma_load_3d(smem + L::kQ + x * L::kTile + bx * L::kBox, &qmap, bx * 64, t.hq + x,
-                        t.qt * kBM, q_full);
-        ++q_use;
-        const int nkv = kr.count();
-        for (int j = 0; j < nkv && ok; ++j) {
-          const int kt = kr.at(j);
-          const int s = kv_use & 1, n = kv_use >> 1;
-          if (n > 0 && !mbar_wait(&k_empty[s], (n - 1) & 1, lim, p.status)) { ok = false; break; }
-          if (kPaged && (s ? owe1 : owe0) && !wait_writer(s)) { ok = false; break; }
-          mbar_arrive_expect_tx(&k_full[s], L::kTile);
-          for (int bx = 0; bx < NBOX; ++bx)
-            tma_load_3d(smem + L::kK + s * L::kTile + bx * L::kBox, &kmap, bx * 64, hkv, kt * kBN,
-                        &k_full[s]);
-          if (n > 0 && !mbar_wait(&v_empty[s], (n - 1) & 1, lim, p.status)) { ok = false; break; }
-          mbar_arrive_expect_tx(&v_full[s], L::kTile);
-          for (int bx = 0; bx < NBOX; ++bx)
-            tma_load_3d(smem + L::kV + s * L::kTile + bx * L::kBox, &vmap, bx * 64, hkv, kt * kBN,
-                        &v_full[s]);
-          if (kPaged) {
-            kv_issued[s] = (uint32_t)n + 1;  // for the page writer
-            if (t.hq % p.G == 0 && kt == t.qt) {  // the writer's tile
-              if (s) owe1 = true;
-              else owe0 = true;
-            }
-          }
-          ++kv_use;
-        }
-      }
     } else if (kPaged && warp == 2) {
       // ------------------------------------------------------------ page writer
-      page_writer<D, L>(p, &kpm, &vpm, smem, k_full, v_full, pg_done, kv_issued, total,
-                        [&](int idx) { return pair_tile_at(p, idx); }, lane);
+      page_writer<D>(p, total, [&](int idx) { return pair_tile_at(p, idx); }, lane);
     } else if (warp == 1 && lane == 0) {
       // ------------------------------------------------------------ MMA issuer
       constexpr uint32_t idesc_s = tc::idesc_bf16_f32(kBM, kBN, false, false);
@@ -1030,15 +876,6 @@ int prefill_entry(const lserve_prefill_desc* d, const void* q, const void* k, co
                              nullptr, nullptr, nullptr, workspace, workspace_bytes, stream);
 }
 
-static int gcd_int(int a, int b) {
-  while (b) {
-    const int t = a % b;
-    a = b;
-    b = t;
-  }
-  return a;
-}
-
 int prefill_paged_entry(const lserve_prefill_desc* d, const lserve_paged_desc* pd, const void* q,
                         const void* k, const void* v, const uint8_t* head_kind_host,
                         float softmax_scale, void* out, float* lse, const int32_t* block_table,
@@ -1099,23 +936,15 @@ int prefill_paged_entry(const lserve_prefill_desc* d, const lserve_paged_desc* p
       !make_map_3d(&km, k, d->seq_len, d->num_kv_heads, d->head_dim) ||
       !make_map_3d(&vm, v, d->seq_len, d->num_kv_heads, d->head_dim))
     return LSERVE_ERR_CUDA;
-  // paged epilogue: the pools as [rows][D] (3-D: 64 channels, D/64 halves,
-  // rows), box = 64 channels x 1 half x gcd(N_P, 128) rows, 128-byte swizzle
-  // (a box is a row range of one swizzled 128-row box of the stage)
-  CUtensorMap kpm = km, vpm = vm;
   if (pd) {
-    const uint64_t rows = (uint64_t)pd->num_pool_pages * pd->num_kv_heads * pd->physical_page;
-    const int br = gcd_int(pd->physical_page, kBN);
-    if (!make_map_tiled(&kpm, k_pool, 3, 64, d->head_dim / 64, rows, 64, 1, (uint32_t)br) ||
-        !make_map_tiled(&vpm, v_pool, 3, 64, d->head_dim / 64, rows, 64, 1, (uint32_t)br))
-      return LSERVE_ERR_CUDA;
+    p.pg_k_in = static_cast<const __nv_bfloat16*>(k);
+    p.pg_v_in = static_cast<const __nv_bfloat16*>(v);
     p.pg_k_pool = static_cast<__nv_bfloat16*>(k_pool);
     p.pg_v_pool = static_cast<__nv_bfloat16*>(v_pool);
     p.pg_stats = static_cast<__nv_bfloat16*>(stats_pool);
     p.pg_block_table = block_table;
     p.pg_np = pd->physical_page;
     p.pg_nl = pd->logical_page;
-    p.pg_box_rows = br;
     p.pg_max_pages = pd->max_pages_per_seq;
     p.pg_num_pool_pages = pd->num_pool_pages;
   }
@@ -1133,27 +962,27 @@ int prefill_paged_entry(const lserve_prefill_desc* d, const lserve_paged_desc* p
       const int smem = std::max(PairLayout<128>::kBytes + 1024, kOneCtaSmem);
       e = set_smem_once(pd ? (const void*)prefill_pair_kernel<128, true> : (const void*)prefill_pair_kernel<128, false>, smem);
       if (e != cudaSuccess) return LSERVE_ERR_CUDA;
-      if (pd) prefill_pair_kernel<128, true><<<grid, kPairThreads, smem, stream>>>(p, qm, km, vm, kpm, vpm);
-      else prefill_pair_kernel<128, false><<<grid, kPairThreads, smem, stream>>>(p, qm, km, vm, kpm, vpm);
+      if (pd) prefill_pair_kernel<128, true><<<grid, kPairThreads, smem, stream>>>(p, qm, km, vm);
+      else prefill_pair_kernel<128, false><<<grid, kPairThreads, smem, stream>>>(p, qm, km, vm);
     } else {
       const int smem = std::max(PairLayout<64>::kBytes + 1024, kOneCtaSmem);
       e = set_smem_once(pd ? (const void*)prefill_pair_kernel<64, true> : (const void*)prefill_pair_kernel<64, false>, smem);
       if (e != cudaSuccess) return LSERVE_ERR_CUDA;
-      if (pd) prefill_pair_kernel<64, true><<<grid, kPairThreads, smem, stream>>>(p, qm, km, vm, kpm, vpm);
-      else prefill_pair_kernel<64, false><<<grid, kPairThreads, smem, stream>>>(p, qm, km, vm, kpm, vpm);
+      if (pd) prefill_pair_kernel<64, true><<<grid, kPairThreads, smem, stream>>>(p, qm, km, vm);
+      else prefill_pair_kernel<64, false><<<grid, kPairThreads, smem, stream>>>(p, qm, km, vm);
     }
   } else if (d->head_dim == 128) {
     const int smem = std::max(Layout<128>::kBytes + 1024, kOneCtaSmem);
     e = set_smem_once(pd ? (const void*)prefill_kernel<128, true> : (const void*)prefill_kernel<128, false>, smem);
     if (e != cudaSuccess) return LSERVE_ERR_CUDA;
-    if (pd) prefill_kernel<128, true><<<grid, kThreads, smem, stream>>>(p, qm, km, vm, kpm, vpm);
-    else prefill_kernel<128, false><<<grid, kThreads - 32, smem, stream>>>(p, qm, km, vm, kpm, vpm);
+    if (pd) prefill_kernel<128, true><<<grid, kThreads, smem, stream>>>(p, qm, km, vm);
+    else prefill_kernel<128, false><<<grid, kThreads - 32, smem, stream>>>(p, qm, km, vm);
   } else {
     const int smem = std::max(Layout<64>::kBytes + 1024, kOneCtaSmem);
     e = set_smem_once(pd ? (const void*)prefill_kernel<64, true> : (const void*)prefill_kernel<64, false>, smem);
     if (e != cudaSuccess) return LSERVE_ERR_CUDA;
-    if (pd) prefill_kernel<64, true><<<grid, kThreads, smem, stream>>>(p, qm, km, vm, kpm, vpm);
-    else prefill_kernel<64, false><<<grid, kThreads - 32, smem, stream>>>(p, qm, km, vm, kpm, vpm);
+    if (pd) prefill_kernel<64, true><<<grid, kThreads, smem, stream>>>(p, qm, km, vm);
+    else prefill_kernel<64, false><<<grid, kThreads - 32, smem, stream>>>(p, qm, km, vm);
   }
   return cudaGetLastError() == cudaSuccess ? LSERVE_OK : LSERVE_ERR_CUDA;
 }

@@ -427,10 +427,10 @@ int lserve_blocksparse_prefill(const lserve_prefill_desc* desc, const void* q, c
  * stats_pool bf16 [num_pool_pages][H_kv][g][2][D] (16-byte aligned).  Token t
  * of KV head h goes to pool id block_table[t / N_P], row t % N_P; rows past
  * seq_len are not written; retrieval heads (head_kind_host[h] == 0) get the
- * k_min / k_max of every logical page.  Each key block of 128 tokens is
- * written by the work tile of its KV head's first query head that ends on it
- * (the diagonal block), while the block is in shared memory.  A bad pool id
- * skips that page and sets LSERVE_ERR_BOUNDS.
+ * k_min / k_max of every logical page.  A warp of the prefill kernel writes
+ * each key block of 128 tokens (the diagonal block of one work tile of its KV
+ * head's first query head), reading it from k / v alongside the attention.
+ * A bad pool id skips that page and sets LSERVE_ERR_BOUNDS.
  */
 int lserve_blocksparse_prefill_paged(const lserve_prefill_desc* desc, const lserve_paged_desc* paged,
                                      const void* q, const void* k, const void* v,
