@@ -3,7 +3,7 @@ whose kernel also hands the sequence to the paged decode cache (K / V through
 the block table into the pools, the retrieval heads' page statistics).
 
 - Its attention output and log-sum-exp equal lserve_blocksparse_prefill's bit
-  for bit (the same kernel schedule; the epilogue only reads the key tiles).
+  for bit (the same kernel schedule; the page writer only reads the inputs).
 - Every valid row of the pools holds the sequence's K / V at its block-table
   position; rows past the sequence and pages the table does not name keep
   their sentinel.
@@ -11,9 +11,9 @@ the block table into the pools, the retrieval heads' page statistics).
   k_max of every logical page; the streaming heads' statistics stay untouched.
 - The result equals what the separate pass lserve_prefill_to_pages writes.
 Shapes cover the paired kernel (G even) and the one-head kernel (G = 1),
-D = 64 and 128, physical pages of 32 to 256 tokens (TMA stores of 32-, 64- and
-128-row boxes, N_P = 192 split across key tiles), logical pages of 8 to 64
-tokens and ragged sequence ends (the last page written by plain stores)."""
+D = 64 and 128, physical pages of 32 to 256 tokens (N_P = 192: pages split
+across 128-token key tiles), logical pages of 8 to 64 tokens and ragged
+sequence ends."""
 import math
 
 import numpy as np
@@ -32,7 +32,7 @@ CASES = [
     (1000, 8, 2, 128, 64, 16, 64, [0, 1]),          # G = 4 (paired kernel), ragged end
     (777, 2, 2, 64, 64, 8, 32, [0, 1]),              # G = 1 (one-head kernel), D = 64, N_P = 32
     (1280, 4, 4, 128, 128, 32, 128, [1, 0, 0, 1]),   # G = 1, N_P = 128, T a multiple of 128
-    (700, 4, 2, 128, 128, 16, 192, [0, 1]),          # N_P = 192: 64-row boxes, pages across tiles
+    (700, 4, 2, 128, 128, 16, 192, [0, 1]),          # N_P = 192: pages across key tiles
     (2100, 8, 2, 64, 64, 64, 256, [0, 0]),           # N_P = 256, N_L = 64, D = 64
     (130, 2, 2, 128, 64, 16, 64, [1, 0]),            # G = 1, two key tiles, 2-token tail
 ]
