@@ -27,6 +27,14 @@ int main(void) {
   /* validation happens before any device work: a null q is rejected */
   if (lserve_page_select(&d, NULL, NULL, NULL, NULL, NULL, 8, NULL, NULL, NULL, NULL, 0, NULL)
       != LSERVE_ERR_INVALID_ARG) return 6;
+  /* the prefill with the paged hand-over: a null block table is rejected */
+  {
+    lserve_prefill_desc pf = {1024, 32, 8, 128, 128, 128, 1, 4};
+    uint8_t kinds[8] = {0, 0, 0, 0, 1, 1, 1, 1};
+    if (lserve_blocksparse_prefill_paged(&pf, &d, NULL, NULL, NULL, kinds, 0.088f, NULL, NULL, NULL,
+                                         NULL, NULL, NULL, NULL, 0, NULL) != LSERVE_ERR_INVALID_ARG)
+      return 7;
+  }
   printf("c client ok\n");
   return 0;
 }
