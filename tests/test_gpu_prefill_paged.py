@@ -35,6 +35,7 @@ CASES = [
     (700, 4, 2, 128, 128, 16, 192, [0, 1]),          # N_P = 192: pages across key tiles
     (2100, 8, 2, 64, 64, 64, 256, [0, 0]),           # N_P = 256, N_L = 64, D = 64
     (130, 2, 2, 128, 64, 16, 64, [1, 0]),            # G = 1, two key tiles, 2-token tail
+    (900, 16, 2, 128, 128, 16, 64, [0, 1]),          # G = 8: four query-head pairs per KV head
 ]
 
 
