@@ -202,11 +202,12 @@ int lserve_page_select(const lserve_paged_desc* desc, const void* q, const void*
  * workspace: lserve_workspace_size(LSERVE_OP_DECODE, desc, top_k) bytes,
  * 256-byte aligned and ZERO-FILLED once before its first use.  It holds the
  * partial results of pairs split over several thread blocks, each word tagged
- * with the pair and a per-pair merge epoch kept in the workspace too; every
- * call advances the epochs it uses, also when it ends in an error (a
- * timeout), so leftovers of any earlier call are never mistaken for this
- * call's: the workspace never needs re-zeroing.  Calls that may run
- * concurrently need separate workspaces.
+ * with the pair and a per-pair merge epoch (20 bits) kept in the workspace
+ * too; every call advances the epochs it uses, also when it ends in an error
+ * (a timeout), so leftovers of earlier calls are not mistaken for this
+ * call's -- only a word left in a slot 2^20 merges of that pair earlier and
+ * never overwritten since could match again: the workspace never needs
+ * re-zeroing.  Calls that may run concurrently need separate workspaces.
  * Limits: B * H_kv <= 2048; N_P = 32 or a multiple of 64.
  */
 int lserve_sparse_decode_attn(const lserve_paged_desc* desc, const void* q, const void* k_pool,
